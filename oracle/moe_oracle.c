@@ -1,0 +1,621 @@
+/*
+ * CPU oracle for the sparse MoE FFN layer forward.
+ *
+ * TEST INFRASTRUCTURE. Only tests/, __graft_entry__.smoke() and bench.py's
+ * cpu_baseline leg may load, call or execute anything under oracle/. The
+ * product path never does; it shares no code, header, table or helper with
+ * this file.
+ *
+ * Plain, slow, obviously correct: every step is the definition written out,
+ * in the order the pages state it. Threads only split independent outputs;
+ * no summation is blocked, split or reordered.
+ *
+ * Precision (and why):
+ *   - router logits: fp32, one accumulator per (token, expert), h ascending.
+ *     The logits decide an integer (the top-k ids), so they are taken in the
+ *     precision of the kernel that must match them. A bf16 x bf16 product is
+ *     exact in fp32 (8 + 8 significand bits), so this is a fully specified
+ *     function of the inputs.
+ *   - routing weights: fp64 exp / sum, rounded once to fp32.
+ *   - expert projections, SwiGLU and the weighted combine: fp64 accumulation,
+ *     each output rounded once to fp32 at the end.
+ *   - FP8: e4m3 codes and their fp32 scales are decided in fp32 (the kernel's
+ *     precision); dequantised values are exact in fp64.
+ *
+ * Parity pins: every function here is checked in tests/ against something
+ * other than itself (fp64 error bounds, brute force, library special cases,
+ * closed forms, exhaustive codec tables).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* small helpers                                                             */
+/* ------------------------------------------------------------------------ */
+static inline float bf16_widen(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+typedef void (*range_fn)(void* ctx, int64_t lo, int64_t hi);
+typedef struct {
+  range_fn fn;
+  void* ctx;
+  int64_t lo, hi;
+} span_t;
+
+static void* span_main(void* a) {
+  span_t* s = (span_t*)a;
+  s->fn(s->ctx, s->lo, s->hi);
+  return NULL;
+}
+
+/* Split [0, n) into nthreads contiguous spans. */
+static void parallel_for(int64_t n, int nthreads, range_fn fn, void* ctx) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if (n < nthreads) nthreads = (int)(n > 0 ? n : 1);
+  pthread_t th[256];
+  span_t sp[256];
+  for (int t = 0; t < nthreads; ++t) {
+    sp[t].fn = fn;
+    sp[t].ctx = ctx;
+    sp[t].lo = n * t / nthreads;
+    sp[t].hi = n * (t + 1) / nthreads;
+    pthread_create(&th[t], NULL, span_main, &sp[t]);
+  }
+  for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Router logits.                                                            */
+/* "Mixture of Experts (MoE): a practical explanation" (lira-now.com), §5    */
+/* "How the Router (Top-k Routing) works step by step", steps 1-2 and the    */
+/* pseudocode's `logits = router(x)`: a linear layer from the token vector   */
+/* to E scores. The bias (when the layer has one) is added to the score.     */
+/*   logits[t, e] = (sum_{h ascending} x[t, h] * Wr[h, e]) + bias[e]         */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+  const uint16_t *x, *wr;
+  const float* bias;
+  const int32_t* tokens;
+  int64_t H, E;
+  float* logits;
+} logits_ctx;
+
+static void logits_rows(void* p, int64_t lo, int64_t hi) {
+  logits_ctx* c = (logits_ctx*)p;
+  enum { EB = 16 }; /* experts computed side by side; each keeps its own h-ascending sum */
+  for (int64_t r = lo; r < hi; ++r) {
+    int64_t t = c->tokens ? c->tokens[r] : r;
+    const uint16_t* xr = c->x + t * c->H;
+    for (int64_t e0 = 0; e0 < c->E; e0 += EB) {
+      int64_t ne = c->E - e0 < EB ? c->E - e0 : EB;
+      float acc[EB];
+      for (int j = 0; j < EB; ++j) acc[j] = 0.0f;
+      for (int64_t h = 0; h < c->H; ++h) {
+        float xv = bf16_widen(xr[h]);
+        const uint16_t* wrow = c->wr + h * c->E + e0;
+        for (int64_t j = 0; j < ne; ++j) acc[j] += xv * bf16_widen(wrow[j]);
+      }
+      for (int64_t j = 0; j < ne; ++j)
+        c->logits[r * c->E + e0 + j] = acc[j] + (c->bias ? c->bias[e0 + j] : 0.0f);
+    }
+  }
+}
+
+/* logits for rows tokens[0..nt) (or 0..nt when tokens == NULL) */
+void oracle_router_logits(const uint16_t* x, const uint16_t* wr, const float* bias,
+                          const int32_t* tokens, int64_t nt, int64_t H, int64_t E, float* logits,
+                          int nthreads) {
+  logits_ctx c = {x, wr, bias, tokens, H, E, logits};
+  parallel_for(nt, nthreads, logits_rows, &c);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Softmax top-k with renormalised weights.                                  */
+/* Same page, §5 steps 3-5 and the pseudocode's `probs = softmax(logits)`,   */
+/* `values, indices = topk(probs, k)`, `weights = values / values.sum()`.    */
+/* softmax is strictly increasing in the logit, so the k largest probs are   */
+/* the k largest logits; ties (equal fp32 logits) go to the lower expert     */
+/* index, and slot j holds the j-th largest. The full softmax denominator    */
+/* cancels in the renormalisation, leaving                                   */
+/*   w_j = exp(l_j - l_max) / sum_{i in selected} exp(l_i - l_max).          */
+/* The toy layer's `+ 1e-9` in the denominator is not used: the denominator  */
+/* is >= 1 because the top term is exp(0).                                   */
+/* ------------------------------------------------------------------------ */
+void oracle_topk(const float* logits, int64_t T, int64_t E, int k, int32_t* ids, float* w) {
+  char* taken = (char*)malloc((size_t)E);
+  double* ex = (double*)malloc(sizeof(double) * (size_t)k);
+  for (int64_t t = 0; t < T; ++t) {
+    const float* l = logits + t * E;
+    memset(taken, 0, (size_t)E);
+    for (int j = 0; j < k; ++j) {
+      int64_t best = -1;
+      for (int64_t e = 0; e < E; ++e) {
+        if (taken[e]) continue;
+        if (best < 0 || l[e] > l[best]) best = e; /* strict >: lower index wins ties */
+      }
+      taken[best] = 1;
+      ids[t * k + j] = (int32_t)best;
+    }
+    double lmax = (double)l[ids[t * k]];
+    double den = 0.0;
+    for (int j = 0; j < k; ++j) {
+      ex[j] = exp((double)l[ids[t * k + j]] - lmax);
+      den += ex[j];
+    }
+    for (int j = 0; j < k; ++j) w[t * k + j] = (float)(ex[j] / den);
+  }
+  free(taken);
+  free(ex);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Permutation by expert.                                                    */
+/* "Experts backends" (HF Transformers docs), backend table, `grouped_mm`    */
+/* row: the routed tokens are sorted by chosen expert so each expert's rows  */
+/* are contiguous for one grouped GEMM. Order is expert-major, then token    */
+/* ascending (a token holds each expert at most once), which makes the       */
+/* result unique:                                                            */
+/*   offsets[0] = 0, offsets[e+1] = offsets[e] + count[e]                    */
+/*   row p in [offsets[e], offsets[e+1]) is (token, slot) pairs with expert  */
+/*   e, in ascending token order; inv_perm[t*k + j] = p.                     */
+/* ------------------------------------------------------------------------ */
+void oracle_permute(const int32_t* ids, int64_t T, int64_t E, int k, int32_t* offsets,
+                    int32_t* perm_token, int32_t* perm_slot, int32_t* inv_perm) {
+  for (int64_t e = 0; e <= E; ++e) offsets[e] = 0;
+  for (int64_t i = 0; i < T * k; ++i) offsets[ids[i] + 1] += 1;
+  for (int64_t e = 0; e < E; ++e) offsets[e + 1] += offsets[e];
+  int64_t p = 0;
+  for (int64_t e = 0; e < E; ++e) {
+    for (int64_t t = 0; t < T; ++t) {
+      for (int j = 0; j < k; ++j) {
+        if (ids[t * k + j] == e) {
+          perm_token[p] = (int32_t)t;
+          perm_slot[p] = j;
+          inv_perm[t * k + j] = (int32_t)p;
+          ++p;
+        }
+      }
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Expert FFN: gated MLP, up/gate projection -> SwiGLU -> down projection.    */
+/* "Experts backends", `deepgemm_megamoe` row and "SonicMoE" section: the     */
+/* expert is a gated MLP (gate and up projections, SwiGLU, down projection). */
+/* SiLU goes on the gate projection, the up projection stays linear:         */
+/*   g_i = sum_h x_h Wg[e,h,i],  u_i = sum_h x_h Wu[e,h,i]                   */
+/*   a_i = silu(g_i) * u_i,      silu(z) = z / (1 + exp(-z))                 */
+/*   y_c = sum_i a_i Wd[e,i,c]                                               */
+/* Weights arrive K-major: w13[e] = [Wg[e]^T ; Wu[e]^T] ([2I, H]) and        */
+/* w2[e] = Wd[e]^T ([H, I]).                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Up to GROUP rows are evaluated side by side so the fp64 sums vectorise
+ * across rows; every (row, output) sum still runs over its index ascending. */
+#define GROUP 8
+
+/* a[n, I] (fp64) from fp64 activation rows xT[H][GROUP] (row r in column r) */
+static void expert_hidden(const double* xT, int64_t n, const uint16_t* w13e, const double* w13e_d,
+                          int64_t H, int64_t I, double* a) {
+  for (int64_t i = 0; i < I; ++i) {
+    double g[GROUP], u[GROUP];
+    for (int r = 0; r < GROUP; ++r) g[r] = u[r] = 0.0;
+    for (int64_t h = 0; h < H; ++h) {
+      double wg, wu;
+      if (w13e_d) {
+        wg = w13e_d[i * H + h];
+        wu = w13e_d[(I + i) * H + h];
+      } else {
+        wg = (double)bf16_widen(w13e[i * H + h]);
+        wu = (double)bf16_widen(w13e[(I + i) * H + h]);
+      }
+      const double* xh = xT + h * GROUP;
+      for (int r = 0; r < GROUP; ++r) {
+        g[r] += xh[r] * wg;
+        u[r] += xh[r] * wu;
+      }
+    }
+    for (int64_t r = 0; r < n; ++r) a[r * I + i] = g[r] / (1.0 + exp(-g[r])) * u[r];
+  }
+}
+
+/* y[n, H] (fp64) from fp64 hidden rows aT[I][GROUP] */
+static void expert_out(const double* aT, int64_t n, const uint16_t* w2e, const double* w2e_d,
+                       int64_t H, int64_t I, double* y) {
+  for (int64_t c = 0; c < H; ++c) {
+    double acc[GROUP];
+    for (int r = 0; r < GROUP; ++r) acc[r] = 0.0;
+    for (int64_t i = 0; i < I; ++i) {
+      double wd = w2e_d ? w2e_d[c * I + i] : (double)bf16_widen(w2e[c * I + i]);
+      const double* ai = aT + i * GROUP;
+      for (int r = 0; r < GROUP; ++r) acc[r] += ai[r] * wd;
+    }
+    for (int64_t r = 0; r < n; ++r) y[r * H + c] = acc[r];
+  }
+}
+
+/* transpose rows [n, C] into [C][GROUP], zero-padding missing rows */
+static void to_cols(const double* rows, int64_t n, int64_t C, double* T) {
+  for (int64_t c = 0; c < C; ++c)
+    for (int r = 0; r < GROUP; ++r) T[c * GROUP + r] = r < n ? rows[r * C + c] : 0.0;
+}
+
+/* Exposed pieces, used by the tests to pin one GEMM stage at a time.
+ * a_rows: [n, H] bf16 rows; out: [n, I] fp32 (each value rounded once). */
+void oracle_expert_swiglu_rows(const uint16_t* a_rows, int64_t n, const uint16_t* w13e, int64_t H,
+                               int64_t I, float* out) {
+  double* xr = (double*)malloc(sizeof(double) * (size_t)(GROUP * H));
+  double* xT = (double*)malloc(sizeof(double) * (size_t)(GROUP * H));
+  double* a = (double*)malloc(sizeof(double) * (size_t)(GROUP * I));
+  for (int64_t r0 = 0; r0 < n; r0 += GROUP) {
+    int64_t m = n - r0 < GROUP ? n - r0 : GROUP;
+    for (int64_t i = 0; i < m * H; ++i) xr[i] = (double)bf16_widen(a_rows[r0 * H + i]);
+    to_cols(xr, m, H, xT);
+    expert_hidden(xT, m, w13e, NULL, H, I, a);
+    for (int64_t i = 0; i < m * I; ++i) out[r0 * I + i] = (float)a[i];
+  }
+  free(xr);
+  free(xT);
+  free(a);
+}
+
+/* h_rows: [n, I] bf16 rows; out: [n, H] fp32 */
+void oracle_expert_down_rows(const uint16_t* h_rows, int64_t n, const uint16_t* w2e, int64_t H,
+                             int64_t I, float* out) {
+  double* a = (double*)malloc(sizeof(double) * (size_t)(GROUP * I));
+  double* aT = (double*)malloc(sizeof(double) * (size_t)(GROUP * I));
+  double* y = (double*)malloc(sizeof(double) * (size_t)(GROUP * H));
+  for (int64_t r0 = 0; r0 < n; r0 += GROUP) {
+    int64_t m = n - r0 < GROUP ? n - r0 : GROUP;
+    for (int64_t i = 0; i < m * I; ++i) a[i] = (double)bf16_widen(h_rows[r0 * I + i]);
+    to_cols(a, m, I, aT);
+    expert_out(aT, m, w2e, NULL, H, I, y);
+    for (int64_t i = 0; i < m * H; ++i) out[r0 * H + i] = (float)y[i];
+  }
+  free(a);
+  free(aT);
+  free(y);
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 e4m3 (OCP E4M3FN: 1 sign, 4 exponent bits with bias 7, 3 mantissa    */
+/* bits; no infinities; S.1111.111 is NaN; largest finite 448).              */
+/* "Fine-grained FP8" (HF Transformers docs), opening list: weights are      */
+/* quantised to 8 bits per 128 x 128 block, activations per token per group  */
+/* of 128 input channels, dynamically.                                       */
+/* ------------------------------------------------------------------------ */
+double oracle_e4m3_decode(uint8_t q) {
+  int s = q >> 7, ef = (q >> 3) & 15, m = q & 7;
+  if (ef == 15 && m == 7) return NAN;
+  double v = ef == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, ef - 7);
+  return s ? -v : v;
+}
+
+/* Round a finite float to the nearest e4m3 code, ties to even, saturating at
+ * +-448 (values this layer encodes never exceed 448 * (1 + 2^-23)). */
+uint8_t oracle_e4m3_encode(float f) {
+  uint8_t s = signbit(f) ? 0x80 : 0;
+  double a = fabs((double)f);
+  if (a >= 464.0) return s | 0x7E; /* beyond the 448/480 midpoint: saturate */
+  if (a < ldexp(1.0, -6)) {      /* subnormal range: multiples of 2^-9 */
+    double m = rint(ldexp(a, 9)); /* default mode rounds ties to even */
+    return s | (uint8_t)m;       /* m == 8 is the code of 2^-6, as wanted */
+  }
+  int ex;
+  frexp(a, &ex); /* a = f * 2^ex, f in [0.5, 1) -> unbiased exponent ex-1 */
+  int e = ex - 1;
+  double m = rint((ldexp(a, -e) - 1.0) * 8.0);
+  if (m == 8.0) {
+    m = 0.0;
+    e += 1;
+  }
+  if (e > 8) return s | 0x7E;
+  return s | (uint8_t)(((e + 7) << 3) | (int)m);
+}
+
+/* amax / 448 in fp32 with IEEE division; an all-zero group gets scale 1 */
+static inline float group_scale(float amax) { return amax > 0.0f ? amax / 448.0f : 1.0f; }
+
+/* Per row, per group of 128 consecutive columns: s = amax/448, q = e4m3(v/s).
+ * vals: [rows, cols] fp32 (already widened); q: [rows, cols]; s: [rows, cols/128]. */
+static void quant_groups_f32(const float* vals, int64_t rows, int64_t cols, uint8_t* q, float* s) {
+  int64_t G = cols / 128;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t g = 0; g < G; ++g) {
+      const float* v = vals + r * cols + g * 128;
+      float amax = 0.0f;
+      for (int c = 0; c < 128; ++c) amax = fmaxf(amax, fabsf(v[c]));
+      float sc = group_scale(amax);
+      s[r * G + g] = sc;
+      for (int c = 0; c < 128; ++c) q[r * cols + g * 128 + c] = oracle_e4m3_encode(v[c] / sc);
+    }
+  }
+}
+
+/* Activation quantisation of bf16 rows [rows, cols]. */
+void oracle_quant_act_fp8(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* s) {
+  float* v = (float*)malloc(sizeof(float) * (size_t)cols);
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < cols; ++c) v[c] = bf16_widen(x[r * cols + c]);
+    quant_groups_f32(v, 1, cols, q + r * cols, s + r * (cols / 128));
+  }
+  free(v);
+}
+
+/* Weight quantisation of nb matrices of bf16 [rows, cols] in 128 x 128
+ * blocks: q [nb, rows, cols], s [nb, rows/128, cols/128]. */
+void oracle_quant_weight_fp8(const uint16_t* w, int64_t nb, int64_t rows, int64_t cols,
+                             uint8_t* q, float* s) {
+  int64_t RB = rows / 128, CB = cols / 128;
+  for (int64_t b = 0; b < nb; ++b) {
+    const uint16_t* wb = w + b * rows * cols;
+    for (int64_t rb = 0; rb < RB; ++rb) {
+      for (int64_t cb = 0; cb < CB; ++cb) {
+        float amax = 0.0f;
+        for (int64_t r = rb * 128; r < rb * 128 + 128; ++r)
+          for (int64_t c = cb * 128; c < cb * 128 + 128; ++c)
+            amax = fmaxf(amax, fabsf(bf16_widen(wb[r * cols + c])));
+        float sc = group_scale(amax);
+        s[(b * RB + rb) * CB + cb] = sc;
+        for (int64_t r = rb * 128; r < rb * 128 + 128; ++r)
+          for (int64_t c = cb * 128; c < cb * 128 + 128; ++c)
+            q[b * rows * cols + r * cols + c] = oracle_e4m3_encode(bf16_widen(wb[r * cols + c]) / sc);
+      }
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* The layer: the eager per-expert loop.                                     */
+/* "Experts backends", backend table, `eager` row (loop over the selected    */
+/* experts, project their tokens), and "Mixture of Experts (MoE): a          */
+/* practical explanation" §13's toy layer: for each slot j, for each expert  */
+/* e, the tokens whose slot-j expert is e get out += w[t, j] * expert_e(x_t). */
+/* Per token the k contributions are summed in slot order j = 0..k-1.        */
+/* Runs on a subset of tokens (each token's output depends on that token     */
+/* only, §5 pseudocode's `y = sum_i weights_i * expert_i(x)`).               */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+  const uint16_t* x;
+  int64_t H, I, E;
+  int k;
+  const int32_t* tokens;
+  int64_t nt;
+  /* bf16 weights, or e4m3 codes + fp32 block scales */
+  const uint16_t *w13, *w2;
+  const uint8_t *w13q, *w2q, *xq;
+  const float *w13s, *w2s, *xs;
+  int fp8;
+  /* work list: items of up to CHUNK (row, slot) pairs of one expert */
+  int64_t* item_e;
+  int64_t* item_start; /* into pairs */
+  int64_t* item_len;
+  int32_t* pair_row;
+  int32_t* pair_slot;
+  int64_t nitems;
+  int64_t next;
+  pthread_mutex_t mu;
+  double* y; /* [nt, k, H]: expert output of (row, slot) */
+} fwd_ctx;
+
+static void dequant_fp8(const uint8_t* q, const float* s, int64_t rows, int64_t cols, double* out) {
+  int64_t CB = cols / 128;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < cols; ++c)
+      out[r * cols + c] = oracle_e4m3_decode(q[r * cols + c]) * (double)s[(r / 128) * CB + c / 128];
+}
+
+static void* fwd_worker(void* p) {
+  fwd_ctx* c = (fwd_ctx*)p;
+  int64_t H = c->H, I = c->I;
+  double* xr = (double*)malloc(sizeof(double) * (size_t)(GROUP * H));
+  double* xT = (double*)malloc(sizeof(double) * (size_t)(GROUP * H));
+  double* a = (double*)malloc(sizeof(double) * (size_t)(GROUP * I));
+  double* aT = (double*)malloc(sizeof(double) * (size_t)(GROUP * I));
+  double* y = (double*)malloc(sizeof(double) * (size_t)(GROUP * H));
+  float* af = (float*)malloc(sizeof(float) * (size_t)I);
+  uint8_t* aq = (uint8_t*)malloc((size_t)I);
+  float* as = (float*)malloc(sizeof(float) * (size_t)(I / 128 + 1));
+  double *w13d = NULL, *w2d = NULL;
+  int64_t cur_e = -1;
+  if (c->fp8) {
+    w13d = (double*)malloc(sizeof(double) * (size_t)(2 * I * H));
+    w2d = (double*)malloc(sizeof(double) * (size_t)(H * I));
+  }
+  for (;;) {
+    pthread_mutex_lock(&c->mu);
+    int64_t it = c->next++;
+    pthread_mutex_unlock(&c->mu);
+    if (it >= c->nitems) break;
+    int64_t e = c->item_e[it];
+    const uint16_t* w13e = c->fp8 ? NULL : c->w13 + e * 2 * I * H;
+    const uint16_t* w2e = c->fp8 ? NULL : c->w2 + e * H * I;
+    if (c->fp8 && e != cur_e) { /* w-hat = e4m3 code * its block scale */
+      dequant_fp8(c->w13q + e * 2 * I * H, c->w13s + e * (2 * I / 128) * (H / 128), 2 * I, H, w13d);
+      dequant_fp8(c->w2q + e * H * I, c->w2s + e * (H / 128) * (I / 128), H, I, w2d);
+      cur_e = e;
+    }
+    for (int64_t g0 = 0; g0 < c->item_len[it]; g0 += GROUP) {
+      int64_t n = c->item_len[it] - g0 < GROUP ? c->item_len[it] - g0 : GROUP;
+      const int32_t* rows = c->pair_row + c->item_start[it] + g0;
+      const int32_t* slots = c->pair_slot + c->item_start[it] + g0;
+      for (int64_t r = 0; r < n; ++r) {
+        int64_t t = c->tokens[rows[r]];
+        for (int64_t h = 0; h < H; ++h) {
+          if (c->fp8) /* x-hat = e4m3(x / s) * s per (token, 128-group) */
+            xr[r * H + h] = oracle_e4m3_decode(c->xq[rows[r] * H + h]) *
+                            (double)c->xs[rows[r] * (H / 128) + h / 128];
+          else
+            xr[r * H + h] = (double)bf16_widen(c->x[t * H + h]);
+        }
+      }
+      to_cols(xr, n, H, xT);
+      expert_hidden(xT, n, w13e, w13d, H, I, a);
+      if (c->fp8) { /* the down projection's input is quantised per (row, 128-group) too */
+        for (int64_t r = 0; r < n; ++r) {
+          for (int64_t i = 0; i < I; ++i) af[i] = (float)a[r * I + i];
+          quant_groups_f32(af, 1, I, aq, as);
+          for (int64_t i = 0; i < I; ++i) a[r * I + i] = oracle_e4m3_decode(aq[i]) * (double)as[i / 128];
+        }
+      }
+      to_cols(a, n, I, aT);
+      expert_out(aT, n, w2e, w2d, H, I, y);
+      for (int64_t r = 0; r < n; ++r)
+        memcpy(c->y + ((int64_t)rows[r] * c->k + slots[r]) * H, y + r * H, sizeof(double) * (size_t)H);
+    }
+  }
+  free(xr);
+  free(xT);
+  free(a);
+  free(aT);
+  free(y);
+  free(af);
+  free(aq);
+  free(as);
+  free(w13d);
+  free(w2d);
+  return NULL;
+}
+
+/* The toy layer's (slot j, expert e) loops evaluate expert e on every token
+ * whose slot-j choice is e. The same (token, slot) evaluations are made here,
+ * grouped by expert so one expert's weights are read together; each is an
+ * independent computation, and the k results of a token are then summed in
+ * slot order j = 0..k-1. */
+static void run_forward(fwd_ctx* c, const int32_t* ids, const float* topk_w, float* out,
+                        int nthreads) {
+  int64_t nt = c->nt, k = c->k, E = c->E, H = c->H;
+  const int64_t CHUNK = 64;
+  int64_t max_items = E + nt * k / CHUNK + 1;
+  c->item_e = (int64_t*)malloc(sizeof(int64_t) * (size_t)max_items);
+  c->item_start = (int64_t*)malloc(sizeof(int64_t) * (size_t)max_items);
+  c->item_len = (int64_t*)malloc(sizeof(int64_t) * (size_t)max_items);
+  c->pair_row = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nt * k + 1));
+  c->pair_slot = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nt * k + 1));
+  c->y = (double*)calloc((size_t)(nt * k * H), sizeof(double));
+  int64_t p = 0, ni = 0;
+  for (int64_t e = 0; e < E; ++e) {
+    int64_t start = p;
+    for (int64_t r = 0; r < nt; ++r)
+      for (int64_t j = 0; j < k; ++j)
+        if (ids[r * k + j] == e) {
+          c->pair_row[p] = (int32_t)r;
+          c->pair_slot[p] = (int32_t)j;
+          ++p;
+        }
+    for (int64_t s0 = start; s0 < p; s0 += CHUNK) {
+      c->item_e[ni] = e;
+      c->item_start[ni] = s0;
+      c->item_len[ni] = p - s0 < CHUNK ? p - s0 : CHUNK;
+      ++ni;
+    }
+  }
+  c->nitems = ni;
+  c->next = 0;
+  pthread_mutex_init(&c->mu, NULL);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  pthread_t th[256];
+  for (int t = 0; t < nthreads; ++t) pthread_create(&th[t], NULL, fwd_worker, c);
+  for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+  pthread_mutex_destroy(&c->mu);
+  /* weighted combine: out[t] = sum_{j ascending} w[t, j] * y[t, j] */
+  for (int64_t r = 0; r < nt; ++r) {
+    for (int64_t h = 0; h < H; ++h) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < k; ++j) acc += (double)topk_w[r * k + j] * c->y[(r * k + j) * H + h];
+      out[r * H + h] = (float)acc;
+    }
+  }
+  free(c->item_e);
+  free(c->item_start);
+  free(c->item_len);
+  free(c->pair_row);
+  free(c->pair_slot);
+  free(c->y);
+}
+
+/* Experts + combine for given routing (ids/w [nt, k]) of tokens[0..nt).
+ * out: [nt, H] fp32. */
+void oracle_experts_combine(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H,
+                            int64_t I, int64_t E, int k, const int32_t* ids, const float* topk_w,
+                            const uint16_t* w13, const uint16_t* w2, float* out, int nthreads) {
+  fwd_ctx c;
+  memset(&c, 0, sizeof(c));
+  c.x = x;
+  c.H = H;
+  c.I = I;
+  c.E = E;
+  c.k = k;
+  c.tokens = tokens;
+  c.nt = nt;
+  c.w13 = w13;
+  c.w2 = w2;
+  run_forward(&c, ids, topk_w, out, nthreads);
+}
+
+/* FP8 experts + combine: x is quantised here per (token, 128-group), weights
+ * are given as e4m3 codes with fp32 128 x 128 block scales. */
+void oracle_experts_combine_fp8(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H,
+                                int64_t I, int64_t E, int k, const int32_t* ids,
+                                const float* topk_w, const uint8_t* w13q, const float* w13s,
+                                const uint8_t* w2q, const float* w2s, float* out, int nthreads) {
+  uint8_t* xq = (uint8_t*)malloc((size_t)(nt * H));
+  float* xs = (float*)malloc(sizeof(float) * (size_t)(nt * (H / 128)));
+  uint16_t* xrows = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)H);
+  for (int64_t r = 0; r < nt; ++r) {
+    memcpy(xrows, x + (int64_t)tokens[r] * H, sizeof(uint16_t) * (size_t)H);
+    oracle_quant_act_fp8(xrows, 1, H, xq + r * H, xs + r * (H / 128));
+  }
+  fwd_ctx c;
+  memset(&c, 0, sizeof(c));
+  c.x = x;
+  c.H = H;
+  c.I = I;
+  c.E = E;
+  c.k = k;
+  c.tokens = tokens;
+  c.nt = nt;
+  c.w13q = w13q;
+  c.w13s = w13s;
+  c.w2q = w2q;
+  c.w2s = w2s;
+  c.xq = xq;
+  c.xs = xs;
+  c.fp8 = 1;
+  run_forward(&c, ids, topk_w, out, nthreads);
+  free(xq);
+  free(xs);
+  free(xrows);
+}
+
+/* The whole layer for tokens[0..nt): logits -> top-k -> experts -> combine.
+ * ids_out/w_out ([nt, k]) and logits_out ([nt, E]) may be NULL. */
+void oracle_moe_forward(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H, int64_t I,
+                        int64_t E, int k, const uint16_t* wr, const float* bias,
+                        const uint16_t* w13, const uint16_t* w2, const uint8_t* w13q,
+                        const float* w13s, const uint8_t* w2q, const float* w2s, float* out,
+                        int32_t* ids_out, float* w_out, float* logits_out, int nthreads) {
+  float* logits = logits_out ? logits_out : (float*)malloc(sizeof(float) * (size_t)(nt * E));
+  int32_t* ids = ids_out ? ids_out : (int32_t*)malloc(sizeof(int32_t) * (size_t)(nt * k));
+  float* w = w_out ? w_out : (float*)malloc(sizeof(float) * (size_t)(nt * k));
+  oracle_router_logits(x, wr, bias, tokens, nt, H, E, logits, nthreads);
+  oracle_topk(logits, nt, E, k, ids, w);
+  if (w13q)
+    oracle_experts_combine_fp8(x, tokens, nt, H, I, E, k, ids, w, w13q, w13s, w2q, w2s, out,
+                               nthreads);
+  else
+    oracle_experts_combine(x, tokens, nt, H, I, E, k, ids, w, w13, w2, out, nthreads);
+  if (!logits_out) free(logits);
+  if (!ids_out) free(ids);
+  if (!w_out) free(w);
+}

@@ -1,0 +1,397 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each test checks one oracle function against a closed form, a rigorous error
+bound, brute force on tiny inputs, an invariant, a library routine, or the
+hand-worked example in tests/golden/. Together they are chosen so that a
+dropped term, a wrong sign or index, a transposed operand or a wrong tie rule
+in the oracle fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _small(name="tiny", **kw):
+    return mi.CONFIGS[name].with_(**kw)
+
+
+def _logical_weights(cfg):
+    """Wg, Wu [E,H,I], Wd [E,I,H] in fp64 drawn in their logical layout (no packing)."""
+    E, H, I = cfg.E, cfg.H, cfg.I
+    wg = mi.bf16_to_f32(mi.normal_bf16(cfg.seed, mi.TAG_WG, cfg.w_sigma, E, H, I)).reshape(E, H, I)
+    wu = mi.bf16_to_f32(mi.normal_bf16(cfg.seed, mi.TAG_WU, cfg.w_sigma, E, H, I)).reshape(E, H, I)
+    wd = mi.bf16_to_f32(mi.normal_bf16(cfg.seed, mi.TAG_WD, cfg.w_sigma, E, I, H)).reshape(E, I, H)
+    return wg.astype(np.float64), wu.astype(np.float64), wd.astype(np.float64)
+
+
+def _bf16(a):
+    return mi.f32_to_bf16(np.asarray(a, dtype=np.float32))
+
+
+# --------------------------------------------------------------------------
+# the hand-worked example (closed forms)
+# --------------------------------------------------------------------------
+def _golden_layer():
+    g = json.load(open(os.path.join(GOLDEN, "hand_worked_layer.json")))
+    d = g["dims"]
+    E, H, I = d["E"], d["H"], d["I"]
+    wg = np.array(g["wg_EHI"], dtype=np.float32)
+    wu = np.array(g["wu_EHI"], dtype=np.float32)
+    wd = np.array(g["wd_EIH"], dtype=np.float32)
+    w13 = np.concatenate([wg.transpose(0, 2, 1), wu.transpose(0, 2, 1)], axis=1)  # [E,2I,H]
+    w2 = wd.transpose(0, 2, 1)  # [E,H,I]
+    return g, dict(x=_bf16(g["x"]), wr=_bf16(g["wr_HE"]), bias=np.array(g["bias"], np.float32),
+                   w13=_bf16(w13), w2=_bf16(w2), k=d["k"], E=E)
+
+
+def test_hand_worked_layer():
+    g, L = _golden_layer()
+    exp = g["expected"]
+    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=L["k"])
+    np.testing.assert_array_equal(r["logits"], np.array(exp["logits"], np.float32))
+    np.testing.assert_array_equal(r["ids"], np.array(exp["ids"]))
+    np.testing.assert_allclose(r["w"], np.array(exp["w"]), rtol=0, atol=2 ** -24)
+    np.testing.assert_allclose(r["out"], np.array(exp["out"]), rtol=2 ** -22, atol=0)
+    offsets, perm_token, _, inv_perm = oracle.permute(r["ids"], L["E"])
+    np.testing.assert_array_equal(offsets, exp["offsets"])
+    np.testing.assert_array_equal(perm_token, exp["perm_token"])
+    np.testing.assert_array_equal(inv_perm, exp["inv_perm"])
+
+
+# --------------------------------------------------------------------------
+# router logits: rigorous fp32 summation bound against an fp64 recomputation
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("H,E,T", [(128, 8, 64), (1024, 32, 16), (96, 5, 7)])
+def test_logits_within_higham_bound(H, E, T):
+    cfg = _small(H=H, E=E, T=T, bias="normal")
+    x = mi.make_x(cfg)
+    wr, b = mi.make_router(cfg)
+    l32 = oracle.router_logits(x, wr, b)
+    xf = mi.bf16_to_f32(x).astype(np.float64)
+    wf = mi.bf16_to_f32(wr).astype(np.float64)
+    l64 = xf @ wf + b.astype(np.float64)
+    # recursive summation of H exact products: |err| <= gamma_{H-1} sum|x w| (Higham Thm 3.1),
+    # plus one rounding of the bias add
+    u = 2.0 ** -24
+    gam = (H - 1) * u / (1 - (H - 1) * u)
+    bound = gam * (np.abs(xf) @ np.abs(wf)) + u * (np.abs(l64) + 1e-30) * 2
+    err = np.abs(l32.astype(np.float64) - l64)
+    assert np.all(err <= bound), float((err - bound).max())
+    # sensitivity: a sum missing one product (a dropped term) breaks the bound almost everywhere
+    dropped = l64 - xf[:, :1] @ wf[:1, :]
+    assert np.mean(np.abs(dropped - l64) > bound) > 0.75
+
+
+def test_logits_subset_rows_match_full():
+    cfg = _small(T=40)
+    x = mi.make_x(cfg)
+    wr, b = mi.make_router(cfg)
+    full = oracle.router_logits(x, wr, b)
+    toks = np.array([3, 17, 39], dtype=np.int32)
+    np.testing.assert_array_equal(oracle.router_logits(x, wr, b, tokens=toks), full[toks])
+
+
+# --------------------------------------------------------------------------
+# top-k selection and weights
+# --------------------------------------------------------------------------
+def _brute_topk(logits, k):
+    ids = np.empty((logits.shape[0], k), np.int32)
+    for t, l in enumerate(logits):
+        order = np.lexsort((np.arange(len(l)), -l.astype(np.float64)))  # logit desc, index asc
+        ids[t] = order[:k]
+    return ids
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (256, 8), (5, 5), (7, 1), (1, 1), (64, 16)])
+def test_topk_matches_lexsort_and_softmax(E, k):
+    rng = np.random.default_rng(E * 100 + k)
+    T = 50
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    logits[::7, : E // 2] = 0.25  # planted exact ties
+    ids, w = oracle.topk(logits, k)
+    np.testing.assert_array_equal(ids, _brute_topk(logits, k))
+    # renormalised weights = softmax over the selected logits (library routine, fp64)
+    sel = np.take_along_axis(logits, ids, 1).astype(np.float64)
+    ref = torch.softmax(torch.from_numpy(sel), dim=1).numpy()
+    np.testing.assert_allclose(w, ref, rtol=0, atol=2 ** -24)
+    assert np.all(np.abs(w.astype(np.float64).sum(1) - 1) <= k * 2 ** -24)
+    # every selected logit >= every unselected one
+    for t in range(T):
+        mask = np.ones(E, bool)
+        mask[ids[t]] = False
+        if mask.any():
+            assert logits[t, ids[t]].min() >= logits[t, mask].max()
+
+
+def test_topk_all_equal_is_first_k_with_uniform_weights():
+    logits = np.full((3, 16), -1.5, np.float32)
+    ids, w = oracle.topk(logits, 4)
+    np.testing.assert_array_equal(ids, np.tile(np.arange(4), (3, 1)))
+    np.testing.assert_array_equal(w, np.full((3, 4), 0.25, np.float32))
+
+
+def test_topk_k_equals_E_is_full_softmax():
+    rng = np.random.default_rng(1)
+    logits = rng.standard_normal((20, 8)).astype(np.float32)
+    ids, w = oracle.topk(logits, 8)
+    full = torch.softmax(torch.from_numpy(logits.astype(np.float64)), 1).numpy()
+    np.testing.assert_allclose(w, np.take_along_axis(full, ids, 1), rtol=0, atol=2 ** -24)
+
+
+def test_topk_k1_weight_is_one():
+    rng = np.random.default_rng(2)
+    logits = rng.standard_normal((30, 8)).astype(np.float32)
+    ids, w = oracle.topk(logits, 1)
+    np.testing.assert_array_equal(w, np.ones((30, 1), np.float32))
+    np.testing.assert_array_equal(ids[:, 0], np.argmax(logits, 1))
+
+
+# --------------------------------------------------------------------------
+# permutation
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("T,E,k", [(64, 8, 2), (33, 256, 8), (1, 4, 4), (100, 1, 1), (17, 3, 2)])
+def test_permute_is_stable_sort_by_expert(T, E, k):
+    rng = np.random.default_rng(T * 7 + E)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    if E > 2:  # skew: expert 1 in slot 0 for the first half (swapped in, no duplicates)
+        for t in range(T // 2):
+            row = list(ids[t])
+            if 1 in row:
+                i = row.index(1)
+                row[0], row[i] = row[i], row[0]
+            else:
+                row[0] = 1
+            ids[t] = row
+    offsets, perm_token, perm_slot, inv_perm = oracle.permute(ids, E)
+    flat = ids.reshape(-1)
+    tok = np.repeat(np.arange(T), k)
+    order = np.argsort(flat.astype(np.int64) * T + tok, kind="stable")  # library stable sort
+    np.testing.assert_array_equal(perm_token, tok[order])
+    np.testing.assert_array_equal(perm_slot, np.tile(np.arange(k), T)[order])
+    counts = np.bincount(flat, minlength=E)
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    assert offsets[-1] == T * k and np.all(np.diff(offsets) >= 0)
+    # bijection, and inv_perm inverts it
+    assert sorted(inv_perm.reshape(-1).tolist()) == list(range(T * k))
+    for t in range(T):
+        for j in range(k):
+            p = inv_perm[t, j]
+            assert perm_token[p] == t and perm_slot[p] == j
+
+
+# --------------------------------------------------------------------------
+# experts + combine
+# --------------------------------------------------------------------------
+def _dense_masked(cfg, L, ids, w):
+    """Every expert on every token (fp64, logical weights), then masked by top-k."""
+    wg, wu, wd = _logical_weights(cfg)
+    x = mi.bf16_to_f32(L["x"]).astype(np.float64)
+    out = np.zeros((cfg.T, cfg.H))
+    for e in range(cfg.E):
+        g = x @ wg[e]
+        u = x @ wu[e]
+        y = (torch.nn.functional.silu(torch.from_numpy(g)).numpy() * u) @ wd[e]
+        for j in range(cfg.k):
+            m = ids[:, j] == e
+            out[m] += w[m, j:j + 1].astype(np.float64) * y[m]
+    return out
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("tiny", dict(T=19, E=5, k=3, H=64, I=96,
+                                                                   bias="normal"))])
+def test_forward_matches_dense_masked_brute_force(name, kw):
+    cfg = _small(name, **kw)
+    L = mi.make_layer(cfg)
+    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k)
+    ref = _dense_masked(cfg, L, r["ids"], r["w"])
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-6, atol=1e-7 * np.abs(ref).max())
+
+
+def test_one_hot_identical_experts_equal_one_dense_ffn():
+    cfg = _small(T=24, E=4, k=1, H=64, I=128)
+    L = mi.make_layer(cfg)
+    w13 = np.repeat(L["w13"][:1], cfg.E, axis=0)
+    w2 = np.repeat(L["w2"][:1], cfg.E, axis=0)
+    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], w13, w2, k=1)
+    x = torch.from_numpy(mi.bf16_to_f32(L["x"]).astype(np.float64))
+    W13 = torch.from_numpy(mi.bf16_to_f32(L["w13"][0]).astype(np.float64))
+    W2 = torch.from_numpy(mi.bf16_to_f32(L["w2"][0]).astype(np.float64))
+    g = torch.nn.functional.linear(x, W13[: cfg.I])
+    u = torch.nn.functional.linear(x, W13[cfg.I:])
+    ref = torch.nn.functional.linear(torch.nn.functional.silu(g) * u, W2).numpy()
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-6, atol=1e-7 * np.abs(ref).max())
+
+
+def test_identical_experts_k2_equal_one_dense_ffn():
+    cfg = _small(T=16, E=6, k=2, H=64, I=64, bias="normal")
+    L = mi.make_layer(cfg)
+    w13 = np.repeat(L["w13"][2:3], cfg.E, axis=0)
+    w2 = np.repeat(L["w2"][2:3], cfg.E, axis=0)
+    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], w13, w2, k=2)
+    one = oracle.moe_forward(L["x"], L["wr"], L["bias"], w13, w2, k=1)
+    np.testing.assert_allclose(r["out"], one["out"], rtol=1e-6, atol=1e-7)
+
+
+def test_stage_pieces_match_dense():
+    cfg = _small(T=10, E=3, k=2, H=64, I=32)
+    L = mi.make_layer(cfg)
+    wg, wu, wd = _logical_weights(cfg)
+    x = mi.bf16_to_f32(L["x"]).astype(np.float64)
+    h = oracle.expert_swiglu_rows(L["x"], L["w13"][1])
+    g, u = x @ wg[1], x @ wu[1]
+    np.testing.assert_allclose(h, g / (1 + np.exp(-g)) * u, rtol=1e-6, atol=1e-9)
+    hb = mi.f32_to_bf16(h)
+    y = oracle.expert_down_rows(hb, L["w2"][1])
+    np.testing.assert_allclose(y, mi.bf16_to_f32(hb).astype(np.float64) @ wd[1], rtol=1e-6,
+                               atol=1e-9)
+
+
+def test_subset_forward_equals_full_forward_rows():
+    cfg = _small(T=48)
+    L = mi.make_layer(cfg)
+    full = oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k)
+    toks = np.array([0, 5, 47], np.int32)
+    sub = oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k, tokens=toks)
+    np.testing.assert_array_equal(sub["out"], full["out"][toks])
+    np.testing.assert_array_equal(sub["ids"], full["ids"][toks])
+
+
+# --------------------------------------------------------------------------
+# FP8 e4m3 codec and block quantisation
+# --------------------------------------------------------------------------
+def test_e4m3_decode_all_codes_match_torch():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([oracle.e4m3_decode(q) for q in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan) and nan.sum() == 2
+    np.testing.assert_array_equal(mine[~nan], ref[~nan])
+
+
+def test_e4m3_encode_roundtrip_and_rne_vs_torch():
+    for q in range(256):
+        v = oracle.e4m3_decode(q)
+        if not math.isnan(v):
+            assert oracle.e4m3_encode(v) == q
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([rng.standard_normal(4000) * s for s in (1e-3, 0.05, 1, 30, 200)])
+    vals = np.clip(vals, -448, 448).astype(np.float32)
+    # exact midpoints between neighbouring codes exercise ties-to-even
+    finite = sorted({oracle.e4m3_decode(q) for q in range(128) if not math.isnan(oracle.e4m3_decode(q))})
+    mids = np.array([(a + b) / 2 for a, b in zip(finite[:-1], finite[1:])], np.float32)
+    vals = np.concatenate([vals, mids, -mids])
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = np.array([oracle.e4m3_encode(v) for v in vals], np.uint8)
+    np.testing.assert_array_equal(mine, ref)
+
+
+def test_act_quant_bounds_and_closed_forms():
+    cfg = _small(T=8, H=512)
+    x = mi.make_x(cfg)
+    x[3, 128:256] = 0  # an all-zero group
+    q, s = oracle.quant_act_fp8(x)
+    xf = mi.bf16_to_f32(x).astype(np.float64)
+    dq = np.vectorize(oracle.e4m3_decode)(q) * np.repeat(s, 128, axis=1)
+    assert s[3, 1] == 1.0 and np.all(q[3, 128:256] == 0)
+    amax = np.abs(xf).reshape(8, 4, 128).max(2)
+    nz = amax > 0
+    np.testing.assert_array_equal(s[nz], (amax[nz].astype(np.float32) / np.float32(448)))
+    # the element holding the group max encodes to +-448 (code 0x7E / 0xFE)
+    for r in range(8):
+        for g in range(4):
+            if nz[r, g]:
+                c = np.argmax(np.abs(xf[r, g * 128:(g + 1) * 128]))
+                assert q[r, g * 128 + c] & 0x7F == 0x7E
+    err = np.abs(dq - xf)
+    sfull = np.repeat(s, 128, axis=1).astype(np.float64)
+    assert np.all(err <= np.maximum(2.0 ** -4 * np.abs(xf), 2.0 ** -10 * sfull) * (1 + 1e-6))
+
+
+def test_weight_quant_blocks():
+    rng = np.random.default_rng(4)
+    w = mi.f32_to_bf16(rng.standard_normal((2, 256, 384)).astype(np.float32) * 0.02)
+    w[1, :128, 128:256] = 0
+    q, s = oracle.quant_weight_fp8(w.reshape(2, 256, 384))
+    assert s.shape == (2, 2, 3) and s[1, 0, 1] == 1.0
+    wf = mi.bf16_to_f32(w).astype(np.float64)
+    for b in range(2):
+        for rb in range(2):
+            for cb in range(3):
+                blk = wf[b, rb * 128:(rb + 1) * 128, cb * 128:(cb + 1) * 128]
+                amax = np.abs(blk).max()
+                if amax > 0:
+                    assert s[b, rb, cb] == np.float32(amax) / np.float32(448)
+                dq = np.vectorize(oracle.e4m3_decode)(
+                    q[b, rb * 128:(rb + 1) * 128, cb * 128:(cb + 1) * 128]) * s[b, rb, cb]
+                assert np.all(np.abs(dq - blk) <= np.maximum(2.0 ** -4 * np.abs(blk),
+                                                              2.0 ** -10 * s[b, rb, cb]) * (1 + 1e-6))
+
+
+def test_fp8_forward_matches_dense_on_dequantised_values():
+    cfg = _small(T=12, E=3, k=2, H=256, I=256)
+    L = mi.make_layer(cfg)
+    w13q, w13s = oracle.quant_weight_fp8(L["w13"])
+    w2q, w2s = oracle.quant_weight_fp8(L["w2"])
+    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], k=2, fp8=(w13q, w13s, w2q, w2s))
+    dec = np.vectorize(oracle.e4m3_decode)
+    W13 = dec(w13q) * np.repeat(np.repeat(w13s, 128, 1), 128, 2)
+    W2 = dec(w2q) * np.repeat(np.repeat(w2s, 128, 1), 128, 2)
+    xq, xs = oracle.quant_act_fp8(L["x"])
+    X = dec(xq) * np.repeat(xs, 128, 1)
+    out = np.zeros((cfg.T, cfg.H))
+    for t in range(cfg.T):
+        for j in range(2):
+            e = r["ids"][t, j]
+            g = W13[e, :cfg.I] @ X[t]
+            u = W13[e, cfg.I:] @ X[t]
+            a = (g / (1 + np.exp(-g)) * u).astype(np.float32)
+            # quantise a (fp32) per 128 group exactly as the layer states
+            ah = np.empty(cfg.I)
+            for g0 in range(0, cfg.I, 128):
+                grp = a[g0:g0 + 128]
+                sc = np.float32(np.abs(grp).max()) / np.float32(448) if np.abs(grp).max() > 0 else 1.0
+                codes = torch.from_numpy((grp / np.float32(sc)).astype(np.float32)).to(
+                    torch.float8_e4m3fn).to(torch.float64).numpy()
+                ah[g0:g0 + 128] = codes * float(sc)
+            out[t] += float(r["w"][t, j]) * (W2[e] @ ah)
+    np.testing.assert_allclose(r["out"], out, rtol=1e-5, atol=1e-6 * np.abs(out).max())
+
+
+# --------------------------------------------------------------------------
+# the input generator itself
+# --------------------------------------------------------------------------
+def test_generator_splitmix_reference_value():
+    # SplitMix64 (Steele, Lea & Flood 2014) seeded with 0: first output
+    assert int(mi.raw_u64(0, 0, 1)[0]) == 0xE220A8397B1DCDAF
+
+
+def test_generator_transposed_store_draws_same_values():
+    cfg = _small(E=3, H=64, I=32)
+    L = mi.make_layer(cfg)
+    wg, wu, wd = _logical_weights(cfg)
+    np.testing.assert_array_equal(mi.bf16_to_f32(L["w13"][:, :cfg.I, :]), wg.transpose(0, 2, 1))
+    np.testing.assert_array_equal(mi.bf16_to_f32(L["w13"][:, cfg.I:, :]), wu.transpose(0, 2, 1))
+    np.testing.assert_array_equal(mi.bf16_to_f32(L["w2"]), wd.transpose(0, 2, 1))
+
+
+def test_generator_moments():
+    v = mi.bf16_to_f32(mi.normal_bf16(0, 99, 0.02, 1, 1000, 1000)).astype(np.float64)
+    assert abs(v.mean()) < 1e-4 and abs(v.std() - 0.02) < 2e-4
+    z = v / 0.02
+    assert 0.040 < np.mean(np.abs(z) > 2) < 0.051  # two-sided normal tail 4.55 %
+
+
+def test_zipf_bias_is_log_pmf_of_a_rank_permutation():
+    cfg = mi.CONFIGS["fine_grained"]
+    _, b = mi.make_router(cfg.with_(H=8))
+    ranks = np.exp(-b.astype(np.float64) / 1.1)
+    np.testing.assert_allclose(np.sort(ranks), np.arange(1, 257), rtol=1e-5)
