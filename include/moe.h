@@ -1,0 +1,238 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts FFN layer
+ * forward: router -> softmax top-k -> permutation by expert -> grouped
+ * gated-MLP GEMMs (gate/up, SwiGLU, down) -> weighted combine, in bf16 and in
+ * fine-grained FP8.
+ *
+ * Passages the operations follow (titles of the pages they come from):
+ *   [R]  "Mixture of Experts (MoE): a practical explanation of how expert
+ *        models work" (lira-now.com), section 5 "How the Router (Top-k
+ *        Routing) works step by step" and its pseudocode; section 13's toy
+ *        layer.
+ *   [X]  "Experts backends" (HF Transformers docs), the backend table
+ *        (`eager`, `grouped_mm`, `deepgemm_megamoe` rows), "Switching at
+ *        decode", "FP8 and FP4 quantized experts".
+ *   [F]  "Fine-grained FP8" (HF Transformers docs), the opening list (128 x 128
+ *        weight blocks; per-token activation groups of 128 input channels).
+ *   [S]  "AWS improves MoE model performance on Amazon SageMaker AI"
+ *        (mikhbar.website), section "Swap-AB advantage in MoE workloads".
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_dev are DEVICE pointers of the current device; nothing
+ *     else in this header takes host memory except moe_forward_hostio's
+ *     x_host/out_host. Every device pointer must be 16-byte aligned.
+ *   - The library never allocates, frees or synchronises: the caller owns
+ *     every buffer, including the workspace `ws` (size from
+ *     moe_workspace_size). Work is enqueued on `stream` (a cudaStream_t; NULL
+ *     is the legacy default stream) and is stream-ordered.
+ *   - bf16 tensors are raw bf16 (IEEE binary16 upper half), e4m3 tensors are
+ *     OCP E4M3FN bytes, all row-major and densely packed.
+ *   - Validation (pointers, alignment, dimensions, workspace size, device
+ *     architecture) happens on the host before any launch. Failure returns a
+ *     status without launching anything; moe_last_error() then describes it.
+ *     Launch failures return MOE_ERR_CUDA. A device-side wait that runs out
+ *     (a bounded spin in a kernel) records MOE_ERR_TIMEOUT in the workspace's
+ *     status word, which moe_get_device_status() reads.
+ *   - Results are deterministic (bitwise identical run to run).
+ *   - NaN or Inf inputs: behaviour unspecified.
+ *
+ * Dimensions (moe_dims_t): T tokens, H hidden, I expert intermediate, E
+ * experts, k experts per token. Supported: T >= 1, H and I multiples of 128,
+ * 1 <= E <= 1024, 1 <= k <= min(E, 16), T*k < 2^31.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* bad pointer, alignment or dimension */
+  MOE_ERR_UNSUPPORTED_DEVICE = 2, /* current device is not compute capability 10.0 */
+  MOE_ERR_WORKSPACE = 3,          /* workspace missing or smaller than required */
+  MOE_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+  MOE_ERR_TIMEOUT = 5             /* a bounded device-side wait ran out */
+} moe_status_t;
+
+typedef enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 } moe_dtype_t;
+
+typedef enum { MOE_EPILOGUE_NONE = 0, MOE_EPILOGUE_SWIGLU = 1 } moe_epilogue_t;
+
+typedef struct {
+  int32_t T, H, I, E, k;
+} moe_dims_t;
+
+/* Thread-local text describing the last failure in this thread ("" if none). */
+const char* moe_last_error(void);
+
+/* MOE_ABI_VERSION of the loaded library. */
+int32_t moe_abi_version(void);
+
+/* Number of kernel launches this library has issued in this process (all
+ * threads). Read it before and after a region to count the launches in it. */
+int64_t moe_launch_count(void);
+
+/* Bytes of workspace moe_forward (dt = BF16) or moe_forward_fp8 (dt = FP8)
+ * needs for dims d, also enough for moe_route_topk, moe_permute and
+ * moe_grouped_gemm on the same dims. 0 for invalid dims. */
+size_t moe_workspace_size(moe_dims_t d, moe_dtype_t dt);
+
+/* Byte offsets of the intermediates moe_forward / moe_forward_fp8 leave in
+ * the workspace (for inspection and tests). -1 marks a buffer the dtype does
+ * not use. Layout (all 256-byte aligned):
+ *   status    int32                      device status word
+ *   logits    fp32 [T, E]
+ *   topk_ids  int32 [T, k]               expert of slot j, slots by descending logit
+ *   topk_w    fp32 [T, k]                renormalised routing weight of slot j
+ *   offsets   int32 [E + 1]              expert e owns permuted rows [offsets[e], offsets[e+1])
+ *   perm_token int32 [T*k]               token of permuted row p
+ *   inv_perm  int32 [T, k]               permuted row of (token t, slot j)
+ *   x_perm    bf16 [T*k, H]  (BF16)      permuted token rows
+ *   xq_perm   e4m3 [T*k, H], xs_perm fp32 [T*k, H/128]   (FP8)
+ *   h         bf16 [T*k, I]  (BF16)      SwiGLU output per permuted row
+ *   hq        e4m3 [T*k, I], hs fp32 [T*k, I/128]        (FP8)
+ *   y_perm    bf16 [T*k, H]              expert output per permuted row          */
+typedef struct {
+  int64_t status, logits, topk_ids, topk_w, offsets, perm_token, inv_perm;
+  int64_t x_perm, xq_perm, xs_perm, h, hq, hs, y_perm, scratch, total;
+} moe_ws_layout_t;
+moe_status_t moe_workspace_layout(moe_dims_t d, moe_dtype_t dt, moe_ws_layout_t* out);
+
+/* Router: logits = x Wr + bias, then softmax top-k with renormalised
+ * weights.  [R] section 5 steps 1-5; the pseudocode's logits / softmax / topk /
+ * `values / values.sum()`.
+ *   x_dev      bf16 [T, H]
+ *   wr_dev     bf16 [H, E]
+ *   bias_dev   fp32 [E] or NULL (added to the logits before selection)
+ *   logits_dev fp32 [T, E] out, or NULL (then kept in the workspace)
+ *   ids_dev    int32 [T, k] out: slot j holds the j-th largest logit; equal
+ *              fp32 logits go to the lower expert index
+ *   w_dev      fp32 [T, k] out: exp(l_j - l_max) / sum over selected
+ *   ws/ws_bytes workspace (needed when logits_dev is NULL; may be NULL else)
+ * The logits are fp32 sums over h in ascending order of exact bf16 x bf16
+ * products, so they (and the ids) are bit-reproducible functions of the
+ * inputs. I is ignored. */
+moe_status_t moe_route_topk(const void* x_dev, const void* wr_dev, const float* bias_dev,
+                            moe_dims_t d, float* logits_dev, int32_t* ids_dev, float* w_dev,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Selection alone, from given logits fp32 [T, E] (same rules as above). */
+moe_status_t moe_topk_from_logits(const float* logits_dev, moe_dims_t d, int32_t* ids_dev,
+                                  float* w_dev, void* stream);
+
+/* Permutation by expert ([X] backend table, grouped_mm row: tokens sorted by
+ * chosen expert so each expert's rows are contiguous). Rows are ordered by
+ * expert, then by token ascending.
+ *   ids_dev        int32 [T, k] in
+ *   offsets_dev    int32 [E + 1] out (exclusive prefix sum of expert counts)
+ *   perm_token_dev int32 [T*k] out
+ *   inv_perm_dev   int32 [T, k] out
+ *   x_dev/x_perm_dev  bf16 [T, H] in / [T*k, H] out, both NULL to skip the row gather
+ *   ws/ws_bytes    workspace of moe_workspace_size(d, BF16) bytes */
+moe_status_t moe_permute(const int32_t* ids_dev, moe_dims_t d, int32_t* offsets_dev,
+                         int32_t* perm_token_dev, int32_t* inv_perm_dev, const void* x_dev,
+                         void* x_perm_dev, void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped GEMM on tcgen05 tensor cores ([X] backend table, grouped_mm and
+ * deepgemm rows: one grouped GEMM over expert-sorted rows).
+ * For each expert e, rows m in [offsets[e], offsets[e+1]) of A:
+ *   NONE:   C[m, n] = sum_k A[m, k] B[e, n, k]                  n < N
+ *   SWIGLU: g = A B[e, 0:N]^T, u = A B[e, N:2N]^T, C = silu(g) * u,
+ *           silu(z) = z / (1 + e^-z)   ([X] deepgemm_megamoe row)
+ *   A_dev  [M_total, K] (bf16, or e4m3 with a_scales fp32 [M_total, K/128])
+ *   B_dev  [E, N or 2N, K] K-major (bf16, or e4m3 with b_scales fp32
+ *          [E, rows/128, K/128], one scale per 128 x 128 block, [F])
+ *   C_dev  bf16 [M_total, N]; for FP8 SWIGLU with c_scales != NULL, C is
+ *          e4m3 [M_total, N] with c_scales fp32 [M_total, N/128] (each
+ *          128-group scaled by amax/448, [F] activation groups)
+ *   max_rows_per_expert: an upper bound on any expert's row count (0 =
+ *          unknown). Bounds <= 64 select the small-M variant that puts the
+ *          weight rows in the MMA M slot ([S]).
+ * N, K multiples of 128. Accumulation is fp32. ws: the forward's workspace
+ * (its status word is used). */
+moe_status_t moe_grouped_gemm(const void* A_dev, const void* B_dev, const int32_t* offsets_dev,
+                              int32_t M_total, int32_t E, int32_t N, int32_t K, moe_dtype_t dt,
+                              moe_epilogue_t ep, void* C_dev, const float* a_scales_dev,
+                              const float* b_scales_dev, float* c_scales_dev,
+                              int32_t max_rows_per_expert, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Weighted combine ([R] pseudocode `y = sum_i weights_i * expert_i(x)`):
+ *   out[t, :] = sum_{j = 0..k-1} w[t, j] * y_perm[inv_perm[t, j], :]
+ * summed in fp32 in slot order, rounded once to bf16.
+ *   y_perm_dev bf16 [T*k, H], w_dev fp32 [T, k], inv_perm_dev int32 [T, k],
+ *   out_dev bf16 [T, H] */
+moe_status_t moe_combine(const void* y_perm_dev, const float* w_dev, const int32_t* inv_perm_dev,
+                         moe_dims_t d, void* out_dev, void* stream);
+
+/* The whole layer, bf16: route -> permute -> GEMM1 (+SwiGLU) -> GEMM2 ->
+ * combine ([X] backend table; [R] section 5).
+ *   x_dev   bf16 [T, H];  wr_dev bf16 [H, E];  bias_dev fp32 [E] or NULL
+ *   w13_dev bf16 [E, 2I, H]: rows [0, I) = Wg[e]^T, rows [I, 2I) = Wu[e]^T
+ *   w2_dev  bf16 [E, H, I]  = Wd[e]^T
+ *   out_dev bf16 [T, H]
+ *   ws      >= moe_workspace_size(d, MOE_DTYPE_BF16) bytes
+ * No host synchronisation; capturable in a CUDA graph. */
+moe_status_t moe_forward(const void* x_dev, const void* wr_dev, const float* bias_dev,
+                         const void* w13_dev, const void* w2_dev, moe_dims_t d, void* out_dev,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer with fine-grained FP8 experts ([F]; [X] "FP8 and FP4
+ * quantized experts"): x is quantised per (token, 128-channel group) to e4m3
+ * with scale amax/448, the SwiGLU output likewise per (row, 128-group of I),
+ * and the expert weights come as e4m3 with one fp32 scale per 128 x 128
+ * block. The router stays bf16 on x.
+ *   w13q_dev e4m3 [E, 2I, H], w13s_dev fp32 [E, 2I/128, H/128]
+ *   w2q_dev  e4m3 [E, H, I],  w2s_dev  fp32 [E, H/128, I/128]
+ *   ws >= moe_workspace_size(d, MOE_DTYPE_FP8_E4M3) bytes */
+moe_status_t moe_forward_fp8(const void* x_dev, const void* wr_dev, const float* bias_dev,
+                             const void* w13q_dev, const float* w13s_dev, const void* w2q_dev,
+                             const float* w2s_dev, moe_dims_t d, void* out_dev, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* moe_forward with the token rows in HOST memory: copies x_host ([T, H]
+ * bf16) to the workspace, runs the layer, copies the result to out_host
+ * ([T, H] bf16), all on `stream`. Pinned host buffers make the copies
+ * asynchronous; the call returns after enqueueing (synchronise `stream`
+ * before reading out_host). ws >= moe_workspace_size(d, BF16) + 2*T*H*2. */
+moe_status_t moe_forward_hostio(const void* x_host, const void* wr_dev, const float* bias_dev,
+                                const void* w13_dev, const void* w2_dev, moe_dims_t d,
+                                void* out_host, void* ws, size_t ws_bytes, void* stream);
+
+/* Activation quantisation ([F]): per row, per group of 128 columns,
+ * s = amax/448 (1 for an all-zero group), q = e4m3_rn(v / s) with IEEE fp32
+ * division and round-to-nearest-even.
+ *   x_dev bf16 [rows, cols] -> q_dev e4m3 [rows, cols], s_dev fp32 [rows, cols/128] */
+moe_status_t moe_quantize_act_fp8(const void* x_dev, int64_t rows, int64_t cols, void* q_dev,
+                                  float* s_dev, void* stream);
+
+/* Weight quantisation ([F]): nb matrices bf16 [rows, cols] in 128 x 128
+ * blocks, same scale and rounding rule -> q_dev e4m3 [nb, rows, cols],
+ * s_dev fp32 [nb, rows/128, cols/128]. A one-time preparation step. */
+moe_status_t moe_quantize_weight_fp8(const void* w_dev, int64_t nb, int64_t rows, int64_t cols,
+                                     void* q_dev, float* s_dev, void* stream);
+
+/* Reads the workspace's device status word (MOE_OK or MOE_ERR_TIMEOUT) into
+ * *status_out. Synchronises the device (a blocking copy); not for hot loops. */
+moe_status_t moe_get_device_status(const void* ws, int32_t* status_out);
+
+/* Clears the workspace's device status word (stream-ordered). */
+moe_status_t moe_clear_device_status(void* ws, void* stream);
+
+/* Stage timing for moe_forward / moe_forward_fp8 on the calling thread: when
+ * set, the next forwards record events[0..5] (cudaEvent_t) on their stream at
+ * entry, after routing, after the permutation, after GEMM1, after GEMM2 and
+ * after the combine. Pass NULL to stop. */
+moe_status_t moe_set_stage_events(void* const* events, int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

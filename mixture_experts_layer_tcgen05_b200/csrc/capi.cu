@@ -1,0 +1,510 @@
+// C ABI of the MoE layer (include/moe.h): argument validation, workspace
+// layout, device check and the launch sequence of each entry point. Every
+// step of the layer runs in this library's kernels; nothing here computes
+// on the host.
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+
+namespace moe {
+
+// kernels (router.cu, permute.cu, gemm.cu, fp8.cu)
+cudaError_t launch_router_logits(const void* x, const void* wr, const float* bias, int T, int H,
+                                 int E, float* logits, cudaStream_t s);
+cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                        cudaStream_t s);
+int64_t permute_scratch_bytes(int T, int E);
+cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
+                           int32_t* perm_token, int32_t* inv_perm, void* scratch, int32_t* status,
+                           cudaStream_t s);
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, int T,
+                               int row_bytes, void* x_perm, int32_t* status, cudaStream_t s);
+cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_perm, int T,
+                           int H, int k, void* out, int32_t* status, cudaStream_t s);
+cudaError_t launch_grouped_gemm_bf16(const void* A, const void* B, const int32_t* offsets,
+                                     int M_total, int E, int N, int K, bool swiglu, void* C,
+                                     int max_rows_per_expert, int32_t* status, cudaStream_t s,
+                                     const char** why);
+cudaError_t launch_grouped_gemm_fp8(const void* A, const float* a_scales, const void* B,
+                                    const float* b_scales, const int32_t* offsets, int M_total,
+                                    int E, int N, int K, bool swiglu, void* C, float* c_scales,
+                                    int max_rows_per_expert, int32_t* status, cudaStream_t s,
+                                    const char** why);
+cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
+                             const int32_t* row_map, cudaStream_t s);
+cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
+                                float* sc, cudaStream_t s);
+
+static std::atomic<int64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string t_err;
+thread_local void* t_events[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+thread_local bool t_events_on = false;
+
+moe_status_t fail(moe_status_t st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+moe_status_t fail(moe_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return st;
+}
+
+moe_status_t ok() {
+  t_err.clear();
+  return MOE_OK;
+}
+
+moe_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t check_dims(moe_dims_t d, bool need_I) {
+  if (d.T < 1) return fail(MOE_ERR_INVALID_ARG, "T must be >= 1 (got %d)", d.T);
+  if (d.H < 128 || d.H % 128)
+    return fail(MOE_ERR_INVALID_ARG, "H must be a positive multiple of 128 (got %d)", d.H);
+  if (need_I && (d.I < 128 || d.I % 128))
+    return fail(MOE_ERR_INVALID_ARG, "I must be a positive multiple of 128 (got %d)", d.I);
+  if (d.E < 1 || d.E > 1024) return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 1024] (got %d)", d.E);
+  if (d.k < 1 || d.k > 16 || d.k > d.E)
+    return fail(MOE_ERR_INVALID_ARG, "k must be in [1, min(E, 16)] (got k=%d, E=%d)", d.k, d.E);
+  if ((int64_t)d.T * d.k >= (int64_t)1 << 31)
+    return fail(MOE_ERR_INVALID_ARG, "T*k must be < 2^31");
+  return MOE_OK;
+}
+
+moe_status_t check_ptr(const void* p, const char* name, bool allow_null = false) {
+  if (!p) {
+    if (allow_null) return MOE_OK;
+    return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+  }
+  if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return MOE_OK;
+}
+
+#define MOE_TRY(x)                      \
+  do {                                  \
+    moe_status_t _st = (x);             \
+    if (_st != MOE_OK) return _st;      \
+  } while (0)
+
+moe_status_t check_device() {
+  const char* fake = getenv("MOE_FAKE_CC");
+  int major = 0, minor = 0;
+  if (fake) {
+    major = atoi(fake) / 10;
+    minor = atoi(fake) % 10;
+  } else {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(MOE_ERR_UNSUPPORTED_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+    static int cache_major[64] = {0}, cache_minor[64] = {0};
+    if (dev < 64 && cache_major[dev]) {
+      major = cache_major[dev];
+      minor = cache_minor[dev];
+    } else {
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+      if (dev < 64) {
+        cache_major[dev] = major;
+        cache_minor[dev] = minor;
+      }
+    }
+  }
+  if (major != 10 || minor != 0)
+    return fail(MOE_ERR_UNSUPPORTED_DEVICE,
+                "this library is built for sm_100a (compute capability 10.0); device is %d.%d",
+                major, minor);
+  return MOE_OK;
+}
+
+// Workspace layout shared by every entry point.
+moe_ws_layout_t layout(moe_dims_t d, moe_dtype_t dt) {
+  moe_ws_layout_t L;
+  int64_t off = 0;
+  auto take = [&](int64_t bytes) {
+    int64_t o = off;
+    off += align_up(bytes > 0 ? bytes : 0, 256);
+    return o;
+  };
+  const int64_t T = d.T, H = d.H, I = d.I, E = d.E, k = d.k, R = T * k;
+  L.status = take(256);
+  L.logits = take(T * E * 4);
+  L.topk_ids = take(R * 4);
+  L.topk_w = take(R * 4);
+  L.offsets = take((E + 1) * 4);
+  L.perm_token = take(R * 4);
+  L.inv_perm = take(R * 4);
+  L.scratch = take(permute_scratch_bytes((int)T, (int)E));
+  if (dt == MOE_DTYPE_BF16) {
+    L.x_perm = take(R * H * 2);
+    L.xq_perm = L.xs_perm = -1;
+    L.h = take(R * I * 2);
+    L.hq = L.hs = -1;
+  } else {
+    L.x_perm = -1;
+    L.xq_perm = take(R * H);
+    L.xs_perm = take(R * (H / 128) * 4);
+    L.h = -1;
+    L.hq = take(R * I);
+    L.hs = take(R * (I / 128) * 4);
+  }
+  L.y_perm = take(R * H * 2);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, int64_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+void record(cudaStream_t s, int i) {
+  if (t_events_on && t_events[i]) cudaEventRecord(static_cast<cudaEvent_t>(t_events[i]), s);
+}
+
+moe_status_t check_ws(moe_dims_t d, moe_dtype_t dt, const void* ws, size_t ws_bytes,
+                      size_t extra = 0) {
+  MOE_TRY(check_ptr(ws, "ws"));
+  size_t need = (size_t)layout(d, dt).total + extra;
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error(void) { return t_err.c_str(); }
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+int64_t moe_launch_count(void) { return g_launches.load(); }
+
+size_t moe_workspace_size(moe_dims_t d, moe_dtype_t dt) {
+  if (check_dims(d, true) != MOE_OK) return 0;
+  if (dt != MOE_DTYPE_BF16 && dt != MOE_DTYPE_FP8_E4M3) return 0;
+  return (size_t)layout(d, dt).total;
+}
+
+moe_status_t moe_workspace_layout(moe_dims_t d, moe_dtype_t dt, moe_ws_layout_t* out) {
+  MOE_TRY(check_dims(d, true));
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  if (dt != MOE_DTYPE_BF16 && dt != MOE_DTYPE_FP8_E4M3) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
+  *out = layout(d, dt);
+  return ok();
+}
+
+moe_status_t moe_route_topk(const void* x, const void* wr, const float* bias, moe_dims_t d,
+                            float* logits, int32_t* ids, float* w, void* ws, size_t ws_bytes,
+                            void* stream) {
+  MOE_TRY(check_dims(d, false));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(wr, "w_router"));
+  MOE_TRY(check_ptr(bias, "bias", true));
+  MOE_TRY(check_ptr(logits, "logits", true));
+  MOE_TRY(check_ptr(ids, "topk_ids"));
+  MOE_TRY(check_ptr(w, "topk_w"));
+  if (!logits) {
+    moe_dims_t d2 = d;
+    d2.I = 128;
+    MOE_TRY(check_ws(d2, MOE_DTYPE_BF16, ws, ws_bytes));
+    logits = at<float>(ws, layout(d2, MOE_DTYPE_BF16).logits);
+  }
+  MOE_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_router_logits(x, wr, bias, d.T, d.H, d.E, logits, s);
+  if (e != cudaSuccess) return cuda_fail(e, "router logits");
+  e = launch_topk(logits, d.T, d.E, d.k, ids, w, s);
+  if (e != cudaSuccess) return cuda_fail(e, "top-k");
+  return ok();
+}
+
+moe_status_t moe_topk_from_logits(const float* logits, moe_dims_t d, int32_t* ids, float* w,
+                                  void* stream) {
+  if (d.T < 1 || d.E < 1 || d.E > 1024 || d.k < 1 || d.k > 16 || d.k > d.E)
+    return fail(MOE_ERR_INVALID_ARG, "bad dims (T=%d E=%d k=%d)", d.T, d.E, d.k);
+  MOE_TRY(check_ptr(logits, "logits"));
+  MOE_TRY(check_ptr(ids, "topk_ids"));
+  MOE_TRY(check_ptr(w, "topk_w"));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_topk(logits, d.T, d.E, d.k, ids, w, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "top-k");
+  return ok();
+}
+
+moe_status_t moe_permute(const int32_t* ids, moe_dims_t d, int32_t* offsets, int32_t* perm_token,
+                         int32_t* inv_perm, const void* x, void* x_perm, void* ws,
+                         size_t ws_bytes, void* stream) {
+  moe_dims_t d2 = d;
+  if (d2.I < 128) d2.I = 128;
+  MOE_TRY(check_dims(d2, true));
+  MOE_TRY(check_ptr(ids, "topk_ids"));
+  MOE_TRY(check_ptr(offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(perm_token, "perm_token"));
+  MOE_TRY(check_ptr(inv_perm, "inv_perm"));
+  if ((x == nullptr) != (x_perm == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "x and x_perm must both be given or both be NULL");
+  MOE_TRY(check_ptr(x, "x", true));
+  MOE_TRY(check_ptr(x_perm, "x_perm", true));
+  MOE_TRY(check_ws(d2, MOE_DTYPE_BF16, ws, ws_bytes));
+  MOE_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  moe_ws_layout_t L = layout(d2, MOE_DTYPE_BF16);
+  cudaError_t e = launch_permute(ids, d.T, d.E, d.k, offsets, perm_token, inv_perm,
+                                 at<char>(ws, L.scratch), at<int32_t>(ws, L.status), s);
+  if (e != cudaSuccess) return cuda_fail(e, "permute");
+  if (x) {
+    e = launch_gather_rows(x, perm_token, d.T * d.k, d.T, d.H * 2, x_perm,
+                           at<int32_t>(ws, L.status), s);
+    if (e != cudaSuccess) return cuda_fail(e, "gather");
+  }
+  return ok();
+}
+
+moe_status_t moe_grouped_gemm(const void* A, const void* B, const int32_t* offsets,
+                              int32_t M_total, int32_t E, int32_t N, int32_t K, moe_dtype_t dt,
+                              moe_epilogue_t ep, void* C, const float* a_scales,
+                              const float* b_scales, float* c_scales, int32_t max_rows_per_expert,
+                              void* ws, size_t ws_bytes, void* stream) {
+  if (M_total < 1) return fail(MOE_ERR_INVALID_ARG, "M_total must be >= 1");
+  if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 1024]");
+  if (N < 128 || N % 128 || K < 128 || K % 128)
+    return fail(MOE_ERR_INVALID_ARG, "N and K must be positive multiples of 128 (N=%d K=%d)", N, K);
+  if (ep != MOE_EPILOGUE_NONE && ep != MOE_EPILOGUE_SWIGLU) return fail(MOE_ERR_INVALID_ARG, "bad epilogue");
+  if (dt != MOE_DTYPE_BF16 && dt != MOE_DTYPE_FP8_E4M3) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
+  MOE_TRY(check_ptr(A, "A"));
+  MOE_TRY(check_ptr(B, "B"));
+  MOE_TRY(check_ptr(offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(C, "C"));
+  if (dt == MOE_DTYPE_FP8_E4M3) {
+    MOE_TRY(check_ptr(a_scales, "a_scales"));
+    MOE_TRY(check_ptr(b_scales, "b_scales"));
+    MOE_TRY(check_ptr(c_scales, "c_scales", true));
+    if (c_scales && ep != MOE_EPILOGUE_SWIGLU)
+      return fail(MOE_ERR_INVALID_ARG, "c_scales (quantised output) needs the SWIGLU epilogue");
+  }
+  MOE_TRY(check_ptr(ws, "ws"));
+  if (ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes", ws_bytes);
+  MOE_TRY(check_device());
+  const char* why = "";
+  cudaError_t e;
+  if (dt == MOE_DTYPE_BF16)
+    e = launch_grouped_gemm_bf16(A, B, offsets, M_total, E, N, K, ep == MOE_EPILOGUE_SWIGLU, C,
+                                 max_rows_per_expert, at<int32_t>(ws, 0),
+                                 static_cast<cudaStream_t>(stream), &why);
+  else
+    e = launch_grouped_gemm_fp8(A, a_scales, B, b_scales, offsets, M_total, E, N, K,
+                                ep == MOE_EPILOGUE_SWIGLU, C, c_scales, max_rows_per_expert,
+                                at<int32_t>(ws, 0), static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "grouped GEMM: %s %s", cudaGetErrorString(e), why);
+  return ok();
+}
+
+moe_status_t moe_combine(const void* y_perm, const float* w, const int32_t* inv_perm, moe_dims_t d,
+                         void* out, void* stream) {
+  moe_dims_t d2 = d;
+  if (d2.I < 128) d2.I = 128;
+  MOE_TRY(check_dims(d2, true));
+  MOE_TRY(check_ptr(y_perm, "y_perm"));
+  MOE_TRY(check_ptr(w, "topk_w"));
+  MOE_TRY(check_ptr(inv_perm, "inv_perm"));
+  MOE_TRY(check_ptr(out, "out"));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_combine(y_perm, w, inv_perm, d.T, d.H, d.k, out, nullptr,
+                                 static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine");
+  return ok();
+}
+
+static moe_status_t forward_impl(const void* x, const void* wr, const float* bias, const void* w13,
+                                 const float* w13s, const void* w2, const float* w2s, moe_dims_t d,
+                                 void* out, void* ws, moe_dtype_t dt, cudaStream_t s) {
+  const moe_ws_layout_t L = layout(d, dt);
+  const int T = d.T, H = d.H, I = d.I, E = d.E, k = d.k, R = T * k;
+  int32_t* status = at<int32_t>(ws, L.status);
+  float* logits = at<float>(ws, L.logits);
+  int32_t* ids = at<int32_t>(ws, L.topk_ids);
+  float* tw = at<float>(ws, L.topk_w);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm_token = at<int32_t>(ws, L.perm_token);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  void* y_perm = at<void>(ws, L.y_perm);
+  const char* why = "";
+  cudaError_t e;
+  record(s, 0);
+  if ((e = launch_router_logits(x, wr, bias, T, H, E, logits, s)) != cudaSuccess)
+    return cuda_fail(e, "router logits");
+  if ((e = launch_topk(logits, T, E, k, ids, tw, s)) != cudaSuccess) return cuda_fail(e, "top-k");
+  record(s, 1);
+  if ((e = launch_permute(ids, T, E, k, offsets, perm_token, inv_perm, at<char>(ws, L.scratch),
+                          status, s)) != cudaSuccess)
+    return cuda_fail(e, "permute");
+  if (dt == MOE_DTYPE_BF16) {
+    void* x_perm = at<void>(ws, L.x_perm);
+    void* h = at<void>(ws, L.h);
+    if ((e = launch_gather_rows(x, perm_token, R, T, H * 2, x_perm, status, s)) != cudaSuccess)
+      return cuda_fail(e, "gather");
+    record(s, 2);
+    if ((e = launch_grouped_gemm_bf16(x_perm, w13, offsets, R, E, I, H, true, h, T, status, s,
+                                      &why)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "GEMM1: %s %s", cudaGetErrorString(e), why);
+    record(s, 3);
+    if ((e = launch_grouped_gemm_bf16(h, w2, offsets, R, E, H, I, false, y_perm, T, status, s,
+                                      &why)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "GEMM2: %s %s", cudaGetErrorString(e), why);
+    record(s, 4);
+  } else {
+    void* xq = at<void>(ws, L.xq_perm);
+    float* xs = at<float>(ws, L.xs_perm);
+    void* hq = at<void>(ws, L.hq);
+    float* hs = at<float>(ws, L.hs);
+    if ((e = launch_quant_act(x, R, H, xq, xs, perm_token, s)) != cudaSuccess)
+      return cuda_fail(e, "activation quantisation");
+    record(s, 2);
+    if ((e = launch_grouped_gemm_fp8(xq, xs, w13, w13s, offsets, R, E, I, H, true, hq, hs, T,
+                                     status, s, &why)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "FP8 GEMM1: %s %s", cudaGetErrorString(e), why);
+    record(s, 3);
+    if ((e = launch_grouped_gemm_fp8(hq, hs, w2, w2s, offsets, R, E, H, I, false, y_perm, nullptr,
+                                     T, status, s, &why)) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "FP8 GEMM2: %s %s", cudaGetErrorString(e), why);
+    record(s, 4);
+  }
+  if ((e = launch_combine(y_perm, tw, inv_perm, T, H, k, out, status, s)) != cudaSuccess)
+    return cuda_fail(e, "combine");
+  record(s, 5);
+  return ok();
+}
+
+moe_status_t moe_forward(const void* x, const void* wr, const float* bias, const void* w13,
+                         const void* w2, moe_dims_t d, void* out, void* ws, size_t ws_bytes,
+                         void* stream) {
+  MOE_TRY(check_dims(d, true));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(wr, "w_router"));
+  MOE_TRY(check_ptr(bias, "bias", true));
+  MOE_TRY(check_ptr(w13, "w13"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  MOE_TRY(check_ptr(out, "out"));
+  MOE_TRY(check_ws(d, MOE_DTYPE_BF16, ws, ws_bytes));
+  MOE_TRY(check_device());
+  return forward_impl(x, wr, bias, w13, nullptr, w2, nullptr, d, out, ws, MOE_DTYPE_BF16,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward_fp8(const void* x, const void* wr, const float* bias, const void* w13q,
+                             const float* w13s, const void* w2q, const float* w2s, moe_dims_t d,
+                             void* out, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_dims(d, true));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(wr, "w_router"));
+  MOE_TRY(check_ptr(bias, "bias", true));
+  MOE_TRY(check_ptr(w13q, "w13q"));
+  MOE_TRY(check_ptr(w13s, "w13s"));
+  MOE_TRY(check_ptr(w2q, "w2q"));
+  MOE_TRY(check_ptr(w2s, "w2s"));
+  MOE_TRY(check_ptr(out, "out"));
+  MOE_TRY(check_ws(d, MOE_DTYPE_FP8_E4M3, ws, ws_bytes));
+  MOE_TRY(check_device());
+  return forward_impl(x, wr, bias, w13q, w13s, w2q, w2s, d, out, ws, MOE_DTYPE_FP8_E4M3,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward_hostio(const void* x_host, const void* wr, const float* bias,
+                                const void* w13, const void* w2, moe_dims_t d, void* out_host,
+                                void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_dims(d, true));
+  if (!x_host || !out_host) return fail(MOE_ERR_INVALID_ARG, "x_host and out_host must be given");
+  MOE_TRY(check_ptr(wr, "w_router"));
+  MOE_TRY(check_ptr(bias, "bias", true));
+  MOE_TRY(check_ptr(w13, "w13"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  const size_t io = (size_t)d.T * d.H * 2;
+  const size_t io_al = (size_t)align_up((int64_t)io, 256);
+  MOE_TRY(check_ws(d, MOE_DTYPE_BF16, ws, ws_bytes, 2 * io_al));
+  MOE_TRY(check_device());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t base = layout(d, MOE_DTYPE_BF16).total;
+  void* x_dev = at<void>(ws, base);
+  void* out_dev = at<void>(ws, base + (int64_t)io_al);
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, io, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy x to device");
+  MOE_TRY(forward_impl(x_dev, wr, bias, w13, nullptr, w2, nullptr, d, out_dev, ws, MOE_DTYPE_BF16, s));
+  e = cudaMemcpyAsync(out_host, out_dev, io, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy out to host");
+  return ok();
+}
+
+moe_status_t moe_quantize_act_fp8(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
+                                  void* stream) {
+  if (rows < 1 || cols < 128 || cols % 128) return fail(MOE_ERR_INVALID_ARG, "rows >= 1, cols a multiple of 128");
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(q, "q"));
+  MOE_TRY(check_ptr(sc, "s"));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_quant_act(x, rows, cols, q, sc, nullptr, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "activation quantisation");
+  return ok();
+}
+
+moe_status_t moe_quantize_weight_fp8(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
+                                     float* sc, void* stream) {
+  if (nb < 1 || rows < 128 || rows % 128 || cols < 128 || cols % 128)
+    return fail(MOE_ERR_INVALID_ARG, "nb >= 1, rows and cols multiples of 128");
+  MOE_TRY(check_ptr(w, "w"));
+  MOE_TRY(check_ptr(q, "q"));
+  MOE_TRY(check_ptr(sc, "s"));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_quant_weight(w, nb, rows, cols, q, sc, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "weight quantisation");
+  return ok();
+}
+
+moe_status_t moe_get_device_status(const void* ws, int32_t* status_out) {
+  MOE_TRY(check_ptr(ws, "ws"));
+  if (!status_out) return fail(MOE_ERR_INVALID_ARG, "status_out is NULL");
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  *status_out = v;
+  return ok();
+}
+
+moe_status_t moe_clear_device_status(void* ws, void* stream) {
+  MOE_TRY(check_ptr(ws, "ws"));
+  cudaError_t e = cudaMemsetAsync(ws, 0, 4, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  return ok();
+}
+
+moe_status_t moe_set_stage_events(void* const* events, int32_t n) {
+  if (!events) {
+    t_events_on = false;
+    return ok();
+  }
+  if (n != 6) return fail(MOE_ERR_INVALID_ARG, "expected 6 events (got %d)", n);
+  for (int i = 0; i < 6; ++i) t_events[i] = events[i];
+  t_events_on = true;
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,111 @@
+// Fine-grained FP8 quantisation kernels.
+//
+// "Fine-grained FP8" (HF Transformers docs), opening list: weights are
+// quantised to 8 bits per 128 x 128 block; activations per token per group
+// of 128 input channels, dynamically. Scale rule (both): s = amax / 448 in
+// fp32 (IEEE division), s = 1 for an all-zero group, code = e4m3 of v / s
+// rounded to nearest even (the hardware cvt with satfinite; |v / s| <= 448
+// up to one rounding, so saturation never changes a value).
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ float group_scale(float amax) {
+  return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+// One warp per (output row, 128-column group). Output row p reads input row
+// row_map[p] (the expert permutation) or p when row_map is NULL.
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint2* __restrict__ x, int64_t rows,
+                                                        int64_t cols,
+                                                        const int32_t* __restrict__ row_map,
+                                                        uint32_t* __restrict__ q,
+                                                        float* __restrict__ s) {
+  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t groups = cols / 128;
+  if (gw >= rows * groups) return;
+  const int64_t p = gw / groups, g = gw % groups;
+  const int64_t src = row_map ? row_map[p] : p;
+  // 4 bf16 per lane
+  uint2 v = x[(src * cols + g * 128) / 4 + lane];
+  float f0 = bf16lo_to_f32(v.x), f1 = bf16hi_to_f32(v.x), f2 = bf16lo_to_f32(v.y),
+        f3 = bf16hi_to_f32(v.y);
+  float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float sc = group_scale(amax);
+  q[(p * cols + g * 128) / 4 + lane] =
+      e4m3x4(__fdiv_rn(f0, sc), __fdiv_rn(f1, sc), __fdiv_rn(f2, sc), __fdiv_rn(f3, sc));
+  if (lane == 0) s[p * groups + g] = sc;
+}
+
+// One block (256 threads) per 128 x 128 weight block.
+__global__ void __launch_bounds__(256) quant_weight_kernel(const __nv_bfloat16* __restrict__ w,
+                                                           int64_t rows, int64_t cols,
+                                                           uint8_t* __restrict__ q,
+                                                           float* __restrict__ s) {
+  const int64_t RB = rows / 128, CB = cols / 128;
+  const int64_t blk = blockIdx.x;
+  const int64_t b = blk / (RB * CB), rb = (blk / CB) % RB, cb = blk % CB;
+  const int64_t base = b * rows * cols + rb * 128 * cols + cb * 128;
+  const uint16_t* wp = reinterpret_cast<const uint16_t*>(w);
+  __shared__ float red[8];
+  float amax = 0.0f;
+  // thread t: row t / 2, columns (t % 2) * 64 .. +64
+  const int r = threadIdx.x >> 1, c0 = (threadIdx.x & 1) * 64;
+  const uint16_t* rowp = wp + base + (int64_t)r * cols + c0;
+  float vals[64];
+#pragma unroll
+  for (int i = 0; i < 64; i += 8) {
+    uint4 u = *reinterpret_cast<const uint4*>(rowp + i);
+    vals[i + 0] = bf16lo_to_f32(u.x), vals[i + 1] = bf16hi_to_f32(u.x);
+    vals[i + 2] = bf16lo_to_f32(u.y), vals[i + 3] = bf16hi_to_f32(u.y);
+    vals[i + 4] = bf16lo_to_f32(u.z), vals[i + 5] = bf16hi_to_f32(u.z);
+    vals[i + 6] = bf16lo_to_f32(u.w), vals[i + 7] = bf16hi_to_f32(u.w);
+  }
+#pragma unroll
+  for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(vals[i]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = group_scale(amax);
+  uint32_t* qp = reinterpret_cast<uint32_t*>(q + base + (int64_t)r * cols + c0);
+#pragma unroll
+  for (int i = 0; i < 64; i += 4)
+    qp[i / 4] = e4m3x4(__fdiv_rn(vals[i], sc), __fdiv_rn(vals[i + 1], sc),
+                       __fdiv_rn(vals[i + 2], sc), __fdiv_rn(vals[i + 3], sc));
+  if (threadIdx.x == 0) s[blk] = sc;
+}
+
+cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
+                             const int32_t* row_map, cudaStream_t s) {
+  const int64_t warps = rows * (cols / 128);
+  quant_act_kernel<<<(unsigned)ceil_div(warps * 32, 256), 256, 0, s>>>(
+      static_cast<const uint2*>(x), rows, cols, row_map, static_cast<uint32_t*>(q), sc);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
+                                float* sc, cudaStream_t s) {
+  const int64_t blocks = nb * (rows / 128) * (cols / 128);
+  quant_weight_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), rows,
+                                                       cols, static_cast<uint8_t*>(q), sc);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,617 @@
+// Grouped GEMMs of the expert MLP on sm_100a tensor cores (tcgen05 + TMEM,
+// operands staged by TMA), with the SwiGLU epilogue fused.
+//
+// "Experts backends" (HF Transformers docs), backend table: grouped_mm /
+// deepgemm rows (tokens sorted by expert, one grouped GEMM for all experts)
+// and deepgemm_megamoe row (gated MLP: gate/up projection, SwiGLU, down
+// projection). Rows of expert e are [offsets[e], offsets[e+1]) of A; the
+// offsets are read on the device, so nothing here waits for the host.
+//
+// Two kernels:
+//  * gemm_rows_kernel  -- tokens in the MMA M slot (M = 128 rows), weights in
+//    N (256 or 128). Persistent: one CTA per SM walks a linear tile list
+//    (expert, band of m-tiles, n-tile, m-tile) so the CTAs running together
+//    share weight strips and activation bands through L2.
+//  * gemm_swap_kernel  -- the small-M variant: weight rows in the MMA M slot
+//    (M = 128) and the few token rows of an expert in N (16, 32 or 64).
+//    "AWS improves MoE model performance on Amazon SageMaker AI", section
+//    "Swap-AB advantage in MoE workloads": with few tokens per expert the
+//    large expert dimension fills the MMA's fixed-size M.
+//
+// Both use the same warp roles (192 threads):
+//   warp 0      TMA producer (one lane) through a STAGES-deep smem ring
+//   warp 1      TMEM allocator + MMA issuer (one lane)
+//   warps 2..5  epilogue: TMEM -> registers -> (SwiGLU) -> bf16 -> global
+// with two accumulator buffers in TMEM so the epilogue of one tile overlaps
+// the mainloop of the next. Every wait is bounded (see ptx::mbar_wait).
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace moe {
+namespace gg {
+
+constexpr int BM = 128;         // MMA M
+constexpr int BK = 64;          // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int UK = 16;          // K per tcgen05.mma (16-bit inputs)
+constexpr int kThreads = 192;
+constexpr int kTileA = BM * BK * 2;  // 16 KB
+constexpr int kMaxE = 1024;
+constexpr int kSmemBudget = 200 * 1024;
+
+struct Args {
+  const int32_t* offsets;  // [E + 1]
+  int E;
+  int K;
+  int ldc;         // output columns
+  int NT;          // weight tiles per expert
+  int b_rows;      // rows of B (weights) per expert
+  int up_off;      // SwiGLU: row offset of the up half inside an expert
+  int band;        // m-tiles per raster band (rows kernel)
+  int M_total;     // rows of A (and C); stores never leave [0, M_total)
+  __nv_bfloat16* C;
+  int32_t* status;
+};
+
+// ------------------------------------------------------------- scheduling
+// tile_start[e] = sum_{e' < e} tiles(e'), tile_start[E] = total. Warp-wide.
+template <int kRowsPerTile>
+__device__ void build_tile_starts(const int32_t* offsets, int E, int NT, int32_t* tile_start) {
+  const int lane = threadIdx.x & 31;
+  int32_t carry = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    int e = e0 + lane;
+    int32_t cnt = e < E ? max(offsets[e + 1] - offsets[e], 0) : 0;
+    int32_t t = (int32_t)((cnt + kRowsPerTile - 1) / kRowsPerTile) * NT;
+    int32_t incl = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (e < E) tile_start[e] = carry + incl - t;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) tile_start[E] = carry;
+}
+
+// Largest e with tile_start[e] <= tile (that expert is non-empty).
+__device__ __forceinline__ int find_expert(const int32_t* tile_start, int E, int tile) {
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (tile_start[mid] <= tile) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// ------------------------------------------------------------------ utils
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 o;
+    o.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = o;
+  }
+}
+
+// Producer drain: wait for the last in-flight loads of the ring to land so no
+// TMA write targets shared memory after the CTA has gone.
+template <int STAGES>
+__device__ void drain_loads(uint32_t full0, int64_t issued, int32_t* status) {
+  for (int64_t i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i) {
+    uint32_t bar = full0 + (uint32_t)(i % STAGES) * 8;
+    ptx::mbar_wait(bar, (uint32_t)((i / STAGES) & 1), status, kSiteDrain);
+  }
+}
+
+// ==========================================================================
+// tokens-in-M kernel
+// ==========================================================================
+template <bool SWIGLU, int BN>
+struct RowsCfg {
+  static constexpr int kTileB = BN * BK * 2;
+  static constexpr int kStage = kTileA + kTileB;
+  static constexpr int STAGES = kSmemBudget / kStage;
+  static constexpr int kAccCols = 256;  // column stride between the two accumulators
+  static constexpr uint32_t kIdesc = ptx::make_idesc(BM, BN, 1, 1);  // bf16 x bf16 -> fp32
+  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4;
+};
+
+template <bool SWIGLU, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_rows_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB, Args args) {
+  using C = RowsCfg<SWIGLU, BN>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStage);
+  // bars: full[STAGES], empty[STAGES], accf[2], acce[2], drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(smem + STAGES * C::kStage + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const uint32_t full0 = ptx::smem_addr(bars), empty0 = full0 + STAGES * 8;
+  const uint32_t accf0 = empty0 + STAGES * 8, acce0 = accf0 + 16, drain = acce0 + 16;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full0 + s * 8, 1);
+      ptx::mbar_init(empty0 + s * 8, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(accf0 + a * 8, 1);
+      ptx::mbar_init(acce0 + a * 8, 4);
+    }
+    ptx::mbar_init(drain, 1);
+    ptx::fence_barrier_init();
+    ptx::tma_prefetch_desc(&tmA);
+    ptx::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 2) build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = tile_start[args.E];
+  const int nkb = args.K / BK;
+
+  auto decode = [&](int tile, int& e, int& m, int& n) {
+    e = find_expert(tile_start, args.E, tile);
+    const int local = tile - tile_start[e];
+    const int cnt = args.offsets[e + 1] - args.offsets[e];
+    const int mt = (cnt + BM - 1) / BM;
+    const int bsz = args.band * args.NT;
+    const int b = local / bsz;
+    const int rows = min(args.band, mt - b * args.band);
+    const int l2 = local - b * bsz;
+    n = l2 / rows;
+    m = b * args.band + l2 % rows;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, m, n;
+        decode(tile, e, m, n);
+        const int row_a = args.offsets[e] + m * BM;
+        int rb0, rb1;
+        if (SWIGLU) {
+          rb0 = e * args.b_rows + n * 128;
+          rb1 = rb0 + args.up_off;
+        } else {
+          rb0 = e * args.b_rows + n * BN;
+          rb1 = rb0 + 128;
+        }
+        for (int kb = 0; kb < nkb; ++kb, ++issued) {
+          const int s = (int)(issued % STAGES);
+          const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
+          if (!ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + s * C::kStage, sb = sa + kTileA;
+          ptx::mbar_arrive_expect_tx(full0 + s * 8, C::kStage);
+          ptx::tma_load_2d(sa, &tmA, kb * BK, row_a, full0 + s * 8);
+          ptx::tma_load_2d(sb, &tmB, kb * BK, rb0, full0 + s * 8);
+          if (BN == 256) ptx::tma_load_2d(sb + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
+        }
+      }
+      drain_loads<STAGES>(full0, issued, args.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int64_t consumed = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        if (!ptx::mbar_wait(acce0 + acc * 8, acc_ph ^ 1, args.status, kSiteMmaAccEmpty)) break;
+        ptx::tc_fence_after();
+        const uint32_t d = tmem_base + acc * C::kAccCols;
+        for (int kb = 0; kb < nkb; ++kb, ++consumed) {
+          const int s = (int)(consumed % STAGES);
+          const uint32_t ph = (uint32_t)((consumed / STAGES) & 1);
+          if (!ptx::mbar_wait(full0 + s * 8, ph, args.status, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa = sbase + s * C::kStage, sb = sa + kTileA;
+          const uint64_t da = ptx::sw128_kmajor_desc(sa), db = ptx::sw128_kmajor_desc(sb);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk)
+            ptx::mma_f16(d, da + (uint64_t)(kk * UK * 2 / 16), db + (uint64_t)(kk * UK * 2 / 16),
+                         C::kIdesc, (kb | kk) != 0);
+          ptx::mma_commit(empty0 + s * 8);
+        }
+        if (!ok) break;
+        ptx::mma_commit(accf0 + acc * 8);
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1;
+      }
+      // every MMA this thread issued has completed once `drain` fires
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, args.status, kSiteDrain);
+    }
+  } else {
+    // epilogue warps 2..5 -> TMEM lane quarter warp % 4
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int e, m, n;
+      decode(tile, e, m, n);
+      const int row = args.offsets[e] + m * BM + q * 32 + lane;
+      const bool valid = row >= 0 && row < args.offsets[e + 1] && row < args.M_total;
+      if (!ptx::mbar_wait(accf0 + acc * 8, acc_ph, args.status, kSiteEpiAccFull)) break;
+      ptx::tc_fence_after();
+      const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
+      if (SWIGLU) {
+        __nv_bfloat16* dst = args.C + (int64_t)row * args.ldc + n * 128;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t g[32], u[32];
+          ptx::tmem_ld32(t0 + c, g);
+          ptx::tmem_ld32(t0 + 128 + c, u);
+          ptx::tmem_wait_ld();
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) h[i] = silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i]));
+          if (valid) store_row32(dst + c, h);
+        }
+      } else {
+        __nv_bfloat16* dst = args.C + (int64_t)row * args.ldc + n * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld32(t0 + c, v);
+          ptx::tmem_wait_ld();
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
+          if (valid) store_row32(dst + c, y);
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acce0 + acc * 8);
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ==========================================================================
+// small-M (swap-AB) kernel: weights in M, tokens in N
+// ==========================================================================
+template <bool SWIGLU, int BNT>
+struct SwapCfg {
+  static constexpr int kNA = SWIGLU ? 2 : 1;                 // weight tiles per stage
+  static constexpr int kTileB = BNT * BK * 2;
+  static constexpr int kStage = kNA * kTileA + kTileB;       // multiple of 1024
+  static constexpr int STAGES = (kSmemBudget / kStage) > 12 ? 12 : (kSmemBudget / kStage);
+  static constexpr int kAccCols = kNA * BNT;                 // per accumulator buffer
+  static constexpr int kTmemCols = (2 * kAccCols) <= 32 ? 32 : (2 * kAccCols) <= 64 ? 64
+                                   : (2 * kAccCols) <= 128 ? 128 : 256;
+  static constexpr uint32_t kIdesc = ptx::make_idesc(BM, BNT, 1, 1);
+  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4;
+};
+
+// tmA: weights [E*b_rows, K]; tmB: activation rows [M_total, K].
+// Tile = (expert e, token tile tt, weight tile n); order: e, tt, n.
+template <bool SWIGLU, int BNT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_swap_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB, Args args) {
+  using C = SwapCfg<SWIGLU, BNT>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStage);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(smem + STAGES * C::kStage + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const uint32_t full0 = ptx::smem_addr(bars), empty0 = full0 + STAGES * 8;
+  const uint32_t accf0 = empty0 + STAGES * 8, acce0 = accf0 + 16, drain = acce0 + 16;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full0 + s * 8, 1);
+      ptx::mbar_init(empty0 + s * 8, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(accf0 + a * 8, 1);
+      ptx::mbar_init(acce0 + a * 8, 4);
+    }
+    ptx::mbar_init(drain, 1);
+    ptx::fence_barrier_init();
+    ptx::tma_prefetch_desc(&tmA);
+    ptx::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_slot), C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 2) build_tile_starts<BNT>(args.offsets, args.E, args.NT, tile_start);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = tile_start[args.E];
+  const int nkb = args.K / BK;
+
+  auto decode = [&](int tile, int& e, int& tt, int& n) {
+    e = find_expert(tile_start, args.E, tile);
+    const int local = tile - tile_start[e];
+    tt = local / args.NT;
+    n = local % args.NT;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, tt, n;
+        decode(tile, e, tt, n);
+        const int row_b = args.offsets[e] + tt * BNT;
+        const int ra = e * args.b_rows + n * 128;
+        for (int kb = 0; kb < nkb; ++kb, ++issued) {
+          const int s = (int)(issued % STAGES);
+          const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
+          if (!ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + s * C::kStage, sb = sa + C::kNA * kTileA;
+          ptx::mbar_arrive_expect_tx(full0 + s * 8, C::kStage);
+          ptx::tma_load_2d(sa, &tmA, kb * BK, ra, full0 + s * 8);
+          if (SWIGLU) ptx::tma_load_2d(sa + kTileA, &tmA, kb * BK, ra + args.up_off, full0 + s * 8);
+          ptx::tma_load_2d(sb, &tmB, kb * BK, row_b, full0 + s * 8);
+        }
+      }
+      drain_loads<STAGES>(full0, issued, args.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int64_t consumed = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        if (!ptx::mbar_wait(acce0 + acc * 8, acc_ph ^ 1, args.status, kSiteMmaAccEmpty)) break;
+        ptx::tc_fence_after();
+        const uint32_t d = tmem_base + acc * C::kAccCols;
+        for (int kb = 0; kb < nkb; ++kb, ++consumed) {
+          const int s = (int)(consumed % STAGES);
+          const uint32_t ph = (uint32_t)((consumed / STAGES) & 1);
+          if (!ptx::mbar_wait(full0 + s * 8, ph, args.status, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa = sbase + s * C::kStage, sb = sa + C::kNA * kTileA;
+          const uint64_t da = ptx::sw128_kmajor_desc(sa), db = ptx::sw128_kmajor_desc(sb);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk) {
+            const uint64_t ko = (uint64_t)(kk * UK * 2 / 16);
+            ptx::mma_f16(d, da + ko, db + ko, C::kIdesc, (kb | kk) != 0);
+            if (SWIGLU)
+              ptx::mma_f16(d + BNT, da + (uint64_t)(kTileA >> 4) + ko, db + ko, C::kIdesc,
+                           (kb | kk) != 0);
+          }
+          ptx::mma_commit(empty0 + s * 8);
+        }
+        if (!ok) break;
+        ptx::mma_commit(accf0 + acc * 8);
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1;
+      }
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, args.status, kSiteDrain);
+    }
+  } else {
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int e, tt, n;
+      decode(tile, e, tt, n);
+      const int row0 = args.offsets[e] + tt * BNT;
+      const int nrows = min(min(BNT, args.offsets[e + 1] - row0), args.M_total - row0);
+      const int col = n * 128 + q * 32 + lane;  // output column owned by this thread
+      if (!ptx::mbar_wait(accf0 + acc * 8, acc_ph, args.status, kSiteEpiAccFull)) break;
+      ptx::tc_fence_after();
+      const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
+#pragma unroll 1
+      for (int c = 0; c < BNT; c += 16) {
+        uint32_t g[16], u[16];
+        ptx::tmem_ld16(t0 + c, g);
+        if (SWIGLU) ptx::tmem_ld16(t0 + BNT + c, u);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (c + i < nrows && row0 + c + i >= 0) {
+            float v = SWIGLU ? silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i]))
+                             : __uint_as_float(g[i]);
+            args.C[(int64_t)(row0 + c + i) * args.ldc + col] = __float2bfloat16_rn(v);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acce0 + acc * 8);
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace gg
+
+// ==========================================================================
+// host side
+// ==========================================================================
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  }
+  return fn;
+}
+
+// 2-D K-major operand [rows, K] with 128-byte swizzled boxes {64 (K), box_rows}.
+static bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                      int64_t K, int64_t rows, int box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K * elem_bytes)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <typename KernelT>
+static cudaError_t set_smem(KernelT k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// bf16 grouped GEMM. B: [E, b_rows, K]; for SWIGLU b_rows = 2N.
+cudaError_t launch_grouped_gemm_bf16(const void* A, const void* B, const int32_t* offsets,
+                                     int M_total, int E, int N, int K, bool swiglu, void* Cout,
+                                     int max_rows_per_expert, int32_t* status, cudaStream_t s,
+                                     const char** why) {
+  const int b_rows = swiglu ? 2 * N : N;
+  CUtensorMap tmA, tmB;
+  gg::Args a;
+  a.offsets = offsets;
+  a.E = E;
+  a.K = K;
+  a.ldc = N;
+  a.b_rows = b_rows;
+  a.up_off = swiglu ? N : 0;
+  a.C = static_cast<__nv_bfloat16*>(Cout);
+  a.M_total = M_total;
+  a.status = status;
+  const int mrpe = max_rows_per_expert > 0 ? max_rows_per_expert : M_total;
+  const int sms = num_sms();
+  if (mrpe <= 64) {
+    // small-M variant: A operand = weights, B operand = tokens
+    const int bnt = mrpe <= 16 ? 16 : mrpe <= 32 ? 32 : 64;
+    if (!make_tmap(&tmA, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, (int64_t)E * b_rows, 128) ||
+        !make_tmap(&tmB, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M_total, bnt)) {
+      *why = "cuTensorMapEncodeTiled failed";
+      return cudaErrorInvalidValue;
+    }
+    a.NT = N / 128;
+    a.band = 1;
+    const int64_t tiles_ub = ((int64_t)M_total / bnt + (M_total < E ? M_total : E)) * a.NT;
+    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_ub));
+#define MOE_SWAP(SW, BNT)                                                                \
+  do {                                                                                   \
+    auto k = gg::gemm_swap_kernel<SW, BNT>;                                              \
+    cudaError_t e = set_smem(k, gg::SwapCfg<SW, BNT>::kSmem);                            \
+    if (e != cudaSuccess) return e;                                                      \
+    k<<<grid, gg::kThreads, gg::SwapCfg<SW, BNT>::kSmem, s>>>(tmA, tmB, a);              \
+  } while (0)
+    if (swiglu) {
+      if (bnt == 16) MOE_SWAP(true, 16);
+      else if (bnt == 32) MOE_SWAP(true, 32);
+      else MOE_SWAP(true, 64);
+    } else {
+      if (bnt == 16) MOE_SWAP(false, 16);
+      else if (bnt == 32) MOE_SWAP(false, 32);
+      else MOE_SWAP(false, 64);
+    }
+#undef MOE_SWAP
+    note_launch();
+    return cudaGetLastError();
+  }
+  const int BN = swiglu ? 256 : (N % 256 == 0 ? 256 : 128);
+  if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M_total, 128) ||
+      !make_tmap(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, (int64_t)E * b_rows, 128)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  a.NT = swiglu ? N / 128 : N / BN;
+  a.band = 8;
+  const int64_t tiles_ub = ((int64_t)M_total / gg::BM + (M_total < E ? M_total : E)) * a.NT;
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_ub));
+#define MOE_ROWS(SW, BNV)                                                                \
+  do {                                                                                   \
+    auto k = gg::gemm_rows_kernel<SW, BNV>;                                              \
+    cudaError_t e = set_smem(k, gg::RowsCfg<SW, BNV>::kSmem);                            \
+    if (e != cudaSuccess) return e;                                                      \
+    k<<<grid, gg::kThreads, gg::RowsCfg<SW, BNV>::kSmem, s>>>(tmA, tmB, a);              \
+  } while (0)
+  if (swiglu)
+    MOE_ROWS(true, 256);
+  else if (BN == 256)
+    MOE_ROWS(false, 256);
+  else
+    MOE_ROWS(false, 128);
+#undef MOE_ROWS
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,237 @@
+// Permutation of routed (token, slot) pairs by expert, the row gather, and
+// the weighted combine.
+//
+// "Experts backends" (HF Transformers docs), backend table, grouped_mm row:
+// the routed tokens are sorted by chosen expert so one grouped GEMM covers
+// every expert. The order is expert-major, then token ascending; a token
+// holds each expert at most once, so this order is unique. It is built
+// without atomics on the order itself:
+//   1. per 32-token chunk (one warp), a bitmask per expert of the chunk's
+//      lanes (tokens) that chose it;
+//   2. per expert, an exclusive scan of popcount(mask) over chunks, and the
+//      expert totals;
+//   3. offsets = exclusive scan of the totals over experts; the row of
+//      (token t, slot j) with expert e is
+//        offsets[e] + chunk_base[chunk(t)][e] + popc(mask[chunk(t)][e] & lanes below t).
+#include "common.cuh"
+
+namespace moe {
+
+// ---- 1. chunk masks ---------------------------------------------------------
+// grid: one warp per chunk of 32 tokens, 4 warps per block; smem E words per warp.
+__global__ void __launch_bounds__(128) permute_mask_kernel(const int32_t* __restrict__ ids, int T,
+                                                           int E, int k, int nchunks,
+                                                           uint32_t* __restrict__ masks,
+                                                           int32_t* status) {
+  extern __shared__ uint32_t pm_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * 4 + warp;
+  uint32_t* m = pm_smem + warp * E;
+  for (int e = lane; e < E; e += 32) m[e] = 0;
+  __syncwarp();
+  if (chunk < nchunks) {
+    int t = chunk * 32 + lane;
+    if (t < T)
+      for (int j = 0; j < k; ++j) {
+        const int e = ids[(int64_t)t * k + j];
+        if ((unsigned)e < (unsigned)E) atomicOr(&m[e], 1u << lane);
+        else record_bad_index(status);
+      }
+  }
+  __syncwarp();
+  if (chunk < nchunks)
+    for (int e = lane; e < E; e += 32) masks[(int64_t)chunk * E + e] = m[e];
+}
+
+// ---- 2. per-expert scan over chunks ----------------------------------------
+// block: 32 experts (lanes) x 32 warps; warp w scans chunks [w*S, (w+1)*S).
+__global__ void __launch_bounds__(1024) permute_scan_kernel(const uint32_t* __restrict__ masks,
+                                                            int E, int nchunks,
+                                                            int32_t* __restrict__ chunk_base,
+                                                            int32_t* __restrict__ counts) {
+  __shared__ int32_t seg_total[32][33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 32 + lane;
+  const int S = (nchunks + 31) / 32;
+  const int c0 = warp * S, c1 = min(nchunks, c0 + S);
+  int32_t run = 0;
+  if (e < E)
+    for (int c = c0; c < c1; ++c) run += __popc(masks[(int64_t)c * E + e]);
+  seg_total[warp][lane] = run;
+  __syncthreads();
+  int32_t base = 0;
+  for (int w = 0; w < warp; ++w) base += seg_total[w][lane];
+  if (e < E) {
+    for (int c = c0; c < c1; ++c) {
+      chunk_base[(int64_t)c * E + e] = base;
+      base += __popc(masks[(int64_t)c * E + e]);
+    }
+    if (warp == 31) counts[e] = base;
+  }
+}
+
+// ---- 3. offsets + scatter ---------------------------------------------------
+// Each block first scans the E totals into offsets (block 0 stores them),
+// then one warp per chunk places its (token, slot) pairs.
+__global__ void __launch_bounds__(128) permute_scatter_kernel(
+    const int32_t* __restrict__ ids, const uint32_t* __restrict__ masks,
+    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ counts, int T, int E,
+    int k, int nchunks, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+    int32_t* __restrict__ inv_perm, int32_t* status) {
+  extern __shared__ int32_t off_smem[];  // E + 1
+  __shared__ int32_t warp_sums[4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // exclusive scan of counts over E with 128 threads: each owns a contiguous slice
+  const int per = (E + 127) / 128;
+  const int lo = threadIdx.x * per, hi = min(E, lo + per);
+  int32_t local = 0;
+  for (int e = lo; e < hi; ++e) local += counts[e];
+  int32_t incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  int32_t wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += warp_sums[w];
+  int32_t run = wbase + incl - local;
+  for (int e = lo; e < hi; ++e) {
+    off_smem[e] = run;
+    run += counts[e];
+  }
+  if (threadIdx.x == 127) off_smem[E] = wbase + incl;
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= E; e += 128) offsets[e] = off_smem[e];
+
+  const int chunk = blockIdx.x * 4 + warp;
+  if (chunk >= nchunks) return;
+  const int t = chunk * 32 + lane;
+  if (t >= T) return;
+  const uint32_t below = (1u << lane) - 1u;
+  for (int j = 0; j < k; ++j) {
+    int e = ids[(int64_t)t * k + j];
+    if ((unsigned)e >= (unsigned)E) continue;  // recorded by the mask kernel
+    uint32_t m = masks[(int64_t)chunk * E + e];
+    int32_t p = off_smem[e] + chunk_base[(int64_t)chunk * E + e] + __popc(m & below);
+    if ((unsigned)p >= (unsigned)(T * k)) {  // repeated expert within a token
+      record_bad_index(status);
+      continue;
+    }
+    perm_token[p] = t;
+    inv_perm[(int64_t)t * k + j] = p;
+  }
+}
+
+// ---- row gather: x_perm[p, :] = x[perm_token[p], :] --------------------------
+// one warp per row, 16-byte vectors
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                          const int32_t* __restrict__ perm_token,
+                                                          int R, int T, int vec_per_row,
+                                                          uint4* __restrict__ x_perm,
+                                                          int32_t* status) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= R) return;
+  const int t = perm_token[row];
+  if ((unsigned)t >= (unsigned)T) {
+    if (lane == 0) record_bad_index(status);
+    return;
+  }
+  const uint4* src = x + (int64_t)t * vec_per_row;
+  uint4* dst = x_perm + (int64_t)row * vec_per_row;
+  for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+}
+
+// ---- weighted combine ---------------------------------------------------------
+// "Mixture of Experts (MoE): a practical explanation", section 5 pseudocode
+// `y = sum_i weights_i * expert_i(x)`:
+//   out[t, c] = sum_{j ascending} w[t, j] * y_perm[inv_perm[t, j], c]  (fp32) -> bf16
+// Each thread owns 8 consecutive columns (one 16-byte vector) of one token.
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
+                                                      const float* __restrict__ w,
+                                                      const int32_t* __restrict__ inv_perm, int T,
+                                                      int vec_per_row, int k,
+                                                      uint4* __restrict__ out, int32_t* status) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)T * vec_per_row) return;
+  const int t = (int)(i / vec_per_row), v = (int)(i % vec_per_row);
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    const float wj = __ldg(w + (int64_t)t * k + j);
+    const int p = __ldg(inv_perm + (int64_t)t * k + j);
+    if ((unsigned)p >= (unsigned)(T * k)) {
+      record_bad_index(status);
+      continue;
+    }
+    uint4 y = __ldg(y_perm + (int64_t)p * vec_per_row + v);
+    acc[0] = __fmaf_rn(wj, bf16lo_to_f32(y.x), acc[0]);
+    acc[1] = __fmaf_rn(wj, bf16hi_to_f32(y.x), acc[1]);
+    acc[2] = __fmaf_rn(wj, bf16lo_to_f32(y.y), acc[2]);
+    acc[3] = __fmaf_rn(wj, bf16hi_to_f32(y.y), acc[3]);
+    acc[4] = __fmaf_rn(wj, bf16lo_to_f32(y.z), acc[4]);
+    acc[5] = __fmaf_rn(wj, bf16hi_to_f32(y.z), acc[5]);
+    acc[6] = __fmaf_rn(wj, bf16lo_to_f32(y.w), acc[6]);
+    acc[7] = __fmaf_rn(wj, bf16hi_to_f32(y.w), acc[7]);
+  }
+  uint4 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  o.z = pack_bf16x2(acc[4], acc[5]);
+  o.w = pack_bf16x2(acc[6], acc[7]);
+  out[i] = o;
+}
+
+// ---- launchers ------------------------------------------------------------------
+int64_t permute_scratch_bytes(int T, int E) {
+  int64_t nchunks = ceil_div(T, 32);
+  return align_up(nchunks * E * 4, 256) * 2 + align_up((int64_t)E * 4, 256);
+}
+
+cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
+                           int32_t* perm_token, int32_t* inv_perm, void* scratch,
+                           int32_t* status, cudaStream_t s) {
+  const int nchunks = (int)ceil_div(T, 32);
+  char* sp = static_cast<char*>(scratch);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(sp);
+  sp += align_up((int64_t)nchunks * E * 4, 256);
+  int32_t* chunk_base = reinterpret_cast<int32_t*>(sp);
+  sp += align_up((int64_t)nchunks * E * 4, 256);
+  int32_t* counts = reinterpret_cast<int32_t*>(sp);
+
+  const unsigned nblk = (unsigned)ceil_div(nchunks, 4);
+  permute_mask_kernel<<<nblk, 128, 4 * E * sizeof(uint32_t), s>>>(ids, T, E, k, nchunks, masks,
+                                                                  status);
+  note_launch();
+  permute_scan_kernel<<<(unsigned)ceil_div(E, 32), 1024, 0, s>>>(masks, E, nchunks, chunk_base,
+                                                                   counts);
+  note_launch();
+  permute_scatter_kernel<<<nblk, 128, (E + 1) * sizeof(int32_t), s>>>(
+      ids, masks, chunk_base, counts, T, E, k, nchunks, offsets, perm_token, inv_perm, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, int T,
+                               int row_bytes, void* x_perm, int32_t* status, cudaStream_t s) {
+  gather_rows_kernel<<<(unsigned)ceil_div(R, 8), 256, 0, s>>>(
+      static_cast<const uint4*>(x), perm_token, R, T, row_bytes / 16,
+      static_cast<uint4*>(x_perm), status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_perm, int T,
+                           int H, int k, void* out, int32_t* status, cudaStream_t s) {
+  const int vpr = H / 8;
+  const int64_t n = (int64_t)T * vpr;
+  combine_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(
+      static_cast<const uint4*>(y_perm), w, inv_perm, T, vpr, k, static_cast<uint4*>(out), status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,60 @@
+"""Shared test helpers: device transfer of raw bf16 bits, the output tolerance
+check, and cached full-size layer inputs."""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+
+import moe_inputs as mi
+
+# Output tolerance for bf16 inputs with fp32 accumulation (the layer's stated bar):
+#   max |out - ref| <= 2e-2 * max |ref|   and   sum |out - ref| / sum |ref| <= 5e-3
+BF16_TOL = (2e-2, 5e-3)
+# FP8 path, against the oracle run on the dequantised values
+FP8_TOL = (6e-2, 2e-2)
+
+
+def check_close(out, ref, tol=BF16_TOL, what="output"):
+    out = np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert out.shape == ref.shape, (out.shape, ref.shape)
+    assert np.all(np.isfinite(out)), f"{what}: non-finite values"
+    err = np.abs(out - ref)
+    max_rel = err.max() / max(np.abs(ref).max(), 1e-30)
+    l1_rel = err.sum() / max(np.abs(ref).sum(), 1e-30)
+    assert max_rel <= tol[0] and l1_rel <= tol[1], (
+        f"{what}: max|err|/max|ref| = {max_rel:.3e} (<= {tol[0]}), "
+        f"sum|err|/sum|ref| = {l1_rel:.3e} (<= {tol[1]})")
+    return max_rel, l1_rel
+
+
+def dev_bf16(a: np.ndarray):
+    import torch
+    a = np.ascontiguousarray(a, dtype=np.uint16)
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def host_bf16(t) -> np.ndarray:
+    import torch
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def dev(a: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def dev_u8(a: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+
+@functools.lru_cache(maxsize=2)
+def layer_host(name: str, **over) -> tuple:
+    cfg = mi.CONFIGS[name].with_(**over) if over else mi.CONFIGS[name]
+    return cfg, mi.make_layer(cfg)
+
+
+def dims(cfg):
+    return (cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)

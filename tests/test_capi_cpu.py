@@ -1,0 +1,114 @@
+"""The C ABI library on the CPU: it loads, exports every symbol include/moe.h
+declares, and its host-side validation rejects bad calls before any launch.
+No GPU is touched (pointers below are never dereferenced: every call fails
+validation or the device check first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_layer_tcgen05_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x7F0000001000  # 16-byte aligned address, never dereferenced
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = moe.lib()
+    names = _declared()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(moe.EXPORTED)
+    assert moe.moe_abi_version() == 1
+
+
+def test_workspace_size_and_layout():
+    d = (64, 128, 256, 8, 2)
+    n = moe.moe_workspace_size(d, moe.MOE_DTYPE_BF16)
+    L = moe.moe_workspace_layout(d, moe.MOE_DTYPE_BF16)
+    assert n == L.total > 0
+    R, H, I = 128, 128, 256
+    assert L.y_perm >= L.h + R * I * 2 and L.h >= L.x_perm + R * H * 2
+    for f in ("logits", "topk_ids", "topk_w", "offsets", "perm_token", "inv_perm", "x_perm", "h",
+              "y_perm"):
+        assert getattr(L, f) % 256 == 0
+    L8 = moe.moe_workspace_layout(d, moe.MOE_DTYPE_FP8_E4M3)
+    assert L8.x_perm == -1 and L8.h == -1 and L8.xq_perm > 0 and L8.hs > 0
+    assert moe.moe_workspace_size((64, 100, 256, 8, 2), moe.MOE_DTYPE_BF16) == 0
+
+
+@pytest.mark.parametrize("d,msg", [
+    ((0, 128, 256, 8, 2), "T must be"),
+    ((4, 100, 256, 8, 2), "H must be"),
+    ((4, 128, 200, 8, 2), "I must be"),
+    ((4, 128, 256, 2000, 2), "E must be"),
+    ((4, 128, 256, 8, 9), "k must be"),
+    ((4, 128, 256, 8, 17), "k must be"),
+])
+def test_forward_rejects_bad_dims(d, msg):
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_forward(FAKE, FAKE, None, FAKE, FAKE, d, FAKE, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG and msg in str(ei.value)
+
+
+def test_forward_rejects_null_and_misaligned_pointers():
+    d = (4, 128, 256, 8, 2)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_forward(None, FAKE, None, FAKE, FAKE, d, FAKE, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG and "x is NULL" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_forward(FAKE + 2, FAKE, None, FAKE, FAKE, d, FAKE, FAKE, 1 << 30, stream=0)
+    assert "aligned" in str(ei.value)
+
+
+def test_forward_rejects_small_workspace():
+    d = (4, 128, 256, 8, 2)
+    need = moe.moe_workspace_size(d)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_forward(FAKE, FAKE, None, FAKE, FAKE, d, FAKE, FAKE, need - 1, stream=0)
+    assert ei.value.status == moe.MOE_ERR_WORKSPACE
+
+
+def test_wrong_architecture_is_refused(monkeypatch):
+    monkeypatch.setenv("MOE_FAKE_CC", "90")
+    d = (4, 128, 256, 8, 2)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_forward(FAKE, FAKE, None, FAKE, FAKE, d, FAKE, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_DEVICE and "9.0" in str(ei.value)
+
+
+def test_grouped_gemm_validation():
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_grouped_gemm(FAKE, FAKE, FAKE, 10, 4, 100, 128, moe.MOE_DTYPE_BF16,
+                             moe.MOE_EPILOGUE_NONE, FAKE, ws=FAKE, ws_bytes=4096, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoeError) as ei:  # FP8 needs scales
+        moe.moe_grouped_gemm(FAKE, FAKE, FAKE, 10, 4, 128, 128, moe.MOE_DTYPE_FP8_E4M3,
+                             moe.MOE_EPILOGUE_NONE, FAKE, ws=FAKE, ws_bytes=4096, stream=0)
+    assert "a_scales" in str(ei.value)
+
+
+def test_permute_requires_x_and_x_perm_together():
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_permute(FAKE, (4, 128, 256, 8, 2), FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30,
+                        stream=0)
+    assert "both" in str(ei.value)
+
+
+def test_stage_events_need_six():
+    with pytest.raises(moe.MoeError):
+        moe.moe_set_stage_events([1, 2, 3])
+    moe.moe_set_stage_events(None)
+
+
+def test_last_error_is_thread_local_and_cleared():
+    moe.moe_set_stage_events(None)
+    assert moe.moe_last_error() == ""
