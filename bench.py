@@ -1,0 +1,356 @@
+"""Benchmark of the sparse MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+A step is one forward of the whole layer (router, permutation, GEMM1 +
+SwiGLU, GEMM2, combine) over one batch of synthetic tokens, with every input
+already resident in HBM. K steps are timed with CUDA events between a barrier
+and a device synchronisation on both sides; the maximum over ranks is taken.
+Under torchrun every rank runs its own replica on its own token batch (tokens
+are independent, no collective on the data path): weak scaling.
+
+Prints one JSON line (rank 0). ``--impl reference`` times the CPU oracle on
+the host cores instead (bounded token samples of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE layer tokens/s + achieved TFLOP/s or HBM GB/s as % of B200 roofline"
+DEFAULT_CONFIG = "mixtral_prefill"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
+
+
+class Clocks:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def touched_weight_bytes(cfg, offsets, bytes_per_w=2.0):
+    counts = np.diff(offsets)
+    ne = int(np.sum(counts > 0))
+    return ne * 3 * cfg.H * cfg.I * bytes_per_w, ne
+
+
+def kernel_traffic(cfg_name: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    ent = d.get(cfg_name, {}).get(kernel)
+    if not ent:
+        return None
+    src = open(os.path.join(ROOT, "mixture_experts_layer_tcgen05_b200", "csrc", ent["source"]), "rb").read()
+    if hashlib.sha256(src).hexdigest()[:16] != ent["source_sha"]:
+        return None
+    return ent["dram_bytes_per_launch"]
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline only)
+# ---------------------------------------------------------------------------
+def oracle_tokens_per_s(cfg, L, budget_s: float, seed_tag: int = 0):
+    import oracle
+
+    T = cfg.T
+
+    def run(n):
+        toks = mi.token_subset(cfg, n) if n < T else np.arange(T, dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k, tokens=toks)
+        return time.perf_counter() - t0
+
+    n0 = min(T, max(1, oracle.threads()))
+    t0 = run(n0)
+    per_tok = t0 / n0
+    n = int(min(T, max(n0, budget_s / max(per_tok, 1e-9))))
+    t = run(n) if n != n0 else t0
+    return n / t, n, t
+
+
+def reference_arm(args, cfg):
+    import oracle
+
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    L = mi.make_layer(cfg)
+    total_budget = float(os.environ.get("MOE_REF_BUDGET_S", "120"))
+    per_step = max(2.0, total_budget / max(1, args.steps + args.warmup))
+    # calibrate the sample size to the per-step budget
+    _, n, t = oracle_tokens_per_s(cfg, L, per_step)
+    toks = mi.token_subset(cfg, n) if n < cfg.T else np.arange(cfg.T, dtype=np.int32)
+    for _ in range(args.warmup):
+        oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k, tokens=toks)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k, tokens=toks)
+        times.append(time.perf_counter() - t0)
+    value = len(toks) * args.steps / sum(times)
+    sample = f"{len(toks)} of {cfg.T} tokens per step (seeded subset), whole layer per token"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.desc, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def gpu_arm(args, cfg):
+    import torch
+
+    import mixture_experts_layer_tcgen05_b200 as moe
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # each rank draws its own token batch (seed = rank); weights are shared
+    rcfg = cfg.with_(seed=cfg.seed)
+    L = mi.make_layer(rcfg)
+    if rank > 0:
+        L["x"] = mi.make_x(cfg.with_(seed=rank))
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    x, wr = bf(L["x"]), bf(L["wr"])
+    bias = torch.from_numpy(L["bias"]).cuda()
+    w13, w2 = bf(L["w13"]), bf(L["w2"])
+    d = (cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
+    ws_bytes = moe.moe_workspace_size(d)
+    io_bytes = cfg.T * cfg.H * 2
+    io_al = (io_bytes + 255) // 256 * 256
+    ws = torch.zeros(ws_bytes + 2 * io_al, dtype=torch.uint8, device="cuda")
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.moe_forward(x, wr, bias, w13, w2, d, out, ws, ws_bytes)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    status = moe.moe_get_device_status(ws)
+    if status != 0:
+        raise SystemExit(f"device status {status} after warm-up")
+    lay = moe.moe_workspace_layout(d)
+    offsets = ws[lay.offsets:lay.offsets + 4 * (cfg.E + 1)].cpu().numpy().view(np.int32)
+
+    # ---- timed region: K forwards, stage events per step ----
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(torch.cuda.current_device())
+    if rank == 0:
+        clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    n0 = moe.moe_launch_count()
+    t_start.record(stream)
+    for i in range(args.steps):
+        moe.moe_set_stage_events(stage_ev[i])
+        step()
+    t_end.record(stream)
+    moe.moe_set_stage_events(None)
+    torch.cuda.synchronize()
+    barrier()
+    launches = moe.moe_launch_count() - n0
+    clk = clocks.stop() if rank == 0 else None
+    ms = t_start.elapsed_time(t_end)
+    stages = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(5)] for ev in stage_ev])
+    stage_ms = stages.mean(0)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * cfg.T / (ms_per_step / 1e3)
+
+    # ---- end to end through the host-buffer entry point ----
+    x_host = torch.from_numpy(np.ascontiguousarray(L["x"]).view(np.int16)).pin_memory()
+    out_host = torch.empty(cfg.T * cfg.H, dtype=torch.int16).pin_memory()
+    for _ in range(2):
+        moe.moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        moe.moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ems = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ems], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = world * cfg.T / (ems / args.steps / 1e3)
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    flops = 6.0 * cfg.T * cfg.k * cfg.H * cfg.I
+    wbytes, n_exp = touched_weight_bytes(cfg, offsets)
+    layer_bytes = wbytes + 2 * cfg.T * cfg.H * 2 + cfg.H * cfg.E * 2
+    gemm1_ms = float(stage_ms[2])
+    decode = cfg.T * cfg.k <= 64 * cfg.E and cfg.T <= 64
+    if decode:
+        g1_bytes = n_exp * 2 * cfg.H * cfg.I * 2.0
+        ach = g1_bytes / (gemm1_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"],
+                "traffic": kernel_traffic(cfg.name, "gemm1"),
+                "kernel": "gemm_swap_kernel<SwiGLU> (GEMM1, small-M)",
+                "algorithmic_bytes_per_launch": g1_bytes, "peak_source": peak_src}
+    else:
+        g1_flops = 4.0 * cfg.T * cfg.k * cfg.H * cfg.I
+        ach = g1_flops / (gemm1_ms / 1e3) / 1e12
+        pk = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
+                "traffic": kernel_traffic(cfg.name, "gemm1"),
+                "kernel": "gemm_rows_kernel<SwiGLU,256> (GEMM1 + SwiGLU)",
+                "algorithmic_flops_per_launch": g1_flops,
+                "peak_source": f"{peak_src} (sustained; burst {peaks['bf16_tflops']} -> frac "
+                               f"{ach / peaks['bf16_tflops']:.3f})"}
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights)",
+        "config": {"workload": cfg.desc, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+                   "parallelism": f"token-parallel replicas x{world}",
+                   "l2": f"inputs larger than L2: {wbytes / 1e9:.2f} GB of expert weights read "
+                         "per step, no flush"},
+        "roofline": roof,
+        "layer": {"tflops": flops / (ms_per_step / 1e3) / 1e12,
+                  "tflops_frac": flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                  "gbs": layer_bytes / (ms_per_step / 1e3) / 1e9,
+                  "gbs_frac": layer_bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
+                  "touched_experts": n_exp},
+        "stages_us": {n: round(float(v) * 1e3, 2) for n, v in
+                      zip(["route", "permute", "gemm1", "gemm2", "combine"], stage_ms)},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
+                "d2h_bytes_per_step": io_bytes},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        v, n, t = oracle_tokens_per_s(cfg, L, float(os.environ.get("MOE_CPU_BUDGET_S", "20")))
+        res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle.threads(),
+                               "kind": "oracle",
+                               "sample": f"{n} of {cfg.T} tokens (seeded subset), whole layer "
+                                         f"per token, {t:.1f} s"}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(mi.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = mi.CONFIGS[args.config]
+    if args.impl == "reference":
+        reference_arm(args, cfg)
+    else:
+        gpu_arm(args, cfg)
+
+
+if __name__ == "__main__":
+    main()
