@@ -423,6 +423,7 @@ moe_status_t moe_forward_fp8(const void* x, const void* wr, const float* bias, c
   MOE_TRY(check_ptr(w2q, "w2q"));
   MOE_TRY(check_ptr(w2s, "w2s"));
   MOE_TRY(check_ptr(out, "out"));
+  if (d.H % 256) return fail(MOE_ERR_INVALID_ARG, "the FP8 layer needs H %% 256 == 0 (got %d)", d.H);
   MOE_TRY(check_ws(d, MOE_DTYPE_FP8_E4M3, ws, ws_bytes));
   MOE_TRY(check_device());
   return forward_impl(x, wr, bias, w13q, w13s, w2q, w2s, d, out, ws, MOE_DTYPE_FP8_E4M3,

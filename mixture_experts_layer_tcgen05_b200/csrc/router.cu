@@ -36,73 +36,101 @@ __device__ __forceinline__ void load_bf16_vec(const uint16_t* p, float (&v)[N]) 
   }
 }
 
-// blockDim.x = NE * NTT threads; thread (te_grp = tid % NE, tt_grp = tid / NE)
-// owns experts e0 + te_grp*TE + [0,TE) and tokens t0 + tt_grp*TT + [0,TT).
-template <int TE, int TT>
-__global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16* __restrict__ x,
-                                                            const __nv_bfloat16* __restrict__ wr,
-                                                            const float* __restrict__ bias, int T,
-                                                            int H, int E, int NE, int NTT,
-                                                            float* __restrict__ logits) {
-  const int EC = NE * TE;   // experts per block
-  const int BT = NTT * TT;  // tokens per block
+// Wide router (E > 32). Block = 32 expert groups x 8 token groups (256
+// threads); thread owns TT=4 tokens x TE=8 consecutive experts, so a block
+// covers 32 tokens x 256 experts (grid.y walks expert chunks of 256). Chunks
+// of kRouterKC h values are staged in shared memory as bf16 (x transposed to
+// [h][token], Wr as [h][expert]) with 16-byte loads, double-buffered through
+// registers so the next chunk's global loads overlap this chunk's FMAs.
+template <bool VEC>
+__global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16* __restrict__ x,
+                                                             const __nv_bfloat16* __restrict__ wr,
+                                                             const float* __restrict__ bias,
+                                                             int T, int H, int E,
+                                                             float* __restrict__ logits) {
+  constexpr int TE = 8, TT = 4, NE = 32, NTT = 8, BT = NTT * TT, EC = NE * TE;
+  constexpr int KC = kRouterKC;
+  constexpr int WVEC = KC * EC / 8 / 256;  // 16-byte w vectors per thread per chunk (8)
   extern __shared__ __align__(16) unsigned char router_smem[];
-  // xs[h][t] (token contiguous) and ws[h][e] (expert contiguous), bf16 bits
-  uint16_t* xs = reinterpret_cast<uint16_t*>(router_smem);
-  uint16_t* ws = xs + kRouterKC * BT;
-
+  uint16_t* xs = reinterpret_cast<uint16_t*>(router_smem);  // [2][KC][BT]
+  uint16_t* ws = xs + 2 * KC * BT;                           // [2][KC][EC]
   const int tid = threadIdx.x;
   const int te_grp = tid % NE, tt_grp = tid / NE;
-  const int t0 = blockIdx.x * BT;
-  const int e0 = blockIdx.y * EC;
+  const int t0 = blockIdx.x * BT, e0 = blockIdx.y * EC;
   const uint16_t* xg = reinterpret_cast<const uint16_t*>(x);
   const uint16_t* wg = reinterpret_cast<const uint16_t*>(wr);
+
+  uint4 xr, wreg[WVEC];
+  auto load = [&](int k0) {
+    {  // x: BT tokens x KC h = 256 vectors of 8
+      const int t = tid / (KC / 8), c8 = (tid % (KC / 8)) * 8;
+      xr = (t0 + t < T) ? *reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + t) * H + k0 + c8)
+                        : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < WVEC; ++i) {
+      const int v = tid + i * 256, h = v / (EC / 8), e8 = (v % (EC / 8)) * 8;
+      if (VEC) {
+        wreg[i] = (e0 + e8 < E) ? *reinterpret_cast<const uint4*>(wg + (int64_t)(k0 + h) * E + e0 + e8)
+                                : make_uint4(0, 0, 0, 0);
+      } else {
+        uint16_t tmp[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          tmp[j] = (e0 + e8 + j < E) ? wg[(int64_t)(k0 + h) * E + e0 + e8 + j] : (uint16_t)0;
+        wreg[i] = *reinterpret_cast<uint4*>(tmp);
+      }
+    }
+  };
+  auto store = [&](int b) {
+    {
+      const int t = tid / (KC / 8), c8 = (tid % (KC / 8)) * 8;
+      const uint16_t* pv = reinterpret_cast<const uint16_t*>(&xr);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xs[(b * KC + c8 + j) * BT + t] = pv[j];
+    }
+#pragma unroll
+    for (int i = 0; i < WVEC; ++i) {
+      const int v = tid + i * 256, h = v / (EC / 8), e8 = (v % (EC / 8)) * 8;
+      *reinterpret_cast<uint4*>(ws + (b * KC + h) * EC + e8) = wreg[i];
+    }
+  };
 
   float acc[TT][TE];
 #pragma unroll
   for (int a = 0; a < TT; ++a)
 #pragma unroll
-    for (int b = 0; b < TE; ++b) acc[a][b] = 0.0f;
-
-  const int nthreads = NE * NTT;
-  for (int k0 = 0; k0 < H; k0 += kRouterKC) {
-    // stage x[t0.., k0..k0+KC) transposed, 8 bf16 (16 B) per load
-    for (int i = tid; i < BT * (kRouterKC / 8); i += nthreads) {
-      int t = i / (kRouterKC / 8), c8 = (i % (kRouterKC / 8)) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t0 + t < T) v = *reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + t) * H + k0 + c8);
-      const uint16_t* pv = reinterpret_cast<const uint16_t*>(&v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xs[(c8 + j) * BT + t] = pv[j];
-    }
-    // stage wr[k0.., e0..e0+EC), zero beyond E
-    for (int i = tid; i < kRouterKC * EC; i += nthreads) {
-      int h = i / EC, e = i % EC;
-      ws[h * EC + e] = (e0 + e < E) ? wg[(int64_t)(k0 + h) * E + e0 + e] : (uint16_t)0;
-    }
-    __syncthreads();
+    for (int c = 0; c < TE; ++c) acc[a][c] = 0.0f;
+  const int nchunks = H / KC;
+  load(0);
+  store(0);
+  __syncthreads();
+  for (int c = 0; c < nchunks; ++c) {
+    const int b = c & 1;
+    if (c + 1 < nchunks) load((c + 1) * KC);
+    const uint16_t* xb = xs + b * KC * BT + tt_grp * TT;
+    const uint16_t* wb = ws + b * KC * EC + te_grp * TE;
 #pragma unroll 4
-    for (int h = 0; h < kRouterKC; ++h) {
+    for (int h = 0; h < KC; ++h) {
       float xv[TT], wv[TE];
-      const uint16_t* xp = xs + h * BT + tt_grp * TT;
-      const uint16_t* wp = ws + h * EC + te_grp * TE;
-      load_bf16_vec<TT>(xp, xv);
-      load_bf16_vec<TE>(wp, wv);
+      load_bf16_vec<TT>(xb + h * BT, xv);
+      load_bf16_vec<TE>(wb + h * EC, wv);
 #pragma unroll
       for (int a = 0; a < TT; ++a)
 #pragma unroll
-        for (int b = 0; b < TE; ++b) acc[a][b] = __fmaf_rn(xv[a], wv[b], acc[a][b]);
+        for (int e = 0; e < TE; ++e) acc[a][e] = __fmaf_rn(xv[a], wv[e], acc[a][e]);
     }
+    if (c + 1 < nchunks) store(b ^ 1);
     __syncthreads();
   }
 #pragma unroll
   for (int a = 0; a < TT; ++a) {
-    int t = t0 + tt_grp * TT + a;
+    const int t = t0 + tt_grp * TT + a;
     if (t >= T) continue;
 #pragma unroll
-    for (int b = 0; b < TE; ++b) {
-      int e = e0 + te_grp * TE + b;
-      if (e < E) logits[(int64_t)t * E + e] = __fadd_rn(acc[a][b], bias ? bias[e] : 0.0f);
+    for (int e = 0; e < TE; ++e) {
+      const int ee = e0 + te_grp * TE + e;
+      if (ee < E) logits[(int64_t)t * E + ee] = __fadd_rn(acc[a][e], bias ? bias[ee] : 0.0f);
     }
   }
 }
@@ -169,32 +197,133 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (my_slot >= 0) w[(int64_t)warp * k + my_slot] = __fdiv_rn(my_ex, denom);
 }
 
-struct RouterShape {
-  int TE, TT, NE, NTT;
+// Narrow router (E <= 32): one thread per (token, expert), so the T*E
+// sequential sums run side by side across the whole GPU. Chunks of 128 h
+// values of x and Wr are staged in shared memory as fp32 (Wr transposed, one
+// padded row per expert) in two buffers; global loads run two chunks ahead
+// through two register sets, so their latency hides behind the FMA chain.
+constexpr int kNarrowKC = 128;
+constexpr int kNarrowPad = 4;  // floats of padding per expert row (bank spread)
+
+template <int EB>
+struct NarrowStage {
+  static constexpr int BT = 256 / EB;
+  static constexpr int XV = BT * kNarrowKC / 8;         // 16-byte x vectors per chunk
+  static constexpr int XPT = (XV + 255) / 256;          // ... per thread
+  static constexpr int WV = kNarrowKC * EB / 256;       // w values per thread
+  uint4 x[XPT];
+  uint16_t w[WV];
 };
 
-static RouterShape router_shape(int E) {
-  if (E <= 32) return {8, 1, (E + 7) / 8, 64};
-  int ne = (E + 7) / 8;
-  if (ne > 32) ne = 32;
-  return {8, 4, ne, 256 / ne};
+template <int EB>
+__global__ void __launch_bounds__(256) router_narrow_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            const __nv_bfloat16* __restrict__ wr,
+                                                            const float* __restrict__ bias, int T,
+                                                            int H, int E,
+                                                            float* __restrict__ logits) {
+  using S = NarrowStage<EB>;
+  constexpr int BT = S::BT;
+  constexpr int WROW = kNarrowKC + kNarrowPad;
+  static_assert(S::XPT >= 1 && S::WV >= 1, "staging covers the chunk");
+  __shared__ __align__(16) float xs[2][BT][kNarrowKC];
+  __shared__ __align__(16) float wt[2][EB][WROW];
+  const int tid = threadIdx.x;
+  const int tl = tid / EB, el = tid % EB;
+  const int t0 = blockIdx.x * BT;
+  const uint16_t* xg = reinterpret_cast<const uint16_t*>(x);
+  const uint16_t* wg = reinterpret_cast<const uint16_t*>(wr);
+
+  auto load = [&](S& r, int k0) {
+#pragma unroll
+    for (int i = 0; i < S::XPT; ++i) {
+      const int v = tid + i * 256, t = v / (kNarrowKC / 8), c8 = (v % (kNarrowKC / 8)) * 8;
+      if (v >= S::XV) break;
+      r.x[i] = (t0 + t < T) ? *reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + t) * H + k0 + c8)
+                            : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < S::WV; ++i) {
+      const int idx = tid + i * 256, h = idx / EB, e = idx % EB;
+      r.w[i] = (e < E) ? wg[(int64_t)(k0 + h) * E + e] : (uint16_t)0;
+    }
+  };
+  auto store = [&](const S& r, int b) {
+#pragma unroll
+    for (int i = 0; i < S::XPT; ++i) {
+      const int v = tid + i * 256, t = v / (kNarrowKC / 8), c8 = (v % (kNarrowKC / 8)) * 8;
+      if (v >= S::XV) break;
+      float4* d = reinterpret_cast<float4*>(&xs[b][t][c8]);
+      const uint4 u = r.x[i];
+      d[0] = make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
+      d[1] = make_float4(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w));
+    }
+#pragma unroll
+    for (int i = 0; i < S::WV; ++i) {
+      const int idx = tid + i * 256, h = idx / EB, e = idx % EB;
+      wt[b][e][h] = __uint_as_float((uint32_t)r.w[i] << 16);
+    }
+  };
+  float acc = 0.0f;
+  auto compute = [&](int b) {
+    const float* xp = &xs[b][tl][0];
+    const float* wp = &wt[b][el][0];
+#pragma unroll 8
+    for (int h = 0; h < kNarrowKC; h += 4) {
+      const float4 xv = *reinterpret_cast<const float4*>(xp + h);
+      const float4 wv = *reinterpret_cast<const float4*>(wp + h);
+      acc = __fmaf_rn(xv.x, wv.x, acc);
+      acc = __fmaf_rn(xv.y, wv.y, acc);
+      acc = __fmaf_rn(xv.z, wv.z, acc);
+      acc = __fmaf_rn(xv.w, wv.w, acc);
+    }
+  };
+  const int n = H / kNarrowKC;
+  S ra, rb;
+  load(ra, 0);
+  if (n > 1) load(rb, kNarrowKC);
+  store(ra, 0);
+  __syncthreads();
+  // chunk c lives in buffer c & 1; chunk c+1 waits in a register set; chunk
+  // c+2 is requested before chunk c is summed.
+  for (int c = 0; c < n; c += 2) {
+    if (c + 2 < n) load(ra, (c + 2) * kNarrowKC);
+    compute(0);
+    if (c + 1 < n) store(rb, 1);
+    __syncthreads();
+    if (c + 1 >= n) break;
+    if (c + 3 < n) load(rb, (c + 3) * kNarrowKC);
+    compute(1);
+    if (c + 2 < n) store(ra, 0);
+    __syncthreads();
+  }
+  const int t = t0 + tl;
+  if (t < T && el < E) logits[(int64_t)t * E + el] = __fadd_rn(acc, bias ? bias[el] : 0.0f);
 }
 
 cudaError_t launch_router_logits(const void* x, const void* wr, const float* bias, int T, int H,
                                  int E, float* logits, cudaStream_t s) {
-  RouterShape rs = router_shape(E);
-  int EC = rs.NE * rs.TE, BT = rs.NTT * rs.TT;
-  dim3 grid((unsigned)ceil_div(T, BT), (unsigned)ceil_div(E, EC));
-  size_t smem = (size_t)kRouterKC * (BT + EC) * 2;
-  int threads = rs.NE * rs.NTT;
   const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
   const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(wr);
-  if (rs.TT == 1)
-    router_logits_kernel<8, 1><<<grid, threads, smem, s>>>(xp, wp, bias, T, H, E, rs.NE, rs.NTT,
-                                                           logits);
-  else
-    router_logits_kernel<8, 4><<<grid, threads, smem, s>>>(xp, wp, bias, T, H, E, rs.NE, rs.NTT,
-                                                           logits);
+  if (E <= 32) {
+#define MOE_NARROW(EBV)                                                                        \
+  router_narrow_kernel<EBV><<<(unsigned)ceil_div(T, 256 / EBV), 256, 0, s>>>(xp, wp, bias, T, H, \
+                                                                            E, logits)
+    if (E <= 8) MOE_NARROW(8);
+    else if (E <= 16) MOE_NARROW(16);
+    else MOE_NARROW(32);
+#undef MOE_NARROW
+    note_launch();
+    return cudaGetLastError();
+  }
+  const size_t smem = 2 * (size_t)kRouterKC * (32 + 256) * 2;
+  dim3 grid((unsigned)ceil_div(T, 32), (unsigned)ceil_div(E, 256));
+  if (E % 8 == 0) {
+    cudaFuncSetAttribute(router_wide_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    router_wide_kernel<true><<<grid, 256, smem, s>>>(xp, wp, bias, T, H, E, logits);
+  } else {
+    cudaFuncSetAttribute(router_wide_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    router_wide_kernel<false><<<grid, 256, smem, s>>>(xp, wp, bias, T, H, E, logits);
+  }
   note_launch();
   return cudaGetLastError();
 }

@@ -49,7 +49,7 @@ def _L():
             "oracle_expert_swiglu_rows": [vp, i64, vp, i64, i64, vp],
             "oracle_expert_down_rows": [vp, i64, vp, i64, i64, vp],
             "oracle_quant_act_fp8": [vp, i64, i64, vp, vp],
-            "oracle_quant_weight_fp8": [vp, i64, i64, i64, vp, vp],
+            "oracle_quant_weight_fp8": [vp, i64, i64, i64, vp, vp, i32],
             "oracle_experts_combine": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, i32],
             "oracle_experts_combine_fp8": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp,
                                            vp, i32],
@@ -154,13 +154,13 @@ def quant_act_fp8(x):
     return q, s
 
 
-def quant_weight_fp8(w):
+def quant_weight_fp8(w, nthreads=None):
     """128 x 128 blocks of w [nb, rows, cols]: q [nb, rows, cols], s [nb, rows/128, cols/128]."""
     w = _c(w, np.uint16)
     nb, rows, cols = w.shape
     q = np.empty((nb, rows, cols), dtype=np.uint8)
     s = np.empty((nb, rows // 128, cols // 128), dtype=np.float32)
-    _L().oracle_quant_weight_fp8(_p(w), nb, rows, cols, _p(q), _p(s))
+    _L().oracle_quant_weight_fp8(_p(w), nb, rows, cols, _p(q), _p(s), nthreads or threads())
     return q, s
 
 

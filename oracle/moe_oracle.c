@@ -352,26 +352,37 @@ void oracle_quant_act_fp8(const uint16_t* x, int64_t rows, int64_t cols, uint8_t
 }
 
 /* Weight quantisation of nb matrices of bf16 [rows, cols] in 128 x 128
- * blocks: q [nb, rows, cols], s [nb, rows/128, cols/128]. */
-void oracle_quant_weight_fp8(const uint16_t* w, int64_t nb, int64_t rows, int64_t cols,
-                             uint8_t* q, float* s) {
-  int64_t RB = rows / 128, CB = cols / 128;
-  for (int64_t b = 0; b < nb; ++b) {
-    const uint16_t* wb = w + b * rows * cols;
-    for (int64_t rb = 0; rb < RB; ++rb) {
-      for (int64_t cb = 0; cb < CB; ++cb) {
-        float amax = 0.0f;
-        for (int64_t r = rb * 128; r < rb * 128 + 128; ++r)
-          for (int64_t c = cb * 128; c < cb * 128 + 128; ++c)
-            amax = fmaxf(amax, fabsf(bf16_widen(wb[r * cols + c])));
-        float sc = group_scale(amax);
-        s[(b * RB + rb) * CB + cb] = sc;
-        for (int64_t r = rb * 128; r < rb * 128 + 128; ++r)
-          for (int64_t c = cb * 128; c < cb * 128 + 128; ++c)
-            q[b * rows * cols + r * cols + c] = oracle_e4m3_encode(bf16_widen(wb[r * cols + c]) / sc);
-      }
-    }
+ * blocks: q [nb, rows, cols], s [nb, rows/128, cols/128]. Blocks are
+ * independent; threads take whole blocks. */
+typedef struct {
+  const uint16_t* w;
+  int64_t rows, cols;
+  uint8_t* q;
+  float* s;
+} wq_ctx;
+
+static void wq_blocks(void* p, int64_t lo, int64_t hi) {
+  wq_ctx* c = (wq_ctx*)p;
+  int64_t RB = c->rows / 128, CB = c->cols / 128, rows = c->rows, cols = c->cols;
+  for (int64_t blk = lo; blk < hi; ++blk) {
+    int64_t b = blk / (RB * CB), rb = (blk / CB) % RB, cb = blk % CB;
+    const uint16_t* wb = c->w + b * rows * cols;
+    float amax = 0.0f;
+    for (int64_t r = rb * 128; r < rb * 128 + 128; ++r)
+      for (int64_t cc = cb * 128; cc < cb * 128 + 128; ++cc)
+        amax = fmaxf(amax, fabsf(bf16_widen(wb[r * cols + cc])));
+    float sc = group_scale(amax);
+    c->s[blk] = sc;
+    for (int64_t r = rb * 128; r < rb * 128 + 128; ++r)
+      for (int64_t cc = cb * 128; cc < cb * 128 + 128; ++cc)
+        c->q[b * rows * cols + r * cols + cc] = oracle_e4m3_encode(bf16_widen(wb[r * cols + cc]) / sc);
   }
+}
+
+void oracle_quant_weight_fp8(const uint16_t* w, int64_t nb, int64_t rows, int64_t cols,
+                             uint8_t* q, float* s, int nthreads) {
+  wq_ctx c = {w, rows, cols, q, s};
+  parallel_for(nb * (rows / 128) * (cols / 128), nthreads, wq_blocks, &c);
 }
 
 /* ------------------------------------------------------------------------ */

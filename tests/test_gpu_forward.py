@@ -111,4 +111,6 @@ def test_mixtral_prefill_full_size_sampled():
 def test_fine_grained_full_size_sampled():
     cfg, L = layer_host("fine_grained")
     _, off = check_layer(cfg, L)
-    assert np.sum(np.diff(off) == 0) >= 1
+    counts = np.diff(off)
+    # Zipf-skewed load: the largest expert holds many times the mean
+    assert counts.max() > 8 * counts.mean()
