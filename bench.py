@@ -94,6 +94,27 @@ class Clocks:
                 "samples": len(sm)}
 
 
+def rank_tokens(cfg, rank: int) -> np.ndarray:
+    """Token batch of one replica: rank r draws its own x (seed r); the
+    weights and router are shared by every rank."""
+    return mi.make_x(cfg.with_(seed=cfg.seed + rank))
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """All ranks take the same collective step; returns the max of `value`."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(T: int, world: int, ms_per_step: float) -> float:
+    """Weak scaling: every rank processes T tokens per step; the job's time is the slowest rank's."""
+    return world * T / (ms_per_step / 1e3)
+
+
 def touched_weight_bytes(cfg, offsets, bytes_per_w=2.0):
     counts = np.diff(offsets)
     ne = int(np.sum(counts > 0))
@@ -192,11 +213,10 @@ def gpu_arm(args, cfg):
         if dist is not None:
             dist.barrier()
 
-    # each rank draws its own token batch (seed = rank); weights are shared
-    rcfg = cfg.with_(seed=cfg.seed)
-    L = mi.make_layer(rcfg)
+    # each rank draws its own token batch; weights are shared
+    L = mi.make_layer(cfg)
     if rank > 0:
-        L["x"] = mi.make_x(cfg.with_(seed=rank))
+        L["x"] = rank_tokens(cfg, rank)
 
     def bf(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
@@ -246,12 +266,9 @@ def gpu_arm(args, cfg):
     ms = t_start.elapsed_time(t_end)
     stages = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(5)] for ev in stage_ev])
     stage_ms = stages.mean(0)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, "cuda")
     ms_per_step = ms / args.steps
-    value = world * cfg.T / (ms_per_step / 1e3)
+    value = whole_job_tokens_per_s(cfg.T, world, ms_per_step)
 
     # ---- end to end through the host-buffer entry point ----
     x_host = torch.from_numpy(np.ascontiguousarray(L["x"]).view(np.int16)).pin_memory()
@@ -268,11 +285,8 @@ def gpu_arm(args, cfg):
     torch.cuda.synchronize()
     barrier()
     ems = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ems], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e_value = world * cfg.T / (ems / args.steps / 1e3)
+    ems = max_over_ranks(ems, dist, "cuda")
+    e2e_value = whole_job_tokens_per_s(cfg.T, world, ems / args.steps)
 
     if dist is not None:
         dist.destroy_process_group()

@@ -22,30 +22,39 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return lo | (hi << 16);
 }
 
-// One warp per (output row, 128-column group). Output row p reads input row
+// One warp per output row; each step covers two 128-column groups (lanes
+// 0-15 and 16-31, eight values each). Output row p reads input row
 // row_map[p] (the expert permutation) or p when row_map is NULL.
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint2* __restrict__ x, int64_t rows,
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint4* __restrict__ x, int64_t rows,
                                                         int64_t cols,
                                                         const int32_t* __restrict__ row_map,
-                                                        uint32_t* __restrict__ q,
+                                                        uint2* __restrict__ q,
                                                         float* __restrict__ s) {
-  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t groups = cols / 128;
-  if (gw >= rows * groups) return;
-  const int64_t p = gw / groups, g = gw % groups;
+  if (p >= rows) return;
   const int64_t src = row_map ? row_map[p] : p;
-  // 4 bf16 per lane
-  uint2 v = x[(src * cols + g * 128) / 4 + lane];
-  float f0 = bf16lo_to_f32(v.x), f1 = bf16hi_to_f32(v.x), f2 = bf16lo_to_f32(v.y),
-        f3 = bf16hi_to_f32(v.y);
-  float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+  const int64_t vpr = cols / 8, groups = cols / 128;
+  const uint4* xr = x + src * vpr;
+  uint2* qr = q + p * vpr;
+  for (int64_t v0 = 0; v0 < vpr; v0 += 32) {
+    const int64_t v = v0 + lane;
+    const bool on = v < vpr;  // a trailing single group leaves lanes 16-31 idle
+    const uint4 u = on ? xr[v] : make_uint4(0, 0, 0, 0);
+    const float f[8] = {bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y),
+                        bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w)};
+    float amax = 0.0f;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float sc = group_scale(amax);
-  q[(p * cols + g * 128) / 4 + lane] =
-      e4m3x4(__fdiv_rn(f0, sc), __fdiv_rn(f1, sc), __fdiv_rn(f2, sc), __fdiv_rn(f3, sc));
-  if (lane == 0) s[p * groups + g] = sc;
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float sc = group_scale(amax);
+    if (on) {
+      qr[v] = make_uint2(e4m3x4(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc), __fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc)),
+                         e4m3x4(__fdiv_rn(f[4], sc), __fdiv_rn(f[5], sc), __fdiv_rn(f[6], sc), __fdiv_rn(f[7], sc)));
+      if ((lane & 15) == 0) s[p * groups + v / 16] = sc;
+    }
+  }
 }
 
 // One block (256 threads) per 128 x 128 weight block.
@@ -92,9 +101,8 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const __nv_bfloat16* 
 
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
                              const int32_t* row_map, cudaStream_t s) {
-  const int64_t warps = rows * (cols / 128);
-  quant_act_kernel<<<(unsigned)ceil_div(warps * 32, 256), 256, 0, s>>>(
-      static_cast<const uint2*>(x), rows, cols, row_map, static_cast<uint32_t*>(q), sc);
+  quant_act_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, s>>>(
+      static_cast<const uint4*>(x), rows, cols, row_map, static_cast<uint2*>(q), sc);
   note_launch();
   return cudaGetLastError();
 }

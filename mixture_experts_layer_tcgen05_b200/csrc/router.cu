@@ -16,8 +16,6 @@
 
 namespace moe {
 
-constexpr int kRouterKC = 64;  // h values staged per shared-memory chunk
-
 // N consecutive bf16 from shared memory, widened to fp32 (vector loads).
 template <int N>
 __device__ __forceinline__ void load_bf16_vec(const uint16_t* p, float (&v)[N]) {
@@ -37,23 +35,29 @@ __device__ __forceinline__ void load_bf16_vec(const uint16_t* p, float (&v)[N]) 
 }
 
 // Wide router (E > 32). Block = 32 expert groups x 8 token groups (256
-// threads); thread owns TT=4 tokens x TE=8 consecutive experts, so a block
-// covers 32 tokens x 256 experts (grid.y walks expert chunks of 256). Chunks
-// of kRouterKC h values are staged in shared memory as bf16 (x transposed to
-// [h][token], Wr as [h][expert]) with 16-byte loads, double-buffered through
-// registers so the next chunk's global loads overlap this chunk's FMAs.
+// threads); a thread owns TT=8 tokens x TE=8 consecutive experts, a block 64
+// tokens x 256 experts (grid.y walks expert chunks of 256). Chunks of KC h
+// values are converted to fp32 while being staged in shared memory (x as
+// [h][token], Wr as [h][expert]), double-buffered through registers so the
+// next chunk's global loads overlap this chunk's FMAs. The inner loop uses
+// paired FMAs (__ffma2_rn: two independent IEEE fmas per instruction), so
+// each (token, expert) sum is still one fp32 fma per h in ascending order.
+constexpr int kWideKC = 32;
+
 template <bool VEC>
 __global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16* __restrict__ x,
                                                              const __nv_bfloat16* __restrict__ wr,
                                                              const float* __restrict__ bias,
                                                              int T, int H, int E,
                                                              float* __restrict__ logits) {
-  constexpr int TE = 8, TT = 4, NE = 32, NTT = 8, BT = NTT * TT, EC = NE * TE;
-  constexpr int KC = kRouterKC;
-  constexpr int WVEC = KC * EC / 8 / 256;  // 16-byte w vectors per thread per chunk (8)
+  constexpr int TE = 8, TT = 8, NE = 32, NTT = 8, BT = NTT * TT, EC = NE * TE;
+  constexpr int KC = kWideKC;
+  constexpr int XVEC = BT * KC / 8 / 256;  // 16-byte x vectors per thread per chunk (1)
+  constexpr int WVEC = KC * EC / 8 / 256;  // 16-byte w vectors per thread per chunk (4)
+  static_assert(XVEC == 1 && WVEC == 4, "staging layout");
   extern __shared__ __align__(16) unsigned char router_smem[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(router_smem);  // [2][KC][BT]
-  uint16_t* ws = xs + 2 * KC * BT;                           // [2][KC][EC]
+  float* xs = reinterpret_cast<float*>(router_smem);  // [2][KC][BT]
+  float* ws = xs + 2 * KC * BT;                        // [2][KC][EC]
   const int tid = threadIdx.x;
   const int te_grp = tid % NE, tt_grp = tid / NE;
   const int t0 = blockIdx.x * BT, e0 = blockIdx.y * EC;
@@ -85,22 +89,28 @@ __global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16
   auto store = [&](int b) {
     {
       const int t = tid / (KC / 8), c8 = (tid % (KC / 8)) * 8;
-      const uint16_t* pv = reinterpret_cast<const uint16_t*>(&xr);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xs[(b * KC + c8 + j) * BT + t] = pv[j];
+      float* d = xs + (b * KC + c8) * BT + t;
+      d[0 * BT] = bf16lo_to_f32(xr.x), d[1 * BT] = bf16hi_to_f32(xr.x);
+      d[2 * BT] = bf16lo_to_f32(xr.y), d[3 * BT] = bf16hi_to_f32(xr.y);
+      d[4 * BT] = bf16lo_to_f32(xr.z), d[5 * BT] = bf16hi_to_f32(xr.z);
+      d[6 * BT] = bf16lo_to_f32(xr.w), d[7 * BT] = bf16hi_to_f32(xr.w);
     }
 #pragma unroll
     for (int i = 0; i < WVEC; ++i) {
       const int v = tid + i * 256, h = v / (EC / 8), e8 = (v % (EC / 8)) * 8;
-      *reinterpret_cast<uint4*>(ws + (b * KC + h) * EC + e8) = wreg[i];
+      float4* d = reinterpret_cast<float4*>(ws + (b * KC + h) * EC + e8);
+      const uint4 u = wreg[i];
+      d[0] = make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
+      d[1] = make_float4(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w));
     }
   };
 
-  float acc[TT][TE];
+  // acc[a][p] holds experts (2p, 2p+1) of token a
+  float2 acc[TT][TE / 2];
 #pragma unroll
   for (int a = 0; a < TT; ++a)
 #pragma unroll
-    for (int c = 0; c < TE; ++c) acc[a][c] = 0.0f;
+    for (int p = 0; p < TE / 2; ++p) acc[a][p] = make_float2(0.0f, 0.0f);
   const int nchunks = H / KC;
   load(0);
   store(0);
@@ -108,17 +118,23 @@ __global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
     if (c + 1 < nchunks) load((c + 1) * KC);
-    const uint16_t* xb = xs + b * KC * BT + tt_grp * TT;
-    const uint16_t* wb = ws + b * KC * EC + te_grp * TE;
+    const float* xb = xs + b * KC * BT + tt_grp * TT;
+    const float* wb = ws + b * KC * EC + te_grp * TE;
 #pragma unroll 4
     for (int h = 0; h < KC; ++h) {
-      float xv[TT], wv[TE];
-      load_bf16_vec<TT>(xb + h * BT, xv);
-      load_bf16_vec<TE>(wb + h * EC, wv);
+      const float4 x0 = *reinterpret_cast<const float4*>(xb + h * BT);
+      const float4 x1 = *reinterpret_cast<const float4*>(xb + h * BT + 4);
+      const float4 w0 = *reinterpret_cast<const float4*>(wb + h * EC);
+      const float4 w1 = *reinterpret_cast<const float4*>(wb + h * EC + 4);
+      const float xv[TT] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const float2 wv[TE / 2] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
+                                 make_float2(w1.x, w1.y), make_float2(w1.z, w1.w)};
 #pragma unroll
-      for (int a = 0; a < TT; ++a)
+      for (int a = 0; a < TT; ++a) {
+        const float2 xa = make_float2(xv[a], xv[a]);
 #pragma unroll
-        for (int e = 0; e < TE; ++e) acc[a][e] = __fmaf_rn(xv[a], wv[e], acc[a][e]);
+        for (int p = 0; p < TE / 2; ++p) acc[a][p] = __ffma2_rn(xa, wv[p], acc[a][p]);
+      }
     }
     if (c + 1 < nchunks) store(b ^ 1);
     __syncthreads();
@@ -128,9 +144,10 @@ __global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16
     const int t = t0 + tt_grp * TT + a;
     if (t >= T) continue;
 #pragma unroll
-    for (int e = 0; e < TE; ++e) {
-      const int ee = e0 + te_grp * TE + e;
-      if (ee < E) logits[(int64_t)t * E + ee] = __fadd_rn(acc[a][e], bias ? bias[ee] : 0.0f);
+    for (int p = 0; p < TE / 2; ++p) {
+      const int ee = e0 + te_grp * TE + 2 * p;
+      if (ee < E) logits[(int64_t)t * E + ee] = __fadd_rn(acc[a][p].x, bias ? bias[ee] : 0.0f);
+      if (ee + 1 < E) logits[(int64_t)t * E + ee + 1] = __fadd_rn(acc[a][p].y, bias ? bias[ee + 1] : 0.0f);
     }
   }
 }
@@ -216,7 +233,7 @@ struct NarrowStage {
 };
 
 template <int EB>
-__global__ void __launch_bounds__(256) router_narrow_kernel(const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(256, 1) router_narrow_kernel(const __nv_bfloat16* __restrict__ x,
                                                             const __nv_bfloat16* __restrict__ wr,
                                                             const float* __restrict__ bias, int T,
                                                             int H, int E,
@@ -264,17 +281,32 @@ __global__ void __launch_bounds__(256) router_narrow_kernel(const __nv_bfloat16*
     }
   };
   float acc = 0.0f;
+  // The chain is latency-bound (one fma per h). Operands move from shared
+  // memory to registers 16 h at a time, one group ahead of the fmas that use
+  // them, so the chain never waits on a shared load.
   auto compute = [&](int b) {
-    const float* xp = &xs[b][tl][0];
-    const float* wp = &wt[b][el][0];
-#pragma unroll 8
-    for (int h = 0; h < kNarrowKC; h += 4) {
-      const float4 xv = *reinterpret_cast<const float4*>(xp + h);
-      const float4 wv = *reinterpret_cast<const float4*>(wp + h);
-      acc = __fmaf_rn(xv.x, wv.x, acc);
-      acc = __fmaf_rn(xv.y, wv.y, acc);
-      acc = __fmaf_rn(xv.z, wv.z, acc);
-      acc = __fmaf_rn(xv.w, wv.w, acc);
+    const float4* xp = reinterpret_cast<const float4*>(&xs[b][tl][0]);
+    const float4* wp = reinterpret_cast<const float4*>(&wt[b][el][0]);
+    float4 xa[4], wa[4], xn[4], wn[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) xa[j] = xp[j], wa[j] = wp[j];
+#pragma unroll
+    for (int g = 0; g < kNarrowKC / 16; ++g) {
+      if (g + 1 < kNarrowKC / 16) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xn[j] = xp[4 * (g + 1) + j], wn[j] = wp[4 * (g + 1) + j];
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc = __fmaf_rn(xa[j].x, wa[j].x, acc);
+        acc = __fmaf_rn(xa[j].y, wa[j].y, acc);
+        acc = __fmaf_rn(xa[j].z, wa[j].z, acc);
+        acc = __fmaf_rn(xa[j].w, wa[j].w, acc);
+      }
+      if (g + 1 < kNarrowKC / 16) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xa[j] = xn[j], wa[j] = wn[j];
+      }
     }
   };
   const int n = H / kNarrowKC;
@@ -315,8 +347,8 @@ cudaError_t launch_router_logits(const void* x, const void* wr, const float* bia
     note_launch();
     return cudaGetLastError();
   }
-  const size_t smem = 2 * (size_t)kRouterKC * (32 + 256) * 2;
-  dim3 grid((unsigned)ceil_div(T, 32), (unsigned)ceil_div(E, 256));
+  const size_t smem = 2 * (size_t)kWideKC * (64 + 256) * 4;
+  dim3 grid((unsigned)ceil_div(T, 64), (unsigned)ceil_div(E, 256));
   if (E % 8 == 0) {
     cudaFuncSetAttribute(router_wide_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     router_wide_kernel<true><<<grid, 256, smem, s>>>(xp, wp, bias, T, H, E, logits);

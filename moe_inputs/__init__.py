@@ -63,6 +63,8 @@ def _L():
         lib.gen_normal_f32.argtypes = [u64, u32, f32, i64, i64, i64, i32, i64, vp, i32]
         lib.gen_permutation.argtypes = [u64, u32, i64, vp]
         lib.gen_raw_u64.argtypes = [u64, u32, i64, vp]
+        lib.gen_splitmix64.argtypes = [u64]
+        lib.gen_splitmix64.restype = u64
         for f in (lib.gen_normal_bf16, lib.gen_normal_f32, lib.gen_permutation, lib.gen_raw_u64):
             f.restype = None
         _lib = lib
@@ -76,6 +78,10 @@ def _threads() -> int:
 def _ptr(a: np.ndarray) -> int:
     assert a.flags["C_CONTIGUOUS"]
     return a.ctypes.data
+
+
+def splitmix64(z: int) -> int:
+    return int(_L().gen_splitmix64(z))
 
 
 def raw_u64(seed: int, tag: int, n: int) -> np.ndarray:

@@ -7,7 +7,7 @@
  *
  * Generator (counter based, so any element can be drawn independently and in
  * parallel):
- *   key    = seed ^ (tag << 56)
+ *   key    = splitmix64(seed ^ (tag << 56))         one well-mixed key per (seed, tensor)
  *   u64    = splitmix64(key ^ (idx >> 1))           one draw per index pair
  *   u1, u2 = ((u64 >> 32) + 0.5) / 2^32, ((u64 & 0xffffffff) + 0.5) / 2^32
  *   z      = sqrt(-2 ln u1) * (idx even ? cos(2 pi u2) : sin(2 pi u2))
@@ -33,7 +33,7 @@ static inline uint64_t splitmix64(uint64_t z) {
 }
 
 static inline uint64_t gen_key(uint64_t seed, uint32_t tag) {
-  return seed ^ ((uint64_t)tag << 56);
+  return splitmix64(seed ^ ((uint64_t)tag << 56));
 }
 
 static inline float normal_at(uint64_t key, uint64_t idx) {
@@ -135,7 +135,10 @@ void gen_permutation(uint64_t seed, uint32_t tag, int64_t n, int32_t* perm) {
   }
 }
 
-/* Raw 64-bit draws, exposed so tests can pin the generator itself. */
+/* The SplitMix64 finaliser itself, exposed so tests can pin it. */
+uint64_t gen_splitmix64(uint64_t z) { return splitmix64(z); }
+
+/* Raw 64-bit draws of one stream. */
 void gen_raw_u64(uint64_t seed, uint32_t tag, int64_t n, uint64_t* out) {
   uint64_t key = gen_key(seed, tag);
   for (int64_t i = 0; i < n; ++i) out[i] = splitmix64(key ^ (uint64_t)i);

@@ -1,0 +1,55 @@
+"""Host-side logic of the multi-GPU bench on CPU ranks (gloo, world size 2):
+token-parallel replicas share the weights, draw their own token batches, and
+report the whole-job rate from the slowest rank's time."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import moe_inputs as mi
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cfg = mi.CONFIGS["tiny"]
+        x = bench.rank_tokens(cfg, rank)
+        wr, b = mi.make_router(cfg)
+        # fake per-rank step times: rank 1 is slower
+        ms = 10.0 + 5.0 * rank
+        mx = bench.max_over_ranks(ms, dist)
+        rate = bench.whole_job_tokens_per_s(cfg.T, world, mx)
+        digest = torch.tensor([float(x.astype(np.float64).sum()), float(wr.astype(np.float64).sum())],
+                              dtype=torch.float64)
+        allx = [torch.zeros(2, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(allx, digest)
+        out[rank] = (mx, rate, [t.tolist() for t in allx])
+    finally:
+        dist.destroy_process_group()
+
+
+def test_token_parallel_replicas_gloo_world2():
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+    cfg = mi.CONFIGS["tiny"]
+    for r in range(world):
+        mx, rate, digests = out[r]
+        assert mx == 15.0  # the slowest rank's time
+        assert rate == pytest.approx(world * cfg.T / 0.015)
+        assert digests[0][1] == digests[1][1]  # same router weights
+        assert digests[0][0] != digests[1][0]  # different token batches

@@ -371,7 +371,13 @@ def test_fp8_forward_matches_dense_on_dequantised_values():
 # --------------------------------------------------------------------------
 def test_generator_splitmix_reference_value():
     # SplitMix64 (Steele, Lea & Flood 2014) seeded with 0: first output
-    assert int(mi.raw_u64(0, 0, 1)[0]) == 0xE220A8397B1DCDAF
+    assert mi.splitmix64(0) == 0xE220A8397B1DCDAF
+
+
+def test_generator_streams_of_different_seeds_are_unrelated():
+    a = mi.normal_bf16(0, mi.TAG_X, 1.0, 1, 64, 128)
+    b = mi.normal_bf16(1, mi.TAG_X, 1.0, 1, 64, 128)
+    assert np.sort(a).tolist() != np.sort(b).tolist()
 
 
 def test_generator_transposed_store_draws_same_values():
