@@ -140,6 +140,30 @@ moe_status_t moe_permute(const int32_t* ids_dev, moe_dims_t d, int32_t* offsets_
                          int32_t* perm_token_dev, int32_t* inv_perm_dev, const void* x_dev,
                          void* x_perm_dev, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_permute without a workspace. No passage on the pages corresponds to
+ * this entry point: it exists for callers that cannot allocate device memory
+ * when they call it -- for example an engine that plans all of its memory
+ * once at start-up and must not call cudaMalloc (or a caching allocator)
+ * while serving, or code that runs where allocation is not allowed. Results
+ * are identical to moe_permute's.
+ *
+ * The scratch lives in one fixed device array inside this library,
+ * MOE_NOALLOC_SCRATCH_BYTES bytes on every device that loads it, held until
+ * the process exits. Dims whose scratch exceeds it (2 * ceil(T/32) * E * 4
+ * bytes, each part rounded up to 256, plus E * 4) are rejected with
+ * MOE_ERR_INVALID_ARG before anything is launched; E = 256 allows T up to
+ * 16352, E = 8 about a million. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. Every call uses the same array and leaves its
+ * contents behind (nothing in it needs clearing: each call writes every word
+ * it reads), so calls that can overlap on the GPU -- two streams, or two
+ * threads -- race on it: order them on one stream. Nothing here allocates or
+ * frees memory. Arguments as for moe_permute (no ws). */
+#define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+moe_status_t moe_permute_noalloc(const int32_t* ids_dev, moe_dims_t d, int32_t* offsets_dev,
+                                 int32_t* perm_token_dev, int32_t* inv_perm_dev,
+                                 const void* x_dev, void* x_perm_dev, void* stream);
+
 /* Grouped GEMM on tcgen05 tensor cores ([X] backend table, grouped_mm and
  * deepgemm rows: one grouped GEMM over expert-sorted rows).
  * For each expert e, rows m in [offsets[e], offsets[e+1]) of A:

@@ -23,6 +23,7 @@ __all__ = [
     "MOE_DTYPE_BF16", "MOE_DTYPE_FP8_E4M3", "MOE_EPILOGUE_NONE", "MOE_EPILOGUE_SWIGLU",
     "moe_last_error", "moe_abi_version", "moe_launch_count", "moe_workspace_size",
     "moe_workspace_layout", "moe_route_topk", "moe_topk_from_logits", "moe_permute",
+    "moe_permute_noalloc",
     "moe_grouped_gemm", "moe_combine", "moe_forward", "moe_forward_fp8", "moe_forward_hostio",
     "moe_quantize_act_fp8", "moe_quantize_weight_fp8", "moe_get_device_status",
     "moe_clear_device_status", "moe_set_stage_events", "EXPORTED",
@@ -65,6 +66,7 @@ _SIGS = {
     "moe_route_topk": (_i32, [_vp, _vp, _vp, Dims, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_topk_from_logits": (_i32, [_vp, Dims, _vp, _vp, _vp]),
     "moe_permute": (_i32, [_vp, Dims, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_noalloc": (_i32, [_vp, Dims, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_grouped_gemm": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
                                 _vp, _i32, _vp, _sz, _vp]),
     "moe_combine": (_i32, [_vp, _vp, _vp, Dims, _vp, _vp]),
@@ -175,6 +177,12 @@ def moe_topk_from_logits(logits, d, ids, w, stream=None):
 def moe_permute(ids, d, offsets, perm_token, inv_perm, x, x_perm, ws, ws_bytes=None, stream=None):
     _check(lib().moe_permute(_p(ids), _dims(d), _p(offsets), _p(perm_token), _p(inv_perm), _p(x),
                              _p(x_perm), _p(ws), _nbytes(ws, ws_bytes), _s(stream)))
+
+
+def moe_permute_noalloc(ids, d, offsets, perm_token, inv_perm, x=None, x_perm=None, stream=None):
+    """moe_permute with the library's fixed scratch array (no workspace, no allocation)."""
+    _check(lib().moe_permute_noalloc(_p(ids), _dims(d), _p(offsets), _p(perm_token), _p(inv_perm),
+                                     _p(x), _p(x_perm), _s(stream)))
 
 
 def moe_grouped_gemm(A, B, offsets, M_total, E, N, K, dt, ep, C, a_scales=None, b_scales=None,

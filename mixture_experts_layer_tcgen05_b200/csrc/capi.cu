@@ -41,6 +41,11 @@ cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q,
 cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                 float* sc, cudaStream_t s);
 
+int64_t noalloc_scratch_capacity();
+cudaError_t launch_permute_noalloc(const int32_t* ids, int T, int H, int E, int k, int32_t* offsets,
+                                   int32_t* perm_token, int32_t* inv_perm, const void* x,
+                                   void* x_perm, cudaStream_t s);
+
 static std::atomic<int64_t> g_launches{0};
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -277,6 +282,33 @@ moe_status_t moe_permute(const int32_t* ids, moe_dims_t d, int32_t* offsets, int
                            at<int32_t>(ws, L.status), s);
     if (e != cudaSuccess) return cuda_fail(e, "gather");
   }
+  return ok();
+}
+
+moe_status_t moe_permute_noalloc(const int32_t* ids, moe_dims_t d, int32_t* offsets,
+                                 int32_t* perm_token, int32_t* inv_perm, const void* x,
+                                 void* x_perm, void* stream) {
+  moe_dims_t d2 = d;
+  if (d2.I < 128) d2.I = 128;
+  MOE_TRY(check_dims(d2, true));
+  MOE_TRY(check_ptr(ids, "topk_ids"));
+  MOE_TRY(check_ptr(offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(perm_token, "perm_token"));
+  MOE_TRY(check_ptr(inv_perm, "inv_perm"));
+  if ((x == nullptr) != (x_perm == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "x and x_perm must both be given or both be NULL");
+  MOE_TRY(check_ptr(x, "x", true));
+  MOE_TRY(check_ptr(x_perm, "x_perm", true));
+  const int64_t need = permute_scratch_bytes(d.T, d.E);
+  if (need > noalloc_scratch_capacity())
+    return fail(MOE_ERR_INVALID_ARG,
+                "T=%d, E=%d need %lld bytes of permutation scratch; the fixed array holds %lld "
+                "(MOE_NOALLOC_SCRATCH_BYTES); use moe_permute with a workspace",
+                d.T, d.E, (long long)need, (long long)noalloc_scratch_capacity());
+  MOE_TRY(check_device());
+  cudaError_t e = launch_permute_noalloc(ids, d.T, d.H, d.E, d.k, offsets, perm_token, inv_perm, x,
+                                         x_perm, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "permute (fixed scratch)");
   return ok();
 }
 

@@ -1,0 +1,68 @@
+// moe_permute_noalloc: the permutation by expert with its scratch in a
+// fixed device array that this library owns, for callers that cannot hand
+// the library a workspace.
+//
+// The scratch is a file-scope __device__ array, so it exists once per device
+// that loads the library and stays allocated until the process exits. In host
+// code its name only stands in for the symbol (it is not a device address),
+// so the address the kernels receive comes from cudaGetSymbolAddress, looked
+// up once per device with that device current.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace moe {
+
+cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
+                           int32_t* perm_token, int32_t* inv_perm, void* scratch, int32_t* status,
+                           cudaStream_t s);
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, int T,
+                               int row_bytes, void* x_perm, int32_t* status, cudaStream_t s);
+
+// The largest scratch the fixed array provides (see MOE_NOALLOC_SCRATCH_BYTES).
+constexpr int64_t kNoAllocScratch = MOE_NOALLOC_SCRATCH_BYTES;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_addr[kMaxDevices] = {};
+
+// Device address of the array on the current device (looked up once per device).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_addr[dev] = p;
+  }
+  *out = g_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+int64_t noalloc_scratch_capacity() { return kNoAllocScratch; }
+
+// Same kernels as moe_permute, with the scratch taken from the fixed array.
+cudaError_t launch_permute_noalloc(const int32_t* ids, int T, int H, int E, int k, int32_t* offsets,
+                                   int32_t* perm_token, int32_t* inv_perm, const void* x,
+                                   void* x_perm, cudaStream_t s) {
+  void* scratch = nullptr;
+  cudaError_t e = scratch_address(&scratch);
+  if (e != cudaSuccess) return e;
+  // Every scratch word the permutation reads is written earlier in the same
+  // call (chunk masks, chunk bases, counts), so the array needs no clearing.
+  e = launch_permute(ids, T, E, k, offsets, perm_token, inv_perm, scratch, nullptr, s);
+  if (e == cudaSuccess && x) e = launch_gather_rows(x, perm_token, T * k, T, H * 2, x_perm, nullptr, s);
+  return e;
+}
+
+}  // namespace moe
