@@ -139,15 +139,27 @@ def kernel_traffic(cfg_name: str, kernel: str):
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline only)
 # ---------------------------------------------------------------------------
-def oracle_tokens_per_s(cfg, L, budget_s: float, seed_tag: int = 0):
+def oracle_inputs(cfg, L):
+    """Keyword arguments for oracle.moe_forward; FP8 weights are quantised by the oracle itself."""
+    import oracle
+
+    if cfg.fp8:
+        w13q, w13s = oracle.quant_weight_fp8(L["w13"])
+        w2q, w2s = oracle.quant_weight_fp8(L["w2"])
+        return {"fp8": (w13q, w13s, w2q, w2s)}
+    return {"w13": L["w13"], "w2": L["w2"]}
+
+
+def oracle_tokens_per_s(cfg, L, budget_s: float, kw=None):
     import oracle
 
     T = cfg.T
+    kw = oracle_inputs(cfg, L) if kw is None else kw
 
     def run(n):
         toks = mi.token_subset(cfg, n) if n < T else np.arange(T, dtype=np.int32)
         t0 = time.perf_counter()
-        oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k, tokens=toks)
+        oracle.moe_forward(L["x"], L["wr"], L["bias"], k=cfg.k, tokens=toks, **kw)
         return time.perf_counter() - t0
 
     n0 = min(T, max(1, oracle.threads()))
@@ -165,17 +177,18 @@ def reference_arm(args, cfg):
     if rank != 0:
         return
     L = mi.make_layer(cfg)
+    kw = oracle_inputs(cfg, L)
     total_budget = float(os.environ.get("MOE_REF_BUDGET_S", "120"))
     per_step = max(2.0, total_budget / max(1, args.steps + args.warmup))
     # calibrate the sample size to the per-step budget
-    _, n, t = oracle_tokens_per_s(cfg, L, per_step)
+    _, n, t = oracle_tokens_per_s(cfg, L, per_step, kw)
     toks = mi.token_subset(cfg, n) if n < cfg.T else np.arange(cfg.T, dtype=np.int32)
     for _ in range(args.warmup):
-        oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k, tokens=toks)
+        oracle.moe_forward(L["x"], L["wr"], L["bias"], k=cfg.k, tokens=toks, **kw)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k, tokens=toks)
+        oracle.moe_forward(L["x"], L["wr"], L["bias"], k=cfg.k, tokens=toks, **kw)
         times.append(time.perf_counter() - t0)
     value = len(toks) * args.steps / sum(times)
     sample = f"{len(toks)} of {cfg.T} tokens per step (seeded subset), whole layer per token"
@@ -225,15 +238,30 @@ def gpu_arm(args, cfg):
     bias = torch.from_numpy(L["bias"]).cuda()
     w13, w2 = bf(L["w13"]), bf(L["w2"])
     d = (cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
-    ws_bytes = moe.moe_workspace_size(d)
+    dt = moe.MOE_DTYPE_FP8_E4M3 if cfg.fp8 else moe.MOE_DTYPE_BF16
+    if cfg.fp8:
+        # one-time weight preparation (untimed): e4m3 with one fp32 scale per 128 x 128 block
+        w13q = torch.empty(cfg.E, 2 * cfg.I, cfg.H, dtype=torch.uint8, device="cuda")
+        w13s = torch.empty(cfg.E, 2 * cfg.I // 128, cfg.H // 128, dtype=torch.float32, device="cuda")
+        w2q = torch.empty(cfg.E, cfg.H, cfg.I, dtype=torch.uint8, device="cuda")
+        w2s = torch.empty(cfg.E, cfg.H // 128, cfg.I // 128, dtype=torch.float32, device="cuda")
+        moe.moe_quantize_weight_fp8(w13, cfg.E, 2 * cfg.I, cfg.H, w13q, w13s)
+        moe.moe_quantize_weight_fp8(w2, cfg.E, cfg.H, cfg.I, w2q, w2s)
+        torch.cuda.synchronize()
+        del w13, w2
+    ws_bytes = moe.moe_workspace_size(d, dt)
     io_bytes = cfg.T * cfg.H * 2
     io_al = (io_bytes + 255) // 256 * 256
     ws = torch.zeros(ws_bytes + 2 * io_al, dtype=torch.uint8, device="cuda")
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step():
-        moe.moe_forward(x, wr, bias, w13, w2, d, out, ws, ws_bytes)
+    def step(xin=None):
+        xin = x if xin is None else xin
+        if cfg.fp8:
+            moe.moe_forward_fp8(xin, wr, bias, w13q, w13s, w2q, w2s, d, out, ws, ws_bytes)
+        else:
+            moe.moe_forward(xin, wr, bias, w13, w2, d, out, ws, ws_bytes)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -270,17 +298,27 @@ def gpu_arm(args, cfg):
     ms_per_step = ms / args.steps
     value = whole_job_tokens_per_s(cfg.T, world, ms_per_step)
 
-    # ---- end to end through the host-buffer entry point ----
+    # ---- end to end: pinned host tokens in, pinned host result out, every step ----
     x_host = torch.from_numpy(np.ascontiguousarray(L["x"]).view(np.int16)).pin_memory()
     out_host = torch.empty(cfg.T * cfg.H, dtype=torch.int16).pin_memory()
+    x_dev = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+
+    def e2e_step():
+        if cfg.fp8:
+            x_dev.view(torch.int16).copy_(x_host.view(cfg.T, cfg.H), non_blocking=True)
+            step(x_dev)
+            out_host.copy_(out.view(torch.int16).view(-1), non_blocking=True)
+        else:  # the C ABI's host-buffer entry point does both copies on the stream
+            moe.moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws)
+
     for _ in range(2):
-        moe.moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws)
+        e2e_step()
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        moe.moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -295,7 +333,7 @@ def gpu_arm(args, cfg):
 
     peaks, peak_src = load_peaks()
     flops = 6.0 * cfg.T * cfg.k * cfg.H * cfg.I
-    wbytes, n_exp = touched_weight_bytes(cfg, offsets)
+    wbytes, n_exp = touched_weight_bytes(cfg, offsets, 1.0 if cfg.fp8 else 2.0)
     layer_bytes = wbytes + 2 * cfg.T * cfg.H * 2 + cfg.H * cfg.E * 2
     gemm1_ms = float(stage_ms[2])
     decode = cfg.T * cfg.k <= 64 * cfg.E and cfg.T <= 64
@@ -310,17 +348,21 @@ def gpu_arm(args, cfg):
     else:
         g1_flops = 4.0 * cfg.T * cfg.k * cfg.H * cfg.I
         ach = g1_flops / (gemm1_ms / 1e3) / 1e12
-        pk = peaks["bf16_tflops_sustained"]
+        # FP8 peak = the measured bf16 peak x the nominal fp8/bf16 ratio (2)
+        ratio = 2.0 if cfg.fp8 else 1.0
+        pk, pk_burst = ratio * peaks["bf16_tflops_sustained"], ratio * peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                 "traffic": kernel_traffic(cfg.name, "gemm1"),
-                "kernel": "gemm_rows_kernel<SwiGLU,256> (GEMM1 + SwiGLU)",
+                "kernel": ("gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)" if cfg.fp8
+                           else "gemm_rows_kernel<SwiGLU,256> (GEMM1 + SwiGLU, rows gathered)"),
                 "algorithmic_flops_per_launch": g1_flops,
-                "peak_source": f"{peak_src} (sustained; burst {peaks['bf16_tflops']} -> frac "
-                               f"{ach / peaks['bf16_tflops']:.3f})"}
+                "peak_source": f"{peak_src} bf16 x {ratio:g} (sustained; burst {pk_burst:.1f} -> frac "
+                               f"{ach / pk_burst:.3f})"}
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 -> fp32 (experts), bf16 router" if cfg.fp8 else "bf16 x bf16 -> fp32",
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights)",
         "config": {"workload": cfg.desc, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
                    "parallelism": f"token-parallel replicas x{world}",
@@ -328,7 +370,8 @@ def gpu_arm(args, cfg):
                          "per step, no flush"},
         "roofline": roof,
         "layer": {"tflops": flops / (ms_per_step / 1e3) / 1e12,
-                  "tflops_frac": flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                  "tflops_frac": flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]
+                  / (2.0 if cfg.fp8 else 1.0),
                   "gbs": layer_bytes / (ms_per_step / 1e3) / 1e9,
                   "gbs_frac": layer_bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
                   "touched_experts": n_exp},

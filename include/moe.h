@@ -95,13 +95,15 @@ size_t moe_workspace_size(moe_dims_t d, moe_dtype_t dt);
  *   perm_token int32 [T*k]               token of permuted row p
  *   inv_perm  int32 [T, k]               permuted row of (token t, slot j)
  *   x_perm    bf16 [T*k, H]  (BF16)      permuted token rows
- *   xq_perm   e4m3 [T*k, H], xs_perm fp32 [T*k, H/128]   (FP8)
+ *   xq        e4m3 [T, H], xs fp32 [T, H/128]            (FP8: x quantised per token)
+ *   xq_perm   e4m3 [T*k, H], xs_perm fp32 [T*k, H/128]   (FP8: their permuted rows)
  *   h         bf16 [T*k, I]  (BF16)      SwiGLU output per permuted row
  *   hq        e4m3 [T*k, I], hs fp32 [T*k, I/128]        (FP8)
+ *   splitk    fp32 partial sums of the small-M GEMMs (BF16 with T <= 64)
  *   y_perm    bf16 [T*k, H]              expert output per permuted row          */
 typedef struct {
   int64_t status, logits, topk_ids, topk_w, offsets, perm_token, inv_perm;
-  int64_t x_perm, xq_perm, xs_perm, h, hq, hs, y_perm, scratch, total;
+  int64_t x_perm, xq, xs, xq_perm, xs_perm, h, hq, hs, splitk, y_perm, scratch, total;
 } moe_ws_layout_t;
 moe_status_t moe_workspace_layout(moe_dims_t d, moe_dtype_t dt, moe_ws_layout_t* out);
 
@@ -166,11 +168,16 @@ moe_status_t moe_permute_noalloc(const int32_t* ids_dev, moe_dims_t d, int32_t* 
 
 /* Grouped GEMM on tcgen05 tensor cores ([X] backend table, grouped_mm and
  * deepgemm rows: one grouped GEMM over expert-sorted rows).
- * For each expert e, rows m in [offsets[e], offsets[e+1]) of A:
+ * For each expert e, routed rows m in [offsets[e], offsets[e+1]) of A:
  *   NONE:   C[m, n] = sum_k A[m, k] B[e, n, k]                  n < N
  *   SWIGLU: g = A B[e, 0:N]^T, u = A B[e, N:2N]^T, C = silu(g) * u,
  *           silu(z) = z / (1 + e^-z)   ([X] deepgemm_megamoe row)
- *   A_dev  [M_total, K] (bf16, or e4m3 with a_scales fp32 [M_total, K/128])
+ *   A_dev  [M_total, K] (bf16, or e4m3 with a_scales fp32 [M_total, K/128]);
+ *          with a_rows_dev, routed row m is row a_rows_dev[m] of A_dev
+ *          [a_src_rows, K] (and of a_scales [a_src_rows, K/128]) -- the
+ *          permutation's row gather done inside the GEMM (rows outside
+ *          [0, a_src_rows) read as zeros). Rows-per-expert bounds <= 64 with
+ *          a_rows take the large-M kernel.
  *   B_dev  [E, N or 2N, K] K-major (bf16, or e4m3 with b_scales fp32
  *          [E, rows/128, K/128], one scale per 128 x 128 block, [F])
  *   C_dev  bf16 [M_total, N]; for FP8 SWIGLU with c_scales != NULL, C is
@@ -179,9 +186,11 @@ moe_status_t moe_permute_noalloc(const int32_t* ids_dev, moe_dims_t d, int32_t* 
  *   max_rows_per_expert: an upper bound on any expert's row count (0 =
  *          unknown). Bounds <= 64 select the small-M variant that puts the
  *          weight rows in the MMA M slot ([S]).
- * N, K multiples of 128. Accumulation is fp32. ws: the forward's workspace
- * (its status word is used). */
-moe_status_t moe_grouped_gemm(const void* A_dev, const void* B_dev, const int32_t* offsets_dev,
+ * N, K multiples of 128. Accumulation is fp32. ws: its first 256 bytes hold
+ * the status word; the small-M kernel may use the rest for fp32 split-K
+ * partials (summed in a fixed order, so results stay deterministic). */
+moe_status_t moe_grouped_gemm(const void* A_dev, const int32_t* a_rows_dev, int32_t a_src_rows,
+                              const void* B_dev, const int32_t* offsets_dev,
                               int32_t M_total, int32_t E, int32_t N, int32_t K, moe_dtype_t dt,
                               moe_epilogue_t ep, void* C_dev, const float* a_scales_dev,
                               const float* b_scales_dev, float* c_scales_dev,

@@ -52,7 +52,7 @@ class Dims(ctypes.Structure):
 class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "status", "logits", "topk_ids", "topk_w", "offsets", "perm_token", "inv_perm", "x_perm",
-        "xq_perm", "xs_perm", "h", "hq", "hs", "y_perm", "scratch", "total")]
+        "xq", "xs", "xq_perm", "xs_perm", "h", "hq", "hs", "splitk", "y_perm", "scratch", "total")]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -67,8 +67,8 @@ _SIGS = {
     "moe_topk_from_logits": (_i32, [_vp, Dims, _vp, _vp, _vp]),
     "moe_permute": (_i32, [_vp, Dims, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (_i32, [_vp, Dims, _vp, _vp, _vp, _vp, _vp, _vp]),
-    "moe_grouped_gemm": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
-                                _vp, _i32, _vp, _sz, _vp]),
+    "moe_grouped_gemm": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp,
+                                _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "moe_combine": (_i32, [_vp, _vp, _vp, Dims, _vp, _vp]),
     "moe_forward": (_i32, [_vp, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _sz, _vp]),
     "moe_forward_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _sz, _vp]),
@@ -186,8 +186,10 @@ def moe_permute_noalloc(ids, d, offsets, perm_token, inv_perm, x=None, x_perm=No
 
 
 def moe_grouped_gemm(A, B, offsets, M_total, E, N, K, dt, ep, C, a_scales=None, b_scales=None,
-                     c_scales=None, max_rows_per_expert=0, ws=None, ws_bytes=None, stream=None):
-    _check(lib().moe_grouped_gemm(_p(A), _p(B), _p(offsets), M_total, E, N, K, dt, ep, _p(C),
+                     c_scales=None, max_rows_per_expert=0, ws=None, ws_bytes=None, stream=None,
+                     a_rows=None, a_src_rows=0):
+    _check(lib().moe_grouped_gemm(_p(A), _p(a_rows), a_src_rows, _p(B), _p(offsets), M_total, E, N,
+                                  K, dt, ep, _p(C),
                                   _p(a_scales), _p(b_scales), _p(c_scales), max_rows_per_expert,
                                   _p(ws), _nbytes(ws, ws_bytes), _s(stream)))
 

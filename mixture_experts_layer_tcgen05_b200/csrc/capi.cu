@@ -27,13 +27,15 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, 
                                int row_bytes, void* x_perm, int32_t* status, cudaStream_t s);
 cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_perm, int T,
                            int H, int k, void* out, int32_t* status, cudaStream_t s);
-cudaError_t launch_grouped_gemm_bf16(const void* A, const void* B, const int32_t* offsets,
-                                     int M_total, int E, int N, int K, bool swiglu, void* C,
-                                     int max_rows_per_expert, int32_t* status, cudaStream_t s,
-                                     const char** why);
-cudaError_t launch_grouped_gemm_fp8(const void* A, const float* a_scales, const void* B,
-                                    const float* b_scales, const int32_t* offsets, int M_total,
-                                    int E, int N, int K, bool swiglu, void* C, float* c_scales,
+cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A_src_rows,
+                                     const void* B, const int32_t* offsets, int M_total, int E,
+                                     int N, int K, bool swiglu, void* C,
+                                     int max_rows_per_expert, int32_t* status, void* scratch,
+                                     size_t scratch_bytes, cudaStream_t s, const char** why);
+cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_src_rows,
+                                    const float* a_scales, const void* B, const float* b_scales,
+                                    const int32_t* offsets, int M_total, int E, int N, int K,
+                                    bool swiglu, void* C, float* c_scales,
                                     int max_rows_per_expert, int32_t* status, cudaStream_t s,
                                     const char** why);
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
@@ -160,16 +162,21 @@ moe_ws_layout_t layout(moe_dims_t d, moe_dtype_t dt) {
   L.scratch = take(permute_scratch_bytes((int)T, (int)E));
   if (dt == MOE_DTYPE_BF16) {
     L.x_perm = take(R * H * 2);
-    L.xq_perm = L.xs_perm = -1;
+    L.xq = L.xs = L.xq_perm = L.xs_perm = -1;
     L.h = take(R * I * 2);
     L.hq = L.hs = -1;
+    // split-K partials of the small-M (decode) kernels: up to 8 fp32 slices
+    L.splitk = T <= 64 ? take(8 * R * std::max(2 * I, H) * 4) : -1;
   } else {
     L.x_perm = -1;
+    L.xq = take(T * H);
+    L.xs = take(T * (H / 128) * 4);
     L.xq_perm = take(R * H);
     L.xs_perm = take(R * (H / 128) * 4);
     L.h = -1;
     L.hq = take(R * I);
     L.hs = take(R * (I / 128) * 4);
+    L.splitk = -1;
   }
   L.y_perm = take(R * H * 2);
   L.total = off;
@@ -312,7 +319,8 @@ moe_status_t moe_permute_noalloc(const int32_t* ids, moe_dims_t d, int32_t* offs
   return ok();
 }
 
-moe_status_t moe_grouped_gemm(const void* A, const void* B, const int32_t* offsets,
+moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_src_rows,
+                              const void* B, const int32_t* offsets,
                               int32_t M_total, int32_t E, int32_t N, int32_t K, moe_dtype_t dt,
                               moe_epilogue_t ep, void* C, const float* a_scales,
                               const float* b_scales, float* c_scales, int32_t max_rows_per_expert,
@@ -324,6 +332,8 @@ moe_status_t moe_grouped_gemm(const void* A, const void* B, const int32_t* offse
   if (ep != MOE_EPILOGUE_NONE && ep != MOE_EPILOGUE_SWIGLU) return fail(MOE_ERR_INVALID_ARG, "bad epilogue");
   if (dt != MOE_DTYPE_BF16 && dt != MOE_DTYPE_FP8_E4M3) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
   MOE_TRY(check_ptr(A, "A"));
+  MOE_TRY(check_ptr(a_rows, "a_rows", true));
+  if (a_rows && a_src_rows < 1) return fail(MOE_ERR_INVALID_ARG, "a_src_rows must be >= 1 with a_rows");
   MOE_TRY(check_ptr(B, "B"));
   MOE_TRY(check_ptr(offsets, "expert_offsets"));
   MOE_TRY(check_ptr(C, "C"));
@@ -340,11 +350,13 @@ moe_status_t moe_grouped_gemm(const void* A, const void* B, const int32_t* offse
   const char* why = "";
   cudaError_t e;
   if (dt == MOE_DTYPE_BF16)
-    e = launch_grouped_gemm_bf16(A, B, offsets, M_total, E, N, K, ep == MOE_EPILOGUE_SWIGLU, C,
-                                 max_rows_per_expert, at<int32_t>(ws, 0),
-                                 static_cast<cudaStream_t>(stream), &why);
+    e = launch_grouped_gemm_bf16(A, a_rows, a_rows ? a_src_rows : M_total, B, offsets, M_total, E,
+                                 N, K, ep == MOE_EPILOGUE_SWIGLU, C,
+                                 max_rows_per_expert, at<int32_t>(ws, 0), at<char>(ws, 256),
+                                 ws_bytes - 256, static_cast<cudaStream_t>(stream), &why);
   else
-    e = launch_grouped_gemm_fp8(A, a_scales, B, b_scales, offsets, M_total, E, N, K,
+    e = launch_grouped_gemm_fp8(A, a_rows, a_rows ? a_src_rows : M_total, a_scales, B, b_scales,
+                                offsets, M_total, E, N, K,
                                 ep == MOE_EPILOGUE_SWIGLU, C, c_scales, max_rows_per_expert,
                                 at<int32_t>(ws, 0), static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "grouped GEMM: %s %s", cudaGetErrorString(e), why);
@@ -393,31 +405,41 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
   if (dt == MOE_DTYPE_BF16) {
     void* x_perm = at<void>(ws, L.x_perm);
     void* h = at<void>(ws, L.h);
+    // The permuted copy of x feeds GEMM1's TMA tile loads (a gather inside the
+    // GEMM costs the tensor cores more than this copy costs).
     if ((e = launch_gather_rows(x, perm_token, R, T, H * 2, x_perm, status, s)) != cudaSuccess)
       return cuda_fail(e, "gather");
     record(s, 2);
-    if ((e = launch_grouped_gemm_bf16(x_perm, w13, offsets, R, E, I, H, true, h, T, status, s,
-                                      &why)) != cudaSuccess)
+    void* splitk = L.splitk >= 0 ? at<void>(ws, L.splitk) : nullptr;
+    const size_t splitk_bytes = L.splitk >= 0 ? (size_t)(L.y_perm - L.splitk) : 0;
+    if ((e = launch_grouped_gemm_bf16(x_perm, nullptr, R, w13, offsets, R, E, I, H, true, h, T,
+                                      status, splitk, splitk_bytes, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "GEMM1: %s %s", cudaGetErrorString(e), why);
     record(s, 3);
-    if ((e = launch_grouped_gemm_bf16(h, w2, offsets, R, E, H, I, false, y_perm, T, status, s,
-                                      &why)) != cudaSuccess)
+    if ((e = launch_grouped_gemm_bf16(h, nullptr, R, w2, offsets, R, E, H, I, false, y_perm, T,
+                                      status, splitk, splitk_bytes, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "GEMM2: %s %s", cudaGetErrorString(e), why);
     record(s, 4);
   } else {
-    void* xq = at<void>(ws, L.xq_perm);
-    float* xs = at<float>(ws, L.xs_perm);
+    void* xq = at<void>(ws, L.xq);
+    float* xs = at<float>(ws, L.xs);
+    void* xq_perm = at<void>(ws, L.xq_perm);
+    float* xs_perm = at<float>(ws, L.xs_perm);
     void* hq = at<void>(ws, L.hq);
     float* hs = at<float>(ws, L.hs);
-    if ((e = launch_quant_act(x, R, H, xq, xs, perm_token, s)) != cudaSuccess)
+    // x is quantised once per token, then its codes and scales are permuted
+    if ((e = launch_quant_act(x, T, H, xq, xs, nullptr, s)) != cudaSuccess)
       return cuda_fail(e, "activation quantisation");
+    if ((e = launch_gather_rows(xq, perm_token, R, T, H, xq_perm, status, s)) != cudaSuccess ||
+        (e = launch_gather_rows(xs, perm_token, R, T, (H / 128) * 4, xs_perm, status, s)) != cudaSuccess)
+      return cuda_fail(e, "gather");
     record(s, 2);
-    if ((e = launch_grouped_gemm_fp8(xq, xs, w13, w13s, offsets, R, E, I, H, true, hq, hs, T,
-                                     status, s, &why)) != cudaSuccess)
+    if ((e = launch_grouped_gemm_fp8(xq_perm, nullptr, R, xs_perm, w13, w13s, offsets, R, E, I, H,
+                                     true, hq, hs, T, status, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "FP8 GEMM1: %s %s", cudaGetErrorString(e), why);
     record(s, 3);
-    if ((e = launch_grouped_gemm_fp8(hq, hs, w2, w2s, offsets, R, E, H, I, false, y_perm, nullptr,
-                                     T, status, s, &why)) != cudaSuccess)
+    if ((e = launch_grouped_gemm_fp8(hq, nullptr, R, hs, w2, w2s, offsets, R, E, H, I, false, y_perm,
+                                     nullptr, T, status, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "FP8 GEMM2: %s %s", cudaGetErrorString(e), why);
     record(s, 4);
   }

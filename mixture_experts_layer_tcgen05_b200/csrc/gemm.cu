@@ -24,6 +24,8 @@
 //   warps 2..5  epilogue: TMEM -> registers -> (SwiGLU) -> bf16 -> global
 // with two accumulator buffers in TMEM so the epilogue of one tile overlaps
 // the mainloop of the next. Every wait is bounded (see ptx::mbar_wait).
+#include <cmath>
+
 #include "gemm_common.cuh"
 
 namespace moe {
@@ -42,7 +44,9 @@ struct RowsCfg {
   static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4;
 };
 
-template <bool SWIGLU, int BN>
+// GATHER: A rows are copied by index (args.a_rows) from args.a_src by the
+// whole producer warp instead of being loaded from a permuted copy by TMA.
+template <bool SWIGLU, int BN, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_rows_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, Args args) {
@@ -101,7 +105,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (GATHER) {
+      // all 32 lanes gather A rows (4 each); lane 0 also owns the barriers and the B loads
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, m, n;
+        decode(tile, e, m, n);
+        int src_row[4];
+        gather4_tile_rows(args.a_rows, args.offsets[e] + m * BM, args.M_total, args.a_src_rows, lane,
+                         src_row);
+        int rb0, rb1;
+        if (SWIGLU) {
+          rb0 = e * args.b_rows + n * 128;
+          rb1 = rb0 + args.up_off;
+        } else {
+          rb0 = e * args.b_rows + n * BN;
+          rb1 = rb0 + 128;
+        }
+        for (int kb = 0; kb < nkb; ++kb, ++issued) {
+          const int s = (int)(issued % STAGES);
+          const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
+          int got = 1;
+          if (lane == 0) got = ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty);
+          if (!__shfl_sync(0xffffffffu, got, 0)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + s * C::kStage, sb = sa + kTileA;
+          if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(full0 + s * 8, C::kStage);
+            ptx::tma_load_2d(sb, &tmB, kb * BK, rb0, full0 + s * 8);
+            if (BN == 256) ptx::tma_load_2d(sb + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
+          }
+          __syncwarp();
+          ptx::tma_gather4(sa + lane * 512, &tmA, kb * BK, src_row[0], src_row[1], src_row[2],
+                           src_row[3], full0 + s * 8);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) drain_loads<STAGES>(full0, issued, args.status);
+    } else if (lane == 0) {
       int64_t issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
@@ -280,10 +324,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = tile_start[args.E];
-  const int nkb = args.K / BK;
+  // work unit = (tile, k range): with ksplit > 1 each tile's K is cut into
+  // ksplit ranges that run as separate units and leave fp32 partial sums
+  const int S = args.ksplit;
+  const int total = tile_start[args.E] * S;
+  const int nkb = args.K / BK / S;  // k-blocks per unit
 
-  auto decode = [&](int tile, int& e, int& tt, int& n) {
+  auto decode = [&](int unit, int& e, int& tt, int& n, int& kb0) {
+    const int tile = unit / S;
+    kb0 = (unit % S) * nkb;
     e = find_expert(tile_start, args.E, tile);
     const int local = tile - tile_start[e];
     tt = local / args.NT;
@@ -295,11 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        int e, tt, n;
-        decode(tile, e, tt, n);
+        int e, tt, n, kb0;
+        decode(tile, e, tt, n, kb0);
         const int row_b = args.offsets[e] + tt * BNT;
         const int ra = e * args.b_rows + n * 128;
-        for (int kb = 0; kb < nkb; ++kb, ++issued) {
+        for (int kb = kb0; kb < kb0 + nkb; ++kb, ++issued) {
           const int s = (int)(issued % STAGES);
           const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
           if (!ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty)) {
@@ -325,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ptx::mbar_wait(acce0 + acc * 8, acc_ph ^ 1, args.status, kSiteMmaAccEmpty)) break;
         ptx::tc_fence_after();
         const uint32_t d = tmem_base + acc * C::kAccCols;
-        for (int kb = 0; kb < nkb; ++kb, ++consumed) {
+        for (int kb = 0; kb < nkb; ++kb, ++consumed) {  // kb counts within the unit
           const int s = (int)(consumed % STAGES);
           const uint32_t ph = (uint32_t)((consumed / STAGES) & 1);
           if (!ptx::mbar_wait(full0 + s * 8, ph, args.status, kSiteMmaFull)) {
@@ -358,8 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      int e, tt, n;
-      decode(tile, e, tt, n);
+      int e, tt, n, kb0;
+      decode(tile, e, tt, n, kb0);
       const int row0 = args.offsets[e] + tt * BNT;
       const int nrows = min(min(BNT, args.offsets[e + 1] - row0), args.M_total - row0);
       const int col = n * 128 + q * 32 + lane;  // output column owned by this thread
@@ -372,12 +421,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_ld16(t0 + c, g);
         if (SWIGLU) ptx::tmem_ld16(t0 + BNT + c, u);
         ptx::tmem_wait_ld();
+        if (S == 1) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (c + i < nrows && row0 + c + i >= 0) {
-            float v = SWIGLU ? silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i]))
-                             : __uint_as_float(g[i]);
-            args.C[(int64_t)(row0 + c + i) * args.ldc + col] = __float2bfloat16_rn(v);
+          for (int i = 0; i < 16; ++i) {
+            if (c + i < nrows && row0 + c + i >= 0) {
+              float v = SWIGLU ? silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i]))
+                               : __uint_as_float(g[i]);
+              args.C[(int64_t)(row0 + c + i) * args.ldc + col] = __float2bfloat16_rn(v);
+            }
+          }
+        } else {  // partial sums of this K range: gate in [0, ldc), up in [ldc, 2 ldc)
+          const int pld = (SWIGLU ? 2 : 1) * args.ldc;
+          float* P = args.partial + (int64_t)(kb0 / nkb) * args.M_total * pld;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (c + i < nrows && row0 + c + i >= 0) {
+              float* prow = P + (int64_t)(row0 + c + i) * pld;
+              prow[col] = __uint_as_float(g[i]);
+              if (SWIGLU) prow[args.ldc + col] = __uint_as_float(u[i]);
+            }
           }
         }
       }
@@ -396,16 +458,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Sum of the ksplit fp32 partials of each output in split order, then the
+// epilogue the unsplit kernel would have applied (SwiGLU or none), to bf16.
+template <bool SWIGLU>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial,
+                                                            int S, int M, int N,
+                                                            __nv_bfloat16* __restrict__ C) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)M * N) return;
+  const int64_t r = i / N, c = i % N;
+  const int pld = (SWIGLU ? 2 : 1) * N;
+  const int64_t slice = (int64_t)M * pld;
+  float g = 0.0f, u = 0.0f;
+  for (int s = 0; s < S; ++s) {
+    g += partial[s * slice + r * pld + c];
+    if (SWIGLU) u += partial[s * slice + r * pld + N + c];
+  }
+  C[i] = __float2bfloat16_rn(SWIGLU ? silu_mul(g, u) : g);
+}
+
 }  // namespace gg
 
 // ==========================================================================
 // host side
 // ==========================================================================
 // bf16 grouped GEMM. B: [E, b_rows, K]; for SWIGLU b_rows = 2N.
-cudaError_t launch_grouped_gemm_bf16(const void* A, const void* B, const int32_t* offsets,
-                                     int M_total, int E, int N, int K, bool swiglu, void* Cout,
-                                     int max_rows_per_expert, int32_t* status, cudaStream_t s,
-                                     const char** why) {
+// A_rows != nullptr: routed row r of A is row A_rows[r] of A ([A_src_rows, K]).
+// scratch (may be null): room for the small-M kernel's split-K partials.
+cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A_src_rows,
+                                     const void* B, const int32_t* offsets, int M_total, int E,
+                                     int N, int K, bool swiglu, void* Cout,
+                                     int max_rows_per_expert, int32_t* status, void* scratch,
+                                     size_t scratch_bytes, cudaStream_t s, const char** why) {
   const int b_rows = swiglu ? 2 * N : N;
   CUtensorMap tmA, tmB;
   gg::Args a;
@@ -417,10 +501,16 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const void* B, const int32_t
   a.up_off = swiglu ? N : 0;
   a.C = static_cast<__nv_bfloat16*>(Cout);
   a.M_total = M_total;
+  a.a_rows = A_rows;
+  a.a_src = A;
+  a.a_src_rows = A_src_rows;
+  a.ksplit = 1;
+  a.partial = nullptr;
+  const int64_t a_tmap_rows = A_rows ? A_src_rows : M_total;
   a.status = status;
   const int mrpe = max_rows_per_expert > 0 ? max_rows_per_expert : M_total;
   const int sms = num_sms();
-  if (mrpe <= 64) {
+  if (mrpe <= 64 && !A_rows) {
     // small-M variant: A operand = weights, B operand = tokens
     const int bnt = mrpe <= 16 ? 16 : mrpe <= 32 ? 32 : 64;
     if (!make_tmap(&tmA, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, (int64_t)E * b_rows, 128) ||
@@ -431,7 +521,29 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const void* B, const int32_t
     a.NT = N / 128;
     a.band = 1;
     const int64_t tiles_ub = ((int64_t)M_total / bnt + (M_total < E ? M_total : E)) * a.NT;
-    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_ub));
+    // Split K so the units fill whole waves of SMs: a weight-streaming kernel
+    // with a partial last wave leaves HBM bandwidth unused.
+    const int nkb = K / gg::BK;
+    const int64_t pld = (int64_t)(swiglu ? 2 : 1) * N;
+    // Splitting costs pipeline ramps and the fp32 partials, so it is used only
+    // when the unsplit units leave at least a fifth of the SMs' time idle.
+    auto wave_eff = [&](int S) {
+      const double waves = (double)tiles_ub * S / sms;
+      return waves / std::ceil(waves);
+    };
+    double best = wave_eff(1);
+    if (best < 0.8) {
+      for (int S = 2; S <= 8; S *= 2) {
+        if (nkb % S || nkb / S < 8) continue;
+        if (!scratch || (int64_t)S * M_total * pld * 4 > (int64_t)scratch_bytes) continue;
+        if (wave_eff(S) > best + 0.05) {
+          best = wave_eff(S);
+          a.ksplit = S;
+        }
+      }
+    }
+    if (a.ksplit > 1) a.partial = static_cast<float*>(scratch);
+    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_ub * a.ksplit));
 #define MOE_SWAP(SW, BNT)                                                                \
   do {                                                                                   \
     auto k = gg::gemm_swap_kernel<SW, BNT>;                                              \
@@ -450,10 +562,21 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const void* B, const int32_t
     }
 #undef MOE_SWAP
     note_launch();
+    if (a.ksplit > 1) {
+      const int64_t n = (int64_t)M_total * N;
+      if (swiglu)
+        gg::splitk_reduce_kernel<true><<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(
+            a.partial, a.ksplit, M_total, N, a.C);
+      else
+        gg::splitk_reduce_kernel<false><<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(
+            a.partial, a.ksplit, M_total, N, a.C);
+      note_launch();
+    }
     return cudaGetLastError();
   }
   const int BN = swiglu ? 256 : (N % 256 == 0 ? 256 : 128);
-  if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M_total, 128) ||
+  // a gathered A is read by tile::gather4 from a map whose box is one row high
+  if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, a_tmap_rows, A_rows ? 1 : 128) ||
       !make_tmap(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, (int64_t)E * b_rows, 128)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
@@ -464,7 +587,7 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const void* B, const int32_t
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_ub));
 #define MOE_ROWS(SW, BNV)                                                                \
   do {                                                                                   \
-    auto k = gg::gemm_rows_kernel<SW, BNV>;                                              \
+    auto k = a.a_rows ? gg::gemm_rows_kernel<SW, BNV, true> : gg::gemm_rows_kernel<SW, BNV, false>; \
     cudaError_t e = set_smem(k, gg::RowsCfg<SW, BNV>::kSmem);                            \
     if (e != cudaSuccess) return e;                                                      \
     k<<<grid, gg::kThreads, gg::RowsCfg<SW, BNV>::kSmem, s>>>(tmA, tmB, a);              \

@@ -30,6 +30,11 @@ struct Args {
   int up_off;      // SwiGLU: row offset of the up half inside an expert
   int band;        // m-tiles per raster band (rows kernel)
   int M_total;     // rows of A (and C); stores never leave [0, M_total)
+  const int32_t* a_rows;  // gather: source row of each routed row (nullptr: A is dense)
+  const void* a_src;      // gather: source matrix [a_src_rows, K]
+  int a_src_rows;
+  int ksplit;        // small-M kernel: K split into ksplit ranges, fp32 partials
+  float* partial;    // [ksplit, M_total, pld] with pld = (SwiGLU ? 2 : 1) * ldc
   __nv_bfloat16* C;
   int32_t* status;
 };
@@ -92,6 +97,27 @@ __device__ void drain_loads(uint32_t full0, int64_t issued, int32_t* status) {
   for (int64_t i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i) {
     uint32_t bar = full0 + (uint32_t)(i % STAGES) * 8;
     ptx::mbar_wait(bar, (uint32_t)((i / STAGES) & 1), status, kSiteDrain);
+  }
+}
+
+// ---------------------------------------------------------- row gather
+// A-operand rows fetched by index instead of from a permuted copy: lane l of
+// the producer warp loads tile rows 4l..4l+3 with one TMA tile::gather4
+// (tensor map box one row high, 128-byte swizzle), 512 bytes at offset 512*l
+// of the stage, so the 32 lanes fill the same 128-row layout a tile load
+// leaves. Rows past M_total (or with an index out of range) get row index
+// `src_rows`, outside the tensor, and are zero-filled.
+__device__ __forceinline__ void gather4_tile_rows(const int32_t* row_map, int base, int M_total,
+                                                  int src_rows, int lane, int (&out)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int r = base + 4 * lane + j;
+    int t = src_rows;
+    if (r >= 0 && r < M_total) {
+      const int v = row_map[r];
+      if ((unsigned)v < (unsigned)src_rows) t = v;
+    }
+    out[j] = t;
   }
 }
 

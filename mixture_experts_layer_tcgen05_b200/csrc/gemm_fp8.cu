@@ -39,11 +39,14 @@ constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4 
 struct Args {
   const int32_t* offsets;
   int E, K, ldc, NT, b_rows, up_off, band, M_total;
+  const int32_t* a_rows;  // gather: source row of each routed row (nullptr: A is dense)
+  const void* a_src;      // gather: source matrix [a_src_rows, K] (e4m3)
+  int a_src_rows;
   int kblocks;  // K / 128
   int b_nblk;   // 128-row blocks of B per expert
   void* C;      // bf16 [M_total, ldc], or e4m3 when c_scales != nullptr
   float* c_scales;
-  const float* a_scales;  // [M_total, kblocks]
+  const float* a_scales;  // [M_total, kblocks], or [a_src_rows, kblocks] with a gather
   const float* b_scales;  // [E, b_nblk, kblocks]
   int32_t* status;
 };
@@ -58,7 +61,7 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return lo | (hi << 16);
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_rows_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, Args args) {
@@ -119,7 +122,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (GATHER) {
+      // all 32 lanes gather A rows (4 each); lane 0 also owns the barriers and the B loads
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, m, n;
+        decode(tile, e, m, n);
+        int src_row[4];
+        gg::gather4_tile_rows(args.a_rows, args.offsets[e] + m * BM, args.M_total, args.a_src_rows,
+                             lane, src_row);
+        int rb0, rb1;
+        if (SWIGLU) {
+          rb0 = e * args.b_rows + n * 128;
+          rb1 = rb0 + args.up_off;
+        } else {
+          rb0 = e * args.b_rows + n * BN;
+          rb1 = rb0 + 128;
+        }
+        for (int kb = 0; kb < nkb; ++kb, ++issued) {
+          const int s = (int)(issued % STAGES);
+          const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
+          int got = 1;
+          if (lane == 0) got = ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty);
+          if (!__shfl_sync(0xffffffffu, got, 0)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + s * kStage, sb = sa + kTileA;
+          if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(full0 + s * 8, kStage);
+            ptx::tma_load_2d(sb, &tmB, kb * BK, rb0, full0 + s * 8);
+            ptx::tma_load_2d(sb + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
+          }
+          __syncwarp();
+          ptx::tma_gather4(sa + lane * 512, &tmA, kb * BK, src_row[0], src_row[1], src_row[2],
+                           src_row[3], full0 + s * 8);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) gg::drain_loads<STAGES>(full0, issued, args.status);
+    } else if (lane == 0) {
       int64_t issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
@@ -194,7 +237,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = args.offsets[e] + m * BM + rl;
       const bool valid = row >= 0 && row < args.offsets[e + 1] && row < args.M_total;
       const int row_c = min(max(row, 0), args.M_total - 1);
-      const float* sa_p = args.a_scales + (int64_t)row_c * nkb;
+      int srow = row_c;
+      if (GATHER) {
+        srow = args.a_rows[row_c];
+        if ((unsigned)srow >= (unsigned)args.a_src_rows) srow = 0;  // such rows are not stored
+      }
+      const float* sa_p = args.a_scales + (int64_t)srow * nkb;
       // B scale rows (128-row blocks of this expert's B) for this thread's columns
       int nb0, nb1;
       if (SWIGLU) {
@@ -313,9 +361,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace gg8
 
-cudaError_t launch_grouped_gemm_fp8(const void* A, const float* a_scales, const void* B,
-                                    const float* b_scales, const int32_t* offsets, int M_total,
-                                    int E, int N, int K, bool swiglu, void* Cout, float* c_scales,
+// A_rows != nullptr: routed row r of A (and of a_scales) is row A_rows[r] of
+// A [A_src_rows, K] (and of a_scales [A_src_rows, K/128]).
+cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_src_rows,
+                                    const float* a_scales, const void* B, const float* b_scales,
+                                    const int32_t* offsets, int M_total, int E, int N, int K,
+                                    bool swiglu, void* Cout, float* c_scales,
                                     int /*max_rows_per_expert*/, int32_t* status, cudaStream_t s,
                                     const char** why) {
   const int b_rows = swiglu ? 2 * N : N;
@@ -324,7 +375,9 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const float* a_scales, const 
     return cudaErrorInvalidValue;
   }
   CUtensorMap tmA, tmB;
-  if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M_total, 128) ||
+  // a gathered A is read by tile::gather4 from a map whose box is one row high
+  if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, A_rows ? A_src_rows : M_total,
+                 A_rows ? 1 : 128) ||
       !make_tmap(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (int64_t)E * b_rows, 128)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
@@ -339,6 +392,9 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const float* a_scales, const 
   a.up_off = swiglu ? N : 0;
   a.band = 8;
   a.M_total = M_total;
+  a.a_rows = A_rows;
+  a.a_src = A;
+  a.a_src_rows = A_src_rows;
   a.kblocks = K / 128;
   a.b_nblk = b_rows / 128;
   a.C = Cout;
@@ -348,16 +404,20 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const float* a_scales, const 
   a.status = status;
   const int64_t tiles_ub = ((int64_t)M_total / gg8::BM + (M_total < E ? M_total : E)) * a.NT;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_ub));
-  cudaError_t e;
+#define MOE_FP8(SW, G)                                                                    \
+  do {                                                                                    \
+    cudaError_t e = set_smem(gg8::gemm_rows_fp8_kernel<SW, G>, gg8::kSmem);               \
+    if (e != cudaSuccess) return e;                                                       \
+    gg8::gemm_rows_fp8_kernel<SW, G><<<grid, gg8::kThreads, gg8::kSmem, s>>>(tmA, tmB, a); \
+  } while (0)
   if (swiglu) {
-    e = set_smem(gg8::gemm_rows_fp8_kernel<true>, gg8::kSmem);
-    if (e != cudaSuccess) return e;
-    gg8::gemm_rows_fp8_kernel<true><<<grid, gg8::kThreads, gg8::kSmem, s>>>(tmA, tmB, a);
+    if (A_rows) MOE_FP8(true, true);
+    else MOE_FP8(true, false);
   } else {
-    e = set_smem(gg8::gemm_rows_fp8_kernel<false>, gg8::kSmem);
-    if (e != cudaSuccess) return e;
-    gg8::gemm_rows_fp8_kernel<false><<<grid, gg8::kThreads, gg8::kSmem, s>>>(tmA, tmB, a);
+    if (A_rows) MOE_FP8(false, true);
+    else MOE_FP8(false, false);
   }
+#undef MOE_FP8
   note_launch();
   return cudaGetLastError();
 }

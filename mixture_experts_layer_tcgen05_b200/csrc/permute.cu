@@ -126,12 +126,13 @@ __global__ void __launch_bounds__(128) permute_scatter_kernel(
 }
 
 // ---- row gather: x_perm[p, :] = x[perm_token[p], :] --------------------------
-// one warp per row, 16-byte vectors
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+// one warp per row, 16-byte vectors (4-byte words for rows that are not a
+// multiple of 16 bytes, e.g. a few fp32 scales)
+template <typename V>
+__global__ void __launch_bounds__(256) gather_rows_kernel(const V* __restrict__ x,
                                                           const int32_t* __restrict__ perm_token,
                                                           int R, int T, int vec_per_row,
-                                                          uint4* __restrict__ x_perm,
-                                                          int32_t* status) {
+                                                          V* __restrict__ x_perm, int32_t* status) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= R) return;
   const int t = perm_token[row];
@@ -139,8 +140,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
     if (lane == 0) record_bad_index(status);
     return;
   }
-  const uint4* src = x + (int64_t)t * vec_per_row;
-  uint4* dst = x_perm + (int64_t)row * vec_per_row;
+  const V* src = x + (int64_t)t * vec_per_row;
+  V* dst = x_perm + (int64_t)row * vec_per_row;
   for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
 }
 
@@ -217,9 +218,14 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* off
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, int T,
                                int row_bytes, void* x_perm, int32_t* status, cudaStream_t s) {
-  gather_rows_kernel<<<(unsigned)ceil_div(R, 8), 256, 0, s>>>(
-      static_cast<const uint4*>(x), perm_token, R, T, row_bytes / 16,
-      static_cast<uint4*>(x_perm), status);
+  if (row_bytes % 16 == 0)
+    gather_rows_kernel<uint4><<<(unsigned)ceil_div(R, 8), 256, 0, s>>>(
+        static_cast<const uint4*>(x), perm_token, R, T, row_bytes / 16,
+        static_cast<uint4*>(x_perm), status);
+  else
+    gather_rows_kernel<uint32_t><<<(unsigned)ceil_div(R, 8), 256, 0, s>>>(
+        static_cast<const uint32_t*>(x), perm_token, R, T, row_bytes / 4,
+        static_cast<uint32_t*>(x_perm), status);
   note_launch();
   return cudaGetLastError();
 }

@@ -12,7 +12,7 @@
 // function of the inputs. The work is register-tiled on CUDA cores (each
 // thread owns TT tokens x TE experts); tensor cores are not used here because
 // their internal accumulation order is not specified.
-#include "common.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -214,122 +214,99 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (my_slot >= 0) w[(int64_t)warp * k + my_slot] = __fdiv_rn(my_ex, denom);
 }
 
-// Narrow router (E <= 32): one thread per (token, expert), so the T*E
-// sequential sums run side by side across the whole GPU. Chunks of 128 h
-// values of x and Wr are staged in shared memory as fp32 (Wr transposed, one
-// padded row per expert) in two buffers; global loads run two chunks ahead
-// through two register sets, so their latency hides behind the FMA chain.
-constexpr int kNarrowKC = 128;
-constexpr int kNarrowPad = 4;  // floats of padding per expert row (bank spread)
+// Narrow router (E <= 32). Thread = (token t, pair of experts): two
+// independent sequential sums per thread. These kernels are latency-bound
+// (a handful of tokens per SM), so nothing global sits on the critical path:
+// the whole of Wr (bf16, expert pairs padded) is loaded into shared memory
+// once, and the token rows stream through an NS-deep ring of cp.async
+// copies, so each chunk of x landed long before its sums need it.
+constexpr int kNarrowKC = 64;  // h per x chunk
+constexpr int kNarrowNS = 8;   // x chunks in flight
 
-template <int EB>
-struct NarrowStage {
-  static constexpr int BT = 256 / EB;
-  static constexpr int XV = BT * kNarrowKC / 8;         // 16-byte x vectors per chunk
-  static constexpr int XPT = (XV + 255) / 256;          // ... per thread
-  static constexpr int WV = kNarrowKC * EB / 256;       // w values per thread
-  uint4 x[XPT];
-  uint16_t w[WV];
-};
-
-template <int EB>
-__global__ void __launch_bounds__(256, 1) router_narrow_kernel(const __nv_bfloat16* __restrict__ x,
-                                                            const __nv_bfloat16* __restrict__ wr,
-                                                            const float* __restrict__ bias, int T,
-                                                            int H, int E,
-                                                            float* __restrict__ logits) {
-  using S = NarrowStage<EB>;
-  constexpr int BT = S::BT;
-  constexpr int WROW = kNarrowKC + kNarrowPad;
-  static_assert(S::XPT >= 1 && S::WV >= 1, "staging covers the chunk");
-  __shared__ __align__(16) float xs[2][BT][kNarrowKC];
-  __shared__ __align__(16) float wt[2][EB][WROW];
+template <int EPP>  // expert pairs per token, padded to a power of two (1..16)
+__global__ void __launch_bounds__(64) router_narrow_kernel(const __nv_bfloat16* __restrict__ x,
+                                                           const __nv_bfloat16* __restrict__ wr,
+                                                           const float* __restrict__ bias, int T,
+                                                           int H, int E,
+                                                           float* __restrict__ logits) {
+  constexpr int BT = 64 / EPP;                    // tokens per block
+  constexpr int XROW = kNarrowKC * 2;             // bytes of one token's chunk
+  constexpr int XSTAGE = BT * XROW;               // bytes of one ring stage
+  extern __shared__ __align__(16) unsigned char narrow_smem[];
+  unsigned char* xring = narrow_smem;                                    // [NS][BT][KC] bf16
+  uint32_t* wsm = reinterpret_cast<uint32_t*>(narrow_smem + kNarrowNS * XSTAGE);  // [H][EPP] bf16 pairs
   const int tid = threadIdx.x;
-  const int tl = tid / EB, el = tid % EB;
+  const int ep = tid % EPP, tl = tid / EPP;
   const int t0 = blockIdx.x * BT;
-  const uint16_t* xg = reinterpret_cast<const uint16_t*>(x);
+  const int nchunks = H / kNarrowKC;
+  const char* xg = reinterpret_cast<const char*>(x);
   const uint16_t* wg = reinterpret_cast<const uint16_t*>(wr);
 
-  auto load = [&](S& r, int k0) {
-#pragma unroll
-    for (int i = 0; i < S::XPT; ++i) {
-      const int v = tid + i * 256, t = v / (kNarrowKC / 8), c8 = (v % (kNarrowKC / 8)) * 8;
-      if (v >= S::XV) break;
-      r.x[i] = (t0 + t < T) ? *reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + t) * H + k0 + c8)
-                            : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int i = 0; i < S::WV; ++i) {
-      const int idx = tid + i * 256, h = idx / EB, e = idx % EB;
-      r.w[i] = (e < E) ? wg[(int64_t)(k0 + h) * E + e] : (uint16_t)0;
-    }
-  };
-  auto store = [&](const S& r, int b) {
-#pragma unroll
-    for (int i = 0; i < S::XPT; ++i) {
-      const int v = tid + i * 256, t = v / (kNarrowKC / 8), c8 = (v % (kNarrowKC / 8)) * 8;
-      if (v >= S::XV) break;
-      float4* d = reinterpret_cast<float4*>(&xs[b][t][c8]);
-      const uint4 u = r.x[i];
-      d[0] = make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
-      d[1] = make_float4(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w));
-    }
-#pragma unroll
-    for (int i = 0; i < S::WV; ++i) {
-      const int idx = tid + i * 256, h = idx / EB, e = idx % EB;
-      wt[b][e][h] = __uint_as_float((uint32_t)r.w[i] << 16);
-    }
-  };
-  float acc = 0.0f;
-  // The chain is latency-bound (one fma per h). Operands move from shared
-  // memory to registers 16 h at a time, one group ahead of the fmas that use
-  // them, so the chain never waits on a shared load.
-  auto compute = [&](int b) {
-    const float4* xp = reinterpret_cast<const float4*>(&xs[b][tl][0]);
-    const float4* wp = reinterpret_cast<const float4*>(&wt[b][el][0]);
-    float4 xa[4], wa[4], xn[4], wn[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) xa[j] = xp[j], wa[j] = wp[j];
-#pragma unroll
-    for (int g = 0; g < kNarrowKC / 16; ++g) {
-      if (g + 1 < kNarrowKC / 16) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) xn[j] = xp[4 * (g + 1) + j], wn[j] = wp[4 * (g + 1) + j];
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc = __fmaf_rn(xa[j].x, wa[j].x, acc);
-        acc = __fmaf_rn(xa[j].y, wa[j].y, acc);
-        acc = __fmaf_rn(xa[j].z, wa[j].z, acc);
-        acc = __fmaf_rn(xa[j].w, wa[j].w, acc);
-      }
-      if (g + 1 < kNarrowKC / 16) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) xa[j] = xn[j], wa[j] = wn[j];
+  // x chunk c -> ring stage c % NS: BT rows x 128 B = BT*8 copies of 16 B
+  auto issue = [&](int c) {
+    if (c < nchunks) {
+      const uint32_t st = ptx::smem_addr(xring + (c % kNarrowNS) * XSTAGE);
+      for (int i = tid; i < BT * (XROW / 16); i += 64) {
+        const int r = i / (XROW / 16), v = i % (XROW / 16);
+        const int t = t0 + r;
+        const char* src = xg + ((int64_t)(t < T ? t : 0) * H + (int64_t)c * kNarrowKC) * 2 + v * 16;
+        ptx::cp_async16(st + r * XROW + v * 16, src, t < T ? 16u : 0u);
       }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  const int n = H / kNarrowKC;
-  S ra, rb;
-  load(ra, 0);
-  if (n > 1) load(rb, kNarrowKC);
-  store(ra, 0);
-  __syncthreads();
-  // chunk c lives in buffer c & 1; chunk c+1 waits in a register set; chunk
-  // c+2 is requested before chunk c is summed.
-  for (int c = 0; c < n; c += 2) {
-    if (c + 2 < n) load(ra, (c + 2) * kNarrowKC);
-    compute(0);
-    if (c + 1 < n) store(rb, 1);
-    __syncthreads();
-    if (c + 1 >= n) break;
-    if (c + 3 < n) load(rb, (c + 3) * kNarrowKC);
-    compute(1);
-    if (c + 2 < n) store(ra, 0);
-    __syncthreads();
+#pragma unroll
+  for (int c = 0; c < kNarrowNS - 1; ++c) issue(c);
+  // Wr -> shared memory, once: pair p of row h = (Wr[h, 2p], Wr[h, 2p+1]).
+  // When the padded layout equals Wr's own (E = 2 * EPP, rows of 16-byte
+  // multiples) it is one stream of asynchronous 16-byte copies.
+  if (E == 2 * EPP && (E * 2) % 16 == 0) {
+    const uint32_t wdst = ptx::smem_addr(wsm);
+    const char* wsrc = reinterpret_cast<const char*>(wr);
+    for (int i = tid; i < H * E * 2 / 16; i += 64) ptx::cp_async16(wdst + i * 16, wsrc + i * 16, 16u);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else {
+    for (int i = tid; i < H * EPP; i += 64) {
+      const int h = i / EPP, p = i % EPP, e = 2 * p;
+      const uint32_t lo = e < E ? wg[(int64_t)h * E + e] : 0u;
+      const uint32_t hi = e + 1 < E ? wg[(int64_t)h * E + e + 1] : 0u;
+      wsm[i] = lo | (hi << 16);
+    }
   }
+  float a0 = 0.0f, a1 = 0.0f;
+  for (int c = 0; c < nchunks; ++c) {
+    issue(c + kNarrowNS - 1);
+    asm volatile("cp.async.wait_group %0;" ::"n"(kNarrowNS - 1) : "memory");
+    __syncthreads();  // chunk c (and, the first time, Wr) visible to all threads
+    const uint4* xs = reinterpret_cast<const uint4*>(xring + (c % kNarrowNS) * XSTAGE + tl * XROW);
+    const uint32_t* wc = wsm + (int64_t)c * kNarrowKC * EPP + ep;
+#pragma unroll
+    for (int v = 0; v < kNarrowKC / 8; ++v) {
+      const uint4 u = xs[v];
+      const float xf[8] = {bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y),
+                           bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w)};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t w2 = wc[(v * 8 + j) * EPP];
+        a0 = __fmaf_rn(xf[j], bf16lo_to_f32(w2), a0);
+        a1 = __fmaf_rn(xf[j], bf16hi_to_f32(w2), a1);
+      }
+    }
+    __syncthreads();  // stage c % NS is refilled by the next iteration's issue
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   const int t = t0 + tl;
-  if (t < T && el < E) logits[(int64_t)t * E + el] = __fadd_rn(acc, bias ? bias[el] : 0.0f);
+  if (t < T) {
+    const int e = 2 * ep;
+    if (e < E) logits[(int64_t)t * E + e] = __fadd_rn(a0, bias ? bias[e] : 0.0f);
+    if (e + 1 < E) logits[(int64_t)t * E + e + 1] = __fadd_rn(a1, bias ? bias[e + 1] : 0.0f);
+  }
+}
+
+template <int EPP>
+size_t narrow_smem_bytes(int H) {
+  return (size_t)kNarrowNS * (64 / EPP) * kNarrowKC * 2 + (size_t)H * EPP * 4;
 }
 
 cudaError_t launch_router_logits(const void* x, const void* wr, const float* bias, int T, int H,
@@ -337,15 +314,29 @@ cudaError_t launch_router_logits(const void* x, const void* wr, const float* bia
   const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
   const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(wr);
   if (E <= 32) {
-#define MOE_NARROW(EBV)                                                                        \
-  router_narrow_kernel<EBV><<<(unsigned)ceil_div(T, 256 / EBV), 256, 0, s>>>(xp, wp, bias, T, H, \
-                                                                            E, logits)
-    if (E <= 8) MOE_NARROW(8);
-    else if (E <= 16) MOE_NARROW(16);
-    else MOE_NARROW(32);
+    const int ep = (E + 1) / 2;
+    const int epp = ep <= 1 ? 1 : ep <= 2 ? 2 : ep <= 4 ? 4 : ep <= 8 ? 8 : 16;
+    // the whole of Wr must fit in shared memory next to the x ring
+    const size_t need = epp == 1 ? narrow_smem_bytes<1>(H) : epp == 2 ? narrow_smem_bytes<2>(H)
+                        : epp == 4 ? narrow_smem_bytes<4>(H) : epp == 8 ? narrow_smem_bytes<8>(H)
+                        : narrow_smem_bytes<16>(H);
+    if (need <= 200 * 1024) {
+#define MOE_NARROW(EPPV)                                                                       \
+  do {                                                                                         \
+    cudaFuncSetAttribute(router_narrow_kernel<EPPV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                         (int)need);                                                           \
+    router_narrow_kernel<EPPV><<<(unsigned)ceil_div(T, 64 / EPPV), 64, need, s>>>(xp, wp, bias, T, \
+                                                                                 H, E, logits);   \
+  } while (0)
+      if (epp == 1) MOE_NARROW(1);
+      else if (epp == 2) MOE_NARROW(2);
+      else if (epp == 4) MOE_NARROW(4);
+      else if (epp == 8) MOE_NARROW(8);
+      else MOE_NARROW(16);
 #undef MOE_NARROW
-    note_launch();
-    return cudaGetLastError();
+      note_launch();
+      return cudaGetLastError();
+    }
   }
   const size_t smem = 2 * (size_t)kWideKC * (64 + 256) * 4;
   dim3 grid((unsigned)ceil_div(T, 64), (unsigned)ceil_div(E, 256));

@@ -164,3 +164,33 @@ def test_fp8_layer_small(kw):
 def test_fp8_layer_full_size_sampled():
     cfg, L = layer_host("fine_grained_fp8")
     check_fp8_layer(cfg, L)
+
+
+def test_fp8_grouped_gemm_row_gather():
+    """FP8 GEMM-1 fetching its routed rows (and their activation scales) by index."""
+    counts, N, K, Tsrc = [0, 3, 200, 129], 256, 384, 61
+    E = len(counts)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    M = int(offsets[-1])
+    X = mi.normal_bf16(0, 75, 1.0, 1, Tsrc, K).reshape(Tsrc, K)
+    xq, xs = oracle.quant_act_fp8(X)
+    rows = np.random.default_rng(3).integers(0, Tsrc, size=M).astype(np.int32)
+    B = mi.normal_bf16(0, 76, 0.05, E, 2 * N, K).reshape(E, 2 * N, K)
+    bq, bs = oracle.quant_weight_fp8(B)
+    C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    moe.moe_grouped_gemm(dev_u8(xq), dev_u8(bq), dev(offsets), M, E, N, K, moe.MOE_DTYPE_FP8_E4M3,
+                         moe.MOE_EPILOGUE_SWIGLU, C, dev(xs), dev(bs), None, ws=ws,
+                         a_rows=dev(rows), a_src_rows=Tsrc)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    dec = _dec_table()
+    A = (dec[xq] * np.repeat(xs, 128, 1))[rows]
+    Bd = dec[bq] * np.repeat(np.repeat(bs, 128, 1), 128, 2)
+    got = mi.bf16_to_f32(host_bf16(C))
+    for e in range(E):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            g = A[lo:hi] @ Bd[e, :N].T
+            u = A[lo:hi] @ Bd[e, N:].T
+            check_close(got[lo:hi], g / (1 + np.exp(-g)) * u, (2e-2, 5e-3), f"expert {e}")

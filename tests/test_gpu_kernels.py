@@ -122,6 +122,9 @@ GEMM_CASES = [
     ([0, 1, 17, 64], 256, 256, 64),
     ([3, 0, 16], 128, 512, 16),
     ([31, 2, 32, 0, 9], 384, 256, 32),
+    # large experts: many m-tiles per expert, banded raster
+    ([1500, 0, 700], 256, 384, 0),
+    ([2048, 1, 255], 512, 256, 0),
 ]
 
 
@@ -174,3 +177,56 @@ def test_combine_exact_given_y():
     # against the definition in fp64: only the fp32 sum and one bf16 rounding differ
     exact = sum(w[:, j:j + 1].astype(np.float64) * yf[inv[:, j]] for j in range(k))
     check_close(got, exact, (2 ** -7, 2 ** -8), "combine")
+
+
+@pytest.mark.parametrize("counts,N,K", [([0, 1, 130, 300], 256, 384), ([700, 5], 128, 256),
+                                        ([129, 0, 257], 384, 128)])
+def test_grouped_gemm_swiglu_row_gather(counts, N, K):
+    """A's routed rows fetched by index from a source matrix inside the GEMM
+    (the permutation's gather fused into the producer); rows of the tail past
+    M_total and every other row must match the dense computation."""
+    E = len(counts)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    M = int(offsets[-1])
+    Tsrc = 97
+    X = mi.normal_bf16(0, 33, 1.0, 1, Tsrc, K).reshape(Tsrc, K)
+    rows = np.random.default_rng(9).integers(0, Tsrc, size=M).astype(np.int32)
+    B = mi.normal_bf16(0, 34, 0.05, E, 2 * N, K).reshape(E, 2 * N, K)
+    C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    moe.moe_grouped_gemm(dev_bf16(X), dev_bf16(B), dev(offsets), M, E, N, K, moe.MOE_DTYPE_BF16,
+                         moe.MOE_EPILOGUE_SWIGLU, C, ws=ws, a_rows=dev(rows), a_src_rows=Tsrc)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    got = mi.bf16_to_f32(host_bf16(C))
+    for e in range(E):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            ref = oracle.expert_swiglu_rows(X[rows[lo:hi]], B[e])
+            check_close(got[lo:hi], ref, BF16_TOL, f"expert {e}")
+
+
+@pytest.mark.parametrize("swiglu", [True, False])
+@pytest.mark.parametrize("counts,N,K,hint", [([3, 0, 16], 128, 4096, 16), ([31, 2, 32, 0, 9], 384, 2048, 32)])
+def test_small_m_split_k(swiglu, counts, N, K, hint):
+    """With workspace to spare, the small-M kernel splits K into ranges that
+    fill whole waves; the fp32 partials are summed in a fixed order."""
+    E, offsets, M, A, B = _grouped_problem(counts, (2 if swiglu else 1) * N, K, 51)
+    C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(64 << 20, dtype=torch.uint8, device="cuda")
+    args = (dev_bf16(A), dev_bf16(B), dev(offsets), M, E, N, K, moe.MOE_DTYPE_BF16,
+            moe.MOE_EPILOGUE_SWIGLU if swiglu else moe.MOE_EPILOGUE_NONE, C)
+    moe.moe_grouped_gemm(*args, max_rows_per_expert=hint, ws=ws)
+    torch.cuda.synchronize()
+    first = C.clone()
+    moe.moe_grouped_gemm(*args, max_rows_per_expert=hint, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(first, C)  # deterministic
+    assert moe.moe_get_device_status(ws) == 0
+    got = mi.bf16_to_f32(host_bf16(C))
+    for e in range(E):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            ref = (oracle.expert_swiglu_rows(A[lo:hi], B[e]) if swiglu
+                   else oracle.expert_down_rows(A[lo:hi], B[e]))
+            check_close(got[lo:hi], ref, BF16_TOL, f"expert {e}")
