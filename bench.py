@@ -299,26 +299,37 @@ def gpu_arm(args, cfg):
     value = whole_job_tokens_per_s(cfg.T, world, ms_per_step)
 
     # ---- end to end: pinned host tokens in, pinned host result out, every step ----
+    # Two streams with a workspace each: step i+1's host->device copy runs on
+    # the copy engine while step i computes (as a serving loop would overlap).
     x_host = torch.from_numpy(np.ascontiguousarray(L["x"]).view(np.int16)).pin_memory()
-    out_host = torch.empty(cfg.T * cfg.H, dtype=torch.int16).pin_memory()
-    x_dev = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    streams = [stream, torch.cuda.Stream()]
+    wss = [ws, torch.zeros_like(ws)]
+    outs_host = [torch.empty(cfg.T * cfg.H, dtype=torch.int16).pin_memory() for _ in range(2)]
+    outs_dev = [out, torch.empty_like(out)]
+    xs_dev = [torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
 
-    def e2e_step():
-        if cfg.fp8:
-            x_dev.view(torch.int16).copy_(x_host.view(cfg.T, cfg.H), non_blocking=True)
-            step(x_dev)
-            out_host.copy_(out.view(torch.int16).view(-1), non_blocking=True)
-        else:  # the C ABI's host-buffer entry point does both copies on the stream
-            moe.moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws)
+    def e2e_step(i):
+        j = i & 1
+        with torch.cuda.stream(streams[j]):
+            if cfg.fp8:
+                xs_dev[j].view(torch.int16).copy_(x_host.view(cfg.T, cfg.H), non_blocking=True)
+                moe.moe_forward_fp8(xs_dev[j], wr, bias, w13q, w13s, w2q, w2s, d, outs_dev[j], wss[j],
+                                    ws_bytes, stream=streams[j])
+                outs_host[j].copy_(outs_dev[j].view(torch.int16).view(-1), non_blocking=True)
+            else:  # the C ABI's host-buffer entry point does both copies on its stream
+                moe.moe_forward_hostio(x_host, wr, bias, w13, w2, d, outs_host[j], wss[j],
+                                       stream=streams[j])
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    streams[1].wait_stream(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    stream.wait_stream(streams[1])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
