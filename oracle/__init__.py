@@ -46,15 +46,16 @@ def _L():
             "oracle_router_logits": [vp, vp, vp, vp, i64, i64, i64, vp, i32],
             "oracle_topk": [vp, i64, i64, i32, vp, vp],
             "oracle_permute": [vp, i64, i64, i32, vp, vp, vp, vp],
-            "oracle_expert_swiglu_rows": [vp, i64, vp, i64, i64, vp],
+            "oracle_expert_gated_rows": [vp, i64, vp, i64, i64, i32, vp],
             "oracle_expert_down_rows": [vp, i64, vp, i64, i64, vp],
             "oracle_quant_act_fp8": [vp, i64, i64, vp, vp],
             "oracle_quant_weight_fp8": [vp, i64, i64, i64, vp, vp, i32],
-            "oracle_experts_combine": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, i32],
+            "oracle_experts_combine": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, i32, vp,
+                                       i32],
             "oracle_experts_combine_fp8": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp,
-                                           vp, i32],
+                                           i32, vp, i32],
             "oracle_moe_forward": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp,
-                                   vp, vp, vp, vp, i32],
+                                   i32, vp, vp, vp, vp, i32],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -116,14 +117,23 @@ def permute(ids, E):
     return offsets, perm_token, perm_slot, inv_perm.reshape(T, k)
 
 
-def expert_swiglu_rows(a_rows, w13e):
-    """silu(A Wg) * (A Wu) for bf16 rows A [n, H] and one expert's w13 [2I, H]."""
+# gated activations of the expert MLP (values of the C ABI's epilogue enum)
+ACT_SILU, ACT_GELU, ACT_RELU = 1, 2, 3
+
+
+def expert_gated_rows(a_rows, w13e, act=ACT_SILU):
+    """act(A Wg) * (A Wu) for bf16 rows A [n, H] and one expert's w13 [2I, H]."""
     a_rows, w13e = _c(a_rows, np.uint16), _c(w13e, np.uint16)
     n, H = a_rows.shape
     I = w13e.shape[0] // 2
     out = np.empty((n, I), dtype=np.float32)
-    _L().oracle_expert_swiglu_rows(_p(a_rows), n, _p(w13e), H, I, _p(out))
+    _L().oracle_expert_gated_rows(_p(a_rows), n, _p(w13e), H, I, int(act), _p(out))
     return out
+
+
+def expert_swiglu_rows(a_rows, w13e):
+    """silu(A Wg) * (A Wu) for bf16 rows A [n, H] and one expert's w13 [2I, H]."""
+    return expert_gated_rows(a_rows, w13e, ACT_SILU)
 
 
 def expert_down_rows(h_rows, w2e):
@@ -164,7 +174,7 @@ def quant_weight_fp8(w, nthreads=None):
     return q, s
 
 
-def experts_combine(x, tokens, ids, w, w13, w2, nthreads=None):
+def experts_combine(x, tokens, ids, w, w13, w2, nthreads=None, act=ACT_SILU):
     x, tokens = _c(x, np.uint16), _c(tokens, np.int32)
     ids, w = _c(ids, np.int32), _c(w, np.float32)
     w13, w2 = _c(w13, np.uint16), _c(w2, np.uint16)
@@ -172,11 +182,11 @@ def experts_combine(x, tokens, ids, w, w13, w2, nthreads=None):
     nt, k = ids.shape
     out = np.empty((nt, H), dtype=np.float32)
     _L().oracle_experts_combine(_p(x), _p(tokens), nt, H, I2 // 2, E, k, _p(ids), _p(w), _p(w13),
-                                _p(w2), _p(out), nthreads or threads())
+                                _p(w2), int(act), _p(out), nthreads or threads())
     return out
 
 
-def experts_combine_fp8(x, tokens, ids, w, w13q, w13s, w2q, w2s, nthreads=None):
+def experts_combine_fp8(x, tokens, ids, w, w13q, w13s, w2q, w2s, nthreads=None, act=ACT_SILU):
     x, tokens = _c(x, np.uint16), _c(tokens, np.int32)
     ids, w = _c(ids, np.int32), _c(w, np.float32)
     w13q, w2q = _c(w13q, np.uint8), _c(w2q, np.uint8)
@@ -185,12 +195,13 @@ def experts_combine_fp8(x, tokens, ids, w, w13q, w13s, w2q, w2s, nthreads=None):
     nt, k = ids.shape
     out = np.empty((nt, H), dtype=np.float32)
     _L().oracle_experts_combine_fp8(_p(x), _p(tokens), nt, H, I2 // 2, E, k, _p(ids), _p(w),
-                                    _p(w13q), _p(w13s), _p(w2q), _p(w2s), _p(out),
+                                    _p(w13q), _p(w13s), _p(w2q), _p(w2s), int(act), _p(out),
                                     nthreads or threads())
     return out
 
 
-def moe_forward(x, wr, bias, w13=None, w2=None, k=2, tokens=None, fp8=None, nthreads=None):
+def moe_forward(x, wr, bias, w13=None, w2=None, k=2, tokens=None, fp8=None, nthreads=None,
+                act=ACT_SILU):
     """The whole layer for ``tokens`` (all when None).
 
     ``fp8`` = (w13q, w13s, w2q, w2s) selects the FP8 experts (x is quantised
@@ -216,6 +227,6 @@ def moe_forward(x, wr, bias, w13=None, w2=None, k=2, tokens=None, fp8=None, nthr
     logits = np.empty((nt, E), dtype=np.float32)
     _L().oracle_moe_forward(_p(x), _p(tokens), nt, H, I, E, k, _p(wr), _p(b),
                             _p(w13) if fp8 is None else None, _p(w2) if fp8 is None else None,
-                            _p(w13q), _p(w13s), _p(w2q), _p(w2s), _p(out), _p(ids), _p(w),
-                            _p(logits), nthreads or threads())
+                            _p(w13q), _p(w13s), _p(w2q), _p(w2s), int(act), _p(out), _p(ids),
+                            _p(w), _p(logits), nthreads or threads())
     return {"out": out, "ids": ids, "w": w, "logits": logits}

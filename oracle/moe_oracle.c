@@ -193,11 +193,26 @@ void oracle_permute(const int32_t* ids, int64_t T, int64_t E, int k, int32_t* of
 /* expert is a gated MLP (gate and up projections, SwiGLU, down projection). */
 /* SiLU goes on the gate projection, the up projection stays linear:         */
 /*   g_i = sum_h x_h Wg[e,h,i],  u_i = sum_h x_h Wu[e,h,i]                   */
-/*   a_i = silu(g_i) * u_i,      silu(z) = z / (1 + exp(-z))                 */
+/*   a_i = act(g_i) * u_i,       act = silu by default:                       */
+/*                               silu(z) = z / (1 + exp(-z))                 */
+/* The same page lists experts with other gated activations (silu, gelu or   */
+/* relu: SwiGLU / GeGLU / ReGLU); act selects one:                           */
+/*   ACT_SILU  z / (1 + exp(-z))                                             */
+/*   ACT_GELU  z * Phi(z) = z/2 * (1 + erf(z / sqrt 2))   (the erf form, the */
+/*             one the toy layer's nn.GELU() denotes by default)             */
+/*   ACT_RELU  max(z, 0)                                                     */
 /*   y_c = sum_i a_i Wd[e,i,c]                                               */
 /* Weights arrive K-major: w13[e] = [Wg[e]^T ; Wu[e]^T] ([2I, H]) and        */
 /* w2[e] = Wd[e]^T ([H, I]).                                                 */
 /* ------------------------------------------------------------------------ */
+
+enum { ACT_SILU = 1, ACT_GELU = 2, ACT_RELU = 3 };
+
+static double gate_act(double z, int act) {
+  if (act == ACT_GELU) return 0.5 * z * (1.0 + erf(z / sqrt(2.0)));
+  if (act == ACT_RELU) return z > 0.0 ? z : 0.0;
+  return z / (1.0 + exp(-z));
+}
 
 /* Up to GROUP rows are evaluated side by side so the fp64 sums vectorise
  * across rows; every (row, output) sum still runs over its index ascending. */
@@ -205,7 +220,7 @@ void oracle_permute(const int32_t* ids, int64_t T, int64_t E, int k, int32_t* of
 
 /* a[n, I] (fp64) from fp64 activation rows xT[H][GROUP] (row r in column r) */
 static void expert_hidden(const double* xT, int64_t n, const uint16_t* w13e, const double* w13e_d,
-                          int64_t H, int64_t I, double* a) {
+                          int64_t H, int64_t I, int act, double* a) {
   for (int64_t i = 0; i < I; ++i) {
     double g[GROUP], u[GROUP];
     for (int r = 0; r < GROUP; ++r) g[r] = u[r] = 0.0;
@@ -224,7 +239,7 @@ static void expert_hidden(const double* xT, int64_t n, const uint16_t* w13e, con
         u[r] += xh[r] * wu;
       }
     }
-    for (int64_t r = 0; r < n; ++r) a[r * I + i] = g[r] / (1.0 + exp(-g[r])) * u[r];
+    for (int64_t r = 0; r < n; ++r) a[r * I + i] = gate_act(g[r], act) * u[r];
   }
 }
 
@@ -251,8 +266,8 @@ static void to_cols(const double* rows, int64_t n, int64_t C, double* T) {
 
 /* Exposed pieces, used by the tests to pin one GEMM stage at a time.
  * a_rows: [n, H] bf16 rows; out: [n, I] fp32 (each value rounded once). */
-void oracle_expert_swiglu_rows(const uint16_t* a_rows, int64_t n, const uint16_t* w13e, int64_t H,
-                               int64_t I, float* out) {
+void oracle_expert_gated_rows(const uint16_t* a_rows, int64_t n, const uint16_t* w13e, int64_t H,
+                              int64_t I, int act, float* out) {
   double* xr = (double*)malloc(sizeof(double) * (size_t)(GROUP * H));
   double* xT = (double*)malloc(sizeof(double) * (size_t)(GROUP * H));
   double* a = (double*)malloc(sizeof(double) * (size_t)(GROUP * I));
@@ -260,7 +275,7 @@ void oracle_expert_swiglu_rows(const uint16_t* a_rows, int64_t n, const uint16_t
     int64_t m = n - r0 < GROUP ? n - r0 : GROUP;
     for (int64_t i = 0; i < m * H; ++i) xr[i] = (double)bf16_widen(a_rows[r0 * H + i]);
     to_cols(xr, m, H, xT);
-    expert_hidden(xT, m, w13e, NULL, H, I, a);
+    expert_hidden(xT, m, w13e, NULL, H, I, act, a);
     for (int64_t i = 0; i < m * I; ++i) out[r0 * I + i] = (float)a[i];
   }
   free(xr);
@@ -406,6 +421,7 @@ typedef struct {
   const uint8_t *w13q, *w2q, *xq;
   const float *w13s, *w2s, *xs;
   int fp8;
+  int act; /* gated activation of the expert MLP */
   /* work list: items of up to CHUNK (row, slot) pairs of one expert */
   int64_t* item_e;
   int64_t* item_start; /* into pairs */
@@ -470,7 +486,7 @@ static void* fwd_worker(void* p) {
         }
       }
       to_cols(xr, n, H, xT);
-      expert_hidden(xT, n, w13e, w13d, H, I, a);
+      expert_hidden(xT, n, w13e, w13d, H, I, c->act, a);
       if (c->fp8) { /* the down projection's input is quantised per (row, 128-group) too */
         for (int64_t r = 0; r < n; ++r) {
           for (int64_t i = 0; i < I; ++i) af[i] = (float)a[r * I + i];
@@ -559,9 +575,11 @@ static void run_forward(fwd_ctx* c, const int32_t* ids, const float* topk_w, flo
  * out: [nt, H] fp32. */
 void oracle_experts_combine(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H,
                             int64_t I, int64_t E, int k, const int32_t* ids, const float* topk_w,
-                            const uint16_t* w13, const uint16_t* w2, float* out, int nthreads) {
+                            const uint16_t* w13, const uint16_t* w2, int act, float* out,
+                            int nthreads) {
   fwd_ctx c;
   memset(&c, 0, sizeof(c));
+  c.act = act;
   c.x = x;
   c.H = H;
   c.I = I;
@@ -579,7 +597,8 @@ void oracle_experts_combine(const uint16_t* x, const int32_t* tokens, int64_t nt
 void oracle_experts_combine_fp8(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H,
                                 int64_t I, int64_t E, int k, const int32_t* ids,
                                 const float* topk_w, const uint8_t* w13q, const float* w13s,
-                                const uint8_t* w2q, const float* w2s, float* out, int nthreads) {
+                                const uint8_t* w2q, const float* w2s, int act, float* out,
+                                int nthreads) {
   uint8_t* xq = (uint8_t*)malloc((size_t)(nt * H));
   float* xs = (float*)malloc(sizeof(float) * (size_t)(nt * (H / 128)));
   uint16_t* xrows = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)H);
@@ -603,6 +622,7 @@ void oracle_experts_combine_fp8(const uint16_t* x, const int32_t* tokens, int64_
   c.xq = xq;
   c.xs = xs;
   c.fp8 = 1;
+  c.act = act;
   run_forward(&c, ids, topk_w, out, nthreads);
   free(xq);
   free(xs);
@@ -614,18 +634,19 @@ void oracle_experts_combine_fp8(const uint16_t* x, const int32_t* tokens, int64_
 void oracle_moe_forward(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H, int64_t I,
                         int64_t E, int k, const uint16_t* wr, const float* bias,
                         const uint16_t* w13, const uint16_t* w2, const uint8_t* w13q,
-                        const float* w13s, const uint8_t* w2q, const float* w2s, float* out,
-                        int32_t* ids_out, float* w_out, float* logits_out, int nthreads) {
+                        const float* w13s, const uint8_t* w2q, const float* w2s, int act,
+                        float* out, int32_t* ids_out, float* w_out, float* logits_out,
+                        int nthreads) {
   float* logits = logits_out ? logits_out : (float*)malloc(sizeof(float) * (size_t)(nt * E));
   int32_t* ids = ids_out ? ids_out : (int32_t*)malloc(sizeof(int32_t) * (size_t)(nt * k));
   float* w = w_out ? w_out : (float*)malloc(sizeof(float) * (size_t)(nt * k));
   oracle_router_logits(x, wr, bias, tokens, nt, H, E, logits, nthreads);
   oracle_topk(logits, nt, E, k, ids, w);
   if (w13q)
-    oracle_experts_combine_fp8(x, tokens, nt, H, I, E, k, ids, w, w13q, w13s, w2q, w2s, out,
+    oracle_experts_combine_fp8(x, tokens, nt, H, I, E, k, ids, w, w13q, w13s, w2q, w2s, act, out,
                                nthreads);
   else
-    oracle_experts_combine(x, tokens, nt, H, I, E, k, ids, w, w13, w2, out, nthreads);
+    oracle_experts_combine(x, tokens, nt, H, I, E, k, ids, w, w13, w2, act, out, nthreads);
   if (!logits_out) free(logits);
   if (!ids_out) free(ids);
   if (!w_out) free(w);

@@ -191,7 +191,14 @@ def test_permute_is_stable_sort_by_expert(T, E, k):
 # --------------------------------------------------------------------------
 # experts + combine
 # --------------------------------------------------------------------------
-def _dense_masked(cfg, L, ids, w):
+_TORCH_ACT = {
+    oracle.ACT_SILU: torch.nn.functional.silu,
+    oracle.ACT_GELU: lambda z: torch.nn.functional.gelu(z, approximate="none"),
+    oracle.ACT_RELU: torch.nn.functional.relu,
+}
+
+
+def _dense_masked(cfg, L, ids, w, act=oracle.ACT_SILU):
     """Every expert on every token (fp64, logical weights), then masked by top-k."""
     wg, wu, wd = _logical_weights(cfg)
     x = mi.bf16_to_f32(L["x"]).astype(np.float64)
@@ -199,20 +206,21 @@ def _dense_masked(cfg, L, ids, w):
     for e in range(cfg.E):
         g = x @ wg[e]
         u = x @ wu[e]
-        y = (torch.nn.functional.silu(torch.from_numpy(g)).numpy() * u) @ wd[e]
+        y = (_TORCH_ACT[act](torch.from_numpy(g)).numpy() * u) @ wd[e]
         for j in range(cfg.k):
             m = ids[:, j] == e
             out[m] += w[m, j:j + 1].astype(np.float64) * y[m]
     return out
 
 
+@pytest.mark.parametrize("act", [oracle.ACT_SILU, oracle.ACT_GELU, oracle.ACT_RELU])
 @pytest.mark.parametrize("name,kw", [("tiny", {}), ("tiny", dict(T=19, E=5, k=3, H=64, I=96,
                                                                    bias="normal"))])
-def test_forward_matches_dense_masked_brute_force(name, kw):
+def test_forward_matches_dense_masked_brute_force(name, kw, act):
     cfg = _small(name, **kw)
     L = mi.make_layer(cfg)
-    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k)
-    ref = _dense_masked(cfg, L, r["ids"], r["w"])
+    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], L["w13"], L["w2"], k=cfg.k, act=act)
+    ref = _dense_masked(cfg, L, r["ids"], r["w"], act)
     np.testing.assert_allclose(r["out"], ref, rtol=1e-6, atol=1e-7 * np.abs(ref).max())
 
 
@@ -229,6 +237,37 @@ def test_one_hot_identical_experts_equal_one_dense_ffn():
     u = torch.nn.functional.linear(x, W13[cfg.I:])
     ref = torch.nn.functional.linear(torch.nn.functional.silu(g) * u, W2).numpy()
     np.testing.assert_allclose(r["out"], ref, rtol=1e-6, atol=1e-7 * np.abs(ref).max())
+
+
+def test_gated_activations_closed_forms():
+    """One token x = e_0 and gate weights g_i on channel 0, up weights 1: the
+    expert hidden row is act(g_i) exactly, against textbook values:
+    silu(z) = z sigma(z), gelu(z) = z Phi(z) with Phi the normal CDF
+    (Phi(1) = 0.8413447460685429, Phi(2) = 0.9772498680518208,
+    Phi(-0.5) = 0.3085375387259869), relu(z) = max(z, 0)."""
+    g = np.array([1.0, -1.0, 2.0, -0.5, 0.0], np.float32)
+    I, H = len(g), 16
+    a = np.zeros((1, H), np.float32)
+    a[0, 0] = 1.0
+    w13 = np.zeros((2 * I, H), np.float32)
+    w13[:I, 0] = g
+    w13[I:, 0] = 1.0
+    A, W = _bf16(a), _bf16(w13)
+    sig1 = 1.0 / (1.0 + np.exp(-1.0))
+    want = {
+        oracle.ACT_SILU: [sig1, -(1.0 - sig1), 2.0 / (1.0 + np.exp(-2.0)),
+                          -0.5 / (1.0 + np.exp(0.5)), 0.0],
+        oracle.ACT_GELU: [0.8413447460685429, -(1.0 - 0.8413447460685429), 2 * 0.9772498680518208,
+                          -0.5 * 0.3085375387259869, 0.0],
+        oracle.ACT_RELU: [1.0, 0.0, 2.0, 0.0, 0.0],
+    }
+    for act, ref in want.items():
+        got = oracle.expert_gated_rows(A, W, act)[0]
+        np.testing.assert_allclose(got, np.array(ref), rtol=1e-7, atol=1e-12, err_msg=str(act))
+    # swapping gate and up halves changes the answer (the activation is on the gate)
+    Wsw = np.concatenate([W[I:], W[:I]])
+    assert not np.allclose(oracle.expert_gated_rows(A, Wsw, oracle.ACT_GELU)[0],
+                           oracle.expert_gated_rows(A, W, oracle.ACT_GELU)[0])
 
 
 def test_identical_experts_k2_equal_one_dense_ffn():
