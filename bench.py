@@ -298,6 +298,35 @@ def gpu_arm(args, cfg):
     ms_per_step = ms / args.steps
     value = whole_job_tokens_per_s(cfg.T, world, ms_per_step)
 
+    # ---- the same forward replayed from a CUDA graph (launch overhead removed) ----
+    graph = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream()
+        cs.wait_stream(stream)
+        with torch.cuda.stream(cs):
+            step()  # warm the capture stream
+            cs.synchronize()
+            with torch.cuda.graph(g, stream=cs):
+                step()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        gms = max_over_ranks(g0.elapsed_time(g1), dist, "cuda") / args.steps
+        graph = {"ms_per_step": gms, "value": whole_job_tokens_per_s(cfg.T, world, gms),
+                 "unit": "tokens/s"}
+        del g
+    except Exception as exc:  # reported, not fatal: the eager number above stands
+        graph = {"error": str(exc)[:200]}
+
     # ---- end to end: pinned host tokens in, pinned host result out, every step ----
     # Two streams with a workspace each: step i+1's host->device copy runs on
     # the copy engine while step i computes (as a serving loop would overlap).
@@ -390,6 +419,7 @@ def gpu_arm(args, cfg):
                       zip(["route", "permute", "gemm1", "gemm2", "combine"], stage_ms)},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
                 "d2h_bytes_per_step": io_bytes},
+        "graph": graph,
         "gpu_launches": int(launches),
         "clocks": clk,
     }

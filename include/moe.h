@@ -63,7 +63,18 @@ typedef enum {
 
 typedef enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 } moe_dtype_t;
 
-typedef enum { MOE_EPILOGUE_NONE = 0, MOE_EPILOGUE_SWIGLU = 1 } moe_epilogue_t;
+/* GEMM epilogues. The gated ones compute act(g) * u from the gate projection
+ * g and the up projection u ([X] "Experts backends": experts with a gated
+ * activation -- silu, gelu or relu -- i.e. SwiGLU, GeGLU, ReGLU):
+ *   SWIGLU: silu(g) = g / (1 + e^-g)
+ *   GEGLU:  gelu(g) = g * Phi(g) = 0.5 g (1 + erf(g / sqrt 2))   (erf form)
+ *   REGLU:  relu(g) = max(g, 0) */
+typedef enum {
+  MOE_EPILOGUE_NONE = 0,
+  MOE_EPILOGUE_SWIGLU = 1,
+  MOE_EPILOGUE_GEGLU = 2,
+  MOE_EPILOGUE_REGLU = 3
+} moe_epilogue_t;
 
 typedef struct {
   int32_t T, H, I, E, k;
@@ -172,6 +183,7 @@ moe_status_t moe_permute_noalloc(const int32_t* ids_dev, moe_dims_t d, int32_t* 
  *   NONE:   C[m, n] = sum_k A[m, k] B[e, n, k]                  n < N
  *   SWIGLU: g = A B[e, 0:N]^T, u = A B[e, N:2N]^T, C = silu(g) * u,
  *           silu(z) = z / (1 + e^-z)   ([X] deepgemm_megamoe row)
+ *   GEGLU, REGLU: the same with gelu or relu in place of silu
  *   A_dev  [M_total, K] (bf16, or e4m3 with a_scales fp32 [M_total, K/128]);
  *          with a_rows_dev, routed row m is row a_rows_dev[m] of A_dev
  *          [a_src_rows, K] (and of a_scales [a_src_rows, K/128]) -- the
@@ -180,7 +192,7 @@ moe_status_t moe_permute_noalloc(const int32_t* ids_dev, moe_dims_t d, int32_t* 
  *          a_rows take the large-M kernel.
  *   B_dev  [E, N or 2N, K] K-major (bf16, or e4m3 with b_scales fp32
  *          [E, rows/128, K/128], one scale per 128 x 128 block, [F])
- *   C_dev  bf16 [M_total, N]; for FP8 SWIGLU with c_scales != NULL, C is
+ *   C_dev  bf16 [M_total, N]; for FP8 gated epilogues with c_scales != NULL, C is
  *          e4m3 [M_total, N] with c_scales fp32 [M_total, N/128] (each
  *          128-group scaled by amax/448, [F] activation groups)
  *   max_rows_per_expert: an upper bound on any expert's row count (0 =
@@ -217,6 +229,15 @@ moe_status_t moe_forward(const void* x_dev, const void* wr_dev, const float* bia
                          const void* w13_dev, const void* w2_dev, moe_dims_t d, void* out_dev,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* moe_forward with the expert activation chosen: act is MOE_EPILOGUE_SWIGLU
+ * (what moe_forward uses), MOE_EPILOGUE_GEGLU or MOE_EPILOGUE_REGLU ([X]
+ * "Experts backends": gated silu / gelu / relu experts). Anything else is
+ * MOE_ERR_INVALID_ARG. Other arguments as for moe_forward. */
+moe_status_t moe_forward_gated(const void* x_dev, const void* wr_dev, const float* bias_dev,
+                               const void* w13_dev, const void* w2_dev, moe_dims_t d,
+                               moe_epilogue_t act, void* out_dev, void* ws, size_t ws_bytes,
+                               void* stream);
+
 /* The whole layer with fine-grained FP8 experts ([F]; [X] "FP8 and FP4
  * quantized experts"): x is quantised per (token, 128-channel group) to e4m3
  * with scale amax/448, the SwiGLU output likewise per (row, 128-group of I),
@@ -229,6 +250,14 @@ moe_status_t moe_forward_fp8(const void* x_dev, const void* wr_dev, const float*
                              const void* w13q_dev, const float* w13s_dev, const void* w2q_dev,
                              const float* w2s_dev, moe_dims_t d, void* out_dev, void* ws,
                              size_t ws_bytes, void* stream);
+
+/* moe_forward_fp8 with the expert activation chosen (as moe_forward_gated;
+ * the activation's output is what gets quantised per 128-group). */
+moe_status_t moe_forward_fp8_gated(const void* x_dev, const void* wr_dev, const float* bias_dev,
+                                   const void* w13q_dev, const float* w13s_dev,
+                                   const void* w2q_dev, const float* w2s_dev, moe_dims_t d,
+                                   moe_epilogue_t act, void* out_dev, void* ws, size_t ws_bytes,
+                                   void* stream);
 
 /* moe_forward with the token rows in HOST memory: copies x_host ([T, H]
  * bf16) to the workspace, runs the layer, copies the result to out_host

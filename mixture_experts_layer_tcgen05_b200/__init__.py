@@ -21,6 +21,7 @@ __all__ = [
     "MoeError", "Dims", "WsLayout", "lib", "lib_path", "MOE_OK", "MOE_ERR_INVALID_ARG",
     "MOE_ERR_UNSUPPORTED_DEVICE", "MOE_ERR_WORKSPACE", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
     "MOE_DTYPE_BF16", "MOE_DTYPE_FP8_E4M3", "MOE_EPILOGUE_NONE", "MOE_EPILOGUE_SWIGLU",
+    "MOE_EPILOGUE_GEGLU", "MOE_EPILOGUE_REGLU", "moe_forward_gated", "moe_forward_fp8_gated",
     "moe_last_error", "moe_abi_version", "moe_launch_count", "moe_workspace_size",
     "moe_workspace_layout", "moe_route_topk", "moe_topk_from_logits", "moe_permute",
     "moe_permute_noalloc",
@@ -32,7 +33,7 @@ __all__ = [
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_DEVICE = 0, 1, 2
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 3, 4, 5
 MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3 = 0, 1
-MOE_EPILOGUE_NONE, MOE_EPILOGUE_SWIGLU = 0, 1
+MOE_EPILOGUE_NONE, MOE_EPILOGUE_SWIGLU, MOE_EPILOGUE_GEGLU, MOE_EPILOGUE_REGLU = 0, 1, 2, 3
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libmoe_b200.so")
@@ -73,6 +74,9 @@ _SIGS = {
     "moe_forward": (_i32, [_vp, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _sz, _vp]),
     "moe_forward_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _sz, _vp]),
     "moe_forward_hostio": (_i32, [_vp, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _sz, _vp]),
+    "moe_forward_gated": (_i32, [_vp, _vp, _vp, _vp, _vp, Dims, _i32, _vp, _vp, _sz, _vp]),
+    "moe_forward_fp8_gated": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _i32, _vp, _vp, _sz,
+                                     _vp]),
     "moe_quantize_act_fp8": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "moe_quantize_weight_fp8": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "moe_get_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
@@ -206,6 +210,18 @@ def moe_forward(x, wr, bias, w13, w2, d, out, ws, ws_bytes=None, stream=None):
 def moe_forward_fp8(x, wr, bias, w13q, w13s, w2q, w2s, d, out, ws, ws_bytes=None, stream=None):
     _check(lib().moe_forward_fp8(_p(x), _p(wr), _p(bias), _p(w13q), _p(w13s), _p(w2q), _p(w2s),
                                  _dims(d), _p(out), _p(ws), _nbytes(ws, ws_bytes), _s(stream)))
+
+
+def moe_forward_gated(x, wr, bias, w13, w2, d, act, out, ws, ws_bytes=None, stream=None):
+    _check(lib().moe_forward_gated(_p(x), _p(wr), _p(bias), _p(w13), _p(w2), _dims(d), int(act),
+                                   _p(out), _p(ws), _nbytes(ws, ws_bytes), _s(stream)))
+
+
+def moe_forward_fp8_gated(x, wr, bias, w13q, w13s, w2q, w2s, d, act, out, ws, ws_bytes=None,
+                          stream=None):
+    _check(lib().moe_forward_fp8_gated(_p(x), _p(wr), _p(bias), _p(w13q), _p(w13s), _p(w2q),
+                                       _p(w2s), _dims(d), int(act), _p(out), _p(ws),
+                                       _nbytes(ws, ws_bytes), _s(stream)))
 
 
 def moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws, ws_bytes=None, stream=None):

@@ -15,8 +15,8 @@
 namespace moe {
 
 // kernels (router.cu, permute.cu, gemm.cu, fp8.cu)
-cudaError_t launch_router_logits(const void* x, const void* wr, const float* bias, int T, int H,
-                                 int E, float* logits, cudaStream_t s);
+cudaError_t launch_route(const void* x, const void* wr, const float* bias, int T, int H, int E,
+                         int k, float* logits, int32_t* ids, float* w, cudaStream_t s);
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t s);
 int64_t permute_scratch_bytes(int T, int E);
@@ -29,13 +29,13 @@ cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* in
                            int H, int k, void* out, int32_t* status, cudaStream_t s);
 cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A_src_rows,
                                      const void* B, const int32_t* offsets, int M_total, int E,
-                                     int N, int K, bool swiglu, void* C,
+                                     int N, int K, int act, void* C,
                                      int max_rows_per_expert, int32_t* status, void* scratch,
                                      size_t scratch_bytes, cudaStream_t s, const char** why);
 cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_src_rows,
                                     const float* a_scales, const void* B, const float* b_scales,
                                     const int32_t* offsets, int M_total, int E, int N, int K,
-                                    bool swiglu, void* C, float* c_scales,
+                                    int act, void* C, float* c_scales,
                                     int max_rows_per_expert, int32_t* status, cudaStream_t s,
                                     const char** why);
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
@@ -243,10 +243,8 @@ moe_status_t moe_route_topk(const void* x, const void* wr, const float* bias, mo
   }
   MOE_TRY(check_device());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_router_logits(x, wr, bias, d.T, d.H, d.E, logits, s);
-  if (e != cudaSuccess) return cuda_fail(e, "router logits");
-  e = launch_topk(logits, d.T, d.E, d.k, ids, w, s);
-  if (e != cudaSuccess) return cuda_fail(e, "top-k");
+  cudaError_t e = launch_route(x, wr, bias, d.T, d.H, d.E, d.k, logits, ids, w, s);
+  if (e != cudaSuccess) return cuda_fail(e, "router");
   return ok();
 }
 
@@ -329,7 +327,7 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
   if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 1024]");
   if (N < 128 || N % 128 || K < 128 || K % 128)
     return fail(MOE_ERR_INVALID_ARG, "N and K must be positive multiples of 128 (N=%d K=%d)", N, K);
-  if (ep != MOE_EPILOGUE_NONE && ep != MOE_EPILOGUE_SWIGLU) return fail(MOE_ERR_INVALID_ARG, "bad epilogue");
+  if (ep < MOE_EPILOGUE_NONE || ep > MOE_EPILOGUE_REGLU) return fail(MOE_ERR_INVALID_ARG, "bad epilogue");
   if (dt != MOE_DTYPE_BF16 && dt != MOE_DTYPE_FP8_E4M3) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
   MOE_TRY(check_ptr(A, "A"));
   MOE_TRY(check_ptr(a_rows, "a_rows", true));
@@ -341,8 +339,8 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
     MOE_TRY(check_ptr(a_scales, "a_scales"));
     MOE_TRY(check_ptr(b_scales, "b_scales"));
     MOE_TRY(check_ptr(c_scales, "c_scales", true));
-    if (c_scales && ep != MOE_EPILOGUE_SWIGLU)
-      return fail(MOE_ERR_INVALID_ARG, "c_scales (quantised output) needs the SWIGLU epilogue");
+    if (c_scales && ep == MOE_EPILOGUE_NONE)
+      return fail(MOE_ERR_INVALID_ARG, "c_scales (quantised output) needs a gated epilogue");
   }
   MOE_TRY(check_ptr(ws, "ws"));
   if (ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes", ws_bytes);
@@ -351,13 +349,13 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
   cudaError_t e;
   if (dt == MOE_DTYPE_BF16)
     e = launch_grouped_gemm_bf16(A, a_rows, a_rows ? a_src_rows : M_total, B, offsets, M_total, E,
-                                 N, K, ep == MOE_EPILOGUE_SWIGLU, C,
+                                 N, K, (int)ep, C,
                                  max_rows_per_expert, at<int32_t>(ws, 0), at<char>(ws, 256),
                                  ws_bytes - 256, static_cast<cudaStream_t>(stream), &why);
   else
     e = launch_grouped_gemm_fp8(A, a_rows, a_rows ? a_src_rows : M_total, a_scales, B, b_scales,
                                 offsets, M_total, E, N, K,
-                                ep == MOE_EPILOGUE_SWIGLU, C, c_scales, max_rows_per_expert,
+                                (int)ep, C, c_scales, max_rows_per_expert,
                                 at<int32_t>(ws, 0), static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "grouped GEMM: %s %s", cudaGetErrorString(e), why);
   return ok();
@@ -381,7 +379,7 @@ moe_status_t moe_combine(const void* y_perm, const float* w, const int32_t* inv_
 
 static moe_status_t forward_impl(const void* x, const void* wr, const float* bias, const void* w13,
                                  const float* w13s, const void* w2, const float* w2s, moe_dims_t d,
-                                 void* out, void* ws, moe_dtype_t dt, cudaStream_t s) {
+                                 int act, void* out, void* ws, moe_dtype_t dt, cudaStream_t s) {
   const moe_ws_layout_t L = layout(d, dt);
   const int T = d.T, H = d.H, I = d.I, E = d.E, k = d.k, R = T * k;
   int32_t* status = at<int32_t>(ws, L.status);
@@ -395,9 +393,8 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
   const char* why = "";
   cudaError_t e;
   record(s, 0);
-  if ((e = launch_router_logits(x, wr, bias, T, H, E, logits, s)) != cudaSuccess)
-    return cuda_fail(e, "router logits");
-  if ((e = launch_topk(logits, T, E, k, ids, tw, s)) != cudaSuccess) return cuda_fail(e, "top-k");
+  if ((e = launch_route(x, wr, bias, T, H, E, k, logits, ids, tw, s)) != cudaSuccess)
+    return cuda_fail(e, "router");
   record(s, 1);
   if ((e = launch_permute(ids, T, E, k, offsets, perm_token, inv_perm, at<char>(ws, L.scratch),
                           status, s)) != cudaSuccess)
@@ -412,11 +409,11 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
     record(s, 2);
     void* splitk = L.splitk >= 0 ? at<void>(ws, L.splitk) : nullptr;
     const size_t splitk_bytes = L.splitk >= 0 ? (size_t)(L.y_perm - L.splitk) : 0;
-    if ((e = launch_grouped_gemm_bf16(x_perm, nullptr, R, w13, offsets, R, E, I, H, true, h, T,
+    if ((e = launch_grouped_gemm_bf16(x_perm, nullptr, R, w13, offsets, R, E, I, H, act, h, T,
                                       status, splitk, splitk_bytes, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "GEMM1: %s %s", cudaGetErrorString(e), why);
     record(s, 3);
-    if ((e = launch_grouped_gemm_bf16(h, nullptr, R, w2, offsets, R, E, H, I, false, y_perm, T,
+    if ((e = launch_grouped_gemm_bf16(h, nullptr, R, w2, offsets, R, E, H, I, 0, y_perm, T,
                                       status, splitk, splitk_bytes, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "GEMM2: %s %s", cudaGetErrorString(e), why);
     record(s, 4);
@@ -435,10 +432,10 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
       return cuda_fail(e, "gather");
     record(s, 2);
     if ((e = launch_grouped_gemm_fp8(xq_perm, nullptr, R, xs_perm, w13, w13s, offsets, R, E, I, H,
-                                     true, hq, hs, T, status, s, &why)) != cudaSuccess)
+                                     act, hq, hs, T, status, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "FP8 GEMM1: %s %s", cudaGetErrorString(e), why);
     record(s, 3);
-    if ((e = launch_grouped_gemm_fp8(hq, nullptr, R, hs, w2, w2s, offsets, R, E, H, I, false, y_perm,
+    if ((e = launch_grouped_gemm_fp8(hq, nullptr, R, hs, w2, w2s, offsets, R, E, H, I, 0, y_perm,
                                      nullptr, T, status, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "FP8 GEMM2: %s %s", cudaGetErrorString(e), why);
     record(s, 4);
@@ -449,10 +446,18 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
   return ok();
 }
 
-moe_status_t moe_forward(const void* x, const void* wr, const float* bias, const void* w13,
-                         const void* w2, moe_dims_t d, void* out, void* ws, size_t ws_bytes,
-                         void* stream) {
+static moe_status_t check_act(moe_epilogue_t act) {
+  if (act < MOE_EPILOGUE_SWIGLU || act > MOE_EPILOGUE_REGLU)
+    return fail(MOE_ERR_INVALID_ARG, "the expert activation must be SWIGLU, GEGLU or REGLU (got %d)",
+                (int)act);
+  return MOE_OK;
+}
+
+moe_status_t moe_forward_gated(const void* x, const void* wr, const float* bias, const void* w13,
+                               const void* w2, moe_dims_t d, moe_epilogue_t act, void* out, void* ws,
+                               size_t ws_bytes, void* stream) {
   MOE_TRY(check_dims(d, true));
+  MOE_TRY(check_act(act));
   MOE_TRY(check_ptr(x, "x"));
   MOE_TRY(check_ptr(wr, "w_router"));
   MOE_TRY(check_ptr(bias, "bias", true));
@@ -461,14 +466,22 @@ moe_status_t moe_forward(const void* x, const void* wr, const float* bias, const
   MOE_TRY(check_ptr(out, "out"));
   MOE_TRY(check_ws(d, MOE_DTYPE_BF16, ws, ws_bytes));
   MOE_TRY(check_device());
-  return forward_impl(x, wr, bias, w13, nullptr, w2, nullptr, d, out, ws, MOE_DTYPE_BF16,
+  return forward_impl(x, wr, bias, w13, nullptr, w2, nullptr, d, (int)act, out, ws, MOE_DTYPE_BF16,
                       static_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_forward_fp8(const void* x, const void* wr, const float* bias, const void* w13q,
-                             const float* w13s, const void* w2q, const float* w2s, moe_dims_t d,
-                             void* out, void* ws, size_t ws_bytes, void* stream) {
+moe_status_t moe_forward(const void* x, const void* wr, const float* bias, const void* w13,
+                         const void* w2, moe_dims_t d, void* out, void* ws, size_t ws_bytes,
+                         void* stream) {
+  return moe_forward_gated(x, wr, bias, w13, w2, d, MOE_EPILOGUE_SWIGLU, out, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_forward_fp8_gated(const void* x, const void* wr, const float* bias,
+                                   const void* w13q, const float* w13s, const void* w2q,
+                                   const float* w2s, moe_dims_t d, moe_epilogue_t act, void* out,
+                                   void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(check_dims(d, true));
+  MOE_TRY(check_act(act));
   MOE_TRY(check_ptr(x, "x"));
   MOE_TRY(check_ptr(wr, "w_router"));
   MOE_TRY(check_ptr(bias, "bias", true));
@@ -480,8 +493,15 @@ moe_status_t moe_forward_fp8(const void* x, const void* wr, const float* bias, c
   if (d.H % 256) return fail(MOE_ERR_INVALID_ARG, "the FP8 layer needs H %% 256 == 0 (got %d)", d.H);
   MOE_TRY(check_ws(d, MOE_DTYPE_FP8_E4M3, ws, ws_bytes));
   MOE_TRY(check_device());
-  return forward_impl(x, wr, bias, w13q, w13s, w2q, w2s, d, out, ws, MOE_DTYPE_FP8_E4M3,
+  return forward_impl(x, wr, bias, w13q, w13s, w2q, w2s, d, (int)act, out, ws, MOE_DTYPE_FP8_E4M3,
                       static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward_fp8(const void* x, const void* wr, const float* bias, const void* w13q,
+                             const float* w13s, const void* w2q, const float* w2s, moe_dims_t d,
+                             void* out, void* ws, size_t ws_bytes, void* stream) {
+  return moe_forward_fp8_gated(x, wr, bias, w13q, w13s, w2q, w2s, d, MOE_EPILOGUE_SWIGLU, out, ws,
+                               ws_bytes, stream);
 }
 
 moe_status_t moe_forward_hostio(const void* x_host, const void* wr, const float* bias,
@@ -503,7 +523,8 @@ moe_status_t moe_forward_hostio(const void* x_host, const void* wr, const float*
   void* out_dev = at<void>(ws, base + (int64_t)io_al);
   cudaError_t e = cudaMemcpyAsync(x_dev, x_host, io, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return cuda_fail(e, "copy x to device");
-  MOE_TRY(forward_impl(x_dev, wr, bias, w13, nullptr, w2, nullptr, d, out_dev, ws, MOE_DTYPE_BF16, s));
+  MOE_TRY(forward_impl(x_dev, wr, bias, w13, nullptr, w2, nullptr, d, MOE_EPILOGUE_SWIGLU, out_dev, ws,
+                       MOE_DTYPE_BF16, s));
   e = cudaMemcpyAsync(out_host, out_dev, io, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return cuda_fail(e, "copy out to host");
   return ok();

@@ -43,6 +43,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr int64_t align_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 
+// Gated expert activations: the GEMM-1 epilogue computes act(g) * u from the
+// gate projection g and the up projection u ("Experts backends": experts with
+// a gated activation, silu / gelu / relu, i.e. SwiGLU / GeGLU / ReGLU).
+enum Act : int { kActNone = 0, kActSilu = 1, kActGelu = 2, kActRelu = 3 };
+
+template <int ACT>
+__device__ __forceinline__ float gated(float g, float u) {
+  if constexpr (ACT == kActSilu) {
+    return __fdividef(g, 1.0f + __expf(-g)) * u;  // g * sigmoid(g)
+  } else if constexpr (ACT == kActGelu) {
+    return 0.5f * g * (1.0f + erff(g * 0.7071067811865476f)) * u;  // g * Phi(g), erf form
+  } else {
+    return fmaxf(g, 0.0f) * u;
+  }
+}
+
 // Launch bookkeeping (defined in capi.cu).
 void note_launch();
 

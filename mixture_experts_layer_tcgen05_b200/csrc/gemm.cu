@@ -34,7 +34,7 @@ namespace gg {
 // ==========================================================================
 // tokens-in-M kernel
 // ==========================================================================
-template <bool SWIGLU, int BN>
+template <int ACT, int BN>
 struct RowsCfg {
   static constexpr int kTileB = BN * BK * 2;
   static constexpr int kStage = kTileA + kTileB;
@@ -44,13 +44,15 @@ struct RowsCfg {
   static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4;
 };
 
+// ACT: gated activation of the epilogue (kActNone: plain GEMM).
 // GATHER: A rows are copied by index (args.a_rows) from args.a_src by the
 // whole producer warp instead of being loaded from a permuted copy by TMA.
-template <bool SWIGLU, int BN, bool GATHER>
+template <int ACT, int BN, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_rows_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, Args args) {
-  using C = RowsCfg<SWIGLU, BN>;
+  using C = RowsCfg<ACT, BN>;
+  constexpr bool SWIGLU = ACT != kActNone;
   constexpr int STAGES = C::STAGES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -234,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_wait_ld();
           float h[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) h[i] = silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i]));
+          for (int i = 0; i < 32; ++i) h[i] = gated<ACT>(__uint_as_float(g[i]), __uint_as_float(u[i]));
           if (valid) store_row32(dst + c, h);
         }
       } else {
@@ -268,8 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ==========================================================================
 // small-M (swap-AB) kernel: weights in M, tokens in N
 // ==========================================================================
-template <bool SWIGLU, int BNT>
+template <int ACT, int BNT>
 struct SwapCfg {
+  static constexpr bool SWIGLU = ACT != kActNone;
   static constexpr int kNA = SWIGLU ? 2 : 1;                 // weight tiles per stage
   static constexpr int kTileB = BNT * BK * 2;
   static constexpr int kStage = kNA * kTileA + kTileB;       // multiple of 1024
@@ -283,11 +286,12 @@ struct SwapCfg {
 
 // tmA: weights [E*b_rows, K]; tmB: activation rows [M_total, K].
 // Tile = (expert e, token tile tt, weight tile n); order: e, tt, n.
-template <bool SWIGLU, int BNT>
+template <int ACT, int BNT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_swap_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, Args args) {
-  using C = SwapCfg<SWIGLU, BNT>;
+  using C = SwapCfg<ACT, BNT>;
+  constexpr bool SWIGLU = ACT != kActNone;
   constexpr int STAGES = C::STAGES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -425,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             if (c + i < nrows && row0 + c + i >= 0) {
-              float v = SWIGLU ? silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i]))
+              float v = SWIGLU ? gated<ACT>(__uint_as_float(g[i]), __uint_as_float(u[i]))
                                : __uint_as_float(g[i]);
               args.C[(int64_t)(row0 + c + i) * args.ldc + col] = __float2bfloat16_rn(v);
             }
@@ -460,12 +464,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Sum of the ksplit fp32 partials of each output in split order, then the
 // epilogue the unsplit kernel would have applied (SwiGLU or none), to bf16.
-template <bool SWIGLU>
+template <int ACT>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial,
                                                             int S, int M, int N,
                                                             __nv_bfloat16* __restrict__ C) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (int64_t)M * N) return;
+  constexpr bool SWIGLU = ACT != kActNone;
   const int64_t r = i / N, c = i % N;
   const int pld = (SWIGLU ? 2 : 1) * N;
   const int64_t slice = (int64_t)M * pld;
@@ -474,7 +479,7 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
     g += partial[s * slice + r * pld + c];
     if (SWIGLU) u += partial[s * slice + r * pld + N + c];
   }
-  C[i] = __float2bfloat16_rn(SWIGLU ? silu_mul(g, u) : g);
+  C[i] = __float2bfloat16_rn(SWIGLU ? gated<ACT>(g, u) : g);
 }
 
 }  // namespace gg
@@ -487,9 +492,10 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
 // scratch (may be null): room for the small-M kernel's split-K partials.
 cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A_src_rows,
                                      const void* B, const int32_t* offsets, int M_total, int E,
-                                     int N, int K, bool swiglu, void* Cout,
+                                     int N, int K, int act, void* Cout,
                                      int max_rows_per_expert, int32_t* status, void* scratch,
                                      size_t scratch_bytes, cudaStream_t s, const char** why) {
+  const bool swiglu = act != kActNone;
   const int b_rows = swiglu ? 2 * N : N;
   CUtensorMap tmA, tmB;
   gg::Args a;
@@ -551,25 +557,28 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A
     if (e != cudaSuccess) return e;                                                      \
     k<<<grid, gg::kThreads, gg::SwapCfg<SW, BNT>::kSmem, s>>>(tmA, tmB, a);              \
   } while (0)
-    if (swiglu) {
-      if (bnt == 16) MOE_SWAP(true, 16);
-      else if (bnt == 32) MOE_SWAP(true, 32);
-      else MOE_SWAP(true, 64);
-    } else {
-      if (bnt == 16) MOE_SWAP(false, 16);
-      else if (bnt == 32) MOE_SWAP(false, 32);
-      else MOE_SWAP(false, 64);
-    }
+#define MOE_SWAP_ACT(ACTV)               \
+  do {                                   \
+    if (bnt == 16) MOE_SWAP(ACTV, 16);   \
+    else if (bnt == 32) MOE_SWAP(ACTV, 32); \
+    else MOE_SWAP(ACTV, 64);             \
+  } while (0)
+    if (act == kActSilu) MOE_SWAP_ACT(kActSilu);
+    else if (act == kActGelu) MOE_SWAP_ACT(kActGelu);
+    else if (act == kActRelu) MOE_SWAP_ACT(kActRelu);
+    else MOE_SWAP_ACT(kActNone);
+#undef MOE_SWAP_ACT
 #undef MOE_SWAP
     note_launch();
     if (a.ksplit > 1) {
       const int64_t n = (int64_t)M_total * N;
-      if (swiglu)
-        gg::splitk_reduce_kernel<true><<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(
-            a.partial, a.ksplit, M_total, N, a.C);
-      else
-        gg::splitk_reduce_kernel<false><<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(
-            a.partial, a.ksplit, M_total, N, a.C);
+#define MOE_REDUCE(ACTV) \
+  gg::splitk_reduce_kernel<ACTV><<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(a.partial, a.ksplit, M_total, N, a.C)
+      if (act == kActSilu) MOE_REDUCE(kActSilu);
+      else if (act == kActGelu) MOE_REDUCE(kActGelu);
+      else if (act == kActRelu) MOE_REDUCE(kActRelu);
+      else MOE_REDUCE(kActNone);
+#undef MOE_REDUCE
       note_launch();
     }
     return cudaGetLastError();
@@ -592,12 +601,16 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A
     if (e != cudaSuccess) return e;                                                      \
     k<<<grid, gg::kThreads, gg::RowsCfg<SW, BNV>::kSmem, s>>>(tmA, tmB, a);              \
   } while (0)
-  if (swiglu)
-    MOE_ROWS(true, 256);
+  if (act == kActSilu)
+    MOE_ROWS(kActSilu, 256);
+  else if (act == kActGelu)
+    MOE_ROWS(kActGelu, 256);
+  else if (act == kActRelu)
+    MOE_ROWS(kActRelu, 256);
   else if (BN == 256)
-    MOE_ROWS(false, 256);
+    MOE_ROWS(kActNone, 256);
   else
-    MOE_ROWS(false, 128);
+    MOE_ROWS(kActNone, 128);
 #undef MOE_ROWS
   note_launch();
   return cudaGetLastError();

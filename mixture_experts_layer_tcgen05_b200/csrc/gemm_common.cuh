@@ -73,10 +73,6 @@ __device__ __forceinline__ int find_expert(const int32_t* tile_start, int E, int
 }
 
 // ------------------------------------------------------------------ utils
-__device__ __forceinline__ float silu_mul(float g, float u) {
-  return __fdividef(g, 1.0f + __expf(-g)) * u;
-}
-
 __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float (&v)[32]) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll

@@ -51,20 +51,18 @@ struct Args {
   int32_t* status;
 };
 
-__device__ __forceinline__ float silu_mul(float g, float u) {
-  return __fdividef(g, 1.0f + __expf(-g)) * u;
-}
-
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
   uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
   return lo | (hi << 16);
 }
 
-template <bool SWIGLU, bool GATHER>
+// ACT: gated activation of the epilogue (kActNone: plain GEMM).
+template <int ACT, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_rows_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, Args args) {
+  constexpr bool SWIGLU = ACT != kActNone;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -302,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float amax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          h[i] = silu_mul(acc[i], acc[64 + i]);
+          h[i] = gated<ACT>(acc[i], acc[64 + i]);
           amax = fmaxf(amax, fabsf(h[i]));
         }
         if (args.c_scales) {
@@ -366,9 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_src_rows,
                                     const float* a_scales, const void* B, const float* b_scales,
                                     const int32_t* offsets, int M_total, int E, int N, int K,
-                                    bool swiglu, void* Cout, float* c_scales,
+                                    int act, void* Cout, float* c_scales,
                                     int /*max_rows_per_expert*/, int32_t* status, cudaStream_t s,
                                     const char** why) {
+  const bool swiglu = act != kActNone;
   const int b_rows = swiglu ? 2 * N : N;
   if (!swiglu && N % 256 != 0) {
     *why = "FP8 GEMM without SwiGLU needs N % 256 == 0";
@@ -410,13 +409,16 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_
     if (e != cudaSuccess) return e;                                                       \
     gg8::gemm_rows_fp8_kernel<SW, G><<<grid, gg8::kThreads, gg8::kSmem, s>>>(tmA, tmB, a); \
   } while (0)
-  if (swiglu) {
-    if (A_rows) MOE_FP8(true, true);
-    else MOE_FP8(true, false);
-  } else {
-    if (A_rows) MOE_FP8(false, true);
-    else MOE_FP8(false, false);
-  }
+#define MOE_FP8_ACT(ACTV)           \
+  do {                              \
+    if (A_rows) MOE_FP8(ACTV, true); \
+    else MOE_FP8(ACTV, false);      \
+  } while (0)
+  if (act == kActSilu) MOE_FP8_ACT(kActSilu);
+  else if (act == kActGelu) MOE_FP8_ACT(kActGelu);
+  else if (act == kActRelu) MOE_FP8_ACT(kActRelu);
+  else MOE_FP8_ACT(kActNone);
+#undef MOE_FP8_ACT
 #undef MOE_FP8
   note_launch();
   return cudaGetLastError();

@@ -12,6 +12,7 @@
 // function of the inputs. The work is register-tiled on CUDA cores (each
 // thread owns TT tokens x TE experts); tensor cores are not used here because
 // their internal accumulation order is not specified.
+#include "gemm_common.cuh"  // num_sms
 #include "ptx.cuh"
 
 namespace moe {
@@ -218,120 +219,233 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (my_slot >= 0) w[(int64_t)warp * k + my_slot] = __fdiv_rn(my_ex, denom);
 }
 
-// Narrow router (E <= 32). One thread per (token, expert): one sequential
-// sum each, so a block of 64 threads covers 64/EP tokens (EP = E padded to a
-// power of two) and the T*E sums spread over as many warps as possible.
-// These kernels are latency-bound, so nothing global sits on the critical
-// path: the whole of Wr (bf16, [h][expert], rows padded to EP) is loaded into
-// shared memory once, and the token rows stream through an NS-deep ring of
-// cp.async copies, so each chunk of x landed long before its sums need it.
-constexpr int kNarrowKC = 64;  // h per x chunk
-constexpr int kNarrowNS = 8;   // x chunks in flight
+// Narrow router with fused top-k (E <= 32). One thread per (token, expert
+// pair): each thread carries two sums, one per expert of its pair, advanced
+// together by paired FMAs (__ffma2_rn), so a warp holds 32/EPP tokens and
+// every token's E logits sit in EPP neighbouring lanes (EPP = pairs, a power
+// of two). The sums are sequential chains over h, so their length H times
+// the FMA latency is the floor of this kernel, and the block is split so the
+// chains never wait on anything else:
+//  * CW compute warps run only the chains: per two h steps, two 16-byte
+//    shared loads and two paired FMAs;
+//  * twice as many helper warps stream x rows and Wr rows through an NS-deep ring
+//    of cp.async copies (raw bf16) and widen each chunk into fp32 "ready"
+//    buffers laid out for the compute loop: x as {x_h, x_h, x_h+1, x_h+1}
+//    per token, Wr as {w_h,e, w_h,e+1, w_h+1,e, w_h+1,e+1} per pair;
+//  * one block barrier per chunk of KC h values hands chunk c+1 from the
+//    helpers to the compute warps while they finish chunk c;
+//  * the top-k selection then runs on the logits still in registers: k rounds
+//    of a segmented warp argmax (logit desc, index asc) over the token's lanes.
+constexpr int kNarrowKC = 64;          // h per chunk
+constexpr int kNarrowNS = 8;           // raw chunks in flight
+constexpr int kNarrowXRow = 128 + 16;  // raw x row stride in shared memory (padded)
 
-template <int EP>  // experts per token, padded to a power of two (1..32)
-__global__ void __launch_bounds__(64) router_narrow_kernel(const __nv_bfloat16* __restrict__ x,
-                                                           const __nv_bfloat16* __restrict__ wr,
-                                                           const float* __restrict__ bias, int T,
-                                                           int H, int E,
-                                                           float* __restrict__ logits) {
-  constexpr int BT = 64 / EP;          // tokens per block
-  constexpr int XROW = kNarrowKC * 2;  // bytes of one token's chunk
-  constexpr int XSTAGE = BT * XROW;    // bytes of one ring stage
+template <int EPP>
+struct NarrowCfg {
+  static constexpr int CW = EPP >= 4 ? EPP / 4 : 1;  // compute warps
+  static constexpr int HW = 2 * CW;                   // helper warps
+  static constexpr int kThreads = 32 * (CW + HW);
+  static constexpr int BT = 32 * CW / EPP;            // tokens per block (8, 16 or 32)
+};
+
+__host__ __device__ constexpr size_t narrow_stage_bytes(int BT, int E) {
+  return (size_t)BT * kNarrowXRow + (size_t)kNarrowKC * E * 2;
+}
+__host__ __device__ constexpr size_t narrow_smem_bytes(int BT, int EPP, int E) {
+  return kNarrowNS * narrow_stage_bytes(BT, E) + 2 * (size_t)(kNarrowKC / 2) * 16 * (BT + EPP);
+}
+
+template <int EPP>  // expert pairs per token (power of two, 1..16)
+__global__ void __launch_bounds__(NarrowCfg<EPP>::kThreads) router_narrow_kernel(
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
+    const float* __restrict__ bias, int T, int H, int E, int k, float* __restrict__ logits,
+    int32_t* __restrict__ ids, float* __restrict__ topw) {
+  using Cfg = NarrowCfg<EPP>;
+  constexpr int KC = kNarrowKC, NS = kNarrowNS, XROW = kNarrowXRow, BT = Cfg::BT;
+  constexpr int NH = 32 * Cfg::HW;  // helper threads
+  constexpr int XV = BT * 8;        // 16-byte x vectors per chunk
+  constexpr int WI = (KC / 2) * EPP;  // Wr items (two h x one pair) per chunk
   extern __shared__ __align__(16) unsigned char narrow_smem[];
-  unsigned char* xring = narrow_smem;                                              // [NS][BT][KC] bf16
-  uint16_t* wsm = reinterpret_cast<uint16_t*>(narrow_smem + kNarrowNS * XSTAGE);  // [H][EP] bf16
   const int tid = threadIdx.x;
-  const int e = tid % EP, tl = tid / EP;
+  const bool helper = tid >= 32 * Cfg::CW;
+  const int hid = tid - 32 * Cfg::CW;  // helper thread index
+  const int p = tid % EPP, tl = tid / EPP;  // compute threads: (token, pair)
   const int t0 = blockIdx.x * BT;
-  const int nchunks = H / kNarrowKC;
+  const int nchunks = H / KC;
+  const size_t stage = narrow_stage_bytes(BT, E);
+  unsigned char* ring = narrow_smem;
+  float4* rx = reinterpret_cast<float4*>(narrow_smem + NS * stage);  // [2][KC/2][BT]
+  float4* rw = rx + 2 * (KC / 2) * BT;                                 // [2][KC/2][EPP]
   const char* xg = reinterpret_cast<const char*>(x);
-  const uint16_t* wg = reinterpret_cast<const uint16_t*>(wr);
+  const char* wg = reinterpret_cast<const char*>(wr);
 
-  // x chunk c -> ring stage c % NS: BT rows x 128 B, as 16-byte copies
+  // helpers: raw chunk c -> ring slot c % NS: BT x rows of 128 B, then KC Wr
+  // rows, which are one contiguous 128*E-byte range of Wr [H][E]
   auto issue = [&](int c) {
     if (c < nchunks) {
-      const uint32_t st = ptx::smem_addr(xring + (c % kNarrowNS) * XSTAGE);
-      for (int i = tid; i < BT * (XROW / 16); i += 64) {
-        const int r = i / (XROW / 16), v = i % (XROW / 16);
-        const int t = t0 + r;
-        const char* src = xg + ((int64_t)(t < T ? t : 0) * H + (int64_t)c * kNarrowKC) * 2 + v * 16;
-        ptx::cp_async16(st + r * XROW + v * 16, src, t < T ? 16u : 0u);
+      const uint32_t st = ptx::smem_addr(ring + (c % NS) * stage);
+#pragma unroll
+      for (int it = 0; it < (XV + NH - 1) / NH; ++it) {
+        const int i = hid + it * NH;
+        if (XV % NH == 0 || i < XV) {
+          const int r = i >> 3, v = i & 7, t = t0 + r;
+          const char* src = xg + ((int64_t)(t < T ? t : 0) * H + (int64_t)c * KC) * 2 + v * 16;
+          ptx::cp_async16(st + r * XROW + v * 16, src, t < T ? 16u : 0u);
+        }
       }
+      const char* wsrc = wg + (int64_t)c * KC * E * 2;
+      const uint32_t wdst = st + BT * XROW;
+      for (int i = hid; i < KC * E * 2 / 16; i += NH) ptx::cp_async16(wdst + i * 16, wsrc + i * 16, 16u);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
+  // helpers: widen raw chunk c into ready buffer c & 1
+  auto convert = [&](int c) {
+    const unsigned char* st = ring + (c % NS) * stage;
+    float4* dx = rx + (c & 1) * (KC / 2) * BT;
 #pragma unroll
-  for (int c = 0; c < kNarrowNS - 1; ++c) issue(c);
-  // Wr -> shared memory, once. When the padded layout equals Wr's own (E = EP,
-  // rows of 16-byte multiples) it is one stream of asynchronous copies.
-  if (E == EP && (E * 2) % 16 == 0) {
-    const uint32_t wdst = ptx::smem_addr(wsm);
-    const char* wsrc = reinterpret_cast<const char*>(wr);
-    for (int i = tid; i < H * E * 2 / 16; i += 64) ptx::cp_async16(wdst + i * 16, wsrc + i * 16, 16u);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_all;" ::: "memory");
-  } else {
-    for (int i = tid; i < H * EP; i += 64) {
-      const int h = i / EP, ee = i % EP;
-      wsm[i] = ee < E ? wg[(int64_t)h * E + ee] : (uint16_t)0;
+    for (int it = 0; it < (XV + NH - 1) / NH; ++it) {
+      const int i = hid + it * NH;
+      if (XV % NH == 0 || i < XV) {
+        const int r = i % BT, v = i / BT;
+        const uint4 u = *reinterpret_cast<const uint4*>(st + r * XROW + v * 16);
+        const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float lo = bf16lo_to_f32(q[j]), hi = bf16hi_to_f32(q[j]);
+          dx[(v * 4 + j) * BT + r] = make_float4(lo, lo, hi, hi);
+        }
+      }
     }
+    const unsigned char* sw = st + BT * XROW;  // Wr chunk [KC][E] bf16
+    float4* dw = rw + (c & 1) * (KC / 2) * EPP;
+#pragma unroll
+    for (int it = 0; it < (WI + NH - 1) / NH; ++it) {
+      const int i = hid + it * NH;
+      if (WI % NH == 0 || i < WI) {
+        const int j = i / EPP, pp = i % EPP, e0 = 2 * pp;
+        const int o0 = (2 * j) * E + e0, o1 = o0 + E;  // element offsets of rows 2j, 2j+1
+        uint32_t u0, u1;
+        if ((E & 1) == 0) {  // the pair is one aligned 32-bit word (zero past E)
+          u0 = e0 < E ? *reinterpret_cast<const uint32_t*>(sw + 2 * o0) : 0u;
+          u1 = e0 < E ? *reinterpret_cast<const uint32_t*>(sw + 2 * o1) : 0u;
+        } else {
+          const uint16_t* h16 = reinterpret_cast<const uint16_t*>(sw);
+          u0 = (e0 < E ? (uint32_t)h16[o0] : 0u) | (e0 + 1 < E ? (uint32_t)h16[o0 + 1] << 16 : 0u);
+          u1 = (e0 < E ? (uint32_t)h16[o1] : 0u) | (e0 + 1 < E ? (uint32_t)h16[o1 + 1] << 16 : 0u);
+        }
+        dw[i] = make_float4(bf16lo_to_f32(u0), bf16hi_to_f32(u0), bf16lo_to_f32(u1),
+                            bf16hi_to_f32(u1));
+      }
+    }
+  };
+
+  if (helper) {
+#pragma unroll 1
+    for (int c = 0; c < NS; ++c) issue(c);
+    asm volatile("cp.async.wait_group %0;" ::"n"(NS - 1) : "memory");
   }
-  float acc = 0.0f;
+  __syncthreads();
+  if (helper) convert(0);
+  float2 acc = make_float2(0.0f, 0.0f);  // compute threads: experts (2p, 2p+1) of token tl
+#pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
-    issue(c + kNarrowNS - 1);
-    asm volatile("cp.async.wait_group %0;" ::"n"(kNarrowNS - 1) : "memory");
-    __syncthreads();  // chunk c (and, the first time, Wr) visible to all threads
-    const uint4* xs = reinterpret_cast<const uint4*>(xring + (c % kNarrowNS) * XSTAGE + tl * XROW);
-    const uint16_t* wc = wsm + (int64_t)c * kNarrowKC * EP + e;
+    // helpers' copies of chunk c+1 landed; the barrier publishes them and the
+    // ready buffer of chunk c, and frees ring slot c % NS and buffer (c+1) & 1
+    if (helper) asm volatile("cp.async.wait_group %0;" ::"n"(NS - 2) : "memory");
+    __syncthreads();
+    if (helper) {
+      issue(c + NS);
+      if (c + 1 < nchunks) convert(c + 1);
+    } else {
+      const float4* xb = rx + (c & 1) * (KC / 2) * BT + tl;
+      const float4* wb = rw + (c & 1) * (KC / 2) * EPP + p;
 #pragma unroll
-    for (int v = 0; v < kNarrowKC / 8; ++v) {
-      const uint4 u = xs[v];
-      const float xf[8] = {bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y),
-                           bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w)};
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        acc = __fmaf_rn(xf[j], __uint_as_float((uint32_t)wc[(v * 8 + j) * EP] << 16), acc);
+      for (int j = 0; j < KC / 2; ++j) {
+        const float4 xv = xb[j * BT], wv = wb[j * EPP];
+        acc = __ffma2_rn(make_float2(xv.x, xv.y), make_float2(wv.x, wv.y), acc);
+        acc = __ffma2_rn(make_float2(xv.z, xv.w), make_float2(wv.z, wv.w), acc);
+      }
     }
-    __syncthreads();  // stage c % NS is refilled by the next iteration's issue
   }
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  const int t = t0 + tl;
-  if (t < T && e < E) logits[(int64_t)t * E + e] = __fadd_rn(acc, bias ? bias[e] : 0.0f);
+  if (helper) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    return;
+  }
+
+  const int t = t0 + tl, e0 = 2 * p, e1 = 2 * p + 1;
+  const float l0 = __fadd_rn(acc.x, bias ? bias[e0 < E ? e0 : 0] : 0.0f);
+  const float l1 = __fadd_rn(acc.y, bias ? bias[e1 < E ? e1 : 0] : 0.0f);
+  if (t < T && logits) {
+    if (e0 < E) logits[(int64_t)t * E + e0] = l0;
+    if (e1 < E) logits[(int64_t)t * E + e1] = l1;
+  }
+  // segmented top-k over the EPP lanes of this token (every lane of the warp
+  // takes part; the padding experts past E are never selectable)
+  bool take0 = e0 < E, take1 = e1 < E;  // still selectable
+  float lmax = 0.0f, denom = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+    if (take0) bv = l0, be = e0;
+    if (take1 && (l1 > bv || be == 0x7fffffff)) bv = l1, be = e1;
+#pragma unroll
+    for (int off = EPP / 2; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
+    }
+    if (be == e0) take0 = false;
+    if (be == e1) take1 = false;
+    if (j == 0) lmax = bv;
+    const float ex = expf(bv - lmax);
+    denom += ex;
+    if (t < T && p == j % EPP) {
+      ids[(int64_t)t * k + j] = be;
+      topw[(int64_t)t * k + j] = ex;  // normalised below by the same thread
+    }
+  }
+  if (t < T)
+    for (int j = p; j < k; j += EPP) {
+      const int64_t o = (int64_t)t * k + j;
+      topw[o] = __fdiv_rn(topw[o], denom);
+    }
 }
 
-template <int EP>
-size_t narrow_smem_bytes(int H) {
-  return (size_t)kNarrowNS * (64 / EP) * kNarrowKC * 2 + (size_t)H * EP * 2;
+// Pairs per token for the narrow router (E padded to a power of two >= 2).
+static int narrow_pairs(int E) {
+  const int ep = E <= 2 ? 2 : E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : 32;
+  return ep / 2;
 }
 
-cudaError_t launch_router_logits(const void* x, const void* wr, const float* bias, int T, int H,
-                                 int E, float* logits, cudaStream_t s) {
+cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                        cudaStream_t s);
+
+// Logits and top-k of T tokens: the fused narrow kernel for E <= 32, else the
+// wide logits kernel followed by the warp-per-token selection.
+cudaError_t launch_route(const void* x, const void* wr, const float* bias, int T, int H, int E,
+                         int k, float* logits, int32_t* ids, float* w, cudaStream_t s) {
   const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
   const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(wr);
   if (E <= 32) {
-    const int ep = E <= 1 ? 1 : E <= 2 ? 2 : E <= 4 ? 4 : E <= 8 ? 8 : E <= 16 ? 16 : 32;
-    // the whole of Wr must fit in shared memory next to the x ring
-    const size_t need = ep == 1 ? narrow_smem_bytes<1>(H) : ep == 2 ? narrow_smem_bytes<2>(H)
-                        : ep == 4 ? narrow_smem_bytes<4>(H) : ep == 8 ? narrow_smem_bytes<8>(H)
-                        : ep == 16 ? narrow_smem_bytes<16>(H) : narrow_smem_bytes<32>(H);
-    if (need <= 200 * 1024) {
-#define MOE_NARROW(EPV)                                                                        \
-  do {                                                                                         \
-    cudaFuncSetAttribute(router_narrow_kernel<EPV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                         (int)need);                                                           \
-    router_narrow_kernel<EPV><<<(unsigned)ceil_div(T, 64 / EPV), 64, need, s>>>(xp, wp, bias, T, H, \
-                                                                               E, logits);     \
+    const int epp = narrow_pairs(E);
+#define MOE_NARROW(P)                                                                         \
+  do {                                                                                        \
+    using Cfg = NarrowCfg<P>;                                                                 \
+    const size_t smem = narrow_smem_bytes(Cfg::BT, P, E);                                     \
+    cudaFuncSetAttribute(router_narrow_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                         (int)smem);                                                          \
+    router_narrow_kernel<P><<<(unsigned)ceil_div(T, Cfg::BT), Cfg::kThreads, smem, s>>>(      \
+        xp, wp, bias, T, H, E, k, logits, ids, w);                                            \
   } while (0)
-      if (ep == 1) MOE_NARROW(1);
-      else if (ep == 2) MOE_NARROW(2);
-      else if (ep == 4) MOE_NARROW(4);
-      else if (ep == 8) MOE_NARROW(8);
-      else if (ep == 16) MOE_NARROW(16);
-      else MOE_NARROW(32);
+    if (epp == 1) MOE_NARROW(1);
+    else if (epp == 2) MOE_NARROW(2);
+    else if (epp == 4) MOE_NARROW(4);
+    else if (epp == 8) MOE_NARROW(8);
+    else MOE_NARROW(16);
 #undef MOE_NARROW
-      note_launch();
-      return cudaGetLastError();
-    }
+    note_launch();
+    return cudaGetLastError();
   }
   const size_t smem = 2 * (size_t)kWideKC * (64 + 256) * 4;
   dim3 grid((unsigned)ceil_div(T, 64), (unsigned)ceil_div(E, 256));
@@ -343,7 +457,9 @@ cudaError_t launch_router_logits(const void* x, const void* wr, const float* bia
     router_wide_kernel<false><<<grid, 256, smem, s>>>(xp, wp, bias, T, H, E, logits);
   }
   note_launch();
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_topk(logits, T, E, k, ids, w, s);
 }
 
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,

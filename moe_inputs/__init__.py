@@ -156,6 +156,9 @@ CONFIGS = {
                                     subset=512, fp8=True,
                                     desc="fine-grained prefill, FP8 experts (128x128 weight "
                                          "blocks, 1x128 activation groups)"),
+    "mixtral_decode_fp8": LayerConfig("mixtral_decode_fp8", 16, 4096, 14336, 8, 2, fp8=True,
+                                      desc="Mixtral-shaped decode, FP8 experts: T=16 H=4096 "
+                                           "I=14336 E=8 k=2"),
 }
 
 

@@ -154,10 +154,17 @@ def check_fp8_layer(cfg, L):
 
 
 @pytest.mark.parametrize("kw", [dict(T=200, H=512, I=256, E=16, k=4, subset=0),
-                                dict(T=33, H=256, I=384, E=8, k=2, subset=0)])
+                                dict(T=33, H=256, I=384, E=8, k=2, subset=0),
+                                dict(T=16, H=1024, I=2048, E=8, k=2, bias="zero", subset=0)])
 def test_fp8_layer_small(kw):
     cfg = mi.CONFIGS["fine_grained_fp8"].with_(**kw)
     check_fp8_layer(cfg, mi.make_layer(cfg))
+
+
+@pytest.mark.slow
+def test_fp8_decode_full_size_all_tokens():
+    cfg, L = layer_host("mixtral_decode_fp8")
+    check_fp8_layer(cfg, L)
 
 
 @pytest.mark.slow

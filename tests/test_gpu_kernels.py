@@ -21,7 +21,8 @@ def _route(cfg, x, wr, b):
     logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
     ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
     w = torch.empty(T, k, dtype=torch.float32, device="cuda")
-    moe.moe_route_topk(dev_bf16(x), dev_bf16(wr), dev(b), (T, cfg.H, 128, E, k), logits, ids, w)
+    moe.moe_route_topk(dev_bf16(x), dev_bf16(wr), None if b is None else dev(b), (T, cfg.H, 128, E, k),
+                       logits, ids, w)
     torch.cuda.synchronize()
     return logits.cpu().numpy(), ids.cpu().numpy(), w.cpu().numpy()
 
@@ -36,6 +37,14 @@ ROUTER_CASES = [
     ("mixtral_decode", {}),
     ("mixtral_prefill", {}),
     ("fine_grained", dict(T=1024)),
+    # few experts: one fused logits + top-k kernel, every block shape and pair count
+    ("tiny", dict(T=37, E=2, k=2, bias="normal")),
+    ("tiny", dict(T=300, E=3, k=2)),
+    ("tiny", dict(T=129, E=7, k=3, bias="normal")),
+    ("tiny", dict(T=250, E=16, k=4)),
+    ("tiny", dict(T=70, E=32, k=16, bias="normal")),
+    ("tiny", dict(T=10000, E=8, k=2, H=256)),
+    ("tiny", dict(T=5000, E=24, k=6, H=128)),
 ]
 
 
@@ -48,6 +57,25 @@ def test_router_bit_exact(name, kw):
     ref_l = oracle.router_logits(x, wr, b)
     np.testing.assert_array_equal(logits.view(np.uint32), ref_l.view(np.uint32))
     ref_ids, ref_w = oracle.topk(ref_l, cfg.k)
+    np.testing.assert_array_equal(ids, ref_ids)
+    np.testing.assert_allclose(w, ref_w, rtol=0, atol=1e-6)
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (5, 5), (32, 16), (2, 1)])
+def test_router_exact_ties(E, k):
+    """Equal logits from duplicated router columns and all-zero tokens: the
+    lowest expert index wins every tie, in the fused small-E kernel too."""
+    cfg = mi.CONFIGS["tiny"].with_(T=90, E=E, k=k)
+    x = mi.make_x(cfg)
+    x[::4] = 0  # every logit of these tokens is exactly zero
+    wr, _ = mi.make_router(cfg)
+    wr[:, E - 1] = wr[:, 0]
+    if E > 3:
+        wr[:, 2] = wr[:, 1]
+    logits, ids, w = _route(cfg, x, wr, None)
+    ref_l = oracle.router_logits(x, wr, None)
+    np.testing.assert_array_equal(logits.view(np.uint32), ref_l.view(np.uint32))
+    ref_ids, ref_w = oracle.topk(ref_l, k)
     np.testing.assert_array_equal(ids, ref_ids)
     np.testing.assert_allclose(w, ref_w, rtol=0, atol=1e-6)
 
