@@ -122,7 +122,7 @@ def touched_weight_bytes(cfg, offsets, bytes_per_w=2.0):
 
 
 def kernel_traffic(cfg_name: str, kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's sources are unchanged."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -130,8 +130,10 @@ def kernel_traffic(cfg_name: str, kernel: str):
     ent = d.get(cfg_name, {}).get(kernel)
     if not ent:
         return None
-    src = open(os.path.join(ROOT, "mixture_experts_layer_tcgen05_b200", "csrc", ent["source"]), "rb").read()
-    if hashlib.sha256(src).hexdigest()[:16] != ent["source_sha"]:
+    h = hashlib.sha256()
+    for f in ent["sources"]:
+        h.update(open(os.path.join(ROOT, "mixture_experts_layer_tcgen05_b200", "csrc", f), "rb").read())
+    if h.hexdigest()[:16] != ent["source_sha"]:
         return None
     return ent["dram_bytes_per_launch"]
 

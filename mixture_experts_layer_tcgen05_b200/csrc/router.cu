@@ -240,12 +240,12 @@ constexpr int kNarrowKC = 64;          // h per chunk
 constexpr int kNarrowNS = 8;           // raw chunks in flight
 constexpr int kNarrowXRow = 128 + 16;  // raw x row stride in shared memory (padded)
 
-template <int EPP>
+template <int EPP, int TPT>
 struct NarrowCfg {
   static constexpr int CW = EPP >= 4 ? EPP / 4 : 1;  // compute warps
   static constexpr int HW = 2 * CW;                   // helper warps
   static constexpr int kThreads = 32 * (CW + HW);
-  static constexpr int BT = 32 * CW / EPP;            // tokens per block (8, 16 or 32)
+  static constexpr int BT = TPT * 32 * CW / EPP;      // tokens per block
 };
 
 __host__ __device__ constexpr size_t narrow_stage_bytes(int BT, int E) {
@@ -255,12 +255,45 @@ __host__ __device__ constexpr size_t narrow_smem_bytes(int BT, int EPP, int E) {
   return kNarrowNS * narrow_stage_bytes(BT, E) + 2 * (size_t)(kNarrowKC / 2) * 16 * (BT + EPP);
 }
 
-template <int EPP>  // expert pairs per token (power of two, 1..16)
-__global__ void __launch_bounds__(NarrowCfg<EPP>::kThreads) router_narrow_kernel(
+// Top-k of one token whose logits (l0, l1 for experts e0 = 2p, e1 = 2p + 1)
+// sit in the EPP lanes of its segment; every lane of the warp calls it.
+template <int EPP>
+__device__ __forceinline__ void segment_topk(float l0, float l1, int p, int E, int k, bool valid,
+                                             int32_t* __restrict__ ids, float* __restrict__ topw) {
+  const int e0 = 2 * p, e1 = 2 * p + 1;
+  bool take0 = e0 < E, take1 = e1 < E;  // still selectable (padding experts never are)
+  float lmax = 0.0f, denom = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+    if (take0) bv = l0, be = e0;
+    if (take1 && (l1 > bv || be == 0x7fffffff)) bv = l1, be = e1;
+#pragma unroll
+    for (int off = EPP / 2; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
+    }
+    if (be == e0) take0 = false;
+    if (be == e1) take1 = false;
+    if (j == 0) lmax = bv;
+    const float ex = expf(bv - lmax);
+    denom += ex;
+    if (valid && p == j % EPP) {
+      ids[j] = be;
+      topw[j] = ex;  // normalised below by the same thread
+    }
+  }
+  if (valid)
+    for (int j = p; j < k; j += EPP) topw[j] = __fdiv_rn(topw[j], denom);
+}
+
+template <int EPP, int TPT>  // expert pairs per token (power of two, 1..16); tokens per thread
+__global__ void __launch_bounds__(NarrowCfg<EPP, TPT>::kThreads) router_narrow_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
     const float* __restrict__ bias, int T, int H, int E, int k, float* __restrict__ logits,
     int32_t* __restrict__ ids, float* __restrict__ topw) {
-  using Cfg = NarrowCfg<EPP>;
+  using Cfg = NarrowCfg<EPP, TPT>;
   constexpr int KC = kNarrowKC, NS = kNarrowNS, XROW = kNarrowXRow, BT = Cfg::BT;
   constexpr int NH = 32 * Cfg::HW;  // helper threads
   constexpr int XV = BT * 8;        // 16-byte x vectors per chunk
@@ -269,7 +302,7 @@ __global__ void __launch_bounds__(NarrowCfg<EPP>::kThreads) router_narrow_kernel
   const int tid = threadIdx.x;
   const bool helper = tid >= 32 * Cfg::CW;
   const int hid = tid - 32 * Cfg::CW;  // helper thread index
-  const int p = tid % EPP, tl = tid / EPP;  // compute threads: (token, pair)
+  const int p = tid % EPP, tl = tid / EPP;  // compute threads: (tokens tl + i*BT/TPT, pair)
   const int t0 = blockIdx.x * BT;
   const int nchunks = H / KC;
   const size_t stage = narrow_stage_bytes(BT, E);
@@ -347,7 +380,10 @@ __global__ void __launch_bounds__(NarrowCfg<EPP>::kThreads) router_narrow_kernel
   }
   __syncthreads();
   if (helper) convert(0);
-  float2 acc = make_float2(0.0f, 0.0f);  // compute threads: experts (2p, 2p+1) of token tl
+  // compute threads: acc[i] = experts (2p, 2p+1) of token tl + i * BT/TPT
+  float2 acc[TPT];
+#pragma unroll
+  for (int i = 0; i < TPT; ++i) acc[i] = make_float2(0.0f, 0.0f);
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
     // helpers' copies of chunk c+1 landed; the barrier publishes them and the
@@ -360,11 +396,20 @@ __global__ void __launch_bounds__(NarrowCfg<EPP>::kThreads) router_narrow_kernel
     } else {
       const float4* xb = rx + (c & 1) * (KC / 2) * BT + tl;
       const float4* wb = rw + (c & 1) * (KC / 2) * EPP + p;
+      // TPT independent chains interleave, so a paired FMA rarely waits on its
+      // predecessor
 #pragma unroll
       for (int j = 0; j < KC / 2; ++j) {
-        const float4 xv = xb[j * BT], wv = wb[j * EPP];
-        acc = __ffma2_rn(make_float2(xv.x, xv.y), make_float2(wv.x, wv.y), acc);
-        acc = __ffma2_rn(make_float2(xv.z, xv.w), make_float2(wv.z, wv.w), acc);
+        const float4 wv = wb[j * EPP];
+        float4 xv[TPT];
+#pragma unroll
+        for (int i = 0; i < TPT; ++i) xv[i] = xb[j * BT + i * (BT / TPT)];
+#pragma unroll
+        for (int i = 0; i < TPT; ++i)
+          acc[i] = __ffma2_rn(make_float2(xv[i].x, xv[i].y), make_float2(wv.x, wv.y), acc[i]);
+#pragma unroll
+        for (int i = 0; i < TPT; ++i)
+          acc[i] = __ffma2_rn(make_float2(xv[i].z, xv[i].w), make_float2(wv.z, wv.w), acc[i]);
       }
     }
   }
@@ -373,43 +418,19 @@ __global__ void __launch_bounds__(NarrowCfg<EPP>::kThreads) router_narrow_kernel
     return;
   }
 
-  const int t = t0 + tl, e0 = 2 * p, e1 = 2 * p + 1;
-  const float l0 = __fadd_rn(acc.x, bias ? bias[e0 < E ? e0 : 0] : 0.0f);
-  const float l1 = __fadd_rn(acc.y, bias ? bias[e1 < E ? e1 : 0] : 0.0f);
-  if (t < T && logits) {
-    if (e0 < E) logits[(int64_t)t * E + e0] = l0;
-    if (e1 < E) logits[(int64_t)t * E + e1] = l1;
-  }
-  // segmented top-k over the EPP lanes of this token (every lane of the warp
-  // takes part; the padding experts past E are never selectable)
-  bool take0 = e0 < E, take1 = e1 < E;  // still selectable
-  float lmax = 0.0f, denom = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-    if (take0) bv = l0, be = e0;
-    if (take1 && (l1 > bv || be == 0x7fffffff)) bv = l1, be = e1;
+  const int e0 = 2 * p, e1 = 2 * p + 1;
+  const float b0 = bias ? bias[e0 < E ? e0 : 0] : 0.0f, b1 = bias ? bias[e1 < E ? e1 : 0] : 0.0f;
 #pragma unroll
-    for (int off = EPP / 2; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
+  for (int i = 0; i < TPT; ++i) {
+    const int t = t0 + tl + i * (BT / TPT);
+    const float l0 = __fadd_rn(acc[i].x, b0), l1 = __fadd_rn(acc[i].y, b1);
+    if (t < T && logits) {
+      if (e0 < E) logits[(int64_t)t * E + e0] = l0;
+      if (e1 < E) logits[(int64_t)t * E + e1] = l1;
     }
-    if (be == e0) take0 = false;
-    if (be == e1) take1 = false;
-    if (j == 0) lmax = bv;
-    const float ex = expf(bv - lmax);
-    denom += ex;
-    if (t < T && p == j % EPP) {
-      ids[(int64_t)t * k + j] = be;
-      topw[(int64_t)t * k + j] = ex;  // normalised below by the same thread
-    }
+    const int64_t o = (int64_t)(t < T ? t : 0) * k;
+    segment_topk<EPP>(l0, l1, p, E, k, t < T, ids + o, topw + o);
   }
-  if (t < T)
-    for (int j = p; j < k; j += EPP) {
-      const int64_t o = (int64_t)t * k + j;
-      topw[o] = __fdiv_rn(topw[o], denom);
-    }
 }
 
 // Pairs per token for the narrow router (E padded to a power of two >= 2).
@@ -429,13 +450,15 @@ cudaError_t launch_route(const void* x, const void* wr, const float* bias, int T
   const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(wr);
   if (E <= 32) {
     const int epp = narrow_pairs(E);
+    // one token per compute thread: two tokens per thread (TPT = 2) measured
+    // slower at the decode and prefill shapes
 #define MOE_NARROW(P)                                                                         \
   do {                                                                                        \
-    using Cfg = NarrowCfg<P>;                                                                 \
+    using Cfg = NarrowCfg<P, 1>;                                                              \
     const size_t smem = narrow_smem_bytes(Cfg::BT, P, E);                                     \
-    cudaFuncSetAttribute(router_narrow_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                         (int)smem);                                                          \
-    router_narrow_kernel<P><<<(unsigned)ceil_div(T, Cfg::BT), Cfg::kThreads, smem, s>>>(      \
+    cudaFuncSetAttribute(router_narrow_kernel<P, 1>,                                          \
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);             \
+    router_narrow_kernel<P, 1><<<(unsigned)ceil_div(T, Cfg::BT), Cfg::kThreads, smem, s>>>(   \
         xp, wp, bias, T, H, E, k, logits, ids, w);                                            \
   } while (0)
     if (epp == 1) MOE_NARROW(1);
