@@ -380,12 +380,14 @@ def gpu_arm(args, cfg):
     gemm1_ms = float(stage_ms[2])
     decode = cfg.T * cfg.k <= 64 * cfg.E and cfg.T <= 64
     if decode:
-        g1_bytes = n_exp * 2 * cfg.H * cfg.I * 2.0
+        # touched expert weights of GEMM-1 (e4m3 codes + one fp32 scale per 128 x 128 block)
+        g1_bytes = n_exp * 2 * cfg.H * cfg.I * ((1.0 + 4.0 / (128 * 128)) if cfg.fp8 else 2.0)
         ach = g1_bytes / (gemm1_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"],
                 "traffic": kernel_traffic(cfg.name, "gemm1"),
-                "kernel": "gemm_swap_kernel<SwiGLU> (GEMM1, small-M)",
+                "kernel": ("gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)"
+                           if cfg.fp8 else "gemm_swap_kernel<SwiGLU> (GEMM1, small-M)"),
                 "algorithmic_bytes_per_launch": g1_bytes, "peak_source": peak_src}
     else:
         g1_flops = 4.0 * cfg.T * cfg.k * cfg.H * cfg.I

@@ -37,6 +37,9 @@ ROUTER_CASES = [
     ("mixtral_decode", {}),
     ("mixtral_prefill", {}),
     ("fine_grained", dict(T=1024)),
+    # many experts: odd expert counts (scalar Wr loads), several passes per block
+    ("tiny", dict(T=333, E=300, k=8, H=128, bias="normal")),
+    ("tiny", dict(T=8192, E=1024, k=4, H=128)),
     # few experts: one fused logits + top-k kernel, every block shape and pair count
     ("tiny", dict(T=37, E=2, k=2, bias="normal")),
     ("tiny", dict(T=300, E=3, k=2)),
