@@ -25,6 +25,11 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* off
                            cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, int T,
                                int row_bytes, void* x_perm, int32_t* status, cudaStream_t s);
+cudaError_t launch_permute_gather_small(const int32_t* ids, int T, int E, int k, int32_t* offsets,
+                                        int32_t* perm_token, int32_t* inv_perm, const void* x,
+                                        int row_bytes, void* x_perm, const void* x2,
+                                        int row2_bytes, void* x2_perm, int32_t* status,
+                                        cudaStream_t s);
 cudaError_t launch_combine(const void* y_perm, const float* w, const int32_t* inv_perm, int T,
                            int H, int k, void* out, int32_t* status, cudaStream_t s);
 cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A_src_rows,
@@ -279,8 +284,14 @@ moe_status_t moe_permute(const int32_t* ids, moe_dims_t d, int32_t* offsets, int
   MOE_TRY(check_device());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   moe_ws_layout_t L = layout(d2, MOE_DTYPE_BF16);
-  cudaError_t e = launch_permute(ids, d.T, d.E, d.k, offsets, perm_token, inv_perm,
-                                 at<char>(ws, L.scratch), at<int32_t>(ws, L.status), s);
+  // decode-sized batches: one launch for the permutation and the gather
+  cudaError_t e = launch_permute_gather_small(ids, d.T, d.E, d.k, offsets, perm_token, inv_perm, x,
+                                              d.H * 2, x_perm, nullptr, 0, nullptr,
+                                              at<int32_t>(ws, L.status), s);
+  if (e == cudaSuccess) return ok();
+  if (e != cudaErrorNotSupported) return cuda_fail(e, "permute");
+  e = launch_permute(ids, d.T, d.E, d.k, offsets, perm_token, inv_perm,
+                     at<char>(ws, L.scratch), at<int32_t>(ws, L.status), s);
   if (e != cudaSuccess) return cuda_fail(e, "permute");
   if (x) {
     e = launch_gather_rows(x, perm_token, d.T * d.k, d.T, d.H * 2, x_perm,
@@ -396,16 +407,28 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
   if ((e = launch_route(x, wr, bias, T, H, E, k, logits, ids, tw, s)) != cudaSuccess)
     return cuda_fail(e, "router");
   record(s, 1);
-  if ((e = launch_permute(ids, T, E, k, offsets, perm_token, inv_perm, at<char>(ws, L.scratch),
-                          status, s)) != cudaSuccess)
-    return cuda_fail(e, "permute");
+  // The permuted copy of x feeds GEMM1's TMA tile loads (a gather inside the
+  // GEMM costs the tensor cores more than this copy costs). Decode-sized
+  // batches permute and gather in one launch; larger ones use the chunked
+  // permutation, then the gather.
+  auto permute_gather = [&](const void* a, int a_bytes, void* a_perm, const void* b, int b_bytes,
+                            void* b_perm) -> cudaError_t {
+    cudaError_t r = launch_permute_gather_small(ids, T, E, k, offsets, perm_token, inv_perm, a,
+                                                a_bytes, a_perm, b, b_bytes, b_perm, status, s);
+    if (r != cudaErrorNotSupported) return r;
+    if ((r = launch_permute(ids, T, E, k, offsets, perm_token, inv_perm, at<char>(ws, L.scratch),
+                            status, s)) != cudaSuccess)
+      return r;
+    if ((r = launch_gather_rows(a, perm_token, R, T, a_bytes, a_perm, status, s)) != cudaSuccess)
+      return r;
+    if (b) r = launch_gather_rows(b, perm_token, R, T, b_bytes, b_perm, status, s);
+    return r;
+  };
   if (dt == MOE_DTYPE_BF16) {
     void* x_perm = at<void>(ws, L.x_perm);
     void* h = at<void>(ws, L.h);
-    // The permuted copy of x feeds GEMM1's TMA tile loads (a gather inside the
-    // GEMM costs the tensor cores more than this copy costs).
-    if ((e = launch_gather_rows(x, perm_token, R, T, H * 2, x_perm, status, s)) != cudaSuccess)
-      return cuda_fail(e, "gather");
+    if ((e = permute_gather(x, H * 2, x_perm, nullptr, 0, nullptr)) != cudaSuccess)
+      return cuda_fail(e, "permute");
     record(s, 2);
     void* splitk = L.splitk >= 0 ? at<void>(ws, L.splitk) : nullptr;
     const size_t splitk_bytes = L.splitk >= 0 ? (size_t)(L.y_perm - L.splitk) : 0;
@@ -427,9 +450,8 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
     // x is quantised once per token, then its codes and scales are permuted
     if ((e = launch_quant_act(x, T, H, xq, xs, nullptr, s)) != cudaSuccess)
       return cuda_fail(e, "activation quantisation");
-    if ((e = launch_gather_rows(xq, perm_token, R, T, H, xq_perm, status, s)) != cudaSuccess ||
-        (e = launch_gather_rows(xs, perm_token, R, T, (H / 128) * 4, xs_perm, status, s)) != cudaSuccess)
-      return cuda_fail(e, "gather");
+    if ((e = permute_gather(xq, H, xq_perm, xs, (H / 128) * 4, xs_perm)) != cudaSuccess)
+      return cuda_fail(e, "permute");
     record(s, 2);
     if ((e = launch_grouped_gemm_fp8(xq_perm, nullptr, R, xs_perm, w13, w13s, offsets, R, E, I, H,
                                      act, hq, hs, T, status, s, &why)) != cudaSuccess)

@@ -255,9 +255,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
       bool ok = true;
+      // plain GEMM: scales are read two k-blocks ahead of their use (measured
+      // faster there; with SwiGLU the extra registers cost more than they save)
+      float pa[2], pb0[2];
+      if (!SWIGLU) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int kj = j < nkb ? j : 0;
+          pa[j] = sa_p[kj], pb0[j] = sb0[kj];
+        }
+      }
       for (int kb = 0; kb < nkb; ++kb, ++seq) {
-        const float sa = sa_p[kb];
-        const float s0 = sa * sb0[kb], s1 = sa * sb1[kb];
+        float s0, s1;
+        if (SWIGLU) {
+          const float sa = sa_p[kb];
+          s0 = sa * sb0[kb], s1 = sa * sb1[kb];
+        } else {
+          s0 = s1 = pa[kb & 1] * pb0[kb & 1];
+          if (kb + 2 < nkb) pa[kb & 1] = sa_p[kb + 2], pb0[kb & 1] = sb0[kb + 2];
+        }
         const int pb = (int)(seq & 1);
         const uint32_t pph = (uint32_t)((seq >> 1) & 1);
         if (!ptx::mbar_wait(pfull0 + pb * 8, pph, args.status, kSiteEpiAccFull)) {
@@ -281,13 +297,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
+          const float2 s0p = make_float2(s0, s0);
 #pragma unroll
           for (int c = 0; c < 128; c += 32) {
-            uint32_t v[32];
-            ptx::tmem_ld32(pbase + half * 128 + c, v);
+            uint32_t v0[16], v1[16];
+            ptx::tmem_ld16(pbase + half * 128 + c, v0);
+            ptx::tmem_ld16(pbase + half * 128 + c + 16, v1);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[c + i] = __fmaf_rn(__uint_as_float(v[i]), s0, acc[c + i]);
+            for (int i = 0; i < 16; i += 2) {  // paired FMAs: two IEEE fmas per instruction
+              float2 a = __ffma2_rn(make_float2(__uint_as_float(v0[i]), __uint_as_float(v0[i + 1])), s0p,
+                                    make_float2(acc[c + i], acc[c + i + 1]));
+              acc[c + i] = a.x, acc[c + i + 1] = a.y;
+              float2 b = __ffma2_rn(make_float2(__uint_as_float(v1[i]), __uint_as_float(v1[i + 1])), s0p,
+                                    make_float2(acc[c + 16 + i], acc[c + 17 + i]));
+              acc[c + 16 + i] = b.x, acc[c + 17 + i] = b.y;
+            }
           }
         }
         ptx::tc_fence_before();
@@ -313,20 +338,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           amax = fmaxf(rb[rl], rb[BM + rl]);
           const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+          // one IEEE reciprocal per group, then products: h * (1/s) differs from
+          // h / s by at most one fp32 ulp, which moves an e4m3 code only at a
+          // rounding midpoint
+          const float inv = __frcp_rn(sc);
           if (valid) {
             uint8_t* dst = static_cast<uint8_t*>(args.C) + (int64_t)row * args.ldc + n * 128 + half * 64;
             uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               uint4 o;
-              o.x = e4m3x4(__fdiv_rn(h[16 * v + 0], sc), __fdiv_rn(h[16 * v + 1], sc),
-                           __fdiv_rn(h[16 * v + 2], sc), __fdiv_rn(h[16 * v + 3], sc));
-              o.y = e4m3x4(__fdiv_rn(h[16 * v + 4], sc), __fdiv_rn(h[16 * v + 5], sc),
-                           __fdiv_rn(h[16 * v + 6], sc), __fdiv_rn(h[16 * v + 7], sc));
-              o.z = e4m3x4(__fdiv_rn(h[16 * v + 8], sc), __fdiv_rn(h[16 * v + 9], sc),
-                           __fdiv_rn(h[16 * v + 10], sc), __fdiv_rn(h[16 * v + 11], sc));
-              o.w = e4m3x4(__fdiv_rn(h[16 * v + 12], sc), __fdiv_rn(h[16 * v + 13], sc),
-                           __fdiv_rn(h[16 * v + 14], sc), __fdiv_rn(h[16 * v + 15], sc));
+              o.x = e4m3x4(h[16 * v + 0] * inv, h[16 * v + 1] * inv,
+                           h[16 * v + 2] * inv, h[16 * v + 3] * inv);
+              o.y = e4m3x4(h[16 * v + 4] * inv, h[16 * v + 5] * inv,
+                           h[16 * v + 6] * inv, h[16 * v + 7] * inv);
+              o.z = e4m3x4(h[16 * v + 8] * inv, h[16 * v + 9] * inv,
+                           h[16 * v + 10] * inv, h[16 * v + 11] * inv);
+              o.w = e4m3x4(h[16 * v + 12] * inv, h[16 * v + 13] * inv,
+                           h[16 * v + 14] * inv, h[16 * v + 15] * inv);
               d4[v] = o;
             }
             if (half == 0) args.c_scales[(int64_t)row * (args.ldc / 128) + n] = sc;

@@ -145,6 +145,101 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const V* __restrict__ 
   for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
 }
 
+// ---- small batches: permutation and row gather in one launch ---------------
+// For R = T*k <= 1024 routed rows (decode-sized batches) the three launches of
+// the chunked permutation plus the gather cost more than the work. Here block
+// b handles routed pair b = (token b / k, slot b % k): every block histograms
+// all R expert ids in shared memory (counts, hence offsets, do not depend on
+// the order of the atomic adds), takes the exclusive scan, ranks its pair
+// among the earlier pairs of the same expert (the pairs are in token order, so
+// that rank is the token-ascending position) and copies its token's row(s)
+// to the permuted position. The result equals the chunked permutation's.
+constexpr int kSmallPermMaxR = 1024;
+constexpr int kSmallPermThreads = 128;
+
+__global__ void __launch_bounds__(kSmallPermThreads) permute_gather_small_kernel(
+    const int32_t* __restrict__ ids, int T, int E, int k, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm, const uint4* __restrict__ x,
+    int x_vecs, uint4* __restrict__ x_perm, const uint32_t* __restrict__ x2, int x2_words,
+    uint32_t* __restrict__ x2_perm, int32_t* status) {
+  extern __shared__ int32_t small_smem[];
+  const int R = T * k;
+  int32_t* sid = small_smem;        // [R] expert of each pair (-1: out of range)
+  int32_t* soff = small_smem + R;   // [E + 1] counts, then exclusive offsets
+  __shared__ int32_t red[kSmallPermThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e <= E; e += kSmallPermThreads) soff[e] = 0;
+  __syncthreads();
+  for (int i = tid; i < R; i += kSmallPermThreads) {
+    int e = ids[i];
+    if ((unsigned)e >= (unsigned)E) {
+      if (blockIdx.x == 0) record_bad_index(status);
+      e = -1;
+    } else {
+      atomicAdd(&soff[e], 1);
+    }
+    sid[i] = e;
+  }
+  __syncthreads();
+  // exclusive scan of soff[0..E) (E <= 1024): each thread sums a run of
+  // consecutive experts, the runs are scanned across the block
+  {
+    constexpr int NT = kSmallPermThreads;
+    const int per = (E + NT - 1) / NT, lo = min(tid * per, E), hi = min(lo + per, E);
+    int run = 0;
+    for (int e = lo; e < hi; ++e) run += soff[e];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += red[w];
+    int acc = base + incl - run;  // exclusive prefix of this run
+    __syncthreads();
+    for (int e = lo; e < hi; ++e) {
+      const int c = soff[e];
+      soff[e] = acc;
+      acc += c;
+    }
+    if (tid == NT - 1) soff[E] = acc;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int e = tid; e <= E; e += kSmallPermThreads) offsets[e] = soff[e];
+  const int b = blockIdx.x, t = b / k, e = sid[b];
+  if (e < 0) return;
+  // rank of pair b among the earlier pairs that chose the same expert
+  int cnt = 0;
+  for (int p = tid; p < b; p += kSmallPermThreads) cnt += sid[p] == e;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = cnt;
+  __syncthreads();
+  int rank = 0;
+#pragma unroll
+  for (int w = 0; w < kSmallPermThreads / 32; ++w) rank += red[w];
+  const int pos = soff[e] + rank;
+  if (tid == 0) {
+    perm_token[pos] = t;
+    inv_perm[b] = pos;
+  }
+  if (x) {
+    const uint4* src = x + (int64_t)t * x_vecs;
+    uint4* dst = x_perm + (int64_t)pos * x_vecs;
+    for (int v = tid; v < x_vecs; v += kSmallPermThreads) dst[v] = src[v];
+  }
+  if (x2) {
+    const uint32_t* src = x2 + (int64_t)t * x2_words;
+    uint32_t* dst = x2_perm + (int64_t)pos * x2_words;
+    for (int v = tid; v < x2_words; v += kSmallPermThreads) dst[v] = src[v];
+  }
+}
+
 // ---- weighted combine ---------------------------------------------------------
 // "Mixture of Experts (MoE): a practical explanation", section 5 pseudocode
 // `y = sum_i weights_i * expert_i(x)`:
@@ -212,6 +307,26 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* off
   note_launch();
   permute_scatter_kernel<<<nblk, 128, (E + 1) * sizeof(int32_t), s>>>(
       ids, masks, chunk_base, counts, T, E, k, nchunks, offsets, perm_token, inv_perm, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// Permutation plus the gather of one or two row payloads (row_bytes a
+// multiple of 16; row2_bytes a multiple of 4) in one launch, for
+// R = T*k <= 1024 and E <= 1024; returns cudaErrorNotSupported otherwise.
+cudaError_t launch_permute_gather_small(const int32_t* ids, int T, int E, int k, int32_t* offsets,
+                                        int32_t* perm_token, int32_t* inv_perm, const void* x,
+                                        int row_bytes, void* x_perm, const void* x2,
+                                        int row2_bytes, void* x2_perm, int32_t* status,
+                                        cudaStream_t s) {
+  const int R = T * k;
+  if (R > kSmallPermMaxR || E > 1024 || (x && row_bytes % 16) || (x2 && row2_bytes % 4))
+    return cudaErrorNotSupported;
+  const size_t smem = (size_t)(R + E + 1) * sizeof(int32_t);
+  permute_gather_small_kernel<<<(unsigned)R, kSmallPermThreads, smem, s>>>(
+      ids, T, E, k, offsets, perm_token, inv_perm, static_cast<const uint4*>(x), row_bytes / 16,
+      static_cast<uint4*>(x_perm), static_cast<const uint32_t*>(x2), row2_bytes / 4,
+      static_cast<uint32_t*>(x2_perm), status);
   note_launch();
   return cudaGetLastError();
 }

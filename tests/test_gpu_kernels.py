@@ -100,8 +100,11 @@ def test_topk_from_logits_ties_and_extremes():
 def _ids_cases():
     rng = np.random.default_rng(11)
     cases = []
+    # R = T*k <= 1024 takes the one-launch small-batch permutation, larger R the
+    # chunked one; (512, 8, 2) and (205, 64, 5) sit on either side of the switch
     for T, E, k, skew in [(64, 8, 2, None), (1, 4, 4, None), (100, 1, 1, None), (1000, 256, 8, 1),
-                          (4096, 8, 2, 3), (257, 16, 16, None), (8192, 256, 8, None)]:
+                          (4096, 8, 2, 3), (257, 16, 16, None), (8192, 256, 8, None),
+                          (512, 8, 2, 5), (205, 64, 5, None), (64, 1024, 8, None)]:
         ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
         if skew is not None:  # one expert in every token (slot 0): one expert holds all T
             for t in range(T):
@@ -116,7 +119,7 @@ def _ids_cases():
     return cases
 
 
-@pytest.mark.parametrize("case", range(7))
+@pytest.mark.parametrize("case", range(10))
 def test_permute_bit_exact(case):
     T, E, k, ids = _ids_cases()[case]
     H = 128
