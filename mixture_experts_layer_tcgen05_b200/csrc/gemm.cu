@@ -92,6 +92,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = tile_start[args.E];
   const int nkb = args.K / BK;
+  // Plain GEMM, BN = 256: when the tiles leave a last wave at most half full,
+  // each of its tiles runs as two BN = 128 units (the column halves), so that
+  // wave ends in about half the time. units >= nfull are those halves.
+  constexpr bool kCanSplit = !SWIGLU && BN == 256 && !GATHER;
+  const int G = (int)gridDim.x;
+  const int nfull = (total / G) * G, ntail = total - nfull;
+  const bool split = kCanSplit && args.tail_split && ntail > 0 && 2 * ntail <= G;
+  const int units = split ? nfull + 2 * ntail : total;
+  // unit -> tile and column half (0: all BN columns, 1 / 2: first / second 128)
+  auto unit_tile = [&](int u, int& half) {
+    if (split && u >= nfull) {
+      half = 1 + ((u - nfull) & 1);
+      return nfull + ((u - nfull) >> 1);
+    }
+    half = 0;
+    return u;
+  };
 
   auto decode = [&](int tile, int& e, int& m, int& n) {
     e = find_expert(tile_start, args.E, tile);
@@ -150,7 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (lane == 0) {
       int64_t issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int half;
+        const int tile = unit_tile(u, half);
         int e, m, n;
         decode(tile, e, m, n);
         const int row_a = args.offsets[e] + m * BM;
@@ -159,9 +178,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           rb0 = e * args.b_rows + n * 128;
           rb1 = rb0 + args.up_off;
         } else {
-          rb0 = e * args.b_rows + n * BN;
+          rb0 = e * args.b_rows + n * BN + (half == 2 ? 128 : 0);
           rb1 = rb0 + 128;
         }
+        const bool two_b = BN == 256 && half == 0;  // a column half needs one 128-row B box
         for (int kb = 0; kb < nkb; ++kb, ++issued) {
           const int s = (int)(issued % STAGES);
           const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
@@ -170,10 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t sa = sbase + s * C::kStage, sb = sa + kTileA;
-          ptx::mbar_arrive_expect_tx(full0 + s * 8, C::kStage);
+          ptx::mbar_arrive_expect_tx(full0 + s * 8, two_b ? C::kStage : kTileA + 128 * 128);
           ptx::tma_load_2d(sa, &tmA, kb * BK, row_a, full0 + s * 8);
           ptx::tma_load_2d(sb, &tmB, kb * BK, rb0, full0 + s * 8);
-          if (BN == 256) ptx::tma_load_2d(sb + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
+          if (two_b) ptx::tma_load_2d(sb + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
         }
       }
       drain_loads<STAGES>(full0, issued, args.status);
@@ -184,7 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int acc = 0;
       uint32_t acc_ph = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int half;
+        unit_tile(u, half);
+        const uint32_t idesc = half ? ptx::make_idesc(BM, 128, 1, 1) : C::kIdesc;
         if (!ptx::mbar_wait(acce0 + acc * 8, acc_ph ^ 1, args.status, kSiteMmaAccEmpty)) break;
         ptx::tc_fence_after();
         const uint32_t d = tmem_base + acc * C::kAccCols;
@@ -201,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk)
             ptx::mma_f16(d, da + (uint64_t)(kk * UK * 2 / 16), db + (uint64_t)(kk * UK * 2 / 16),
-                         C::kIdesc, (kb | kk) != 0);
+                         idesc, (kb | kk) != 0);
           ptx::mma_commit(empty0 + s * 8);
         }
         if (!ok) break;
@@ -218,7 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     int acc = 0;
     uint32_t acc_ph = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      int half;
+      const int tile = unit_tile(u, half);
       int e, m, n;
       decode(tile, e, m, n);
       const int row = args.offsets[e] + m * BM + q * 32 + lane;
@@ -240,9 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (valid) store_row32(dst + c, h);
         }
       } else {
-        __nv_bfloat16* dst = args.C + (int64_t)row * args.ldc + n * BN;
+        __nv_bfloat16* dst = args.C + (int64_t)row * args.ldc + n * BN + (half == 2 ? 128 : 0);
+        const int ncols = half ? 128 : BN;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 0; c < ncols; c += 32) {
           uint32_t v[32];
           ptx::tmem_ld32(t0 + c, v);
           ptx::tmem_wait_ld();
@@ -511,6 +537,7 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A
   a.a_src = A;
   a.a_src_rows = A_src_rows;
   a.ksplit = 1;
+  a.tail_split = 1;
   a.partial = nullptr;
   const int64_t a_tmap_rows = A_rows ? A_src_rows : M_total;
   a.status = status;
