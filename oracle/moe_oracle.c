@@ -78,8 +78,17 @@ static void parallel_for(int64_t n, int nthreads, range_fn fn, void* ctx) {
 /* "How the Router (Top-k Routing) works step by step", steps 1-2 and the    */
 /* pseudocode's `logits = router(x)`: a linear layer from the token vector   */
 /* to E scores. The bias (when the layer has one) is added to the score.     */
-/*   logits[t, e] = (sum_{h ascending} x[t, h] * Wr[h, e]) + bias[e]         */
+/*   logits[t, e] = (sum_h x[t, h] * Wr[h, e]) + bias[e]                      */
+/* The logits decide integers (the selected experts), so the fp32 order of  */
+/* the sum is fixed (the page states none): the h range is cut into         */
+/* ROUTER_BLOCKS = 8 contiguous blocks, block b = [b*H/8, (b+1)*H/8) with   */
+/* the bounds rounded down (H/8 each when 8 divides H); each block sum      */
+/* starts at 0                                                               */
+/* and adds its products h ascending, one fp32 add of the exact bf16 x bf16 */
+/* product per term; the block sums are then added left to right:           */
+/*   s = p_0;  s = s + p_1;  ...;  s = s + p_7;  logit = s + bias[e]        */
 /* ------------------------------------------------------------------------ */
+enum { ROUTER_BLOCKS = 8 };
 typedef struct {
   const uint16_t *x, *wr;
   const float* bias;
@@ -97,11 +106,16 @@ static void logits_rows(void* p, int64_t lo, int64_t hi) {
     for (int64_t e0 = 0; e0 < c->E; e0 += EB) {
       int64_t ne = c->E - e0 < EB ? c->E - e0 : EB;
       float acc[EB];
-      for (int j = 0; j < EB; ++j) acc[j] = 0.0f;
-      for (int64_t h = 0; h < c->H; ++h) {
-        float xv = bf16_widen(xr[h]);
-        const uint16_t* wrow = c->wr + h * c->E + e0;
-        for (int64_t j = 0; j < ne; ++j) acc[j] += xv * bf16_widen(wrow[j]);
+      for (int b = 0; b < ROUTER_BLOCKS; ++b) {
+        float part[EB];
+        for (int j = 0; j < EB; ++j) part[j] = 0.0f;
+        const int64_t h0 = b * c->H / ROUTER_BLOCKS, h1 = (b + 1) * c->H / ROUTER_BLOCKS;
+        for (int64_t h = h0; h < h1; ++h) {
+          float xv = bf16_widen(xr[h]);
+          const uint16_t* wrow = c->wr + h * c->E + e0;
+          for (int64_t j = 0; j < ne; ++j) part[j] += xv * bf16_widen(wrow[j]);
+        }
+        for (int j = 0; j < EB; ++j) acc[j] = b == 0 ? part[j] : acc[j] + part[j];
       }
       for (int64_t j = 0; j < ne; ++j)
         c->logits[r * c->E + e0 + j] = acc[j] + (c->bias ? c->bias[e0 + j] : 0.0f);

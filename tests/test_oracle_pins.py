@@ -91,6 +91,21 @@ def test_logits_within_higham_bound(H, E, T):
     assert np.mean(np.abs(dropped - l64) > bound) > 0.75
 
 
+def test_logits_blocked_order_closed_form():
+    """The fixed fp32 order: 8 contiguous h blocks, each summed from 0 in h
+    order, block sums added left to right. With x = 1, a column of Wr holding
+    2^24 then 0 (block 0) and pairs of ones (blocks 1..7) sums to 2^24 + 14
+    exactly: each block of ones gives 2, and 2^24 + 2 is representable. Summed
+    h-sequentially every +1 after 2^24 would round away (2^24 + 1 is a tie to
+    even), and with 4 blocks the answer would be 2^24 + 12."""
+    H, E = 16, 2
+    x = _bf16(np.ones((1, H), np.float32))
+    col = np.array([2.0 ** 24, 0.0] + [1.0, 1.0] * 7, np.float32)
+    wr = np.stack([col, col[::-1]], axis=1)  # expert 1: the big term last
+    got = oracle.router_logits(x, _bf16(wr), None)
+    np.testing.assert_array_equal(got, np.full((1, E), 2.0 ** 24 + 14, np.float32))
+
+
 def test_logits_subset_rows_match_full():
     cfg = _small(T=40)
     x = mi.make_x(cfg)
