@@ -44,12 +44,14 @@ __device__ __forceinline__ void load_bf16_vec(const uint16_t* p, float (&v)[N]) 
 // 16-byte load per lane gives a warp 8 different expert groups without bank
 // conflicts. Per h a warp then moves 4 shared wavefronts for 64 fmas per
 // thread. The inner loop uses paired FMAs (__ffma2_rn: two independent IEEE
-// fmas per instruction), so each (token, expert) sum is still one fp32 fma
-// per h in ascending order.
+// fmas per instruction); each (token, expert) sum follows the fixed blocked
+// order: one fp32 fma per h within each of the 8 h blocks, the block sums
+// added left to right as the blocks end.
+constexpr int kRouterBlocks = 8;  // h blocks of the fixed summation order
 constexpr int kWideKC = 32;
 
 template <bool VEC>
-__global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(256, 1) router_wide_kernel(const __nv_bfloat16* __restrict__ x,
                                                              const __nv_bfloat16* __restrict__ wr,
                                                              const float* __restrict__ bias,
                                                              int T, int H, int E,
@@ -110,13 +112,29 @@ __global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16
     }
   };
 
-  // acc[a][p] holds experts (2p, 2p+1) of token a
-  float2 acc[8][4];
+  // acc[a][p]: the current h block's sums of experts (2p, 2p+1) of token a;
+  // tot[a][p]: the finished blocks' sums, added left to right (the fixed
+  // blocked order: 8 contiguous h blocks, each summed from zero)
+  float2 acc[8][4], tot[8][4];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int p = 0; p < 4; ++p) acc[a][p] = make_float2(0.0f, 0.0f);
+    for (int p = 0; p < 4; ++p) acc[a][p] = tot[a][p] = make_float2(0.0f, 0.0f);
   const int nchunks = H / KC;
+  const int L = H / kRouterBlocks;  // a multiple of 16, so blocks end on 16-h steps
+  int done = 0;                     // finished blocks
+  auto fold = [&]() {
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        tot[a][p] = done == 0 ? acc[a][p]
+                              : make_float2(__fadd_rn(tot[a][p].x, acc[a][p].x),
+                                            __fadd_rn(tot[a][p].y, acc[a][p].y));
+        acc[a][p] = make_float2(0.0f, 0.0f);
+      }
+    ++done;
+  };
   load(0);
   store(0);
   __syncthreads();
@@ -125,21 +143,25 @@ __global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16
     if (c + 1 < nchunks) load((c + 1) * KC);
     const float* xb = xs + b * KC * BT + tok0;
     const float* wb = ws + b * KC * EC + eg * 4;
+#pragma unroll 1
+    for (int h0 = 0; h0 < KC; h0 += 16) {
 #pragma unroll 4
-    for (int h = 0; h < KC; ++h) {
-      const float4 x0 = *reinterpret_cast<const float4*>(xb + h * BT);
-      const float4 x1 = *reinterpret_cast<const float4*>(xb + h * BT + 4);
-      const float4 w0 = *reinterpret_cast<const float4*>(wb + h * EC);
-      const float4 w1 = *reinterpret_cast<const float4*>(wb + h * EC + EC / 2);
-      const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      const float2 wv[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
-                            make_float2(w1.x, w1.y), make_float2(w1.z, w1.w)};
+      for (int h = h0; h < h0 + 16; ++h) {
+        const float4 x0 = *reinterpret_cast<const float4*>(xb + h * BT);
+        const float4 x1 = *reinterpret_cast<const float4*>(xb + h * BT + 4);
+        const float4 w0 = *reinterpret_cast<const float4*>(wb + h * EC);
+        const float4 w1 = *reinterpret_cast<const float4*>(wb + h * EC + EC / 2);
+        const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        const float2 wv[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
+                              make_float2(w1.x, w1.y), make_float2(w1.z, w1.w)};
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const float2 xa = make_float2(xv[a], xv[a]);
+        for (int a = 0; a < 8; ++a) {
+          const float2 xa = make_float2(xv[a], xv[a]);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) acc[a][p] = __ffma2_rn(xa, wv[p], acc[a][p]);
+          for (int p = 0; p < 4; ++p) acc[a][p] = __ffma2_rn(xa, wv[p], acc[a][p]);
+        }
       }
+      if ((c * KC + h0 + 16) % L == 0) fold();
     }
     if (c + 1 < nchunks) store(b ^ 1);
     __syncthreads();
@@ -151,8 +173,8 @@ __global__ void __launch_bounds__(256, 2) router_wide_kernel(const __nv_bfloat16
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const int ee = e0 + eg * 8 + 2 * p;
-      if (ee < E) logits[(int64_t)t * E + ee] = __fadd_rn(acc[a][p].x, bias ? bias[ee] : 0.0f);
-      if (ee + 1 < E) logits[(int64_t)t * E + ee + 1] = __fadd_rn(acc[a][p].y, bias ? bias[ee + 1] : 0.0f);
+      if (ee < E) logits[(int64_t)t * E + ee] = __fadd_rn(tot[a][p].x, bias ? bias[ee] : 0.0f);
+      if (ee + 1 < E) logits[(int64_t)t * E + ee + 1] = __fadd_rn(tot[a][p].y, bias ? bias[ee + 1] : 0.0f);
     }
   }
 }
@@ -219,157 +241,108 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (my_slot >= 0) w[(int64_t)warp * k + my_slot] = __fdiv_rn(my_ex, denom);
 }
 
-// Narrow router with fused top-k (E <= 32). One thread per (token, expert
-// pair): each thread carries two sums, one per expert of its pair, advanced
-// together by paired FMAs (__ffma2_rn), so a warp holds 32/EPP tokens and
-// every token's E logits sit in EPP neighbouring lanes (EPP = pairs, a power
-// of two). The sums are sequential chains over h, so their length H times
-// the FMA latency is the floor of this kernel, and the block is split so the
-// chains never wait on anything else:
-//  * CW compute warps run only the chains: per two h steps, two 16-byte
-//    shared loads and two paired FMAs;
-//  * twice as many helper warps stream x rows and Wr rows through an NS-deep ring
-//    of cp.async copies (raw bf16) and widen each chunk into fp32 "ready"
-//    buffers laid out for the compute loop: x as {x_h, x_h, x_h+1, x_h+1}
-//    per token, Wr as {w_h,e, w_h,e+1, w_h+1,e, w_h+1,e+1} per pair;
-//  * one block barrier per chunk of KC h values hands chunk c+1 from the
-//    helpers to the compute warps while they finish chunk c;
-//  * the top-k selection then runs on the logits still in registers: k rounds
-//    of a segmented warp argmax (logit desc, index asc) over the token's lanes.
-constexpr int kNarrowKC = 64;          // h per chunk
-constexpr int kNarrowNS = 8;           // raw chunks in flight
-constexpr int kNarrowXRow = 128 + 16;  // raw x row stride in shared memory (padded)
-
-template <int EPP, int TPT>
-struct NarrowCfg {
-  static constexpr int CW = EPP >= 4 ? EPP / 4 : 1;  // compute warps
-  static constexpr int HW = 2 * CW;                   // helper warps
-  static constexpr int kThreads = 32 * (CW + HW);
-  static constexpr int BT = TPT * 32 * CW / EPP;      // tokens per block
-};
+// Narrow router with fused top-k (E <= 32). The logit sum runs in the fixed
+// blocked order (8 contiguous h blocks, each summed from zero, then added
+// left to right), and the 8 block sums of a (token, expert pair) are computed
+// by 8 threads at once, so each sequential chain is H/8 paired FMAs long:
+//  * compute thread (token, pair, block b), b in the low 3 bits of the
+//    thread index: two sums (experts 2p, 2p+1) advanced together by paired
+//    FMAs (__ffma2_rn, two IEEE fmas per instruction) over block b's h;
+//  * each chunk covers 16 h of every block; two helper warps stream x rows and
+//    Wr rows through a cp.async ring (raw bf16) and widen each chunk into
+//    fp32 "ready" buffers laid out for the compute loop, b fastest: x as
+//    {x_h, x_h, x_h+1, x_h+1} per (token, block), Wr as
+//    {w_h,e, w_h,e+1, w_h+1,e, w_h+1,e+1} per (pair, block);
+//  * the 8 block sums are combined in order through warp shuffles, and the
+//    top-k selection runs per token over the E logits staged in shared
+//    memory (k rounds of a warp argmax on (logit desc, index asc)).
+constexpr int kNarrowSL = 16;          // h per block per chunk (chunk = 128 h)
+constexpr int kNarrowNS = 4;           // raw chunks in flight
+constexpr int kNarrowCT = 128;         // compute threads per CTA
+constexpr int kNarrowHT = 64;          // helper threads per CTA
+constexpr int kNarrowXP = 256 + 16;    // raw x bytes per token per chunk (8 blocks x 32 B), padded
 
 __host__ __device__ constexpr size_t narrow_stage_bytes(int BT, int E) {
-  return (size_t)BT * kNarrowXRow + (size_t)kNarrowKC * E * 2;
+  return (size_t)BT * kNarrowXP + (size_t)kRouterBlocks * kNarrowSL * E * 2;
 }
 __host__ __device__ constexpr size_t narrow_smem_bytes(int BT, int EPP, int E) {
-  return kNarrowNS * narrow_stage_bytes(BT, E) + 2 * (size_t)(kNarrowKC / 2) * 16 * (BT + EPP);
+  return kNarrowNS * narrow_stage_bytes(BT, E) +
+         2 * (size_t)(kNarrowSL / 2) * kRouterBlocks * 16 * (BT + EPP) + (size_t)BT * 32 * 4;
 }
 
-// Top-k of one token whose logits (l0, l1 for experts e0 = 2p, e1 = 2p + 1)
-// sit in the EPP lanes of its segment; every lane of the warp calls it.
-template <int EPP>
-__device__ __forceinline__ void segment_topk(float l0, float l1, int p, int E, int k, bool valid,
-                                             int32_t* __restrict__ ids, float* __restrict__ topw) {
-  const int e0 = 2 * p, e1 = 2 * p + 1;
-  bool take0 = e0 < E, take1 = e1 < E;  // still selectable (padding experts never are)
-  float lmax = 0.0f, denom = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-    if (take0) bv = l0, be = e0;
-    if (take1 && (l1 > bv || be == 0x7fffffff)) bv = l1, be = e1;
-#pragma unroll
-    for (int off = EPP / 2; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
-    }
-    if (be == e0) take0 = false;
-    if (be == e1) take1 = false;
-    if (j == 0) lmax = bv;
-    const float ex = expf(bv - lmax);
-    denom += ex;
-    if (valid && p == j % EPP) {
-      ids[j] = be;
-      topw[j] = ex;  // normalised below by the same thread
-    }
-  }
-  if (valid)
-    for (int j = p; j < k; j += EPP) topw[j] = __fdiv_rn(topw[j], denom);
-}
-
-template <int EPP, int TPT>  // expert pairs per token (power of two, 1..16); tokens per thread
-__global__ void __launch_bounds__(NarrowCfg<EPP, TPT>::kThreads) router_narrow_kernel(
+template <int EPP>  // expert pairs per token (power of two, 1..16)
+__global__ void __launch_bounds__(kNarrowCT + kNarrowHT) router_narrow_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
     const float* __restrict__ bias, int T, int H, int E, int k, float* __restrict__ logits,
     int32_t* __restrict__ ids, float* __restrict__ topw) {
-  using Cfg = NarrowCfg<EPP, TPT>;
-  constexpr int KC = kNarrowKC, NS = kNarrowNS, XROW = kNarrowXRow, BT = Cfg::BT;
-  constexpr int NH = 32 * Cfg::HW;  // helper threads
-  constexpr int XV = BT * 8;        // 16-byte x vectors per chunk
-  constexpr int WI = (KC / 2) * EPP;  // Wr items (two h x one pair) per chunk
+  constexpr int NB = kRouterBlocks, SL = kNarrowSL, NS = kNarrowNS, XP = kNarrowXP;
+  constexpr int BT = kNarrowCT / (EPP * NB);   // tokens per CTA (16 / EPP)
+  constexpr int NH = kNarrowHT;
+  constexpr int XV = BT * NB * 2;              // 16-byte raw x vectors per chunk
+  constexpr int XI = (SL / 2) * BT * NB;       // x items (h pair, token, block) per chunk
+  constexpr int WI = (SL / 2) * EPP * NB;      // Wr items (h pair, pair, block) per chunk
   extern __shared__ __align__(16) unsigned char narrow_smem[];
   const int tid = threadIdx.x;
-  const bool helper = tid >= 32 * Cfg::CW;
-  const int hid = tid - 32 * Cfg::CW;  // helper thread index
-  const int p = tid % EPP, tl = tid / EPP;  // compute threads: (tokens tl + i*BT/TPT, pair)
+  const bool helper = tid >= kNarrowCT;
+  const int hid = tid - kNarrowCT;
+  const int b = tid & (NB - 1), p = (tid >> 3) % EPP, tl = (tid >> 3) / EPP;
   const int t0 = blockIdx.x * BT;
-  const int nchunks = H / KC;
+  const int L = H / NB;                        // h per block (a multiple of 16)
+  const int nchunks = L / SL;
   const size_t stage = narrow_stage_bytes(BT, E);
   unsigned char* ring = narrow_smem;
-  float4* rx = reinterpret_cast<float4*>(narrow_smem + NS * stage);  // [2][KC/2][BT]
-  float4* rw = rx + 2 * (KC / 2) * BT;                                 // [2][KC/2][EPP]
+  float4* rx = reinterpret_cast<float4*>(narrow_smem + NS * stage);  // [2][SL/2][BT][NB]
+  float4* rw = rx + 2 * (SL / 2) * BT * NB;                            // [2][SL/2][EPP][NB]
+  float* slg = reinterpret_cast<float*>(rw + 2 * (SL / 2) * EPP * NB);  // [BT][32] logits
   const char* xg = reinterpret_cast<const char*>(x);
   const char* wg = reinterpret_cast<const char*>(wr);
 
-  // helpers: raw chunk c -> ring slot c % NS: BT x rows of 128 B, then KC Wr
-  // rows, which are one contiguous 128*E-byte range of Wr [H][E]
+  // helpers: raw chunk c -> ring slot c % NS: per token its 8 block slices of
+  // 16 h (32 B each), then per block 16 Wr rows (one contiguous 32*E bytes)
   auto issue = [&](int c) {
     if (c < nchunks) {
       const uint32_t st = ptx::smem_addr(ring + (c % NS) * stage);
-#pragma unroll
-      for (int it = 0; it < (XV + NH - 1) / NH; ++it) {
-        const int i = hid + it * NH;
-        if (XV % NH == 0 || i < XV) {
-          const int r = i >> 3, v = i & 7, t = t0 + r;
-          const char* src = xg + ((int64_t)(t < T ? t : 0) * H + (int64_t)c * KC) * 2 + v * 16;
-          ptx::cp_async16(st + r * XROW + v * 16, src, t < T ? 16u : 0u);
-        }
+      for (int i = hid; i < XV; i += NH) {
+        const int r = i / (NB * 2), bb = (i / 2) % NB, v = i & 1, t = t0 + r;
+        const char* src = xg + ((int64_t)(t < T ? t : 0) * H + (int64_t)bb * L + c * SL) * 2 + v * 16;
+        ptx::cp_async16(st + r * XP + (bb * 2 + v) * 16, src, t < T ? 16u : 0u);
       }
-      const char* wsrc = wg + (int64_t)c * KC * E * 2;
-      const uint32_t wdst = st + BT * XROW;
-      for (int i = hid; i < KC * E * 2 / 16; i += NH) ptx::cp_async16(wdst + i * 16, wsrc + i * 16, 16u);
+      const int wv = 2 * E;  // 16-byte vectors per block slice
+      const uint32_t wdst = st + BT * XP;
+      for (int i = hid; i < NB * wv; i += NH) {
+        const int bb = i / wv, v = i % wv;
+        const char* src = wg + ((int64_t)bb * L + c * SL) * E * 2 + v * 16;
+        ptx::cp_async16(wdst + (bb * wv + v) * 16, src, 16u);
+      }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
   // helpers: widen raw chunk c into ready buffer c & 1
   auto convert = [&](int c) {
     const unsigned char* st = ring + (c % NS) * stage;
-    float4* dx = rx + (c & 1) * (KC / 2) * BT;
-#pragma unroll
-    for (int it = 0; it < (XV + NH - 1) / NH; ++it) {
-      const int i = hid + it * NH;
-      if (XV % NH == 0 || i < XV) {
-        const int r = i % BT, v = i / BT;
-        const uint4 u = *reinterpret_cast<const uint4*>(st + r * XROW + v * 16);
-        const uint32_t q[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float lo = bf16lo_to_f32(q[j]), hi = bf16hi_to_f32(q[j]);
-          dx[(v * 4 + j) * BT + r] = make_float4(lo, lo, hi, hi);
-        }
-      }
+    float4* dx = rx + (c & 1) * (SL / 2) * BT * NB;
+    for (int i = hid; i < XI; i += NH) {
+      const int bb = i % NB, r = (i / NB) % BT, j = i / (NB * BT);
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(st + r * XP + bb * 32 + j * 4);
+      const float lo = bf16lo_to_f32(u), hi = bf16hi_to_f32(u);
+      dx[(j * BT + r) * NB + bb] = make_float4(lo, lo, hi, hi);
     }
-    const unsigned char* sw = st + BT * XROW;  // Wr chunk [KC][E] bf16
-    float4* dw = rw + (c & 1) * (KC / 2) * EPP;
-#pragma unroll
-    for (int it = 0; it < (WI + NH - 1) / NH; ++it) {
-      const int i = hid + it * NH;
-      if (WI % NH == 0 || i < WI) {
-        const int j = i / EPP, pp = i % EPP, e0 = 2 * pp;
-        const int o0 = (2 * j) * E + e0, o1 = o0 + E;  // element offsets of rows 2j, 2j+1
-        uint32_t u0, u1;
-        if ((E & 1) == 0) {  // the pair is one aligned 32-bit word (zero past E)
-          u0 = e0 < E ? *reinterpret_cast<const uint32_t*>(sw + 2 * o0) : 0u;
-          u1 = e0 < E ? *reinterpret_cast<const uint32_t*>(sw + 2 * o1) : 0u;
-        } else {
-          const uint16_t* h16 = reinterpret_cast<const uint16_t*>(sw);
-          u0 = (e0 < E ? (uint32_t)h16[o0] : 0u) | (e0 + 1 < E ? (uint32_t)h16[o0 + 1] << 16 : 0u);
-          u1 = (e0 < E ? (uint32_t)h16[o1] : 0u) | (e0 + 1 < E ? (uint32_t)h16[o1 + 1] << 16 : 0u);
-        }
-        dw[i] = make_float4(bf16lo_to_f32(u0), bf16hi_to_f32(u0), bf16lo_to_f32(u1),
-                            bf16hi_to_f32(u1));
+    const unsigned char* sw = st + BT * XP;  // [NB][SL][E] bf16
+    float4* dw = rw + (c & 1) * (SL / 2) * EPP * NB;
+    for (int i = hid; i < WI; i += NH) {
+      const int bb = i % NB, pp = (i / NB) % EPP, j = i / (NB * EPP), e0 = 2 * pp;
+      const int o0 = (bb * SL + 2 * j) * E + e0, o1 = o0 + E;  // elements of rows 2j, 2j+1
+      uint32_t u0, u1;
+      if ((E & 1) == 0) {  // the pair is one aligned 32-bit word
+        u0 = e0 < E ? *reinterpret_cast<const uint32_t*>(sw + 2 * o0) : 0u;
+        u1 = e0 < E ? *reinterpret_cast<const uint32_t*>(sw + 2 * o1) : 0u;
+      } else {
+        const uint16_t* h16 = reinterpret_cast<const uint16_t*>(sw);
+        u0 = (e0 < E ? (uint32_t)h16[o0] : 0u) | (e0 + 1 < E ? (uint32_t)h16[o0 + 1] << 16 : 0u);
+        u1 = (e0 < E ? (uint32_t)h16[o1] : 0u) | (e0 + 1 < E ? (uint32_t)h16[o1 + 1] << 16 : 0u);
       }
+      dw[(j * EPP + pp) * NB + bb] = make_float4(bf16lo_to_f32(u0), bf16hi_to_f32(u0),
+                                                 bf16lo_to_f32(u1), bf16hi_to_f32(u1));
     }
   };
 
@@ -380,10 +353,7 @@ __global__ void __launch_bounds__(NarrowCfg<EPP, TPT>::kThreads) router_narrow_k
   }
   __syncthreads();
   if (helper) convert(0);
-  // compute threads: acc[i] = experts (2p, 2p+1) of token tl + i * BT/TPT
-  float2 acc[TPT];
-#pragma unroll
-  for (int i = 0; i < TPT; ++i) acc[i] = make_float2(0.0f, 0.0f);
+  float2 acc = make_float2(0.0f, 0.0f);  // compute threads: block b's sums of experts (2p, 2p+1)
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
     // helpers' copies of chunk c+1 landed; the barrier publishes them and the
@@ -394,22 +364,13 @@ __global__ void __launch_bounds__(NarrowCfg<EPP, TPT>::kThreads) router_narrow_k
       issue(c + NS);
       if (c + 1 < nchunks) convert(c + 1);
     } else {
-      const float4* xb = rx + (c & 1) * (KC / 2) * BT + tl;
-      const float4* wb = rw + (c & 1) * (KC / 2) * EPP + p;
-      // TPT independent chains interleave, so a paired FMA rarely waits on its
-      // predecessor
+      const float4* xb = rx + (c & 1) * (SL / 2) * BT * NB + tl * NB + b;
+      const float4* wb = rw + (c & 1) * (SL / 2) * EPP * NB + p * NB + b;
 #pragma unroll
-      for (int j = 0; j < KC / 2; ++j) {
-        const float4 wv = wb[j * EPP];
-        float4 xv[TPT];
-#pragma unroll
-        for (int i = 0; i < TPT; ++i) xv[i] = xb[j * BT + i * (BT / TPT)];
-#pragma unroll
-        for (int i = 0; i < TPT; ++i)
-          acc[i] = __ffma2_rn(make_float2(xv[i].x, xv[i].y), make_float2(wv.x, wv.y), acc[i]);
-#pragma unroll
-        for (int i = 0; i < TPT; ++i)
-          acc[i] = __ffma2_rn(make_float2(xv[i].z, xv[i].w), make_float2(wv.z, wv.w), acc[i]);
+      for (int j = 0; j < SL / 2; ++j) {
+        const float4 xv = xb[j * BT * NB], wv = wb[j * EPP * NB];
+        acc = __ffma2_rn(make_float2(xv.x, xv.y), make_float2(wv.x, wv.y), acc);
+        acc = __ffma2_rn(make_float2(xv.z, xv.w), make_float2(wv.z, wv.w), acc);
       }
     }
   }
@@ -418,18 +379,57 @@ __global__ void __launch_bounds__(NarrowCfg<EPP, TPT>::kThreads) router_narrow_k
     return;
   }
 
-  const int e0 = 2 * p, e1 = 2 * p + 1;
-  const float b0 = bias ? bias[e0 < E ? e0 : 0] : 0.0f, b1 = bias ? bias[e1 < E ? e1 : 0] : 0.0f;
+  // block sums -> logits, added left to right by the block-0 lane of each group
+  const int lane = tid & 31;
+  float s0 = acc.x, s1 = acc.y;
 #pragma unroll
-  for (int i = 0; i < TPT; ++i) {
-    const int t = t0 + tl + i * (BT / TPT);
-    const float l0 = __fadd_rn(acc[i].x, b0), l1 = __fadd_rn(acc[i].y, b1);
+  for (int i = 1; i < NB; ++i) {
+    const float a0 = __shfl_sync(0xffffffffu, acc.x, (lane & ~(NB - 1)) + i);
+    const float a1 = __shfl_sync(0xffffffffu, acc.y, (lane & ~(NB - 1)) + i);
+    s0 = __fadd_rn(s0, a0);
+    s1 = __fadd_rn(s1, a1);
+  }
+  const int t = t0 + tl, e0 = 2 * p, e1 = 2 * p + 1;
+  if (b == 0) {
+    const float l0 = __fadd_rn(s0, bias ? bias[e0 < E ? e0 : 0] : 0.0f);
+    const float l1 = __fadd_rn(s1, bias ? bias[e1 < E ? e1 : 0] : 0.0f);
+    if (e0 < E) slg[tl * 32 + e0] = l0;
+    if (e1 < E) slg[tl * 32 + e1] = l1;
     if (t < T && logits) {
       if (e0 < E) logits[(int64_t)t * E + e0] = l0;
       if (e1 < E) logits[(int64_t)t * E + e1] = l1;
     }
-    const int64_t o = (int64_t)(t < T ? t : 0) * k;
-    segment_topk<EPP>(l0, l1, p, E, k, t < T, ids + o, topw + o);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kNarrowCT) : "memory");  // compute warps only
+  // top-k: warp w takes tokens w, w + 4, ...; lane = expert
+  const int w = tid >> 5;
+  for (int r = w; r < BT; r += kNarrowCT / 32) {
+    const int tt = t0 + r;
+    if (tt >= T) break;
+    const float v = lane < E ? slg[r * 32 + lane] : -INFINITY;
+    bool taken = lane >= E;
+    float lmax = 0.0f, denom = 0.0f, my_ex = 0.0f;
+    int my_slot = -1;
+    for (int j = 0; j < k; ++j) {
+      float bv = taken ? -INFINITY : v;
+      int be = taken ? 0x7fffffff : lane;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
+      }
+      if (be == lane) taken = true;
+      if (j == 0) lmax = bv;
+      const float ex = expf(bv - lmax);
+      denom += ex;
+      if (lane == j) {
+        my_ex = ex;
+        my_slot = j;
+        ids[(int64_t)tt * k + j] = be;
+      }
+    }
+    if (my_slot >= 0) topw[(int64_t)tt * k + my_slot] = __fdiv_rn(my_ex, denom);
   }
 }
 
@@ -450,15 +450,13 @@ cudaError_t launch_route(const void* x, const void* wr, const float* bias, int T
   const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(wr);
   if (E <= 32) {
     const int epp = narrow_pairs(E);
-    // one token per compute thread: two tokens per thread (TPT = 2) measured
-    // slower at the decode and prefill shapes
 #define MOE_NARROW(P)                                                                         \
   do {                                                                                        \
-    using Cfg = NarrowCfg<P, 1>;                                                              \
-    const size_t smem = narrow_smem_bytes(Cfg::BT, P, E);                                     \
-    cudaFuncSetAttribute(router_narrow_kernel<P, 1>,                                          \
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);             \
-    router_narrow_kernel<P, 1><<<(unsigned)ceil_div(T, Cfg::BT), Cfg::kThreads, smem, s>>>(   \
+    constexpr int BTV = kNarrowCT / (P * kRouterBlocks);                                      \
+    const size_t smem = narrow_smem_bytes(BTV, P, E);                                         \
+    cudaFuncSetAttribute(router_narrow_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                         (int)smem);                                                          \
+    router_narrow_kernel<P><<<(unsigned)ceil_div(T, BTV), kNarrowCT + kNarrowHT, smem, s>>>(  \
         xp, wp, bias, T, H, E, k, logits, ids, w);                                            \
   } while (0)
     if (epp == 1) MOE_NARROW(1);
