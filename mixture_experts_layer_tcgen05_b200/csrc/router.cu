@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 //  * compute thread (token, pair, block b), b in the low 3 bits of the
 //    thread index: two sums (experts 2p, 2p+1) advanced together by paired
 //    FMAs (__ffma2_rn, two IEEE fmas per instruction) over block b's h;
-//  * each chunk covers 16 h of every block; two helper warps stream x rows and
+//  * each chunk covers 16 h of every block; four helper warps stream x rows and
 //    Wr rows through a cp.async ring (raw bf16) and widen each chunk into
 //    fp32 "ready" buffers laid out for the compute loop, b fastest: x as
 //    {x_h, x_h, x_h+1, x_h+1} per (token, block), Wr as
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 constexpr int kNarrowSL = 16;          // h per block per chunk (chunk = 128 h)
 constexpr int kNarrowNS = 4;           // raw chunks in flight
 constexpr int kNarrowCT = 128;         // compute threads per CTA
-constexpr int kNarrowHT = 64;          // helper threads per CTA
+constexpr int kNarrowHT = 128;         // helper threads per CTA
 constexpr int kNarrowXP = 256 + 16;    // raw x bytes per token per chunk (8 blocks x 32 B), padded
 
 __host__ __device__ constexpr size_t narrow_stage_bytes(int BT, int E) {
@@ -321,7 +321,10 @@ __global__ void __launch_bounds__(kNarrowCT + kNarrowHT) router_narrow_kernel(
   auto convert = [&](int c) {
     const unsigned char* st = ring + (c % NS) * stage;
     float4* dx = rx + (c & 1) * (SL / 2) * BT * NB;
-    for (int i = hid; i < XI; i += NH) {
+#pragma unroll
+    for (int it = 0; it < (XI + NH - 1) / NH; ++it) {
+      const int i = hid + it * NH;
+      if (XI % NH != 0 && i >= XI) break;
       const int bb = i % NB, r = (i / NB) % BT, j = i / (NB * BT);
       const uint32_t u = *reinterpret_cast<const uint32_t*>(st + r * XP + bb * 32 + j * 4);
       const float lo = bf16lo_to_f32(u), hi = bf16hi_to_f32(u);
@@ -329,7 +332,10 @@ __global__ void __launch_bounds__(kNarrowCT + kNarrowHT) router_narrow_kernel(
     }
     const unsigned char* sw = st + BT * XP;  // [NB][SL][E] bf16
     float4* dw = rw + (c & 1) * (SL / 2) * EPP * NB;
-    for (int i = hid; i < WI; i += NH) {
+#pragma unroll
+    for (int it = 0; it < (WI + NH - 1) / NH; ++it) {
+      const int i = hid + it * NH;
+      if (WI % NH != 0 && i >= WI) break;
       const int bb = i % NB, pp = (i / NB) % EPP, j = i / (NB * EPP), e0 = 2 * pp;
       const int o0 = (bb * SL + 2 * j) * E + e0, o1 = o0 + E;  // elements of rows 2j, 2j+1
       uint32_t u0, u1;
