@@ -48,14 +48,14 @@ def _L():
             "oracle_permute": [vp, i64, i64, i32, vp, vp, vp, vp],
             "oracle_expert_gated_rows": [vp, i64, vp, i64, i64, i32, vp],
             "oracle_expert_down_rows": [vp, i64, vp, i64, i64, vp],
-            "oracle_quant_act_fp8": [vp, i64, i64, vp, vp],
-            "oracle_quant_weight_fp8": [vp, i64, i64, i64, vp, vp, i32],
+            "oracle_quant_act_fp8": [vp, i64, i64, vp, vp, i32],
+            "oracle_quant_weight_fp8": [vp, i64, i64, i64, vp, vp, i32, i32],
             "oracle_experts_combine": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, i32, vp,
                                        i32],
             "oracle_experts_combine_fp8": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp,
-                                           i32, vp, i32],
+                                           i32, i32, vp, i32],
             "oracle_moe_forward": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp,
-                                   i32, vp, vp, vp, vp, i32],
+                                   i32, i32, vp, vp, vp, vp, i32],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -154,24 +154,34 @@ def e4m3_encode(f: float) -> int:
     return int(_L().oracle_e4m3_encode(float(f)))
 
 
-def quant_act_fp8(x):
-    """Per row, per 128-column group: s = amax/448 (1 if amax == 0), q = e4m3(x/s)."""
+def quant_act_fp8(x, ue8m0=False):
+    """Per row, per 128-column group: s = amax/448 (1 if amax == 0), q = e4m3(x/s).
+    ue8m0: s is the smallest power of two >= amax/448 instead."""
     x = _c(x, np.uint16)
     rows, cols = x.shape
     q = np.empty((rows, cols), dtype=np.uint8)
     s = np.empty((rows, cols // 128), dtype=np.float32)
-    _L().oracle_quant_act_fp8(_p(x), rows, cols, _p(q), _p(s))
+    _L().oracle_quant_act_fp8(_p(x), rows, cols, _p(q), _p(s), int(bool(ue8m0)))
     return q, s
 
 
-def quant_weight_fp8(w, nthreads=None):
+def quant_weight_fp8(w, nthreads=None, ue8m0=False):
     """128 x 128 blocks of w [nb, rows, cols]: q [nb, rows, cols], s [nb, rows/128, cols/128]."""
     w = _c(w, np.uint16)
     nb, rows, cols = w.shape
     q = np.empty((nb, rows, cols), dtype=np.uint8)
     s = np.empty((nb, rows // 128, cols // 128), dtype=np.float32)
-    _L().oracle_quant_weight_fp8(_p(w), nb, rows, cols, _p(q), _p(s), nthreads or threads())
+    _L().oracle_quant_weight_fp8(_p(w), nb, rows, cols, _p(q), _p(s), int(bool(ue8m0)),
+                                 nthreads or threads())
     return q, s
+
+
+def e8m0_code(s):
+    """The float8_e8m0fnu byte of power-of-two scales s (2^(code - 127))."""
+    s = np.asarray(s, dtype=np.float32)
+    m, e = np.frexp(s)
+    assert np.all(m == 0.5), "not powers of two"
+    return (e - 1 + 127).astype(np.uint8)
 
 
 def experts_combine(x, tokens, ids, w, w13, w2, nthreads=None, act=ACT_SILU):
@@ -186,7 +196,8 @@ def experts_combine(x, tokens, ids, w, w13, w2, nthreads=None, act=ACT_SILU):
     return out
 
 
-def experts_combine_fp8(x, tokens, ids, w, w13q, w13s, w2q, w2s, nthreads=None, act=ACT_SILU):
+def experts_combine_fp8(x, tokens, ids, w, w13q, w13s, w2q, w2s, nthreads=None, act=ACT_SILU,
+                        ue8m0=False):
     x, tokens = _c(x, np.uint16), _c(tokens, np.int32)
     ids, w = _c(ids, np.int32), _c(w, np.float32)
     w13q, w2q = _c(w13q, np.uint8), _c(w2q, np.uint8)
@@ -195,13 +206,13 @@ def experts_combine_fp8(x, tokens, ids, w, w13q, w13s, w2q, w2s, nthreads=None, 
     nt, k = ids.shape
     out = np.empty((nt, H), dtype=np.float32)
     _L().oracle_experts_combine_fp8(_p(x), _p(tokens), nt, H, I2 // 2, E, k, _p(ids), _p(w),
-                                    _p(w13q), _p(w13s), _p(w2q), _p(w2s), int(act), _p(out),
-                                    nthreads or threads())
+                                    _p(w13q), _p(w13s), _p(w2q), _p(w2s), int(act),
+                                    int(bool(ue8m0)), _p(out), nthreads or threads())
     return out
 
 
 def moe_forward(x, wr, bias, w13=None, w2=None, k=2, tokens=None, fp8=None, nthreads=None,
-                act=ACT_SILU):
+                act=ACT_SILU, ue8m0=False):
     """The whole layer for ``tokens`` (all when None).
 
     ``fp8`` = (w13q, w13s, w2q, w2s) selects the FP8 experts (x is quantised
@@ -227,6 +238,6 @@ def moe_forward(x, wr, bias, w13=None, w2=None, k=2, tokens=None, fp8=None, nthr
     logits = np.empty((nt, E), dtype=np.float32)
     _L().oracle_moe_forward(_p(x), _p(tokens), nt, H, I, E, k, _p(wr), _p(b),
                             _p(w13) if fp8 is None else None, _p(w2) if fp8 is None else None,
-                            _p(w13q), _p(w13s), _p(w2q), _p(w2s), int(act), _p(out), _p(ids),
-                            _p(w), _p(logits), nthreads or threads())
+                            _p(w13q), _p(w13s), _p(w2q), _p(w2s), int(act), int(bool(ue8m0)),
+                            _p(out), _p(ids), _p(w), _p(logits), nthreads or threads())
     return {"out": out, "ids": ids, "w": w, "logits": logits}

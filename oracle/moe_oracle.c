@@ -351,19 +351,36 @@ uint8_t oracle_e4m3_encode(float f) {
   return s | (uint8_t)(((e + 7) << 3) | (int)m);
 }
 
-/* amax / 448 in fp32 with IEEE division; an all-zero group gets scale 1 */
-static inline float group_scale(float amax) { return amax > 0.0f ? amax / 448.0f : 1.0f; }
+/* amax / 448 in fp32 with IEEE division; an all-zero group gets scale 1.
+ * With power-of-two scales ("Fine-grained FP8" / "Experts backends", UE8M0
+ * scale format: scales stored as 8-bit exponents, float8_e8m0fnu), the scale
+ * is the smallest power of two >= amax / 448 (that fp32 quotient, so no
+ * scaled value exceeds 448), kept within the format's range 2^-127..2^127. */
+enum { SCALE_F32 = 0, SCALE_UE8M0 = 1 };
+
+static inline float group_scale(float amax, int fmt) {
+  if (!(amax > 0.0f)) return 1.0f;
+  const float r = amax / 448.0f;
+  if (fmt != SCALE_UE8M0) return r;
+  int e;
+  const float m = frexpf(r, &e); /* r = m * 2^e, m in [0.5, 1) */
+  int p2 = m == 0.5f ? e - 1 : e;  /* r is a power of two: 2^(e-1); else round up */
+  if (p2 < -127) p2 = -127;
+  if (p2 > 127) p2 = 127;
+  return ldexpf(1.0f, p2);
+}
 
 /* Per row, per group of 128 consecutive columns: s = amax/448, q = e4m3(v/s).
  * vals: [rows, cols] fp32 (already widened); q: [rows, cols]; s: [rows, cols/128]. */
-static void quant_groups_f32(const float* vals, int64_t rows, int64_t cols, uint8_t* q, float* s) {
+static void quant_groups_f32(const float* vals, int64_t rows, int64_t cols, uint8_t* q, float* s,
+                             int fmt) {
   int64_t G = cols / 128;
   for (int64_t r = 0; r < rows; ++r) {
     for (int64_t g = 0; g < G; ++g) {
       const float* v = vals + r * cols + g * 128;
       float amax = 0.0f;
       for (int c = 0; c < 128; ++c) amax = fmaxf(amax, fabsf(v[c]));
-      float sc = group_scale(amax);
+      float sc = group_scale(amax, fmt);
       s[r * G + g] = sc;
       for (int c = 0; c < 128; ++c) q[r * cols + g * 128 + c] = oracle_e4m3_encode(v[c] / sc);
     }
@@ -371,11 +388,12 @@ static void quant_groups_f32(const float* vals, int64_t rows, int64_t cols, uint
 }
 
 /* Activation quantisation of bf16 rows [rows, cols]. */
-void oracle_quant_act_fp8(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* s) {
+void oracle_quant_act_fp8(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* s,
+                          int fmt) {
   float* v = (float*)malloc(sizeof(float) * (size_t)cols);
   for (int64_t r = 0; r < rows; ++r) {
     for (int64_t c = 0; c < cols; ++c) v[c] = bf16_widen(x[r * cols + c]);
-    quant_groups_f32(v, 1, cols, q + r * cols, s + r * (cols / 128));
+    quant_groups_f32(v, 1, cols, q + r * cols, s + r * (cols / 128), fmt);
   }
   free(v);
 }
@@ -388,6 +406,7 @@ typedef struct {
   int64_t rows, cols;
   uint8_t* q;
   float* s;
+  int fmt;
 } wq_ctx;
 
 static void wq_blocks(void* p, int64_t lo, int64_t hi) {
@@ -400,7 +419,7 @@ static void wq_blocks(void* p, int64_t lo, int64_t hi) {
     for (int64_t r = rb * 128; r < rb * 128 + 128; ++r)
       for (int64_t cc = cb * 128; cc < cb * 128 + 128; ++cc)
         amax = fmaxf(amax, fabsf(bf16_widen(wb[r * cols + cc])));
-    float sc = group_scale(amax);
+    float sc = group_scale(amax, c->fmt);
     c->s[blk] = sc;
     for (int64_t r = rb * 128; r < rb * 128 + 128; ++r)
       for (int64_t cc = cb * 128; cc < cb * 128 + 128; ++cc)
@@ -409,8 +428,8 @@ static void wq_blocks(void* p, int64_t lo, int64_t hi) {
 }
 
 void oracle_quant_weight_fp8(const uint16_t* w, int64_t nb, int64_t rows, int64_t cols,
-                             uint8_t* q, float* s, int nthreads) {
-  wq_ctx c = {w, rows, cols, q, s};
+                             uint8_t* q, float* s, int fmt, int nthreads) {
+  wq_ctx c = {w, rows, cols, q, s, fmt};
   parallel_for(nb * (rows / 128) * (cols / 128), nthreads, wq_blocks, &c);
 }
 
@@ -435,7 +454,8 @@ typedef struct {
   const uint8_t *w13q, *w2q, *xq;
   const float *w13s, *w2s, *xs;
   int fp8;
-  int act; /* gated activation of the expert MLP */
+  int scale_fmt; /* FP8 scales: fp32 or power-of-two (UE8M0) */
+  int act;       /* gated activation of the expert MLP */
   /* work list: items of up to CHUNK (row, slot) pairs of one expert */
   int64_t* item_e;
   int64_t* item_start; /* into pairs */
@@ -504,7 +524,7 @@ static void* fwd_worker(void* p) {
       if (c->fp8) { /* the down projection's input is quantised per (row, 128-group) too */
         for (int64_t r = 0; r < n; ++r) {
           for (int64_t i = 0; i < I; ++i) af[i] = (float)a[r * I + i];
-          quant_groups_f32(af, 1, I, aq, as);
+          quant_groups_f32(af, 1, I, aq, as, c->scale_fmt);
           for (int64_t i = 0; i < I; ++i) a[r * I + i] = oracle_e4m3_decode(aq[i]) * (double)as[i / 128];
         }
       }
@@ -611,14 +631,14 @@ void oracle_experts_combine(const uint16_t* x, const int32_t* tokens, int64_t nt
 void oracle_experts_combine_fp8(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H,
                                 int64_t I, int64_t E, int k, const int32_t* ids,
                                 const float* topk_w, const uint8_t* w13q, const float* w13s,
-                                const uint8_t* w2q, const float* w2s, int act, float* out,
-                                int nthreads) {
+                                const uint8_t* w2q, const float* w2s, int act, int scale_fmt,
+                                float* out, int nthreads) {
   uint8_t* xq = (uint8_t*)malloc((size_t)(nt * H));
   float* xs = (float*)malloc(sizeof(float) * (size_t)(nt * (H / 128)));
   uint16_t* xrows = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)H);
   for (int64_t r = 0; r < nt; ++r) {
     memcpy(xrows, x + (int64_t)tokens[r] * H, sizeof(uint16_t) * (size_t)H);
-    oracle_quant_act_fp8(xrows, 1, H, xq + r * H, xs + r * (H / 128));
+    oracle_quant_act_fp8(xrows, 1, H, xq + r * H, xs + r * (H / 128), scale_fmt);
   }
   fwd_ctx c;
   memset(&c, 0, sizeof(c));
@@ -636,6 +656,7 @@ void oracle_experts_combine_fp8(const uint16_t* x, const int32_t* tokens, int64_
   c.xq = xq;
   c.xs = xs;
   c.fp8 = 1;
+  c.scale_fmt = scale_fmt;
   c.act = act;
   run_forward(&c, ids, topk_w, out, nthreads);
   free(xq);
@@ -649,16 +670,16 @@ void oracle_moe_forward(const uint16_t* x, const int32_t* tokens, int64_t nt, in
                         int64_t E, int k, const uint16_t* wr, const float* bias,
                         const uint16_t* w13, const uint16_t* w2, const uint8_t* w13q,
                         const float* w13s, const uint8_t* w2q, const float* w2s, int act,
-                        float* out, int32_t* ids_out, float* w_out, float* logits_out,
-                        int nthreads) {
+                        int scale_fmt, float* out, int32_t* ids_out, float* w_out,
+                        float* logits_out, int nthreads) {
   float* logits = logits_out ? logits_out : (float*)malloc(sizeof(float) * (size_t)(nt * E));
   int32_t* ids = ids_out ? ids_out : (int32_t*)malloc(sizeof(int32_t) * (size_t)(nt * k));
   float* w = w_out ? w_out : (float*)malloc(sizeof(float) * (size_t)(nt * k));
   oracle_router_logits(x, wr, bias, tokens, nt, H, E, logits, nthreads);
   oracle_topk(logits, nt, E, k, ids, w);
   if (w13q)
-    oracle_experts_combine_fp8(x, tokens, nt, H, I, E, k, ids, w, w13q, w13s, w2q, w2s, act, out,
-                               nthreads);
+    oracle_experts_combine_fp8(x, tokens, nt, H, I, E, k, ids, w, w13q, w13s, w2q, w2s, act,
+                               scale_fmt, out, nthreads);
   else
     oracle_experts_combine(x, tokens, nt, H, I, E, k, ids, w, w13, w2, act, out, nthreads);
   if (!logits_out) free(logits);

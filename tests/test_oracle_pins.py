@@ -370,6 +370,63 @@ def test_act_quant_bounds_and_closed_forms():
     assert np.all(err <= np.maximum(2.0 ** -4 * np.abs(xf), 2.0 ** -10 * sfull) * (1 + 1e-6))
 
 
+def test_ue8m0_scales_closed_forms():
+    """Power-of-two (UE8M0) scales: the smallest 2^p >= amax/448. Rows built so
+    amax/448 is exactly 1 (scale 1), just above 1 (scale 2), exactly 1/2
+    (scale 1/2) and 300/448 (scale 1); every scaled group max lands in
+    (224, 448], and the scales are exact powers of two (e8m0 codes 127 + p)."""
+    H = 128
+    rows = np.zeros((5, H), np.float32)
+    rows[0, 7] = 448.0
+    rows[1, 9] = 450.0
+    rows[2, 0] = -224.0
+    rows[3, 100] = 300.0  # row 4 stays all zero: scale 1
+    q, s = oracle.quant_act_fp8(_bf16(rows), ue8m0=True)
+    np.testing.assert_array_equal(s[:, 0], np.array([1.0, 2.0, 0.5, 1.0, 1.0], np.float32))
+    np.testing.assert_array_equal(oracle.e8m0_code(s[:, 0]), [127, 128, 126, 127, 127])
+    assert q[0, 7] == 0x7E and q[2, 0] == 0xFE  # 448 and -448 after scaling
+    assert q[1, 9] == oracle.e4m3_encode(225.0)  # 450 / 2
+    x = mi.make_x(_small(T=16, H=512))
+    q, s = oracle.quant_act_fp8(x, ue8m0=True)
+    amax = np.abs(mi.bf16_to_f32(x)).reshape(16, 4, 128).max(2)
+    ratio = amax / s
+    assert np.all((ratio > 224) & (ratio <= 448))
+    # same codes as the fp32-scale path would give for the scaled values
+    sf = np.repeat(s, 128, axis=1)
+    direct = np.vectorize(oracle.e4m3_encode)((mi.bf16_to_f32(x) / sf).astype(np.float32))
+    np.testing.assert_array_equal(q, direct)
+
+
+def test_ue8m0_weight_blocks_and_forward():
+    cfg = _small(T=12, E=3, k=2, H=256, I=256)
+    L = mi.make_layer(cfg)
+    q13, s13 = oracle.quant_weight_fp8(L["w13"], ue8m0=True)
+    q2, s2 = oracle.quant_weight_fp8(L["w2"], ue8m0=True)
+    for s in (s13, s2):
+        m, _ = np.frexp(s)
+        assert np.all(m == 0.5)
+    # the forward on power-of-two scales equals the dense layer on the dequantised values
+    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], k=cfg.k, fp8=(q13, s13, q2, s2), ue8m0=True)
+    dec = np.vectorize(oracle.e4m3_decode)
+    W13 = dec(q13) * np.repeat(np.repeat(s13, 128, 1), 128, 2)
+    W2 = dec(q2) * np.repeat(np.repeat(s2, 128, 1), 128, 2)
+    xq, xs = oracle.quant_act_fp8(L["x"], ue8m0=True)
+    X = dec(xq) * np.repeat(xs, 128, 1)
+    ref = np.zeros((cfg.T, cfg.H))
+    for t in range(cfg.T):
+        for j in range(cfg.k):
+            e = r["ids"][t, j]
+            g, u = W13[e, :cfg.I] @ X[t], W13[e, cfg.I:] @ X[t]
+            h = (g / (1 + np.exp(-g)) * u).astype(np.float32)
+            # h is re-quantised from fp32 (not bf16) per 128-group with a power-of-two scale
+            amax = np.abs(h).reshape(-1, 128).max(1)
+            sc = np.array([2.0 ** np.ceil(np.log2(np.float32(a) / np.float32(448))) if a > 0 else 1.0
+                           for a in amax])
+            hd = dec(np.vectorize(oracle.e4m3_encode)((h / np.repeat(sc, 128)).astype(np.float32)))
+            ref[t] += r["w"][t, j] * (W2[e] @ (hd * np.repeat(sc, 128)))
+    np.testing.assert_allclose(r["out"], ref, rtol=2e-5, atol=2e-5 * np.abs(ref).max())
+
+
 def test_weight_quant_blocks():
     rng = np.random.default_rng(4)
     w = mi.f32_to_bf16(rng.standard_normal((2, 256, 384)).astype(np.float32) * 0.02)
