@@ -146,9 +146,9 @@ def oracle_inputs(cfg, L):
     import oracle
 
     if cfg.fp8:
-        w13q, w13s = oracle.quant_weight_fp8(L["w13"])
-        w2q, w2s = oracle.quant_weight_fp8(L["w2"])
-        return {"fp8": (w13q, w13s, w2q, w2s)}
+        w13q, w13s = oracle.quant_weight_fp8(L["w13"], ue8m0=cfg.ue8m0)
+        w2q, w2s = oracle.quant_weight_fp8(L["w2"], ue8m0=cfg.ue8m0)
+        return {"fp8": (w13q, w13s, w2q, w2s), "ue8m0": cfg.ue8m0}
     return {"w13": L["w13"], "w2": L["w2"]}
 
 
@@ -240,15 +240,17 @@ def gpu_arm(args, cfg):
     bias = torch.from_numpy(L["bias"]).cuda()
     w13, w2 = bf(L["w13"]), bf(L["w2"])
     d = (cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
-    dt = moe.MOE_DTYPE_FP8_E4M3 if cfg.fp8 else moe.MOE_DTYPE_BF16
+    dt = (moe.MOE_DTYPE_FP8_E4M3_UE8M0 if cfg.ue8m0 else moe.MOE_DTYPE_FP8_E4M3) if cfg.fp8 \
+        else moe.MOE_DTYPE_BF16
+    sfmt = moe.MOE_SCALE_UE8M0 if cfg.ue8m0 else moe.MOE_SCALE_F32
     if cfg.fp8:
-        # one-time weight preparation (untimed): e4m3 with one fp32 scale per 128 x 128 block
+        # one-time weight preparation (untimed): e4m3 with one scale per 128 x 128 block
         w13q = torch.empty(cfg.E, 2 * cfg.I, cfg.H, dtype=torch.uint8, device="cuda")
         w13s = torch.empty(cfg.E, 2 * cfg.I // 128, cfg.H // 128, dtype=torch.float32, device="cuda")
         w2q = torch.empty(cfg.E, cfg.H, cfg.I, dtype=torch.uint8, device="cuda")
         w2s = torch.empty(cfg.E, cfg.H // 128, cfg.I // 128, dtype=torch.float32, device="cuda")
-        moe.moe_quantize_weight_fp8(w13, cfg.E, 2 * cfg.I, cfg.H, w13q, w13s)
-        moe.moe_quantize_weight_fp8(w2, cfg.E, cfg.H, cfg.I, w2q, w2s)
+        moe.moe_quantize_weight_fp8_fmt(w13, cfg.E, 2 * cfg.I, cfg.H, w13q, w13s, sfmt)
+        moe.moe_quantize_weight_fp8_fmt(w2, cfg.E, cfg.H, cfg.I, w2q, w2s, sfmt)
         torch.cuda.synchronize()
         del w13, w2
     ws_bytes = moe.moe_workspace_size(d, dt)
@@ -260,7 +262,10 @@ def gpu_arm(args, cfg):
 
     def step(xin=None):
         xin = x if xin is None else xin
-        if cfg.fp8:
+        if cfg.fp8 and cfg.ue8m0:
+            moe.moe_forward_fp8_ue8m0(xin, wr, bias, w13q, w13s, w2q, w2s, d, moe.MOE_EPILOGUE_SWIGLU,
+                                      out, ws, ws_bytes)
+        elif cfg.fp8:
             moe.moe_forward_fp8(xin, wr, bias, w13q, w13s, w2q, w2s, d, out, ws, ws_bytes)
         else:
             moe.moe_forward(xin, wr, bias, w13, w2, d, out, ws, ws_bytes)
@@ -344,8 +349,13 @@ def gpu_arm(args, cfg):
         with torch.cuda.stream(streams[j]):
             if cfg.fp8:
                 xs_dev[j].view(torch.int16).copy_(x_host.view(cfg.T, cfg.H), non_blocking=True)
-                moe.moe_forward_fp8(xs_dev[j], wr, bias, w13q, w13s, w2q, w2s, d, outs_dev[j], wss[j],
-                                    ws_bytes, stream=streams[j])
+                if cfg.ue8m0:
+                    moe.moe_forward_fp8_ue8m0(xs_dev[j], wr, bias, w13q, w13s, w2q, w2s, d,
+                                              moe.MOE_EPILOGUE_SWIGLU, outs_dev[j], wss[j], ws_bytes,
+                                              stream=streams[j])
+                else:
+                    moe.moe_forward_fp8(xs_dev[j], wr, bias, w13q, w13s, w2q, w2s, d, outs_dev[j],
+                                        wss[j], ws_bytes, stream=streams[j])
                 outs_host[j].copy_(outs_dev[j].view(torch.int16).view(-1), non_blocking=True)
             else:  # the C ABI's host-buffer entry point does both copies on its stream
                 moe.moe_forward_hostio(x_host, wr, bias, w13, w2, d, outs_host[j], wss[j],
@@ -397,7 +407,9 @@ def gpu_arm(args, cfg):
         pk, pk_burst = ratio * peaks["bf16_tflops_sustained"], ratio * peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                 "traffic": kernel_traffic(cfg.name, "gemm1"),
-                "kernel": ("gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)" if cfg.fp8
+                "kernel": ("gemm_mx_kernel<SwiGLU> (block-scaled FP8 GEMM1 + SwiGLU + h quantisation)"
+                           if cfg.ue8m0 else
+                           "gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)" if cfg.fp8
                            else "gemm_rows_kernel<SwiGLU,256> (GEMM1 + SwiGLU, rows gathered)"),
                 "algorithmic_flops_per_launch": g1_flops,
                 "peak_source": f"{peak_src} bf16 x {ratio:g} (sustained; burst {pk_burst:.1f} -> frac "

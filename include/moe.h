@@ -61,7 +61,13 @@ typedef enum {
   MOE_ERR_TIMEOUT = 5             /* a bounded device-side wait ran out */
 } moe_status_t;
 
-typedef enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 } moe_dtype_t;
+/* MOE_DTYPE_FP8_E4M3_UE8M0: e4m3 operands whose scales are powers of two
+ * (MOE_SCALE_UE8M0), which the block-scaled tensor-core MMA applies itself. */
+typedef enum {
+  MOE_DTYPE_BF16 = 0,
+  MOE_DTYPE_FP8_E4M3 = 1,
+  MOE_DTYPE_FP8_E4M3_UE8M0 = 2
+} moe_dtype_t;
 
 /* GEMM epilogues. The gated ones compute act(g) * u from the gate projection
  * g and the up projection u ([X] "Experts backends": experts with a gated
@@ -75,6 +81,12 @@ typedef enum {
   MOE_EPILOGUE_GEGLU = 2,
   MOE_EPILOGUE_REGLU = 3
 } moe_epilogue_t;
+
+/* FP8 scale formats: fp32 values, or powers of two (UE8M0: the 8-bit
+ * exponent format float8_e8m0fnu of [X] "UE8M0 scale format", 2^(code-127)).
+ * With UE8M0 a scale is the smallest power of two >= amax / 448 (that fp32
+ * quotient), clamped to 2^-127..2^127; it is still passed as an fp32 value. */
+typedef enum { MOE_SCALE_F32 = 0, MOE_SCALE_UE8M0 = 1 } moe_scale_fmt_t;
 
 typedef struct {
   int32_t T, H, I, E, k;
@@ -190,6 +202,8 @@ moe_status_t moe_permute_noalloc(const int32_t* ids_dev, moe_dims_t d, int32_t* 
  *          permutation's row gather done inside the GEMM (rows outside
  *          [0, a_src_rows) read as zeros). Rows-per-expert bounds <= 64 with
  *          a_rows take the large-M kernel.
+ *   dt = MOE_DTYPE_FP8_E4M3_UE8M0: the scales are powers of two and the
+ *          block-scaled MMA applies them (no row gather, plain needs N % 256 == 0)
  *   B_dev  [E, N or 2N, K] K-major (bf16, or e4m3 with b_scales fp32
  *          [E, rows/128, K/128], one scale per 128 x 128 block, [F])
  *   C_dev  bf16 [M_total, N]; for FP8 gated epilogues with c_scales != NULL, C is
@@ -251,6 +265,19 @@ moe_status_t moe_forward_fp8(const void* x_dev, const void* wr_dev, const float*
                              const float* w2s_dev, moe_dims_t d, void* out_dev, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* The FP8 layer with power-of-two (UE8M0) scales ([X] "FP8 and FP4 quantized
+ * experts", "UE8M0 scale format"): weights quantised with
+ * moe_quantize_weight_fp8_fmt(..., MOE_SCALE_UE8M0); x and the hidden
+ * activations are quantised the same way inside; both expert GEMMs run on
+ * the block-scaled MMA (kind::mxf8f6f4 with E8M0 scales), so the scales need
+ * no CUDA-core promotion. act as for moe_forward_gated. Buffers as for
+ * moe_forward_fp8; ws >= moe_workspace_size(d, MOE_DTYPE_FP8_E4M3_UE8M0). */
+moe_status_t moe_forward_fp8_ue8m0(const void* x_dev, const void* wr_dev, const float* bias_dev,
+                                   const void* w13q_dev, const float* w13s_dev,
+                                   const void* w2q_dev, const float* w2s_dev, moe_dims_t d,
+                                   moe_epilogue_t act, void* out_dev, void* ws, size_t ws_bytes,
+                                   void* stream);
+
 /* moe_forward_fp8 with the expert activation chosen (as moe_forward_gated;
  * the activation's output is what gets quantised per 128-group). */
 moe_status_t moe_forward_fp8_gated(const void* x_dev, const void* wr_dev, const float* bias_dev,
@@ -280,6 +307,15 @@ moe_status_t moe_quantize_act_fp8(const void* x_dev, int64_t rows, int64_t cols,
  * s_dev fp32 [nb, rows/128, cols/128]. A one-time preparation step. */
 moe_status_t moe_quantize_weight_fp8(const void* w_dev, int64_t nb, int64_t rows, int64_t cols,
                                      void* q_dev, float* s_dev, void* stream);
+
+/* moe_quantize_act_fp8 / moe_quantize_weight_fp8 with the scale format
+ * chosen (MOE_SCALE_F32: what those two do; MOE_SCALE_UE8M0: power-of-two
+ * scales, see moe_scale_fmt_t). Same buffers and layouts. */
+moe_status_t moe_quantize_act_fp8_fmt(const void* x_dev, int64_t rows, int64_t cols, void* q_dev,
+                                      float* s_dev, moe_scale_fmt_t fmt, void* stream);
+moe_status_t moe_quantize_weight_fp8_fmt(const void* w_dev, int64_t nb, int64_t rows,
+                                         int64_t cols, void* q_dev, float* s_dev,
+                                         moe_scale_fmt_t fmt, void* stream);
 
 /* Reads the workspace's device status word (MOE_OK or MOE_ERR_TIMEOUT) into
  * *status_out. Synchronises the device (a blocking copy); not for hot loops. */

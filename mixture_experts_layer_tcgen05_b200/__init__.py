@@ -22,6 +22,8 @@ __all__ = [
     "MOE_ERR_UNSUPPORTED_DEVICE", "MOE_ERR_WORKSPACE", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
     "MOE_DTYPE_BF16", "MOE_DTYPE_FP8_E4M3", "MOE_EPILOGUE_NONE", "MOE_EPILOGUE_SWIGLU",
     "MOE_EPILOGUE_GEGLU", "MOE_EPILOGUE_REGLU", "moe_forward_gated", "moe_forward_fp8_gated",
+    "MOE_SCALE_F32", "MOE_SCALE_UE8M0", "moe_quantize_act_fp8_fmt", "moe_quantize_weight_fp8_fmt",
+    "MOE_DTYPE_FP8_E4M3_UE8M0", "moe_forward_fp8_ue8m0",
     "moe_last_error", "moe_abi_version", "moe_launch_count", "moe_workspace_size",
     "moe_workspace_layout", "moe_route_topk", "moe_topk_from_logits", "moe_permute",
     "moe_permute_noalloc",
@@ -32,8 +34,9 @@ __all__ = [
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_DEVICE = 0, 1, 2
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 3, 4, 5
-MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3 = 0, 1
+MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3, MOE_DTYPE_FP8_E4M3_UE8M0 = 0, 1, 2
 MOE_EPILOGUE_NONE, MOE_EPILOGUE_SWIGLU, MOE_EPILOGUE_GEGLU, MOE_EPILOGUE_REGLU = 0, 1, 2, 3
+MOE_SCALE_F32, MOE_SCALE_UE8M0 = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libmoe_b200.so")
@@ -77,8 +80,12 @@ _SIGS = {
     "moe_forward_gated": (_i32, [_vp, _vp, _vp, _vp, _vp, Dims, _i32, _vp, _vp, _sz, _vp]),
     "moe_forward_fp8_gated": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _i32, _vp, _vp, _sz,
                                      _vp]),
+    "moe_forward_fp8_ue8m0": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _i32, _vp, _vp, _sz,
+                                     _vp]),
     "moe_quantize_act_fp8": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "moe_quantize_weight_fp8": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "moe_quantize_act_fp8_fmt": (_i32, [_vp, _i64, _i64, _vp, _vp, _i32, _vp]),
+    "moe_quantize_weight_fp8_fmt": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp]),
     "moe_get_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_clear_device_status": (_i32, [_vp, _vp]),
     "moe_set_stage_events": (_i32, [ctypes.POINTER(_vp), _i32]),
@@ -224,6 +231,13 @@ def moe_forward_fp8_gated(x, wr, bias, w13q, w13s, w2q, w2s, d, act, out, ws, ws
                                        _nbytes(ws, ws_bytes), _s(stream)))
 
 
+def moe_forward_fp8_ue8m0(x, wr, bias, w13q, w13s, w2q, w2s, d, act, out, ws, ws_bytes=None,
+                          stream=None):
+    _check(lib().moe_forward_fp8_ue8m0(_p(x), _p(wr), _p(bias), _p(w13q), _p(w13s), _p(w2q),
+                                       _p(w2s), _dims(d), int(act), _p(out), _p(ws),
+                                       _nbytes(ws, ws_bytes), _s(stream)))
+
+
 def moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws, ws_bytes=None, stream=None):
     _check(lib().moe_forward_hostio(_p(x_host), _p(wr), _p(bias), _p(w13), _p(w2), _dims(d),
                                     _p(out_host), _p(ws), _nbytes(ws, ws_bytes), _s(stream)))
@@ -235,6 +249,15 @@ def moe_quantize_act_fp8(x, rows, cols, q, s, stream=None):
 
 def moe_quantize_weight_fp8(w, nb, rows, cols, q, s, stream=None):
     _check(lib().moe_quantize_weight_fp8(_p(w), nb, rows, cols, _p(q), _p(s), _s(stream)))
+
+
+def moe_quantize_act_fp8_fmt(x, rows, cols, q, s, fmt, stream=None):
+    _check(lib().moe_quantize_act_fp8_fmt(_p(x), rows, cols, _p(q), _p(s), int(fmt), _s(stream)))
+
+
+def moe_quantize_weight_fp8_fmt(w, nb, rows, cols, q, s, fmt, stream=None):
+    _check(lib().moe_quantize_weight_fp8_fmt(_p(w), nb, rows, cols, _p(q), _p(s), int(fmt),
+                                             _s(stream)))
 
 
 def moe_get_device_status(ws) -> int:

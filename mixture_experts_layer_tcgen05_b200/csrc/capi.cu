@@ -43,10 +43,14 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_
                                     int act, void* C, float* c_scales,
                                     int max_rows_per_expert, int32_t* status, cudaStream_t s,
                                     const char** why);
+cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const void* B,
+                                   const float* b_scales, const int32_t* offsets, int M_total,
+                                   int E, int N, int K, int act, void* Cout, float* c_scales,
+                                   int32_t* status, cudaStream_t s, const char** why);
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
-                             const int32_t* row_map, cudaStream_t s);
+                             const int32_t* row_map, bool ue8m0, cudaStream_t s);
 cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
-                                float* sc, cudaStream_t s);
+                                float* sc, bool ue8m0, cudaStream_t s);
 
 int64_t noalloc_scratch_capacity();
 cudaError_t launch_permute_noalloc(const int32_t* ids, int T, int H, int E, int k, int32_t* offsets,
@@ -218,14 +222,14 @@ int64_t moe_launch_count(void) { return g_launches.load(); }
 
 size_t moe_workspace_size(moe_dims_t d, moe_dtype_t dt) {
   if (check_dims(d, true) != MOE_OK) return 0;
-  if (dt != MOE_DTYPE_BF16 && dt != MOE_DTYPE_FP8_E4M3) return 0;
+  if (dt < MOE_DTYPE_BF16 || dt > MOE_DTYPE_FP8_E4M3_UE8M0) return 0;
   return (size_t)layout(d, dt).total;
 }
 
 moe_status_t moe_workspace_layout(moe_dims_t d, moe_dtype_t dt, moe_ws_layout_t* out) {
   MOE_TRY(check_dims(d, true));
   if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
-  if (dt != MOE_DTYPE_BF16 && dt != MOE_DTYPE_FP8_E4M3) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
+  if (dt < MOE_DTYPE_BF16 || dt > MOE_DTYPE_FP8_E4M3_UE8M0) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
   *out = layout(d, dt);
   return ok();
 }
@@ -339,14 +343,16 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
   if (N < 128 || N % 128 || K < 128 || K % 128)
     return fail(MOE_ERR_INVALID_ARG, "N and K must be positive multiples of 128 (N=%d K=%d)", N, K);
   if (ep < MOE_EPILOGUE_NONE || ep > MOE_EPILOGUE_REGLU) return fail(MOE_ERR_INVALID_ARG, "bad epilogue");
-  if (dt != MOE_DTYPE_BF16 && dt != MOE_DTYPE_FP8_E4M3) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
+  if (dt < MOE_DTYPE_BF16 || dt > MOE_DTYPE_FP8_E4M3_UE8M0) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
+  if (dt == MOE_DTYPE_FP8_E4M3_UE8M0 && a_rows)
+    return fail(MOE_ERR_INVALID_ARG, "the block-scaled GEMM takes no row gather");
   MOE_TRY(check_ptr(A, "A"));
   MOE_TRY(check_ptr(a_rows, "a_rows", true));
   if (a_rows && a_src_rows < 1) return fail(MOE_ERR_INVALID_ARG, "a_src_rows must be >= 1 with a_rows");
   MOE_TRY(check_ptr(B, "B"));
   MOE_TRY(check_ptr(offsets, "expert_offsets"));
   MOE_TRY(check_ptr(C, "C"));
-  if (dt == MOE_DTYPE_FP8_E4M3) {
+  if (dt != MOE_DTYPE_BF16) {
     MOE_TRY(check_ptr(a_scales, "a_scales"));
     MOE_TRY(check_ptr(b_scales, "b_scales"));
     MOE_TRY(check_ptr(c_scales, "c_scales", true));
@@ -363,11 +369,15 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
                                  N, K, (int)ep, C,
                                  max_rows_per_expert, at<int32_t>(ws, 0), at<char>(ws, 256),
                                  ws_bytes - 256, static_cast<cudaStream_t>(stream), &why);
-  else
+  else if (dt == MOE_DTYPE_FP8_E4M3)
     e = launch_grouped_gemm_fp8(A, a_rows, a_rows ? a_src_rows : M_total, a_scales, B, b_scales,
                                 offsets, M_total, E, N, K,
                                 (int)ep, C, c_scales, max_rows_per_expert,
                                 at<int32_t>(ws, 0), static_cast<cudaStream_t>(stream), &why);
+  else
+    e = launch_grouped_gemm_mx(A, a_scales, B, b_scales, offsets, M_total, E, N, K, (int)ep, C,
+                               c_scales, at<int32_t>(ws, 0), static_cast<cudaStream_t>(stream),
+                               &why);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "grouped GEMM: %s %s", cudaGetErrorString(e), why);
   return ok();
 }
@@ -448,18 +458,30 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
     void* hq = at<void>(ws, L.hq);
     float* hs = at<float>(ws, L.hs);
     // x is quantised once per token, then its codes and scales are permuted
-    if ((e = launch_quant_act(x, T, H, xq, xs, nullptr, s)) != cudaSuccess)
+    const bool ue8m0 = dt == MOE_DTYPE_FP8_E4M3_UE8M0;
+    if ((e = launch_quant_act(x, T, H, xq, xs, nullptr, ue8m0, s)) != cudaSuccess)
       return cuda_fail(e, "activation quantisation");
     if ((e = permute_gather(xq, H, xq_perm, xs, (H / 128) * 4, xs_perm)) != cudaSuccess)
       return cuda_fail(e, "permute");
     record(s, 2);
-    if ((e = launch_grouped_gemm_fp8(xq_perm, nullptr, R, xs_perm, w13, w13s, offsets, R, E, I, H,
-                                     act, hq, hs, T, status, s, &why)) != cudaSuccess)
-      return fail(MOE_ERR_CUDA, "FP8 GEMM1: %s %s", cudaGetErrorString(e), why);
-    record(s, 3);
-    if ((e = launch_grouped_gemm_fp8(hq, nullptr, R, hs, w2, w2s, offsets, R, E, H, I, 0, y_perm,
-                                     nullptr, T, status, s, &why)) != cudaSuccess)
-      return fail(MOE_ERR_CUDA, "FP8 GEMM2: %s %s", cudaGetErrorString(e), why);
+    if (ue8m0) {
+      // power-of-two scales: the block-scaled tensor-core path, no promotion
+      if ((e = launch_grouped_gemm_mx(xq_perm, xs_perm, w13, w13s, offsets, R, E, I, H, act, hq, hs,
+                                      status, s, &why)) != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "FP8 GEMM1: %s %s", cudaGetErrorString(e), why);
+      record(s, 3);
+      if ((e = launch_grouped_gemm_mx(hq, hs, w2, w2s, offsets, R, E, H, I, 0, y_perm, nullptr,
+                                      status, s, &why)) != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "FP8 GEMM2: %s %s", cudaGetErrorString(e), why);
+    } else {
+      if ((e = launch_grouped_gemm_fp8(xq_perm, nullptr, R, xs_perm, w13, w13s, offsets, R, E, I, H,
+                                       act, hq, hs, T, status, s, &why)) != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "FP8 GEMM1: %s %s", cudaGetErrorString(e), why);
+      record(s, 3);
+      if ((e = launch_grouped_gemm_fp8(hq, nullptr, R, hs, w2, w2s, offsets, R, E, H, I, 0, y_perm,
+                                       nullptr, T, status, s, &why)) != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "FP8 GEMM2: %s %s", cudaGetErrorString(e), why);
+    }
     record(s, 4);
   }
   if ((e = launch_combine(y_perm, tw, inv_perm, T, H, k, out, status, s)) != cudaSuccess)
@@ -519,6 +541,27 @@ moe_status_t moe_forward_fp8_gated(const void* x, const void* wr, const float* b
                       static_cast<cudaStream_t>(stream));
 }
 
+moe_status_t moe_forward_fp8_ue8m0(const void* x, const void* wr, const float* bias,
+                                   const void* w13q, const float* w13s, const void* w2q,
+                                   const float* w2s, moe_dims_t d, moe_epilogue_t act, void* out,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_dims(d, true));
+  MOE_TRY(check_act(act));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(wr, "w_router"));
+  MOE_TRY(check_ptr(bias, "bias", true));
+  MOE_TRY(check_ptr(w13q, "w13q"));
+  MOE_TRY(check_ptr(w13s, "w13s"));
+  MOE_TRY(check_ptr(w2q, "w2q"));
+  MOE_TRY(check_ptr(w2s, "w2s"));
+  MOE_TRY(check_ptr(out, "out"));
+  if (d.H % 256) return fail(MOE_ERR_INVALID_ARG, "the FP8 layer needs H %% 256 == 0 (got %d)", d.H);
+  MOE_TRY(check_ws(d, MOE_DTYPE_FP8_E4M3_UE8M0, ws, ws_bytes));
+  MOE_TRY(check_device());
+  return forward_impl(x, wr, bias, w13q, w13s, w2q, w2s, d, (int)act, out, ws,
+                      MOE_DTYPE_FP8_E4M3_UE8M0, static_cast<cudaStream_t>(stream));
+}
+
 moe_status_t moe_forward_fp8(const void* x, const void* wr, const float* bias, const void* w13q,
                              const float* w13s, const void* w2q, const float* w2s, moe_dims_t d,
                              void* out, void* ws, size_t ws_bytes, void* stream) {
@@ -552,29 +595,43 @@ moe_status_t moe_forward_hostio(const void* x_host, const void* wr, const float*
   return ok();
 }
 
-moe_status_t moe_quantize_act_fp8(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
-                                  void* stream) {
+moe_status_t moe_quantize_act_fp8_fmt(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
+                                      moe_scale_fmt_t fmt, void* stream) {
   if (rows < 1 || cols < 128 || cols % 128) return fail(MOE_ERR_INVALID_ARG, "rows >= 1, cols a multiple of 128");
+  if (fmt != MOE_SCALE_F32 && fmt != MOE_SCALE_UE8M0) return fail(MOE_ERR_INVALID_ARG, "bad scale format");
   MOE_TRY(check_ptr(x, "x"));
   MOE_TRY(check_ptr(q, "q"));
   MOE_TRY(check_ptr(sc, "s"));
   MOE_TRY(check_device());
-  cudaError_t e = launch_quant_act(x, rows, cols, q, sc, nullptr, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_quant_act(x, rows, cols, q, sc, nullptr, fmt == MOE_SCALE_UE8M0,
+                                   static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "activation quantisation");
+  return ok();
+}
+
+moe_status_t moe_quantize_act_fp8(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
+                                  void* stream) {
+  return moe_quantize_act_fp8_fmt(x, rows, cols, q, sc, MOE_SCALE_F32, stream);
+}
+
+moe_status_t moe_quantize_weight_fp8_fmt(const void* w, int64_t nb, int64_t rows, int64_t cols,
+                                         void* q, float* sc, moe_scale_fmt_t fmt, void* stream) {
+  if (nb < 1 || rows < 128 || rows % 128 || cols < 128 || cols % 128)
+    return fail(MOE_ERR_INVALID_ARG, "nb >= 1, rows and cols multiples of 128");
+  if (fmt != MOE_SCALE_F32 && fmt != MOE_SCALE_UE8M0) return fail(MOE_ERR_INVALID_ARG, "bad scale format");
+  MOE_TRY(check_ptr(w, "w"));
+  MOE_TRY(check_ptr(q, "q"));
+  MOE_TRY(check_ptr(sc, "s"));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_quant_weight(w, nb, rows, cols, q, sc, fmt == MOE_SCALE_UE8M0,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "weight quantisation");
   return ok();
 }
 
 moe_status_t moe_quantize_weight_fp8(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                      float* sc, void* stream) {
-  if (nb < 1 || rows < 128 || rows % 128 || cols < 128 || cols % 128)
-    return fail(MOE_ERR_INVALID_ARG, "nb >= 1, rows and cols multiples of 128");
-  MOE_TRY(check_ptr(w, "w"));
-  MOE_TRY(check_ptr(q, "q"));
-  MOE_TRY(check_ptr(sc, "s"));
-  MOE_TRY(check_device());
-  cudaError_t e = launch_quant_weight(w, nb, rows, cols, q, sc, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "weight quantisation");
-  return ok();
+  return moe_quantize_weight_fp8_fmt(w, nb, rows, cols, q, sc, MOE_SCALE_F32, stream);
 }
 
 moe_status_t moe_get_device_status(const void* ws, int32_t* status_out) {

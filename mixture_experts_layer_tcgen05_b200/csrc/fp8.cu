@@ -3,7 +3,8 @@
 // "Fine-grained FP8" (HF Transformers docs), opening list: weights are
 // quantised to 8 bits per 128 x 128 block; activations per token per group
 // of 128 input channels, dynamically. Scale rule (both): s = amax / 448 in
-// fp32 (IEEE division), s = 1 for an all-zero group, code = e4m3 of v / s
+// fp32 (IEEE division), or the smallest power of two >= it with UE8M0
+// scales, s = 1 for an all-zero group, code = e4m3 of v / s
 // rounded to nearest even (the hardware cvt with satfinite; |v / s| <= 448
 // up to one rounding, so saturation never changes a value).
 #include <cuda_fp8.h>
@@ -12,8 +13,17 @@
 
 namespace moe {
 
-__device__ __forceinline__ float group_scale(float amax) {
-  return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+// ue8m0: power-of-two scales (the UE8M0 scale format of "Experts backends"):
+// the smallest 2^p >= amax / 448 (that fp32 quotient), p clamped to
+// [-127, 127]; dividing by it only shifts exponents.
+__device__ __forceinline__ float group_scale(float amax, bool ue8m0) {
+  if (!(amax > 0.0f)) return 1.0f;
+  const float r = __fdiv_rn(amax, 448.0f);
+  if (!ue8m0) return r;
+  int e;
+  const float m = frexpf(r, &e);  // r = m * 2^e, m in [0.5, 1)
+  const int p2 = min(max(m == 0.5f ? e - 1 : e, -127), 127);
+  return ldexpf(1.0f, p2);
 }
 
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
@@ -29,7 +39,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint4* __restrict_
                                                         int64_t cols,
                                                         const int32_t* __restrict__ row_map,
                                                         uint2* __restrict__ q,
-                                                        float* __restrict__ s) {
+                                                        float* __restrict__ s, bool ue8m0) {
   const int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (p >= rows) return;
@@ -48,7 +58,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint4* __restrict_
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
     for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const float sc = group_scale(amax);
+    const float sc = group_scale(amax, ue8m0);
     if (on) {
       qr[v] = make_uint2(e4m3x4(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc), __fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc)),
                          e4m3x4(__fdiv_rn(f[4], sc), __fdiv_rn(f[5], sc), __fdiv_rn(f[6], sc), __fdiv_rn(f[7], sc)));
@@ -61,7 +71,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint4* __restrict_
 __global__ void __launch_bounds__(256) quant_weight_kernel(const __nv_bfloat16* __restrict__ w,
                                                            int64_t rows, int64_t cols,
                                                            uint8_t* __restrict__ q,
-                                                           float* __restrict__ s) {
+                                                           float* __restrict__ s, bool ue8m0) {
   const int64_t RB = rows / 128, CB = cols / 128;
   const int64_t blk = blockIdx.x;
   const int64_t b = blk / (RB * CB), rb = (blk / CB) % RB, cb = blk % CB;
@@ -90,7 +100,7 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const __nv_bfloat16* 
   amax = red[0];
 #pragma unroll
   for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
-  const float sc = group_scale(amax);
+  const float sc = group_scale(amax, ue8m0);
   uint32_t* qp = reinterpret_cast<uint32_t*>(q + base + (int64_t)r * cols + c0);
 #pragma unroll
   for (int i = 0; i < 64; i += 4)
@@ -100,18 +110,18 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const __nv_bfloat16* 
 }
 
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
-                             const int32_t* row_map, cudaStream_t s) {
+                             const int32_t* row_map, bool ue8m0, cudaStream_t s) {
   quant_act_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, s>>>(
-      static_cast<const uint4*>(x), rows, cols, row_map, static_cast<uint2*>(q), sc);
+      static_cast<const uint4*>(x), rows, cols, row_map, static_cast<uint2*>(q), sc, ue8m0);
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
-                                float* sc, cudaStream_t s) {
+                                float* sc, bool ue8m0, cudaStream_t s) {
   const int64_t blocks = nb * (rows / 128) * (cols / 128);
   quant_weight_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), rows,
-                                                       cols, static_cast<uint8_t*>(q), sc);
+                                                       cols, static_cast<uint8_t*>(q), sc, ue8m0);
   note_launch();
   return cudaGetLastError();
 }

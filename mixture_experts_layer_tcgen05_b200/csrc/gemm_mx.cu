@@ -1,0 +1,440 @@
+// Grouped GEMM with FP8 operands and power-of-two (UE8M0) block scales on the
+// sm_100a block-scaled tensor-core path.
+//
+// "Experts backends" (HF Transformers docs), "FP8 and FP4 quantized experts"
+// and "UE8M0 scale format": with scales stored as 8-bit exponents
+// (float8_e8m0fnu) Blackwell's block-scaled MMA applies them itself, so
+// nothing is promoted on CUDA cores: tcgen05.mma kind::mxf8f6f4.block_scale
+// multiplies e4m3 x e4m3 with one E8M0 scale per row (of A) and per column
+// (of B) per 32-wide K step, accumulating in fp32 across the whole K in TMEM.
+// The layer's scales cover 128-wide K blocks (and 128-row weight blocks), so
+// each 128-K stage repeats a row's scale over its four K steps.
+//
+// Scale factors reach TMEM by tcgen05.cp from a 512-byte shared chunk per
+// 128 rows: the 16 bytes at offset 16*r hold, for rows r, r+32, r+64, r+96
+// (in that order, 4 bytes each), the scales of the stage's four K steps; the
+// copy (32 lanes x 128 bits, replicated to the four lane quarters) puts row
+// group g in TMEM column g and K step j in byte j, which the MMA selects
+// with its scale-factor ids.
+//
+// Warp roles (320 threads): warp 0 TMA producer, all 32 lanes building the
+// scale chunks; warp 1 TMEM allocator + MMA issuer; warps 2..9 epilogue.
+// One accumulator (256 TMEM columns, the rest holds the scale-factor ring):
+// the eight epilogue warps drain it into registers (warp w: lane quarter
+// w % 4, column half (w - 2) / 4) and release it before the SwiGLU /
+// re-quantisation math, so the next tile's MMAs overlap that work.
+#include <cuda_fp8.h>
+
+#include "gemm_common.cuh"
+
+namespace moe {
+namespace ggmx {
+
+constexpr int BM = 128;
+constexpr int BK = 128;  // fp8 elements per stage = one 128-byte swizzle row = one scale block
+constexpr int UK = 32;   // K per block-scaled MMA (8-bit inputs)
+constexpr int BN = 256;
+constexpr int kThreads = 320;
+constexpr int kTileA = BM * BK;  // 16 KB
+constexpr int kTileB = BN * BK;  // 32 KB
+constexpr int kStage = kTileA + kTileB;
+constexpr int STAGES = 4;
+constexpr int kSfA = 512;        // scale chunk bytes for 128 rows of A
+constexpr int kSfStage = 3 * kSfA;  // A chunk + two B chunks
+constexpr int kMaxE = 1024;
+constexpr int kSfCol0 = 256;     // TMEM columns of the scale-factor ring
+constexpr int kSfColsPerStage = 16;
+constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + (size_t)STAGES * kSfStage + 256 +
+                         (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
+
+struct Args {
+  const int32_t* offsets;
+  int E, K, ldc, NT, b_rows, up_off, band, M_total;
+  int kblocks;            // K / 128
+  int b_nblk;             // 128-row blocks of B per expert
+  void* C;                // bf16 [M_total, ldc], or e4m3 when c_scales != nullptr
+  float* c_scales;        // power-of-two scales of C's 128-groups
+  const float* a_scales;  // [M_total, kblocks], powers of two
+  const float* b_scales;  // [E, b_nblk, kblocks], powers of two
+  int32_t* status;
+};
+
+// E8M0 code of a power-of-two fp32 scale (2^-127 is the one subnormal one).
+__device__ __forceinline__ uint32_t e8m0_code(float s) {
+  const uint32_t b = __float_as_uint(s);
+  const uint32_t ex = (b >> 23) & 0xFFu;
+  return ex ? ex : 0u;
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+// Smallest power of two >= amax / 448 (fp32 quotient), 1 for an all-zero group.
+__device__ __forceinline__ float pow2_scale(float amax) {
+  if (!(amax > 0.0f)) return 1.0f;
+  int e;
+  const float m = frexpf(__fdiv_rn(amax, 448.0f), &e);
+  return ldexpf(1.0f, min(max(m == 0.5f ? e - 1 : e, -127), 127));
+}
+
+// Shared-memory descriptor of a scale chunk for tcgen05.cp: K-major, no
+// swizzle, 8-row core matrices of 16-byte rows stacked every 128 bytes.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address
+  d |= (uint64_t)(128u >> 4) << 16;         // leading byte offset (one core matrix along K)
+  d |= (uint64_t)(128u >> 4) << 32;         // stride byte offset: next 8 rows
+  d |= (uint64_t)1u << 46;                  // descriptor version (sm_100)
+  return d;                                 // layout bits 61-63 = 0: no swizzle
+}
+
+__device__ __forceinline__ void sf_copy(uint32_t tmem, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(desc) : "memory");
+}
+
+// Block-scaled instruction descriptor: e4m3 x e4m3, fp32 accumulate, E8M0
+// scales, scale-factor ids (the K step) for A and B.
+__host__ __device__ constexpr uint32_t mx_idesc(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4)                    // B scale-factor id
+         | (0u << 7) | (0u << 10)         // A, B formats: E4M3
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | (1u << 23)                     // scale format E8M0
+         | ((uint32_t)(M >> 4) << 24)     // M / 16
+         | (sf_id << 29);                 // A scale-factor id
+}
+
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// ACT: gated activation of the epilogue (kActNone: plain GEMM).
+template <int ACT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   Args args) {
+  constexpr bool SWIGLU = ACT != kActNone;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sf = smem + STAGES * kStage;  // [STAGES][A chunk, B chunk 0, B chunk 1]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sf + STAGES * kSfStage);
+  // bars: full[STAGES], empty[STAGES], accf, acce, drain, redbar[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(sf + STAGES * kSfStage + 256);
+  float* red = reinterpret_cast<float*>(tile_start + kMaxE + 1);  // [2 tiles][2 halves][BM]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = ptx::smem_addr(smem), sfbase = ptx::smem_addr(sf);
+  const uint32_t full0 = ptx::smem_addr(bars), empty0 = full0 + STAGES * 8;
+  const uint32_t accf = empty0 + STAGES * 8, acce = accf + 8, drain = acce + 8;
+  const uint32_t redbar0 = drain + 8;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full0 + s * 8, 1);
+      ptx::mbar_init(empty0 + s * 8, 1);
+    }
+    ptx::mbar_init(accf, 1);
+    ptx::mbar_init(acce, 8);
+    ptx::mbar_init(drain, 1);
+    ptx::mbar_init(redbar0, 256);
+    ptx::mbar_init(redbar0 + 8, 256);
+    ptx::fence_barrier_init();
+    ptx::tma_prefetch_desc(&tmA);
+    ptx::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 2) gg::build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = tile_start[args.E];
+  const int nkb = args.kblocks;
+
+  auto decode = [&](int tile, int& e, int& m, int& n) {
+    e = gg::find_expert(tile_start, args.E, tile);
+    const int local = tile - tile_start[e];
+    const int cnt = args.offsets[e + 1] - args.offsets[e];
+    const int mt = (cnt + BM - 1) / BM;
+    const int bsz = args.band * args.NT;
+    const int b = local / bsz;
+    const int rows = min(args.band, mt - b * args.band);
+    const int l2 = local - b * bsz;
+    n = l2 / rows;
+    m = b * args.band + l2 % rows;
+  };
+
+  if (warp == 0) {
+    // all lanes: scale chunks (lane l writes the 16 bytes of rows l + 32g);
+    // lane 0: barriers and TMA loads
+    int64_t issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      int e, m, n;
+      decode(tile, e, m, n);
+      const int row0 = args.offsets[e] + m * BM, row_end = args.offsets[e + 1];
+      int rb0, rb1, nb0, nb1;  // B rows of the two 128-row boxes and their scale blocks
+      if (SWIGLU) {
+        rb0 = e * args.b_rows + n * 128;
+        rb1 = rb0 + args.up_off;
+        nb0 = n;
+        nb1 = (args.up_off >> 7) + n;
+      } else {
+        rb0 = e * args.b_rows + n * BN;
+        rb1 = rb0 + 128;
+        nb0 = 2 * n;
+        nb1 = 2 * n + 1;
+      }
+      const float* sb0 = args.b_scales + ((int64_t)e * args.b_nblk + nb0) * nkb;
+      const float* sb1 = args.b_scales + ((int64_t)e * args.b_nblk + nb1) * nkb;
+      const float* sa[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int r = row0 + g * 32 + lane;
+        sa[g] = r < row_end ? args.a_scales + (int64_t)r * nkb : nullptr;  // rows past the expert: scale 1
+      }
+      for (int kb = 0; kb < nkb; ++kb, ++issued) {
+        const int s = (int)(issued % STAGES);
+        const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
+        int got = 1;
+        if (lane == 0) got = ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
+        }
+        // scale chunks of this stage
+        uint32_t w[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t c = sa[g] ? e8m0_code(sa[g][kb]) : 127u;
+          w[g] = c * 0x01010101u;  // the same scale for the stage's four K steps
+        }
+        unsigned char* sfs = sf + s * kSfStage;
+        *reinterpret_cast<uint4*>(sfs + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        const uint32_t c0 = e8m0_code(sb0[kb]) * 0x01010101u, c1 = e8m0_code(sb1[kb]) * 0x01010101u;
+        *reinterpret_cast<uint4*>(sfs + kSfA + lane * 16) = make_uint4(c0, c0, c0, c0);
+        *reinterpret_cast<uint4*>(sfs + 2 * kSfA + lane * 16) = make_uint4(c1, c1, c1, c1);
+        ptx::fence_proxy_async_smem();  // generic-proxy writes -> visible to tcgen05.cp
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t sa_ = sbase + s * kStage, sb_ = sa_ + kTileA;
+          ptx::mbar_arrive_expect_tx(full0 + s * 8, kStage);
+          ptx::tma_load_2d(sa_, &tmA, kb * BK, row0, full0 + s * 8);
+          ptx::tma_load_2d(sb_, &tmB, kb * BK, rb0, full0 + s * 8);
+          ptx::tma_load_2d(sb_ + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) gg::drain_loads<STAGES>(full0, issued, args.status);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int64_t consumed = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        // the single accumulator: wait until the epilogue has drained the previous tile
+        if (!ptx::mbar_wait(acce, acc_ph ^ 1, args.status, kSiteMmaAccEmpty)) break;
+        acc_ph ^= 1;
+        ptx::tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb, ++consumed) {
+          const int s = (int)(consumed % STAGES);
+          const uint32_t ph = (uint32_t)((consumed / STAGES) & 1);
+          if (!ptx::mbar_wait(full0 + s * 8, ph, args.status, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sfcol = tmem_base + kSfCol0 + s * kSfColsPerStage;
+          const uint32_t sfs = sfbase + s * kSfStage;
+          sf_copy(sfcol, sf_desc(sfs));                // A: columns 0..3
+          sf_copy(sfcol + 4, sf_desc(sfs + kSfA));     // B rows 0..127: columns 4..7
+          sf_copy(sfcol + 8, sf_desc(sfs + 2 * kSfA)); // B rows 128..255: columns 8..11
+          const uint32_t sa_ = sbase + s * kStage, sb_ = sa_ + kTileA;
+          const uint64_t da = ptx::sw128_kmajor_desc(sa_), db = ptx::sw128_kmajor_desc(sb_);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk)
+            mma_mx(tmem_base, da + (uint64_t)(kk * UK / 16), db + (uint64_t)(kk * UK / 16),
+                   mx_idesc(BM, BN, (uint32_t)kk), sfcol, sfcol + 4, (kb | kk) != 0);
+          ptx::mma_commit(empty0 + s * 8);
+        }
+        if (!ok) break;
+        ptx::mma_commit(accf);
+      }
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, args.status, kSiteDrain);
+    }
+  } else {
+    const int half = (warp - 2) >> 2;
+    const int q = warp & 3;
+    const int rl = q * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+    uint32_t acc_ph = 0;
+    int tile_iter = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tile_iter) {
+      const int tile_par = tile_iter & 1;
+      int e, m, n;
+      decode(tile, e, m, n);
+      const int row = args.offsets[e] + m * BM + rl;
+      const bool valid = row >= 0 && row < args.offsets[e + 1] && row < args.M_total;
+      if (!ptx::mbar_wait(accf, acc_ph, args.status, kSiteEpiAccFull)) break;
+      acc_ph ^= 1;
+      ptx::tc_fence_after();
+      // drain this thread's 128 accumulator columns, then release the accumulator
+      float acc[128];
+      if (SWIGLU) {
+        // gate cols [half*64, +64) -> acc[0..64), up cols [128 + half*64, +64) -> acc[64..128)
+#pragma unroll
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t g[32], u[32];
+          ptx::tmem_ld32(lane_addr + half * 64 + c, g);
+          ptx::tmem_ld32(lane_addr + 128 + half * 64 + c, u);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[c + i] = __uint_as_float(g[i]), acc[64 + c + i] = __uint_as_float(u[i]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld32(lane_addr + half * 128 + c, v);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[c + i] = __uint_as_float(v[i]);
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acce);
+      if (SWIGLU) {
+        float h[64];
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          h[i] = gated<ACT>(acc[i], acc[64 + i]);
+          amax = fmaxf(amax, fabsf(h[i]));
+        }
+        if (args.c_scales) {
+          // exchange the two halves' row maxima (all 256 epilogue threads arrive)
+          float* rb = red + tile_par * 2 * BM;
+          rb[half * BM + rl] = amax;
+          ptx::mbar_arrive(redbar0 + tile_par * 8);
+          if (!ptx::mbar_wait(redbar0 + tile_par * 8, (uint32_t)((tile_iter >> 1) & 1), args.status,
+                              kSiteEpiAccFull))
+            break;
+          amax = fmaxf(rb[rl], rb[BM + rl]);
+          const float sc = pow2_scale(amax);
+          const float inv = __frcp_rn(sc);  // exact: sc is a power of two
+          if (valid) {
+            uint8_t* dst = static_cast<uint8_t*>(args.C) + (int64_t)row * args.ldc + n * 128 + half * 64;
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 o;
+              o.x = e4m3x4(h[16 * v + 0] * inv, h[16 * v + 1] * inv, h[16 * v + 2] * inv, h[16 * v + 3] * inv);
+              o.y = e4m3x4(h[16 * v + 4] * inv, h[16 * v + 5] * inv, h[16 * v + 6] * inv, h[16 * v + 7] * inv);
+              o.z = e4m3x4(h[16 * v + 8] * inv, h[16 * v + 9] * inv, h[16 * v + 10] * inv, h[16 * v + 11] * inv);
+              o.w = e4m3x4(h[16 * v + 12] * inv, h[16 * v + 13] * inv, h[16 * v + 14] * inv, h[16 * v + 15] * inv);
+              d4[v] = o;
+            }
+            if (half == 0) args.c_scales[(int64_t)row * (args.ldc / 128) + n] = sc;
+          }
+        } else if (valid) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.C) + (int64_t)row * args.ldc + n * 128 + half * 64;
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            d4[v] = make_uint4(pack_bf16x2(h[8 * v], h[8 * v + 1]), pack_bf16x2(h[8 * v + 2], h[8 * v + 3]),
+                               pack_bf16x2(h[8 * v + 4], h[8 * v + 5]), pack_bf16x2(h[8 * v + 6], h[8 * v + 7]));
+        }
+      } else if (valid) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.C) + (int64_t)row * args.ldc + n * BN + half * 128;
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int v = 0; v < 16; ++v)
+          d4[v] = make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                             pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace ggmx
+
+// ==========================================================================
+// host side
+// ==========================================================================
+// Block-scaled FP8 grouped GEMM with power-of-two scales (see
+// launch_grouped_gemm_fp8 for the operands; scales are fp32 powers of two).
+cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const void* B,
+                                   const float* b_scales, const int32_t* offsets, int M_total,
+                                   int E, int N, int K, int act, void* Cout, float* c_scales,
+                                   int32_t* status, cudaStream_t s, const char** why) {
+  const bool swiglu = act != kActNone;
+  const int b_rows = swiglu ? 2 * N : N;
+  if (!swiglu && N % 256 != 0) {
+    *why = "the block-scaled plain GEMM needs N % 256 == 0";
+    return cudaErrorInvalidValue;
+  }
+  CUtensorMap tmA, tmB;
+  if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M_total, 128) ||
+      !make_tmap(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (int64_t)E * b_rows, 128)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  ggmx::Args a;
+  a.offsets = offsets;
+  a.E = E;
+  a.K = K;
+  a.ldc = N;
+  a.NT = swiglu ? N / 128 : N / 256;
+  a.b_rows = b_rows;
+  a.up_off = swiglu ? N : 0;
+  a.band = 8;
+  a.M_total = M_total;
+  a.kblocks = K / 128;
+  a.b_nblk = b_rows / 128;
+  a.C = Cout;
+  a.c_scales = c_scales;
+  a.a_scales = a_scales;
+  a.b_scales = b_scales;
+  a.status = status;
+  const int64_t tiles_ub = ((int64_t)M_total / ggmx::BM + (M_total < E ? M_total : E)) * a.NT;
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_ub));
+#define MOE_MX(ACTV)                                                                      \
+  do {                                                                                    \
+    cudaError_t e = set_smem(ggmx::gemm_mx_kernel<ACTV>, ggmx::kSmem);                    \
+    if (e != cudaSuccess) return e;                                                       \
+    ggmx::gemm_mx_kernel<ACTV><<<grid, ggmx::kThreads, ggmx::kSmem, s>>>(tmA, tmB, a);    \
+  } while (0)
+  if (act == kActSilu) MOE_MX(kActSilu);
+  else if (act == kActGelu) MOE_MX(kActGelu);
+  else if (act == kActRelu) MOE_MX(kActRelu);
+  else MOE_MX(kActNone);
+#undef MOE_MX
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -124,6 +124,7 @@ class LayerConfig:
     bias_sigma: float = 0.5
     zipf_s: float = 1.1
     fp8: bool = False
+    ue8m0: bool = False         # FP8 scales as powers of two (block-scaled tensor-core path)
     x_sigma: float = 1.0
     w_sigma: float = 0.02
     seed: int = 0
@@ -156,6 +157,10 @@ CONFIGS = {
                                     subset=512, fp8=True,
                                     desc="fine-grained prefill, FP8 experts (128x128 weight "
                                          "blocks, 1x128 activation groups)"),
+    "fine_grained_fp8_ue8m0": LayerConfig("fine_grained_fp8_ue8m0", 8192, 7168, 2048, 256, 8,
+                                          bias="zipf", subset=512, fp8=True, ue8m0=True,
+                                          desc="fine-grained prefill, FP8 experts with power-of-two "
+                                               "(UE8M0) scales on the block-scaled MMA"),
     "mixtral_decode_fp8": LayerConfig("mixtral_decode_fp8", 16, 4096, 14336, 8, 2, fp8=True,
                                       desc="Mixtral-shaped decode, FP8 experts: T=16 H=4096 "
                                            "I=14336 E=8 k=2"),

@@ -20,28 +20,32 @@ def _dec_table():
     return np.array([oracle.e4m3_decode(q) for q in range(256)])
 
 
+@pytest.mark.parametrize("ue8m0", [False, True])
 @pytest.mark.parametrize("rows,cols", [(1, 128), (37, 512), (300, 7168)])
-def test_act_quant_bit_exact(rows, cols):
+def test_act_quant_bit_exact(rows, cols, ue8m0):
     x = mi.normal_bf16(0, 61, 1.0, 1, rows, cols).reshape(rows, cols)
     x[0, :128] = 0  # an all-zero group
     q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
     s = torch.empty(rows, cols // 128, dtype=torch.float32, device="cuda")
-    moe.moe_quantize_act_fp8(dev_bf16(x), rows, cols, q, s)
+    moe.moe_quantize_act_fp8_fmt(dev_bf16(x), rows, cols, q, s,
+                                 moe.MOE_SCALE_UE8M0 if ue8m0 else moe.MOE_SCALE_F32)
     torch.cuda.synchronize()
-    rq, rs = oracle.quant_act_fp8(x)
+    rq, rs = oracle.quant_act_fp8(x, ue8m0=ue8m0)
     np.testing.assert_array_equal(q.cpu().numpy(), rq)
     np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
 
 
+@pytest.mark.parametrize("ue8m0", [False, True])
 @pytest.mark.parametrize("nb,rows,cols", [(1, 128, 128), (3, 256, 384), (2, 512, 1024)])
-def test_weight_quant_bit_exact(nb, rows, cols):
+def test_weight_quant_bit_exact(nb, rows, cols, ue8m0):
     w = mi.normal_bf16(0, 62, 0.02, nb, rows, cols).reshape(nb, rows, cols)
     w[0, :128, :128] = 0
     q = torch.empty(nb, rows, cols, dtype=torch.uint8, device="cuda")
     s = torch.empty(nb, rows // 128, cols // 128, dtype=torch.float32, device="cuda")
-    moe.moe_quantize_weight_fp8(dev_bf16(w), nb, rows, cols, q, s)
+    moe.moe_quantize_weight_fp8_fmt(dev_bf16(w), nb, rows, cols, q, s,
+                                    moe.MOE_SCALE_UE8M0 if ue8m0 else moe.MOE_SCALE_F32)
     torch.cuda.synchronize()
-    rq, rs = oracle.quant_weight_fp8(w)
+    rq, rs = oracle.quant_weight_fp8(w, ue8m0=ue8m0)
     np.testing.assert_array_equal(q.cpu().numpy(), rq)
     np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
 
