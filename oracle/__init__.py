@@ -56,6 +56,11 @@ def _L():
                                            i32, i32, vp, i32],
             "oracle_moe_forward": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                    i32, i32, vp, vp, vp, vp, i32],
+            "oracle_quant_weight_fp4": [vp, i64, i64, i64, vp, vp, i32],
+            "oracle_experts_combine_fp4": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp,
+                                           i32, vp, i32],
+            "oracle_moe_forward_fp4": [vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp,
+                                       i32, vp, vp, vp, vp, i32],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -65,6 +70,10 @@ def _L():
         lib.oracle_e4m3_decode.restype = ctypes.c_double
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e2m1_decode.restype = ctypes.c_double
+        lib.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e2m1_encode.restype = ctypes.c_uint8
         _lib = lib
     return _lib
 
@@ -176,6 +185,41 @@ def quant_weight_fp8(w, nthreads=None, ue8m0=False):
     return q, s
 
 
+def e2m1_decode(q: int) -> float:
+    return _L().oracle_e2m1_decode(int(q))
+
+
+def e2m1_encode(f: float) -> int:
+    return int(_L().oracle_e2m1_encode(float(f)))
+
+
+def quant_weight_fp4(w, nthreads=None):
+    """Per row, per 32 consecutive columns of w [nb, rows, cols] (bf16 bits):
+    s = smallest power of two >= amax/6 (1 if amax == 0), q = e2m1(w/s).
+    Returns q [nb, rows, cols/2] (element 2i in the low nibble of byte i) and
+    the e8m0 codes of s [nb, rows, cols/32]."""
+    w = _c(w, np.uint16)
+    nb, rows, cols = w.shape
+    q = np.empty((nb, rows, cols // 2), dtype=np.uint8)
+    sc = np.empty((nb, rows, cols // 32), dtype=np.uint8)
+    _L().oracle_quant_weight_fp4(_p(w), nb, rows, cols, _p(q), _p(sc), nthreads or threads())
+    return q, sc
+
+
+def experts_combine_fp4(x, tokens, ids, w, w13q, w13s, w2q, w2s, nthreads=None, act=ACT_SILU):
+    x, tokens = _c(x, np.uint16), _c(tokens, np.int32)
+    ids, w = _c(ids, np.int32), _c(w, np.float32)
+    w13q, w2q, w13s, w2s = (_c(a, np.uint8) for a in (w13q, w2q, w13s, w2s))
+    E, I2, H2 = w13q.shape
+    nt, k = ids.shape
+    H = 2 * H2
+    out = np.empty((nt, H), dtype=np.float32)
+    _L().oracle_experts_combine_fp4(_p(x), _p(tokens), nt, H, I2 // 2, E, k, _p(ids), _p(w),
+                                    _p(w13q), _p(w13s), _p(w2q), _p(w2s), int(act), _p(out),
+                                    nthreads or threads())
+    return out
+
+
 def e8m0_code(s):
     """The float8_e8m0fnu byte of power-of-two scales s (2^(code - 127))."""
     s = np.asarray(s, dtype=np.float32)
@@ -212,17 +256,31 @@ def experts_combine_fp8(x, tokens, ids, w, w13q, w13s, w2q, w2s, nthreads=None, 
 
 
 def moe_forward(x, wr, bias, w13=None, w2=None, k=2, tokens=None, fp8=None, nthreads=None,
-                act=ACT_SILU, ue8m0=False):
+                act=ACT_SILU, ue8m0=False, fp4=None):
     """The whole layer for ``tokens`` (all when None).
 
     ``fp8`` = (w13q, w13s, w2q, w2s) selects the FP8 experts (x is quantised
-    inside). Returns dict(out [nt,H] f32, ids, w, logits).
+    inside); ``fp4`` = the packed e2m1 codes and e8m0 scale codes of
+    ``quant_weight_fp4`` selects the FP4 experts. Returns dict(out [nt,H]
+    f32, ids, w, logits).
     """
     x, wr = _c(x, np.uint16), _c(wr, np.uint16)
     T, H = x.shape
     E = wr.shape[1]
     tokens = np.arange(T, dtype=np.int32) if tokens is None else _c(tokens, np.int32)
     nt = len(tokens)
+    if fp4 is not None:
+        w13q, w13s, w2q, w2s = (_c(a, np.uint8) for a in fp4)
+        I = w13q.shape[1] // 2
+        b = None if bias is None else _c(bias, np.float32)
+        out = np.empty((nt, H), dtype=np.float32)
+        ids = np.empty((nt, k), dtype=np.int32)
+        w = np.empty((nt, k), dtype=np.float32)
+        logits = np.empty((nt, E), dtype=np.float32)
+        _L().oracle_moe_forward_fp4(_p(x), _p(tokens), nt, H, I, E, k, _p(wr), _p(b), _p(w13q),
+                                    _p(w13s), _p(w2q), _p(w2s), int(act), _p(out), _p(ids), _p(w),
+                                    _p(logits), nthreads or threads())
+        return {"out": out, "ids": ids, "w": w, "logits": logits}
     if fp8 is not None:
         w13q, w13s, w2q, w2s = (_c(fp8[0], np.uint8), _c(fp8[1], np.float32),
                                 _c(fp8[2], np.uint8), _c(fp8[3], np.float32))

@@ -433,6 +433,89 @@ void oracle_quant_weight_fp8(const uint16_t* w, int64_t nb, int64_t rows, int64_
   parallel_for(nb * (rows / 128) * (cols / 128), nthreads, wq_blocks, &c);
 }
 
+
+/* ------------------------------------------------------------------------ */
+/* FP4 e2m1 (OCP: 1 sign, 2 exponent bits with bias 1, 1 mantissa bit; no   */
+/* infinities, no NaN; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6).               */
+/* "Experts backends", "FP8 and FP4 quantized experts": FP4 expert weights   */
+/* packed two per byte, with weight scales in the UE8M0 format (8-bit        */
+/* exponents, float8_e8m0fnu). The pages give no block geometry for them;    */
+/* the OCP microscaling block is taken: one scale per row per 32 consecutive */
+/* elements along K. The scale is the smallest power of two >= amax / 6      */
+/* (that fp32 quotient, so no scaled value exceeds 6), within 2^-127..2^127, */
+/* 1 for an all-zero block, stored as its biased exponent (code = p + 127).  */
+/* Byte c/2 of a row holds element c (c even) in its low four bits and      */
+/* element c + 1 in its high four bits. Activations stay FP8 e4m3 with      */
+/* power-of-two scales per (row, 128-group), as in the UE8M0 FP8 layer.     */
+/* ------------------------------------------------------------------------ */
+double oracle_e2m1_decode(uint8_t q) {
+  int s = (q >> 3) & 1, ef = (q >> 1) & 3, m = q & 1;
+  double v = ef == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, ef - 1);
+  return s ? -v : v;
+}
+
+/* Nearest e2m1 magnitude, ties to the even code (mantissa bit 0); beyond 6
+ * saturates to 6. The sign is kept (a negative value that rounds to zero
+ * gives the code of -0). */
+uint8_t oracle_e2m1_encode(float f) {
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  uint8_t s = signbit(f) ? 8 : 0;
+  double a = fabs((double)f);
+  if (a >= 6.0) return s | 7;
+  int best = 0;
+  for (int c = 1; c < 8; ++c) {
+    double dc = fabs(a - mag[c]), db = fabs(a - mag[best]);
+    if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+  }
+  return s | (uint8_t)best;
+}
+
+static inline float fp4_block_scale(float amax) {
+  if (!(amax > 0.0f)) return 1.0f;
+  const float r = amax / 6.0f;
+  int e;
+  const float m = frexpf(r, &e); /* r = m * 2^e, m in [0.5, 1) */
+  int p2 = m == 0.5f ? e - 1 : e;
+  if (p2 < -127) p2 = -127;
+  if (p2 > 127) p2 = 127;
+  return ldexpf(1.0f, p2);
+}
+
+/* nb matrices of bf16 [rows, cols] -> q [nb, rows, cols/2] (packed codes),
+ * sc [nb, rows, cols/32] (e8m0 codes). Rows are independent. */
+typedef struct {
+  const uint16_t* w;
+  int64_t cols;
+  uint8_t *q, *sc;
+} wq4_ctx;
+
+static void wq4_rows(void* p, int64_t lo, int64_t hi) {
+  wq4_ctx* c = (wq4_ctx*)p;
+  const int64_t cols = c->cols;
+  for (int64_t r = lo; r < hi; ++r) {
+    const uint16_t* wr = c->w + r * cols;
+    for (int64_t b = 0; b < cols / 32; ++b) {
+      float amax = 0.0f;
+      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(bf16_widen(wr[b * 32 + i])));
+      const float sc = fp4_block_scale(amax);
+      int ex;
+      frexpf(sc, &ex); /* sc = 2^(ex - 1) */
+      c->sc[r * (cols / 32) + b] = (uint8_t)(ex - 1 + 127);
+      for (int i = 0; i < 32; i += 2) {
+        uint8_t lo4 = oracle_e2m1_encode(bf16_widen(wr[b * 32 + i]) / sc);
+        uint8_t hi4 = oracle_e2m1_encode(bf16_widen(wr[b * 32 + i + 1]) / sc);
+        c->q[r * (cols / 2) + (b * 32 + i) / 2] = (uint8_t)(lo4 | (hi4 << 4));
+      }
+    }
+  }
+}
+
+void oracle_quant_weight_fp4(const uint16_t* w, int64_t nb, int64_t rows, int64_t cols,
+                             uint8_t* q, uint8_t* sc, int nthreads) {
+  wq4_ctx c = {w, cols, q, sc};
+  parallel_for(nb * rows, nthreads, wq4_rows, &c);
+}
+
 /* ------------------------------------------------------------------------ */
 /* The layer: the eager per-expert loop.                                     */
 /* "Experts backends", backend table, `eager` row (loop over the selected    */
@@ -453,8 +536,10 @@ typedef struct {
   const uint16_t *w13, *w2;
   const uint8_t *w13q, *w2q, *xq;
   const float *w13s, *w2s, *xs;
-  int fp8;
+  int fp8;       /* quantised experts: FP8 activations, e4m3 or e2m1 weights */
   int scale_fmt; /* FP8 scales: fp32 or power-of-two (UE8M0) */
+  int fp4;       /* weights: packed e2m1 codes with e8m0 scales per (row, 32) */
+  const uint8_t *w13s8, *w2s8;
   int act;       /* gated activation of the expert MLP */
   /* work list: items of up to CHUNK (row, slot) pairs of one expert */
   int64_t* item_e;
@@ -473,6 +558,16 @@ static void dequant_fp8(const uint8_t* q, const float* s, int64_t rows, int64_t 
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t c = 0; c < cols; ++c)
       out[r * cols + c] = oracle_e4m3_decode(q[r * cols + c]) * (double)s[(r / 128) * CB + c / 128];
+}
+
+static void dequant_fp4(const uint8_t* q, const uint8_t* sc, int64_t rows, int64_t cols,
+                        double* out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < cols; ++c) {
+      uint8_t byte = q[r * (cols / 2) + c / 2];
+      uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+      out[r * cols + c] = oracle_e2m1_decode(code) * ldexp(1.0, (int)sc[r * (cols / 32) + c / 32] - 127);
+    }
 }
 
 static void* fwd_worker(void* p) {
@@ -500,9 +595,14 @@ static void* fwd_worker(void* p) {
     int64_t e = c->item_e[it];
     const uint16_t* w13e = c->fp8 ? NULL : c->w13 + e * 2 * I * H;
     const uint16_t* w2e = c->fp8 ? NULL : c->w2 + e * H * I;
-    if (c->fp8 && e != cur_e) { /* w-hat = e4m3 code * its block scale */
-      dequant_fp8(c->w13q + e * 2 * I * H, c->w13s + e * (2 * I / 128) * (H / 128), 2 * I, H, w13d);
-      dequant_fp8(c->w2q + e * H * I, c->w2s + e * (H / 128) * (I / 128), H, I, w2d);
+    if (c->fp8 && e != cur_e) {
+      if (c->fp4) { /* w-hat = e2m1 code * 2^(e8m0 code - 127) of its (row, 32) block */
+        dequant_fp4(c->w13q + e * 2 * I * (H / 2), c->w13s8 + e * 2 * I * (H / 32), 2 * I, H, w13d);
+        dequant_fp4(c->w2q + e * H * (I / 2), c->w2s8 + e * H * (I / 32), H, I, w2d);
+      } else { /* w-hat = e4m3 code * its block scale */
+        dequant_fp8(c->w13q + e * 2 * I * H, c->w13s + e * (2 * I / 128) * (H / 128), 2 * I, H, w13d);
+        dequant_fp8(c->w2q + e * H * I, c->w2s + e * (H / 128) * (I / 128), H, I, w2d);
+      }
       cur_e = e;
     }
     for (int64_t g0 = 0; g0 < c->item_len[it]; g0 += GROUP) {
@@ -662,6 +762,63 @@ void oracle_experts_combine_fp8(const uint16_t* x, const int32_t* tokens, int64_
   free(xq);
   free(xs);
   free(xrows);
+}
+
+/* FP4 experts + combine: x is quantised here per (token, 128-group) to e4m3
+ * with power-of-two scales; weights are packed e2m1 codes with e8m0 scales
+ * per (row, 32-element block); the down projection's input is re-quantised
+ * the same way as x. */
+void oracle_experts_combine_fp4(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H,
+                                int64_t I, int64_t E, int k, const int32_t* ids,
+                                const float* topk_w, const uint8_t* w13q, const uint8_t* w13s,
+                                const uint8_t* w2q, const uint8_t* w2s, int act, float* out,
+                                int nthreads) {
+  uint8_t* xq = (uint8_t*)malloc((size_t)(nt * H));
+  float* xs = (float*)malloc(sizeof(float) * (size_t)(nt * (H / 128)));
+  for (int64_t r = 0; r < nt; ++r)
+    oracle_quant_act_fp8(x + (int64_t)tokens[r] * H, 1, H, xq + r * H, xs + r * (H / 128),
+                         SCALE_UE8M0);
+  fwd_ctx c;
+  memset(&c, 0, sizeof(c));
+  c.x = x;
+  c.H = H;
+  c.I = I;
+  c.E = E;
+  c.k = k;
+  c.tokens = tokens;
+  c.nt = nt;
+  c.w13q = w13q;
+  c.w13s8 = w13s;
+  c.w2q = w2q;
+  c.w2s8 = w2s;
+  c.xq = xq;
+  c.xs = xs;
+  c.fp8 = 1;
+  c.fp4 = 1;
+  c.scale_fmt = SCALE_UE8M0;
+  c.act = act;
+  run_forward(&c, ids, topk_w, out, nthreads);
+  free(xq);
+  free(xs);
+}
+
+/* The whole layer with FP4 experts for tokens[0..nt) (see
+ * oracle_experts_combine_fp4); ids_out / w_out / logits_out may be NULL. */
+void oracle_moe_forward_fp4(const uint16_t* x, const int32_t* tokens, int64_t nt, int64_t H,
+                            int64_t I, int64_t E, int k, const uint16_t* wr, const float* bias,
+                            const uint8_t* w13q, const uint8_t* w13s, const uint8_t* w2q,
+                            const uint8_t* w2s, int act, float* out, int32_t* ids_out,
+                            float* w_out, float* logits_out, int nthreads) {
+  float* logits = logits_out ? logits_out : (float*)malloc(sizeof(float) * (size_t)(nt * E));
+  int32_t* ids = ids_out ? ids_out : (int32_t*)malloc(sizeof(int32_t) * (size_t)(nt * k));
+  float* w = w_out ? w_out : (float*)malloc(sizeof(float) * (size_t)(nt * k));
+  oracle_router_logits(x, wr, bias, tokens, nt, H, E, logits, nthreads);
+  oracle_topk(logits, nt, E, k, ids, w);
+  oracle_experts_combine_fp4(x, tokens, nt, H, I, E, k, ids, w, w13q, w13s, w2q, w2s, act, out,
+                             nthreads);
+  if (!logits_out) free(logits);
+  if (!ids_out) free(ids);
+  if (!w_out) free(w);
 }
 
 /* The whole layer for tokens[0..nt): logits -> top-k -> experts -> combine.

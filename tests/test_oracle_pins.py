@@ -478,6 +478,128 @@ def test_fp8_forward_matches_dense_on_dequantised_values():
 
 
 # --------------------------------------------------------------------------
+# FP4 e2m1 experts with e8m0 scales per (row, 32 elements)
+# --------------------------------------------------------------------------
+def _ml_dtypes():
+    return pytest.importorskip("ml_dtypes")
+
+
+def test_e2m1_decode_all_codes_match_ml_dtypes():
+    md = _ml_dtypes()
+    ref = np.arange(16, dtype=np.uint8).view(md.float4_e2m1fn).astype(np.float64)
+    got = np.array([oracle.e2m1_decode(q) for q in range(16)])
+    np.testing.assert_array_equal(got, ref)
+    np.testing.assert_array_equal(np.signbit(got), np.signbit(ref))
+
+
+def test_e2m1_encode_rne_vs_ml_dtypes():
+    """Every grid point, every midpoint (ties to the even code), points just
+    beside the midpoints and random values in [-6, 6]."""
+    md = _ml_dtypes()
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+    mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)
+    pts = np.concatenate([grid.astype(np.float32), mids, np.nextafter(mids, np.float32(0)),
+                          np.nextafter(mids, np.float32(10))])
+    rng = np.random.default_rng(11)
+    pts = np.concatenate([pts, -pts, rng.uniform(-6, 6, 4000).astype(np.float32)])
+    ref = pts.astype(md.float4_e2m1fn).view(np.uint8) & 15
+    got = np.array([oracle.e2m1_encode(v) for v in pts], dtype=np.uint8)
+    nz = (pts != 0) & (np.abs(pts) > 0.25)  # results of +-0 carry the input's sign, checked below
+    np.testing.assert_array_equal(got[nz], ref[nz])
+    assert oracle.e2m1_encode(0.2) == 0 and oracle.e2m1_encode(-0.2) == 8
+    assert oracle.e2m1_encode(5.0) == 6 and oracle.e2m1_encode(0.25) == 0  # ties -> even code
+    assert oracle.e2m1_encode(1.75) == 4 and oracle.e2m1_encode(2.5) == 4
+
+
+def _unpack_fp4(q, sc):
+    """Dense fp64 values of packed e2m1 codes with e8m0 scales per (row, 32),
+    decoded by ml_dtypes."""
+    md = _ml_dtypes()
+    codes = np.stack([q & 15, q >> 4], axis=-1).reshape(*q.shape[:-1], 2 * q.shape[-1])
+    vals = codes.astype(np.uint8).view(md.float4_e2m1fn).astype(np.float64)
+    scale = sc.astype(np.uint8).view(md.float8_e8m0fnu).astype(np.float64)
+    return vals * np.repeat(scale, 32, axis=-1)
+
+
+def test_fp4_weight_quant_closed_forms():
+    """Block scale = smallest power of two >= amax/6, one per (row, 32);
+    element 2i in the low nibble of byte i; an all-zero block has scale 1."""
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((1, 2, 128)) * 0.01).astype(np.float32)
+    w[0, 0, 3] = 6 * 2.0 ** -5          # block 0: amax / 6 is exactly 2^-5
+    w[0, 0, :3] = w[0, 0, 4:32] = 0.01
+    w[0, 0, 32:64] = 0                  # block 1: all zero
+    w[0, 0, 64:96] = np.clip(w[0, 0, 64:96], -0.09, 0.09)
+    w[0, 0, 70] = -0.1                  # block 2: bf16(0.1) / 6 rounds up to 2^-5
+    wb16 = _bf16(w)
+    q, sc = oracle.quant_weight_fp4(wb16)
+    assert q.shape == (1, 2, 64) and sc.shape == (1, 2, 4)
+    assert sc[0, 0, 0] == 127 - 5 and sc[0, 0, 1] == 127 and sc[0, 0, 2] == 127 - 5
+    assert q[0, 0, 1] >> 4 == 7                   # element 3: +6 in the high nibble of byte 1
+    assert q[0, 0, 0] == (1 | (1 << 4))           # 0.01 / 2^-5 = 0.32 -> 0.5 (code 1), twice
+    assert np.all(q[0, 0, 16:32] == 0)
+    assert (q[0, 0, 35] & 15) == 8 | 5            # element 70: -0.1001 / 2^-5 = -3.2 -> -3
+    wf = mi.bf16_to_f32(wb16).astype(np.float64)
+    deq = _unpack_fp4(q, sc)
+    s = np.repeat(2.0 ** (sc.astype(np.float64) - 127), 32, axis=-1)
+    assert np.all(np.abs(wf) <= 6 * s)
+    err = np.abs(deq - wf)
+    assert np.all(err <= s * (1 + 1e-12))                               # largest gap (4..6) / 2
+    small = np.abs(wf) <= 2 * s
+    assert np.all(err[small] <= 0.25 * s[small] * (1 + 1e-12))           # gap 0.5 below 2
+
+
+def _pow2_quant_e4m3(v):
+    """Per 128-group: scale = smallest power of two >= amax/448 (fp32), e4m3 by torch."""
+    v = np.asarray(v, dtype=np.float32).reshape(-1, 128)
+    out = np.empty(v.shape)
+    for i, grp in enumerate(v):
+        amax = np.float32(np.abs(grp).max())
+        sc = 2.0 ** np.ceil(np.log2(np.float32(amax / np.float32(448)))) if amax > 0 else 1.0
+        codes = torch.from_numpy((grp / np.float32(sc)).astype(np.float32)).to(torch.float8_e4m3fn)
+        out[i] = codes.to(torch.float64).numpy() * sc
+    return out.reshape(-1)
+
+
+def test_fp4_forward_matches_dense_on_dequantised_values():
+    cfg = _small(T=12, E=3, k=2, H=256, I=256)
+    L = mi.make_layer(cfg)
+    q13, s13 = oracle.quant_weight_fp4(L["w13"])
+    q2, s2 = oracle.quant_weight_fp4(L["w2"])
+    r = oracle.moe_forward(L["x"], L["wr"], L["bias"], k=cfg.k, fp4=(q13, s13, q2, s2))
+    W13, W2 = _unpack_fp4(q13, s13), _unpack_fp4(q2, s2)
+    xf = mi.bf16_to_f32(L["x"])
+    ref = np.zeros((cfg.T, cfg.H))
+    for t in range(cfg.T):
+        X = _pow2_quant_e4m3(xf[t])
+        for j in range(cfg.k):
+            e = r["ids"][t, j]
+            g, u = W13[e, :cfg.I] @ X, W13[e, cfg.I:] @ X
+            h = (g / (1 + np.exp(-g)) * u).astype(np.float32)
+            ref[t] += float(r["w"][t, j]) * (W2[e] @ _pow2_quant_e4m3(h))
+    np.testing.assert_allclose(r["out"], ref, rtol=2e-5, atol=2e-5 * np.abs(ref).max())
+
+
+def test_fp4_forward_on_fp4_exact_weights_equals_ue8m0_fp8_forward():
+    """Weights already on the e2m1 grid (times 2^-7) quantise without error in
+    both formats, so the FP4 layer must equal the power-of-two FP8 layer."""
+    cfg = _small(T=20, E=4, k=2, H=256, I=384)
+    L = mi.make_layer(cfg)
+    rng = np.random.default_rng(9)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.5, -1, -1.5, -2, -3, -4, -6])
+    w13 = _bf16(rng.choice(grid, size=L["w13"].shape) * 2.0 ** -7)
+    w2 = _bf16(rng.choice(grid, size=L["w2"].shape) * 2.0 ** -7)
+    q13, s13 = oracle.quant_weight_fp4(w13)
+    q2, s2 = oracle.quant_weight_fp4(w2)
+    np.testing.assert_array_equal(_unpack_fp4(q13, s13), mi.bf16_to_f32(w13))
+    f8 = oracle.quant_weight_fp8(w13, ue8m0=True) + oracle.quant_weight_fp8(w2, ue8m0=True)
+    r4 = oracle.moe_forward(L["x"], L["wr"], L["bias"], k=cfg.k, fp4=(q13, s13, q2, s2))
+    r8 = oracle.moe_forward(L["x"], L["wr"], L["bias"], k=cfg.k, fp8=f8, ue8m0=True)
+    np.testing.assert_array_equal(r4["ids"], r8["ids"])
+    np.testing.assert_array_equal(r4["out"], r8["out"])
+
+
+# --------------------------------------------------------------------------
 # the input generator itself
 # --------------------------------------------------------------------------
 def test_generator_splitmix_reference_value():
