@@ -241,6 +241,37 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (my_slot >= 0) w[(int64_t)warp * k + my_slot] = __fdiv_rn(my_ex, denom);
 }
 
+// Top-k of one token's E <= 32 logits held in shared memory, by one warp
+// (lane = expert): k rounds of a warp argmax on (logit desc, index asc); the
+// renormalised weights are exp(l - l_max) over their sum.
+__device__ __forceinline__ void warp_topk32(const float* lg, int E, int k, int64_t tt, int lane,
+                                            int32_t* __restrict__ ids, float* __restrict__ topw) {
+  const float v = lane < E ? lg[lane] : -INFINITY;
+  bool taken = lane >= E;
+  float lmax = 0.0f, denom = 0.0f, my_ex = 0.0f;
+  int my_slot = -1;
+  for (int j = 0; j < k; ++j) {
+    float bv = taken ? -INFINITY : v;
+    int be = taken ? 0x7fffffff : lane;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
+    }
+    if (be == lane) taken = true;
+    if (j == 0) lmax = bv;
+    const float ex = expf(bv - lmax);
+    denom += ex;
+    if (lane == j) {
+      my_ex = ex;
+      my_slot = j;
+      ids[tt * k + j] = be;
+    }
+  }
+  if (my_slot >= 0) topw[tt * k + my_slot] = __fdiv_rn(my_ex, denom);
+}
+
 // Narrow router with fused top-k (E <= 32). The logit sum runs in the fixed
 // blocked order (8 contiguous h blocks, each summed from zero, then added
 // left to right), and the 8 block sums of a (token, expert pair) are computed
@@ -407,36 +438,112 @@ __global__ void __launch_bounds__(kNarrowCT + kNarrowHT) router_narrow_kernel(
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kNarrowCT) : "memory");  // compute warps only
-  // top-k: warp w takes tokens w, w + 4, ...; lane = expert
+  // top-k: warp w takes tokens w, w + 4, ...
   const int w = tid >> 5;
   for (int r = w; r < BT; r += kNarrowCT / 32) {
-    const int tt = t0 + r;
-    if (tt >= T) break;
-    const float v = lane < E ? slg[r * 32 + lane] : -INFINITY;
-    bool taken = lane >= E;
-    float lmax = 0.0f, denom = 0.0f, my_ex = 0.0f;
-    int my_slot = -1;
-    for (int j = 0; j < k; ++j) {
-      float bv = taken ? -INFINITY : v;
-      int be = taken ? 0x7fffffff : lane;
+    if (t0 + r >= T) break;
+    warp_topk32(slg + r * 32, E, k, t0 + r, lane, ids, topw);
+  }
+}
+
+
+// Tall router with fused top-k (E <= 32, many tokens). The CTA holds the
+// whole of Wr, widened to fp32, in shared memory ([H][EV]); warp b owns h
+// block b and lane l token t0 + l, so every shared load of a Wr row is one
+// broadcast to the 32 tokens of the warp. Each thread keeps the EV sums of
+// its (token, block) in registers, one paired FMA per h and expert pair, and
+// reads its x slice straight from global memory, 16 h (32 bytes) per step
+// with two steps in flight. The 8 block sums of a (token, expert) meet in
+// shared memory and are added left to right, then the bias.
+template <int EV>  // experts padded to a power of two (2..32)
+__global__ void __launch_bounds__(256, 1) router_tall_kernel(
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
+    const float* __restrict__ bias, int T, int H, int E, int k, int BT, float* __restrict__ logits,
+    int32_t* __restrict__ ids, float* __restrict__ topw) {
+  constexpr int NB = kRouterBlocks;
+  extern __shared__ __align__(16) float tall_smem[];
+  const int L = H / NB;                  // a multiple of 16 (H % 128 == 0)
+  float* sw = tall_smem;                 // [H][EV] Wr in fp32, padded experts zero
+  float* part = sw + (size_t)H * EV;     // [NB][32][EV] block sums
+  float* slg = part + NB * 32 * EV;      // [32][32] logits for the top-k
+  const int tid = threadIdx.x, b = tid >> 5, lane = tid & 31;
+  const int t0 = blockIdx.x * BT;
+  const int tr = min(t0 + lane, T - 1);  // lanes past the last token read a valid row, never write
+  const uint4* xp = reinterpret_cast<const uint4*>(x + (int64_t)tr * H + (int64_t)b * L);
+  const int nsteps = L / 16;
+  uint4 xa0 = __ldg(xp), xa1 = __ldg(xp + 1), xb0 = xa0, xb1 = xa1;
+  if (nsteps > 1) xb0 = __ldg(xp + 2), xb1 = __ldg(xp + 3);
+
+  // stage Wr: 8 bf16 per 16-byte load, several loads in flight per thread
+  const uint4* w4 = reinterpret_cast<const uint4*>(wr);
+  const int nvec = H * E / 8;
+#pragma unroll 4
+  for (int v = tid; v < nvec; v += blockDim.x) {
+    const uint4 u = __ldg(w4 + v);
+    const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+    int h = (8 * v) / E, e = (8 * v) % E;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
-      }
-      if (be == lane) taken = true;
-      if (j == 0) lmax = bv;
-      const float ex = expf(bv - lmax);
-      denom += ex;
-      if (lane == j) {
-        my_ex = ex;
-        my_slot = j;
-        ids[(int64_t)tt * k + j] = be;
+    for (int q = 0; q < 8; ++q) {
+      sw[h * EV + e] = (q & 1) ? bf16hi_to_f32(uw[q >> 1]) : bf16lo_to_f32(uw[q >> 1]);
+      if (++e == E) e = 0, ++h;
+    }
+  }
+  if (E < EV) {
+    const int pad = EV - E;
+    for (int i = tid; i < H * pad; i += blockDim.x) sw[(i / pad) * EV + E + i % pad] = 0.0f;
+  }
+  __syncthreads();
+
+  float2 acc[EV / 2];
+#pragma unroll
+  for (int i = 0; i < EV / 2; ++i) acc[i] = make_float2(0.0f, 0.0f);
+  const float* wb = sw + (size_t)b * L * EV;
+#pragma unroll 1
+  for (int st = 0; st < nsteps; ++st) {
+    const uint32_t xw[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+    xa0 = xb0, xa1 = xb1;
+    if (st + 2 < nsteps) xb0 = __ldg(xp + 2 * st + 4), xb1 = __ldg(xp + 2 * st + 5);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const float xf = (q & 1) ? bf16hi_to_f32(xw[q >> 1]) : bf16lo_to_f32(xw[q >> 1]);
+      const float2 xx = make_float2(xf, xf);
+      const float* wh = wb + (st * 16 + q) * EV;
+      if constexpr (EV >= 4) {
+#pragma unroll
+        for (int e4 = 0; e4 < EV / 4; ++e4) {
+          const float4 wv = *reinterpret_cast<const float4*>(wh + 4 * e4);
+          acc[2 * e4] = __ffma2_rn(xx, make_float2(wv.x, wv.y), acc[2 * e4]);
+          acc[2 * e4 + 1] = __ffma2_rn(xx, make_float2(wv.z, wv.w), acc[2 * e4 + 1]);
+        }
+      } else {
+        acc[0] = __ffma2_rn(xx, *reinterpret_cast<const float2*>(wh), acc[0]);
       }
     }
-    if (my_slot >= 0) topw[(int64_t)tt * k + my_slot] = __fdiv_rn(my_ex, denom);
   }
+  float* pp = part + (b * 32 + lane) * EV;
+#pragma unroll
+  for (int i = 0; i < EV / 2; ++i) *reinterpret_cast<float2*>(pp + 2 * i) = acc[i];
+  __syncthreads();
+  // block sums -> logits, added left to right, then the bias
+  for (int i = tid; i < BT * E; i += blockDim.x) {
+    const int tl = i / E, e = i % E;
+    float sum = part[tl * EV + e];
+#pragma unroll
+    for (int bb = 1; bb < NB; ++bb) sum = __fadd_rn(sum, part[(bb * 32 + tl) * EV + e]);
+    const float l = __fadd_rn(sum, bias ? bias[e] : 0.0f);
+    slg[tl * 32 + e] = l;
+    if (t0 + tl < T && logits) logits[(int64_t)(t0 + tl) * E + e] = l;
+  }
+  __syncthreads();
+  const int nw = blockDim.x >> 5;
+  for (int r = b; r < BT; r += nw) {
+    if (t0 + r >= T) break;
+    warp_topk32(slg + r * 32, E, k, t0 + r, lane, ids, topw);
+  }
+}
+
+static size_t tall_smem_bytes(int H, int EV) {
+  return ((size_t)H * EV + (size_t)kRouterBlocks * 32 * EV + 32 * 32) * 4;
 }
 
 // Pairs per token for the narrow router (E padded to a power of two >= 2).
@@ -448,12 +555,39 @@ static int narrow_pairs(int E) {
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t s);
 
-// Logits and top-k of T tokens: the fused narrow kernel for E <= 32, else the
-// wide logits kernel followed by the warp-per-token selection.
+// Logits and top-k of T tokens: for E <= 32 the fused tall kernel (many
+// tokens, Wr fits shared memory) or the fused narrow kernel; else the wide
+// logits kernel followed by the warp-per-token selection.
+constexpr int kTallMinT = 1024;
+constexpr size_t kTallMaxSmem = 200 * 1024;
 cudaError_t launch_route(const void* x, const void* wr, const float* bias, int T, int H, int E,
                          int k, float* logits, int32_t* ids, float* w, cudaStream_t s) {
   const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
   const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(wr);
+  if (E <= 32 && T >= kTallMinT) {
+    const int ev = 2 * narrow_pairs(E);
+    // tokens per CTA (lanes of a warp): about one CTA per SM
+    const int sms = num_sms();
+    const int bt = std::min(32, std::max(1, (int)((T + sms - 1) / sms)));
+    const size_t smem = tall_smem_bytes(H, ev);
+    if (smem <= kTallMaxSmem) {
+#define MOE_TALL(EVV)                                                                          \
+  do {                                                                                         \
+    cudaFuncSetAttribute(router_tall_kernel<EVV>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                         (int)smem);                                                           \
+    router_tall_kernel<EVV><<<(unsigned)ceil_div(T, bt), 32 * kRouterBlocks, smem, s>>>(       \
+        xp, wp, bias, T, H, E, k, bt, logits, ids, w);                                         \
+  } while (0)
+      if (ev == 2) MOE_TALL(2);
+      else if (ev == 4) MOE_TALL(4);
+      else if (ev == 8) MOE_TALL(8);
+      else if (ev == 16) MOE_TALL(16);
+      else MOE_TALL(32);
+#undef MOE_TALL
+      note_launch();
+      return cudaGetLastError();
+    }
+  }
   if (E <= 32) {
     const int epp = narrow_pairs(E);
 #define MOE_NARROW(P)                                                                         \

@@ -48,6 +48,12 @@ ROUTER_CASES = [
     ("tiny", dict(T=70, E=32, k=16, bias="normal")),
     ("tiny", dict(T=10000, E=8, k=2, H=256)),
     ("tiny", dict(T=5000, E=24, k=6, H=128)),
+    # many tokens, few experts: the tall kernel (whole Wr in shared memory), its largest table
+    ("tiny", dict(T=1100, E=1, k=1, H=384)),
+    ("tiny", dict(T=1500, E=32, k=8, H=1536, bias="normal")),
+    ("tiny", dict(T=2222, E=13, k=5, H=640, bias="normal")),
+    # Wr too large for shared memory: the narrow kernel at many tokens
+    ("tiny", dict(T=1200, E=16, k=4, H=4096)),
 ]
 
 
@@ -64,11 +70,12 @@ def test_router_bit_exact(name, kw):
     np.testing.assert_allclose(w, ref_w, rtol=0, atol=1e-6)
 
 
+@pytest.mark.parametrize("T", [90, 1200])
 @pytest.mark.parametrize("E,k", [(8, 2), (5, 5), (32, 16), (2, 1)])
-def test_router_exact_ties(E, k):
+def test_router_exact_ties(E, k, T):
     """Equal logits from duplicated router columns and all-zero tokens: the
-    lowest expert index wins every tie, in the fused small-E kernel too."""
-    cfg = mi.CONFIGS["tiny"].with_(T=90, E=E, k=k)
+    lowest expert index wins every tie, in the fused small-E kernels too."""
+    cfg = mi.CONFIGS["tiny"].with_(T=T, E=E, k=k)
     x = mi.make_x(cfg)
     x[::4] = 0  # every logit of these tokens is exactly zero
     wr, _ = mi.make_router(cfg)
