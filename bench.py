@@ -145,6 +145,8 @@ def oracle_inputs(cfg, L):
     """Keyword arguments for oracle.moe_forward; FP8 weights are quantised by the oracle itself."""
     import oracle
 
+    if cfg.fp4:
+        return {"fp4": oracle.quant_weight_fp4(L["w13"]) + oracle.quant_weight_fp4(L["w2"])}
     if cfg.fp8:
         w13q, w13s = oracle.quant_weight_fp8(L["w13"], ue8m0=cfg.ue8m0)
         w2q, w2s = oracle.quant_weight_fp8(L["w2"], ue8m0=cfg.ue8m0)
@@ -240,10 +242,22 @@ def gpu_arm(args, cfg):
     bias = torch.from_numpy(L["bias"]).cuda()
     w13, w2 = bf(L["w13"]), bf(L["w2"])
     d = (cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
-    dt = (moe.MOE_DTYPE_FP8_E4M3_UE8M0 if cfg.ue8m0 else moe.MOE_DTYPE_FP8_E4M3) if cfg.fp8 \
-        else moe.MOE_DTYPE_BF16
+    quant = cfg.fp8 or cfg.fp4
+    dt = (moe.MOE_DTYPE_FP4_E2M1 if cfg.fp4 else
+          (moe.MOE_DTYPE_FP8_E4M3_UE8M0 if cfg.ue8m0 else moe.MOE_DTYPE_FP8_E4M3) if cfg.fp8
+          else moe.MOE_DTYPE_BF16)
     sfmt = moe.MOE_SCALE_UE8M0 if cfg.ue8m0 else moe.MOE_SCALE_F32
-    if cfg.fp8:
+    if cfg.fp4:
+        # one-time weight preparation (untimed): packed e2m1 with one e8m0 scale per (row, 32)
+        w13q = torch.empty(cfg.E, 2 * cfg.I, cfg.H // 2, dtype=torch.uint8, device="cuda")
+        w13s = torch.empty(cfg.E, 2 * cfg.I, cfg.H // 32, dtype=torch.uint8, device="cuda")
+        w2q = torch.empty(cfg.E, cfg.H, cfg.I // 2, dtype=torch.uint8, device="cuda")
+        w2s = torch.empty(cfg.E, cfg.H, cfg.I // 32, dtype=torch.uint8, device="cuda")
+        moe.moe_quantize_weight_fp4(w13, cfg.E, 2 * cfg.I, cfg.H, w13q, w13s)
+        moe.moe_quantize_weight_fp4(w2, cfg.E, cfg.H, cfg.I, w2q, w2s)
+        torch.cuda.synchronize()
+        del w13, w2
+    elif cfg.fp8:
         # one-time weight preparation (untimed): e4m3 with one scale per 128 x 128 block
         w13q = torch.empty(cfg.E, 2 * cfg.I, cfg.H, dtype=torch.uint8, device="cuda")
         w13s = torch.empty(cfg.E, 2 * cfg.I // 128, cfg.H // 128, dtype=torch.float32, device="cuda")
@@ -262,7 +276,10 @@ def gpu_arm(args, cfg):
 
     def step(xin=None):
         xin = x if xin is None else xin
-        if cfg.fp8 and cfg.ue8m0:
+        if cfg.fp4:
+            moe.moe_forward_fp4(xin, wr, bias, w13q, w13s, w2q, w2s, d, moe.MOE_EPILOGUE_SWIGLU, out,
+                                ws, ws_bytes)
+        elif cfg.fp8 and cfg.ue8m0:
             moe.moe_forward_fp8_ue8m0(xin, wr, bias, w13q, w13s, w2q, w2s, d, moe.MOE_EPILOGUE_SWIGLU,
                                       out, ws, ws_bytes)
         elif cfg.fp8:
@@ -347,9 +364,13 @@ def gpu_arm(args, cfg):
     def e2e_step(i):
         j = i & 1
         with torch.cuda.stream(streams[j]):
-            if cfg.fp8:
+            if quant:
                 xs_dev[j].view(torch.int16).copy_(x_host.view(cfg.T, cfg.H), non_blocking=True)
-                if cfg.ue8m0:
+                if cfg.fp4:
+                    moe.moe_forward_fp4(xs_dev[j], wr, bias, w13q, w13s, w2q, w2s, d,
+                                        moe.MOE_EPILOGUE_SWIGLU, outs_dev[j], wss[j], ws_bytes,
+                                        stream=streams[j])
+                elif cfg.ue8m0:
                     moe.moe_forward_fp8_ue8m0(xs_dev[j], wr, bias, w13q, w13s, w2q, w2s, d,
                                               moe.MOE_EPILOGUE_SWIGLU, outs_dev[j], wss[j], ws_bytes,
                                               stream=streams[j])
@@ -385,29 +406,37 @@ def gpu_arm(args, cfg):
 
     peaks, peak_src = load_peaks()
     flops = 6.0 * cfg.T * cfg.k * cfg.H * cfg.I
-    wbytes, n_exp = touched_weight_bytes(cfg, offsets, 1.0 if cfg.fp8 else 2.0)
+    # bytes per expert weight: e2m1 + one e8m0 byte per 32; e4m3 (+ block scales, counted below); bf16
+    wbytes, n_exp = touched_weight_bytes(cfg, offsets, (0.5 + 1.0 / 32) if cfg.fp4 else
+                                         1.0 if cfg.fp8 else 2.0)
     layer_bytes = wbytes + 2 * cfg.T * cfg.H * 2 + cfg.H * cfg.E * 2
     gemm1_ms = float(stage_ms[2])
     decode = cfg.T * cfg.k <= 64 * cfg.E and cfg.T <= 64
     if decode:
         # touched expert weights of GEMM-1 (e4m3 codes + one fp32 scale per 128 x 128 block)
-        g1_bytes = n_exp * 2 * cfg.H * cfg.I * ((1.0 + 4.0 / (128 * 128)) if cfg.fp8 else 2.0)
+        g1_bytes = n_exp * 2 * cfg.H * cfg.I * ((0.5 + 1.0 / 32) if cfg.fp4 else
+                                                (1.0 + 4.0 / (128 * 128)) if cfg.fp8 else 2.0)
         ach = g1_bytes / (gemm1_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"],
                 "traffic": kernel_traffic(cfg.name, "gemm1"),
-                "kernel": ("gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)"
+                "kernel": ("gemm_mx_kernel<SwiGLU, e2m1 B> (FP4 GEMM1 + SwiGLU + h quantisation)"
+                           if cfg.fp4 else
+                           "gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)"
                            if cfg.fp8 else "gemm_swap_kernel<SwiGLU> (GEMM1, small-M)"),
                 "algorithmic_bytes_per_launch": g1_bytes, "peak_source": peak_src}
     else:
         g1_flops = 4.0 * cfg.T * cfg.k * cfg.H * cfg.I
         ach = g1_flops / (gemm1_ms / 1e3) / 1e12
-        # FP8 peak = the measured bf16 peak x the nominal fp8/bf16 ratio (2)
-        ratio = 2.0 if cfg.fp8 else 1.0
+        # FP8 peak = the measured bf16 peak x the nominal fp8/bf16 ratio (2); e4m3 x e2m1 runs on
+        # the same f8f6f4 MMA, at the FP8 rate
+        ratio = 2.0 if quant else 1.0
         pk, pk_burst = ratio * peaks["bf16_tflops_sustained"], ratio * peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s", "frac": ach / pk,
                 "traffic": kernel_traffic(cfg.name, "gemm1"),
-                "kernel": ("gemm_mx_kernel<SwiGLU> (block-scaled FP8 GEMM1 + SwiGLU + h quantisation)"
+                "kernel": ("gemm_mx_kernel<SwiGLU, e2m1 B> (block-scaled FP4 GEMM1 + SwiGLU + h "
+                           "quantisation)" if cfg.fp4 else
+                           "gemm_mx_kernel<SwiGLU> (block-scaled FP8 GEMM1 + SwiGLU + h quantisation)"
                            if cfg.ue8m0 else
                            "gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)" if cfg.fp8
                            else "gemm_rows_kernel<SwiGLU,256> (GEMM1 + SwiGLU, rows gathered)"),
@@ -418,7 +447,8 @@ def gpu_arm(args, cfg):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3 x e4m3 -> fp32 (experts), bf16 router" if cfg.fp8 else "bf16 x bf16 -> fp32",
+        "dtype": ("e4m3 x e2m1 -> fp32 (experts), bf16 router" if cfg.fp4 else
+                  "e4m3 x e4m3 -> fp32 (experts), bf16 router" if cfg.fp8 else "bf16 x bf16 -> fp32"),
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights)",
         "config": {"workload": cfg.desc, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
                    "parallelism": f"token-parallel replicas x{world}",
@@ -427,7 +457,7 @@ def gpu_arm(args, cfg):
         "roofline": roof,
         "layer": {"tflops": flops / (ms_per_step / 1e3) / 1e12,
                   "tflops_frac": flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]
-                  / (2.0 if cfg.fp8 else 1.0),
+                  / (2.0 if quant else 1.0),
                   "gbs": layer_bytes / (ms_per_step / 1e3) / 1e9,
                   "gbs_frac": layer_bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
                   "touched_experts": n_exp},
@@ -458,8 +488,18 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(mi.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default="",
+                    help="override dims of the config, e.g. T=2048,E=64 (for a smaller profiling "
+                         "case; the workload name then says so)")
     args = ap.parse_args()
     cfg = mi.CONFIGS[args.config]
+    if args.shape:
+        over = {k: int(v) for k, v in (kv.split("=") for kv in args.shape.split(","))}
+        bad = set(over) - {"T", "H", "I", "E", "k"}
+        if bad:
+            raise SystemExit(f"--shape takes T, H, I, E, k (got {sorted(bad)})")
+        cfg = cfg.with_(**over, name=f"{cfg.name}@{args.shape}", desc=f"{cfg.desc}; resized to " +
+                        " ".join(f"{k}={v}" for k, v in over.items()))
     if args.impl == "reference":
         reference_arm(args, cfg)
     else:

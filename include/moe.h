@@ -62,11 +62,15 @@ typedef enum {
 } moe_status_t;
 
 /* MOE_DTYPE_FP8_E4M3_UE8M0: e4m3 operands whose scales are powers of two
- * (MOE_SCALE_UE8M0), which the block-scaled tensor-core MMA applies itself. */
+ * (MOE_SCALE_UE8M0), which the block-scaled tensor-core MMA applies itself.
+ * MOE_DTYPE_FP4_E2M1: FP4 expert weights (e2m1, two per byte) with e8m0
+ * scales per (row, 32 K); activations e4m3 with power-of-two scales. Its
+ * workspace layout is the FP8 one. */
 typedef enum {
   MOE_DTYPE_BF16 = 0,
   MOE_DTYPE_FP8_E4M3 = 1,
-  MOE_DTYPE_FP8_E4M3_UE8M0 = 2
+  MOE_DTYPE_FP8_E4M3_UE8M0 = 2,
+  MOE_DTYPE_FP4_E2M1 = 3
 } moe_dtype_t;
 
 /* GEMM epilogues. The gated ones compute act(g) * u from the gate projection
@@ -285,6 +289,47 @@ moe_status_t moe_forward_fp8_gated(const void* x_dev, const void* wr_dev, const 
                                    const void* w2q_dev, const float* w2s_dev, moe_dims_t d,
                                    moe_epilogue_t act, void* out_dev, void* ws, size_t ws_bytes,
                                    void* stream);
+
+/* The layer with FP4 experts ([X] "FP8 and FP4 quantized experts": FP4
+ * expert weights packed two per byte with UE8M0 weight scales). The page
+ * gives no scale block; the OCP microscaling one is used: one scale per row
+ * per 32 consecutive K elements, the smallest power of two >= amax / 6 (1 for
+ * an all-zero block), stored as its e8m0 byte (biased exponent). Byte i of a
+ * row holds element 2i in its low nibble and 2i + 1 in its high nibble.
+ * x and the hidden activations are quantised as in moe_forward_fp8_ue8m0
+ * (e4m3, power-of-two scale per 128-group); both expert GEMMs run on the
+ * block-scaled MMA with e4m3 A and e2m1 B (kind::mxf8f6f4).
+ *   w13q_dev u8 [E, 2I, H/2], w13s_dev u8 [E, 2I, H/32]   (moe_quantize_weight_fp4)
+ *   w2q_dev  u8 [E, H, I/2],  w2s_dev  u8 [E, H, I/32]
+ *   packed weights 32-byte aligned, scales 4-byte aligned; H % 256 == 0
+ *   ws >= moe_workspace_size(d, MOE_DTYPE_FP4_E2M1) bytes; act as for
+ *   moe_forward_gated. */
+moe_status_t moe_forward_fp4(const void* x_dev, const void* wr_dev, const float* bias_dev,
+                             const void* w13q_dev, const uint8_t* w13s_dev, const void* w2q_dev,
+                             const uint8_t* w2s_dev, moe_dims_t d, moe_epilogue_t act,
+                             void* out_dev, void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped GEMM with FP4 weights (the two GEMMs of moe_forward_fp4):
+ *   A_dev        e4m3 [M_total, K], a_scales_dev fp32 [M_total, K/128] powers of two
+ *   B_dev        packed e2m1 [E, N_B, K/2] (32-byte aligned), N_B = 2N for a
+ *                gated epilogue (gate rows then up rows), N otherwise
+ *   b_scales_dev e8m0 bytes [E, N_B, K/32] (4-byte aligned)
+ *   C_dev        bf16 [M_total, N] (plain; N % 256 == 0), or with a gated
+ *                epilogue e4m3 [M_total, N] + c_scales_dev fp32 [M_total, N/128]
+ *                (power-of-two scales), or bf16 when c_scales_dev is NULL
+ *   offsets, E, ws as for moe_grouped_gemm. */
+moe_status_t moe_grouped_gemm_fp4(const void* A_dev, const float* a_scales_dev, const void* B_dev,
+                                  const uint8_t* b_scales_dev, const int32_t* offsets_dev,
+                                  int32_t M_total, int32_t E, int32_t N, int32_t K,
+                                  moe_epilogue_t ep, void* C_dev, float* c_scales_dev, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* FP4 weight quantisation (one-time preparation): nb matrices bf16 [rows,
+ * cols] (cols % 128 == 0) -> q_dev packed e2m1 [nb, rows, cols/2], s_dev e8m0
+ * bytes [nb, rows, cols/32], by the rule of moe_forward_fp4 with IEEE fp32
+ * division and round-to-nearest-even (ties to the even code). */
+moe_status_t moe_quantize_weight_fp4(const void* w_dev, int64_t nb, int64_t rows, int64_t cols,
+                                     void* q_dev, uint8_t* s_dev, void* stream);
 
 /* moe_forward with the token rows in HOST memory: copies x_host ([T, H]
  * bf16) to the workspace, runs the layer, copies the result to out_host

@@ -24,6 +24,7 @@ __all__ = [
     "MOE_EPILOGUE_GEGLU", "MOE_EPILOGUE_REGLU", "moe_forward_gated", "moe_forward_fp8_gated",
     "MOE_SCALE_F32", "MOE_SCALE_UE8M0", "moe_quantize_act_fp8_fmt", "moe_quantize_weight_fp8_fmt",
     "MOE_DTYPE_FP8_E4M3_UE8M0", "moe_forward_fp8_ue8m0",
+    "MOE_DTYPE_FP4_E2M1", "moe_forward_fp4", "moe_grouped_gemm_fp4", "moe_quantize_weight_fp4",
     "moe_last_error", "moe_abi_version", "moe_launch_count", "moe_workspace_size",
     "moe_workspace_layout", "moe_route_topk", "moe_topk_from_logits", "moe_permute",
     "moe_permute_noalloc",
@@ -34,7 +35,7 @@ __all__ = [
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_DEVICE = 0, 1, 2
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 3, 4, 5
-MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3, MOE_DTYPE_FP8_E4M3_UE8M0 = 0, 1, 2
+MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3, MOE_DTYPE_FP8_E4M3_UE8M0, MOE_DTYPE_FP4_E2M1 = 0, 1, 2, 3
 MOE_EPILOGUE_NONE, MOE_EPILOGUE_SWIGLU, MOE_EPILOGUE_GEGLU, MOE_EPILOGUE_REGLU = 0, 1, 2, 3
 MOE_SCALE_F32, MOE_SCALE_UE8M0 = 0, 1
 
@@ -82,6 +83,10 @@ _SIGS = {
                                      _vp]),
     "moe_forward_fp8_ue8m0": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _i32, _vp, _vp, _sz,
                                      _vp]),
+    "moe_forward_fp4": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _i32, _vp, _vp, _sz, _vp]),
+    "moe_grouped_gemm_fp4": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
+                                    _vp, _vp, _sz, _vp]),
+    "moe_quantize_weight_fp4": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "moe_quantize_act_fp8": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "moe_quantize_weight_fp8": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "moe_quantize_act_fp8_fmt": (_i32, [_vp, _i64, _i64, _vp, _vp, _i32, _vp]),
@@ -236,6 +241,24 @@ def moe_forward_fp8_ue8m0(x, wr, bias, w13q, w13s, w2q, w2s, d, act, out, ws, ws
     _check(lib().moe_forward_fp8_ue8m0(_p(x), _p(wr), _p(bias), _p(w13q), _p(w13s), _p(w2q),
                                        _p(w2s), _dims(d), int(act), _p(out), _p(ws),
                                        _nbytes(ws, ws_bytes), _s(stream)))
+
+
+def moe_forward_fp4(x, wr, bias, w13q, w13s, w2q, w2s, d, act, out, ws, ws_bytes=None,
+                    stream=None):
+    _check(lib().moe_forward_fp4(_p(x), _p(wr), _p(bias), _p(w13q), _p(w13s), _p(w2q), _p(w2s),
+                                 _dims(d), int(act), _p(out), _p(ws), _nbytes(ws, ws_bytes),
+                                 _s(stream)))
+
+
+def moe_grouped_gemm_fp4(A, a_scales, B, b_scales, offsets, M_total, E, N, K, ep, C,
+                         c_scales=None, ws=None, ws_bytes=None, stream=None):
+    _check(lib().moe_grouped_gemm_fp4(_p(A), _p(a_scales), _p(B), _p(b_scales), _p(offsets),
+                                      M_total, E, N, K, int(ep), _p(C), _p(c_scales), _p(ws),
+                                      _nbytes(ws, ws_bytes), _s(stream)))
+
+
+def moe_quantize_weight_fp4(w, nb, rows, cols, q, s, stream=None):
+    _check(lib().moe_quantize_weight_fp4(_p(w), nb, rows, cols, _p(q), _p(s), _s(stream)))
 
 
 def moe_forward_hostio(x_host, wr, bias, w13, w2, d, out_host, ws, ws_bytes=None, stream=None):

@@ -44,9 +44,12 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_
                                     int max_rows_per_expert, int32_t* status, cudaStream_t s,
                                     const char** why);
 cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const void* B,
-                                   const float* b_scales, const int32_t* offsets, int M_total,
-                                   int E, int N, int K, int act, void* Cout, float* c_scales,
-                                   int32_t* status, cudaStream_t s, const char** why);
+                                   const float* b_scales, const uint8_t* b_sf8,
+                                   const int32_t* offsets, int M_total, int E, int N, int K, int act,
+                                   void* Cout, float* c_scales, int32_t* status, cudaStream_t s,
+                                   const char** why);
+cudaError_t launch_quant_weight_fp4(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
+                                    uint8_t* sc, cudaStream_t s);
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
                              const int32_t* row_map, bool ue8m0, cudaStream_t s);
 cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
@@ -222,14 +225,14 @@ int64_t moe_launch_count(void) { return g_launches.load(); }
 
 size_t moe_workspace_size(moe_dims_t d, moe_dtype_t dt) {
   if (check_dims(d, true) != MOE_OK) return 0;
-  if (dt < MOE_DTYPE_BF16 || dt > MOE_DTYPE_FP8_E4M3_UE8M0) return 0;
+  if (dt < MOE_DTYPE_BF16 || dt > MOE_DTYPE_FP4_E2M1) return 0;
   return (size_t)layout(d, dt).total;
 }
 
 moe_status_t moe_workspace_layout(moe_dims_t d, moe_dtype_t dt, moe_ws_layout_t* out) {
   MOE_TRY(check_dims(d, true));
   if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
-  if (dt < MOE_DTYPE_BF16 || dt > MOE_DTYPE_FP8_E4M3_UE8M0) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
+  if (dt < MOE_DTYPE_BF16 || dt > MOE_DTYPE_FP4_E2M1) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
   *out = layout(d, dt);
   return ok();
 }
@@ -343,6 +346,8 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
   if (N < 128 || N % 128 || K < 128 || K % 128)
     return fail(MOE_ERR_INVALID_ARG, "N and K must be positive multiples of 128 (N=%d K=%d)", N, K);
   if (ep < MOE_EPILOGUE_NONE || ep > MOE_EPILOGUE_REGLU) return fail(MOE_ERR_INVALID_ARG, "bad epilogue");
+  if (dt == MOE_DTYPE_FP4_E2M1)
+    return fail(MOE_ERR_INVALID_ARG, "FP4 weights take moe_grouped_gemm_fp4 (e8m0 scale bytes)");
   if (dt < MOE_DTYPE_BF16 || dt > MOE_DTYPE_FP8_E4M3_UE8M0) return fail(MOE_ERR_INVALID_ARG, "bad dtype");
   if (dt == MOE_DTYPE_FP8_E4M3_UE8M0 && a_rows)
     return fail(MOE_ERR_INVALID_ARG, "the block-scaled GEMM takes no row gather");
@@ -375,10 +380,43 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
                                 (int)ep, C, c_scales, max_rows_per_expert,
                                 at<int32_t>(ws, 0), static_cast<cudaStream_t>(stream), &why);
   else
-    e = launch_grouped_gemm_mx(A, a_scales, B, b_scales, offsets, M_total, E, N, K, (int)ep, C,
-                               c_scales, at<int32_t>(ws, 0), static_cast<cudaStream_t>(stream),
-                               &why);
+    e = launch_grouped_gemm_mx(A, a_scales, B, b_scales, nullptr, offsets, M_total, E, N, K,
+                               (int)ep, C, c_scales, at<int32_t>(ws, 0),
+                               static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "grouped GEMM: %s %s", cudaGetErrorString(e), why);
+  return ok();
+}
+
+moe_status_t moe_grouped_gemm_fp4(const void* A, const float* a_scales, const void* B,
+                                  const uint8_t* b_scales, const int32_t* offsets, int32_t M_total,
+                                  int32_t E, int32_t N, int32_t K, moe_epilogue_t ep, void* C,
+                                  float* c_scales, void* ws, size_t ws_bytes, void* stream) {
+  if (M_total < 1) return fail(MOE_ERR_INVALID_ARG, "M_total must be >= 1");
+  if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 1024]");
+  if (N < 128 || N % 128 || K < 128 || K % 128)
+    return fail(MOE_ERR_INVALID_ARG, "N and K must be positive multiples of 128 (N=%d K=%d)", N, K);
+  if (ep < MOE_EPILOGUE_NONE || ep > MOE_EPILOGUE_REGLU) return fail(MOE_ERR_INVALID_ARG, "bad epilogue");
+  if (ep == MOE_EPILOGUE_NONE && N % 256)
+    return fail(MOE_ERR_INVALID_ARG, "the plain FP4 GEMM needs N %% 256 == 0 (N=%d)", N);
+  MOE_TRY(check_ptr(A, "A"));
+  MOE_TRY(check_ptr(a_scales, "a_scales"));
+  MOE_TRY(check_ptr(B, "B"));
+  if (reinterpret_cast<uintptr_t>(B) & 31) return fail(MOE_ERR_INVALID_ARG, "B must be 32-byte aligned");
+  if (!b_scales || (reinterpret_cast<uintptr_t>(b_scales) & 3))
+    return fail(MOE_ERR_INVALID_ARG, "b_scales must be non-NULL and 4-byte aligned");
+  MOE_TRY(check_ptr(offsets, "expert_offsets"));
+  MOE_TRY(check_ptr(C, "C"));
+  MOE_TRY(check_ptr(c_scales, "c_scales", true));
+  if (c_scales && ep == MOE_EPILOGUE_NONE)
+    return fail(MOE_ERR_INVALID_ARG, "c_scales (quantised output) needs a gated epilogue");
+  MOE_TRY(check_ptr(ws, "ws"));
+  if (ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes", ws_bytes);
+  MOE_TRY(check_device());
+  const char* why = "";
+  cudaError_t e = launch_grouped_gemm_mx(A, a_scales, B, nullptr, b_scales, offsets, M_total, E, N,
+                                         K, (int)ep, C, c_scales, at<int32_t>(ws, 0),
+                                         static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "FP4 grouped GEMM: %s %s", cudaGetErrorString(e), why);
   return ok();
 }
 
@@ -458,7 +496,8 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
     void* hq = at<void>(ws, L.hq);
     float* hs = at<float>(ws, L.hs);
     // x is quantised once per token, then its codes and scales are permuted
-    const bool ue8m0 = dt == MOE_DTYPE_FP8_E4M3_UE8M0;
+    const bool fp4 = dt == MOE_DTYPE_FP4_E2M1;  // w13s / w2s hold e8m0 bytes then
+    const bool ue8m0 = dt == MOE_DTYPE_FP8_E4M3_UE8M0 || fp4;
     if ((e = launch_quant_act(x, T, H, xq, xs, nullptr, ue8m0, s)) != cudaSuccess)
       return cuda_fail(e, "activation quantisation");
     if ((e = permute_gather(xq, H, xq_perm, xs, (H / 128) * 4, xs_perm)) != cudaSuccess)
@@ -466,13 +505,17 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
     record(s, 2);
     if (ue8m0) {
       // power-of-two scales: the block-scaled tensor-core path, no promotion
-      if ((e = launch_grouped_gemm_mx(xq_perm, xs_perm, w13, w13s, offsets, R, E, I, H, act, hq, hs,
-                                      status, s, &why)) != cudaSuccess)
-        return fail(MOE_ERR_CUDA, "FP8 GEMM1: %s %s", cudaGetErrorString(e), why);
+      const float* f13 = fp4 ? nullptr : w13s;
+      const float* f2 = fp4 ? nullptr : w2s;
+      const uint8_t* b13 = fp4 ? reinterpret_cast<const uint8_t*>(w13s) : nullptr;
+      const uint8_t* b2 = fp4 ? reinterpret_cast<const uint8_t*>(w2s) : nullptr;
+      if ((e = launch_grouped_gemm_mx(xq_perm, xs_perm, w13, f13, b13, offsets, R, E, I, H, act, hq,
+                                      hs, status, s, &why)) != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "%s GEMM1: %s %s", fp4 ? "FP4" : "FP8", cudaGetErrorString(e), why);
       record(s, 3);
-      if ((e = launch_grouped_gemm_mx(hq, hs, w2, w2s, offsets, R, E, H, I, 0, y_perm, nullptr,
+      if ((e = launch_grouped_gemm_mx(hq, hs, w2, f2, b2, offsets, R, E, H, I, 0, y_perm, nullptr,
                                       status, s, &why)) != cudaSuccess)
-        return fail(MOE_ERR_CUDA, "FP8 GEMM2: %s %s", cudaGetErrorString(e), why);
+        return fail(MOE_ERR_CUDA, "%s GEMM2: %s %s", fp4 ? "FP4" : "FP8", cudaGetErrorString(e), why);
     } else {
       if ((e = launch_grouped_gemm_fp8(xq_perm, nullptr, R, xs_perm, w13, w13s, offsets, R, E, I, H,
                                        act, hq, hs, T, status, s, &why)) != cudaSuccess)
@@ -562,6 +605,29 @@ moe_status_t moe_forward_fp8_ue8m0(const void* x, const void* wr, const float* b
                       MOE_DTYPE_FP8_E4M3_UE8M0, static_cast<cudaStream_t>(stream));
 }
 
+moe_status_t moe_forward_fp4(const void* x, const void* wr, const float* bias, const void* w13q,
+                             const uint8_t* w13s, const void* w2q, const uint8_t* w2s, moe_dims_t d,
+                             moe_epilogue_t act, void* out, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_dims(d, true));
+  MOE_TRY(check_act(act));
+  MOE_TRY(check_ptr(x, "x"));
+  MOE_TRY(check_ptr(wr, "w_router"));
+  MOE_TRY(check_ptr(bias, "bias", true));
+  MOE_TRY(check_ptr(w13q, "w13q"));
+  MOE_TRY(check_ptr(w2q, "w2q"));
+  if ((reinterpret_cast<uintptr_t>(w13q) | reinterpret_cast<uintptr_t>(w2q)) & 31)
+    return fail(MOE_ERR_INVALID_ARG, "packed FP4 weights must be 32-byte aligned");
+  if (!w13s || !w2s || ((reinterpret_cast<uintptr_t>(w13s) | reinterpret_cast<uintptr_t>(w2s)) & 3))
+    return fail(MOE_ERR_INVALID_ARG, "w13s / w2s must be non-NULL and 4-byte aligned");
+  MOE_TRY(check_ptr(out, "out"));
+  if (d.H % 256) return fail(MOE_ERR_INVALID_ARG, "the FP4 layer needs H %% 256 == 0 (got %d)", d.H);
+  MOE_TRY(check_ws(d, MOE_DTYPE_FP4_E2M1, ws, ws_bytes));
+  MOE_TRY(check_device());
+  return forward_impl(x, wr, bias, w13q, reinterpret_cast<const float*>(w13s), w2q,
+                      reinterpret_cast<const float*>(w2s), d, (int)act, out, ws, MOE_DTYPE_FP4_E2M1,
+                      static_cast<cudaStream_t>(stream));
+}
+
 moe_status_t moe_forward_fp8(const void* x, const void* wr, const float* bias, const void* w13q,
                              const float* w13s, const void* w2q, const float* w2s, moe_dims_t d,
                              void* out, void* ws, size_t ws_bytes, void* stream) {
@@ -632,6 +698,19 @@ moe_status_t moe_quantize_weight_fp8_fmt(const void* w, int64_t nb, int64_t rows
 moe_status_t moe_quantize_weight_fp8(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                      float* sc, void* stream) {
   return moe_quantize_weight_fp8_fmt(w, nb, rows, cols, q, sc, MOE_SCALE_F32, stream);
+}
+
+moe_status_t moe_quantize_weight_fp4(const void* w, int64_t nb, int64_t rows, int64_t cols,
+                                     void* q, uint8_t* sc, void* stream) {
+  if (nb < 1 || rows < 1 || cols < 128 || cols % 128)
+    return fail(MOE_ERR_INVALID_ARG, "nb >= 1, rows >= 1 and cols a multiple of 128");
+  MOE_TRY(check_ptr(w, "w"));
+  MOE_TRY(check_ptr(q, "q"));
+  if (!sc) return fail(MOE_ERR_INVALID_ARG, "s is NULL");
+  MOE_TRY(check_device());
+  cudaError_t e = launch_quant_weight_fp4(w, nb, rows, cols, q, sc, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "FP4 weight quantisation");
+  return ok();
 }
 
 moe_status_t moe_get_device_status(const void* ws, int32_t* status_out) {

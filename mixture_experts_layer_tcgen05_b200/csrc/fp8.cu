@@ -126,4 +126,71 @@ cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t
   return cudaGetLastError();
 }
 
+// FP4 expert weights ("Experts backends", "FP8 and FP4 quantized experts":
+// e2m1 codes packed two per byte with UE8M0 scales). One scale per row per
+// 32 consecutive K elements (the OCP microscaling block): the smallest power
+// of two >= amax / 6 (fp32 quotient), p clamped to [-127, 127], 1 for an
+// all-zero block, stored as its biased exponent. Element 2i goes to the low
+// nibble of byte i.
+
+// e2m1 code of v (|v| <= 6 here): nearest of 0, 0.5, 1, 1.5, 2, 3, 4, 6, ties
+// to the even code; larger magnitudes saturate to 6; the sign bit is kept.
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  const float a = fabsf(v);
+  uint32_t c;
+  if (a <= 0.25f) c = 0;
+  else if (a < 0.75f) c = 1;
+  else if (a <= 1.25f) c = 2;
+  else if (a < 1.75f) c = 3;
+  else if (a <= 2.5f) c = 4;
+  else if (a < 3.5f) c = 5;
+  else if (a <= 5.0f) c = 6;
+  else c = 7;
+  return (signbit(v) ? 8u : 0u) | c;
+}
+
+// One thread per 32-element block: 64 bytes in, 16 bytes of codes and one
+// scale byte out.
+__global__ void __launch_bounds__(256) quant_weight_fp4_kernel(const uint4* __restrict__ w,
+                                                               int64_t nblocks,
+                                                               uint4* __restrict__ q,
+                                                               uint8_t* __restrict__ sc) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nblocks) return;
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 u = w[i * 4 + j];
+    const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      v[8 * j + 2 * t] = bf16lo_to_f32(uw[t]);
+      v[8 * j + 2 * t + 1] = bf16hi_to_f32(uw[t]);
+    }
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  float s = 1.0f;
+  if (amax > 0.0f) {
+    int e;
+    const float m = frexpf(__fdiv_rn(amax, 6.0f), &e);
+    s = ldexpf(1.0f, min(max(m == 0.5f ? e - 1 : e, -127), 127));
+  }
+  uint32_t out[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 32; ++j) out[j >> 3] |= e2m1_code(__fdiv_rn(v[j], s)) << (4 * (j & 7));
+  q[i] = make_uint4(out[0], out[1], out[2], out[3]);
+  sc[i] = (uint8_t)((__float_as_uint(s) >> 23) & 0xFFu);  // 2^-127 is the one code-0 (subnormal) scale
+}
+
+cudaError_t launch_quant_weight_fp4(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
+                                    uint8_t* sc, cudaStream_t s) {
+  const int64_t nblocks = nb * rows * (cols / 32);
+  quant_weight_fp4_kernel<<<(unsigned)ceil_div(nblocks, 256), 256, 0, s>>>(
+      static_cast<const uint4*>(w), nblocks, static_cast<uint4*>(q), sc);
+  note_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace moe

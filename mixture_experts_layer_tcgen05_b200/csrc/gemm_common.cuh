@@ -62,6 +62,45 @@ __device__ void build_tile_starts(const int32_t* offsets, int E, int NT, int32_t
   if (lane == 0) tile_start[E] = carry;
 }
 
+// The order the persistent CTAs take tiles in. Experts with one row tile
+// stream their whole weight matrix for it (memory-bound tiles); experts with
+// more row tiles share each weight strip among their row tiles (tensor-bound
+// tiles). Both kinds are spread evenly over the schedule, so that at any
+// moment some CTAs stream weights while the others keep the tensor cores
+// busy: ts[0..E] are the tile prefix sums of the multi-tile experts,
+// ts[E+1..2E+1] those of the single-tile experts, and schedule position t is
+// a single-tile one when floor((t+1) NS / N) > floor(t NS / N). Warp-wide.
+template <int kRowsPerTile>
+__device__ void build_tile_starts_mixed(const int32_t* offsets, int E, int NT, int32_t* ts) {
+  const int lane = threadIdx.x & 31;
+  int32_t carry_b = 0, carry_s = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    const int32_t cnt = e < E ? max(offsets[e + 1] - offsets[e], 0) : 0;
+    const int32_t mt = (cnt + kRowsPerTile - 1) / kRowsPerTile;
+    const int32_t tb = mt >= 2 ? mt * NT : 0, tsm = mt == 1 ? NT : 0;
+    int32_t ib = tb, is = tsm;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t vb = __shfl_up_sync(0xffffffffu, ib, off);
+      const int32_t vs = __shfl_up_sync(0xffffffffu, is, off);
+      if (lane >= off) ib += vb, is += vs;
+    }
+    if (e < E) {
+      ts[e] = carry_b + ib - tb;
+      ts[E + 1 + e] = carry_s + is - tsm;
+    }
+    carry_b += __shfl_sync(0xffffffffu, ib, 31);
+    carry_s += __shfl_sync(0xffffffffu, is, 31);
+  }
+  if (lane == 0) {
+    ts[E] = carry_b;
+    ts[2 * E + 1] = carry_s;
+  }
+}
+
+__device__ __forceinline__ int mixed_total(const int32_t* ts, int E) { return ts[E] + ts[2 * E + 1]; }
+
 // Largest e with tile_start[e] <= tile (that expert is non-empty).
 __device__ __forceinline__ int find_expert(const int32_t* tile_start, int E, int tile) {
   int lo = 0, hi = E;
@@ -71,6 +110,24 @@ __device__ __forceinline__ int find_expert(const int32_t* tile_start, int E, int
     else hi = mid;
   }
   return lo;
+}
+
+// Schedule position -> (expert, tile index inside the expert), for the order
+// of build_tile_starts_mixed.
+__device__ __forceinline__ int mixed_decode(const int32_t* ts, int E, int tile, int& local) {
+  const int32_t* big = ts;
+  const int32_t* small = ts + E + 1;
+  const int64_t ns = small[E], n = (int64_t)big[E] + ns;
+  const int sb = (int)((int64_t)tile * ns / n), sa = (int)((int64_t)(tile + 1) * ns / n);
+  if (sa > sb) {
+    const int e = find_expert(small, E, sb);
+    local = sb - small[e];
+    return e;
+  }
+  const int i = tile - sb;
+  const int e = find_expert(big, E, i);
+  local = i - big[e];
+  return e;
 }
 
 // ------------------------------------------------------------------ utils
@@ -150,6 +207,23 @@ inline bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, 
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Packed 4-bit codes [rows, K] (two per byte, element 2i in the low nibble)
+// loaded into the unpacked shared layout (16 codes per 16 bytes), 128 codes
+// (one 128-byte swizzled row) by box_rows rows per box. Needs a 32-byte
+// aligned base and K % 64 == 0.
+inline bool make_tmap_fp4(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

@@ -17,6 +17,12 @@
 // group g in TMEM column g and K step j in byte j, which the MMA selects
 // with its scale-factor ids.
 //
+// FP4 weights (BFP4): B holds packed e2m1 codes, two per byte, loaded by TMA
+// into the 16-byte-aligned unpacked shared layout the f8f6f4 MMA reads (16
+// codes per 16 bytes), so a stage still covers 128 K in 128-byte rows; A stays
+// e4m3 (kind::mxf8f6f4 mixes the two formats). B's scales are e8m0 codes per
+// (row, 32 K): the four bytes of a row for one stage are its four K steps.
+//
 // Warp roles (320 threads): warp 0 TMA producer, all 32 lanes building the
 // scale chunks; warp 1 TMEM allocator + MMA issuer; warps 2..9 epilogue.
 // One accumulator (256 TMEM columns, the rest holds the scale-factor ring):
@@ -39,13 +45,14 @@ constexpr int kTileA = BM * BK;  // 16 KB
 constexpr int kTileB = BN * BK;  // 32 KB
 constexpr int kStage = kTileA + kTileB;
 constexpr int STAGES = 4;
+constexpr int kPre = 4;       // stages of scales the producer loads ahead
 constexpr int kSfA = 512;        // scale chunk bytes for 128 rows of A
 constexpr int kSfStage = 3 * kSfA;  // A chunk + two B chunks
 constexpr int kMaxE = 1024;
 constexpr int kSfCol0 = 256;     // TMEM columns of the scale-factor ring
 constexpr int kSfColsPerStage = 16;
 constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + (size_t)STAGES * kSfStage + 256 +
-                         (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
+                         2 * (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
 
 struct Args {
   const int32_t* offsets;
@@ -55,7 +62,9 @@ struct Args {
   void* C;                // bf16 [M_total, ldc], or e4m3 when c_scales != nullptr
   float* c_scales;        // power-of-two scales of C's 128-groups
   const float* a_scales;  // [M_total, kblocks], powers of two
-  const float* b_scales;  // [E, b_nblk, kblocks], powers of two
+  const float* b_scales;  // [E, b_nblk, kblocks], powers of two (e4m3 B)
+  const uint8_t* b_sf8;   // [E * b_rows, K / 32] e8m0 codes (e2m1 B)
+  int b_sf_ld;            // K / 32
   int32_t* status;
 };
 
@@ -95,11 +104,12 @@ __device__ __forceinline__ void sf_copy(uint32_t tmem, uint64_t desc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(desc) : "memory");
 }
 
-// Block-scaled instruction descriptor: e4m3 x e4m3, fp32 accumulate, E8M0
-// scales, scale-factor ids (the K step) for A and B.
-__host__ __device__ constexpr uint32_t mx_idesc(int M, int N, uint32_t sf_id) {
+// Block-scaled instruction descriptor: e4m3 x (e4m3 or e2m1), fp32
+// accumulate, E8M0 scales, scale-factor ids (the K step) for A and B.
+constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
+__host__ __device__ constexpr uint32_t mx_idesc(int M, int N, uint32_t sf_id, uint32_t b_fmt) {
   return (sf_id << 4)                    // B scale-factor id
-         | (0u << 7) | (0u << 10)         // A, B formats: E4M3
+         | (0u << 7) | (b_fmt << 10)      // A format E4M3; B format E4M3 (0) or E2M1 (5)
          | ((uint32_t)(N >> 3) << 17)     // N / 8
          | (1u << 23)                     // scale format E8M0
          | ((uint32_t)(M >> 4) << 24)     // M / 16
@@ -118,8 +128,9 @@ __device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t
       : "memory");
 }
 
-// ACT: gated activation of the epilogue (kActNone: plain GEMM).
-template <int ACT>
+// ACT: gated activation of the epilogue (kActNone: plain GEMM); BFP4: B is
+// packed e2m1 with e8m0 scales per (row, 32 K).
+template <int ACT, bool BFP4>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    Args args) {
@@ -132,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // bars: full[STAGES], empty[STAGES], accf, acce, drain, redbar[2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
   int32_t* tile_start = reinterpret_cast<int32_t*>(sf + STAGES * kSfStage + 256);
-  float* red = reinterpret_cast<float*>(tile_start + kMaxE + 1);  // [2 tiles][2 halves][BM]
+  float* red = reinterpret_cast<float*>(tile_start + 2 * (kMaxE + 1));  // [2 tiles][2 halves][BM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = ptx::smem_addr(smem), sfbase = ptx::smem_addr(sf);
@@ -158,17 +169,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
     ptx::tmem_relinquish();
   }
-  if (warp == 2) gg::build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start);
+  if (warp == 2) gg::build_tile_starts_mixed<BM>(args.offsets, args.E, args.NT, tile_start);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = tile_start[args.E];
+  const int total = gg::mixed_total(tile_start, args.E);
   const int nkb = args.kblocks;
 
   auto decode = [&](int tile, int& e, int& m, int& n) {
-    e = gg::find_expert(tile_start, args.E, tile);
-    const int local = tile - tile_start[e];
+    int local;
+    e = gg::mixed_decode(tile_start, args.E, tile, local);
     const int cnt = args.offsets[e + 1] - args.offsets[e];
     const int mt = (cnt + BM - 1) / BM;
     const int bsz = args.band * args.NT;
@@ -208,9 +219,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = row0 + g * 32 + lane;
         sa[g] = r < row_end ? args.a_scales + (int64_t)r * nkb : nullptr;  // rows past the expert: scale 1
       }
+      // scales of the next kPre stages, loaded ahead so that their latency
+      // overlaps the wait for a free stage
+      const uint8_t* sf8[8];  // e2m1 B: scale rows lane + 32g of both boxes
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        sf8[g] = BFP4 ? args.b_sf8 + (int64_t)(rb0 + 32 * g + lane) * args.b_sf_ld : nullptr;
+        sf8[4 + g] = BFP4 ? args.b_sf8 + (int64_t)(rb1 + 32 * g + lane) * args.b_sf_ld : nullptr;
+      }
+      float pa[kPre][4], pb[kPre][2];
+      uint32_t pw[kPre][BFP4 ? 8 : 1];
+      auto fetch = [&](int kb, float (&a)[4], float (&b)[2], uint32_t (&wv)[BFP4 ? 8 : 1]) {
+        if (kb < nkb) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) a[g] = sa[g] ? __ldg(sa[g] + kb) : 1.0f;
+          if constexpr (BFP4) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g) wv[g] = __ldg(reinterpret_cast<const uint32_t*>(sf8[g]) + kb);
+          } else {
+            b[0] = __ldg(sb0 + kb);
+            b[1] = __ldg(sb1 + kb);
+          }
+        }
+      };
+#pragma unroll
+      for (int i = 0; i < kPre; ++i) fetch(i, pa[i], pb[i], pw[i]);
       for (int kb = 0; kb < nkb; ++kb, ++issued) {
         const int s = (int)(issued % STAGES);
         const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
+        float ca[4] = {pa[0][0], pa[0][1], pa[0][2], pa[0][3]};
+        const float cb0 = pb[0][0], cb1 = pb[0][1];
+        uint32_t cw[BFP4 ? 8 : 1];
+#pragma unroll
+        for (int g = 0; g < (BFP4 ? 8 : 1); ++g) cw[g] = pw[0][g];
+#pragma unroll
+        for (int i = 0; i + 1 < kPre; ++i) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) pa[i][g] = pa[i + 1][g];
+          pb[i][0] = pb[i + 1][0];
+          pb[i][1] = pb[i + 1][1];
+#pragma unroll
+          for (int g = 0; g < (BFP4 ? 8 : 1); ++g) pw[i][g] = pw[i + 1][g];
+        }
+        fetch(kb + kPre, pa[kPre - 1], pb[kPre - 1], pw[kPre - 1]);
         int got = 1;
         if (lane == 0) got = ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty);
         if (!__shfl_sync(0xffffffffu, got, 0)) {
@@ -220,20 +271,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // scale chunks of this stage
         uint32_t w[4];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t c = sa[g] ? e8m0_code(sa[g][kb]) : 127u;
-          w[g] = c * 0x01010101u;  // the same scale for the stage's four K steps
-        }
+        for (int g = 0; g < 4; ++g) w[g] = e8m0_code(ca[g]) * 0x01010101u;  // same for the four K steps
         unsigned char* sfs = sf + s * kSfStage;
         *reinterpret_cast<uint4*>(sfs + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        const uint32_t c0 = e8m0_code(sb0[kb]) * 0x01010101u, c1 = e8m0_code(sb1[kb]) * 0x01010101u;
-        *reinterpret_cast<uint4*>(sfs + kSfA + lane * 16) = make_uint4(c0, c0, c0, c0);
-        *reinterpret_cast<uint4*>(sfs + 2 * kSfA + lane * 16) = make_uint4(c1, c1, c1, c1);
+        if constexpr (BFP4) {  // per-row codes, one byte per K step
+          *reinterpret_cast<uint4*>(sfs + kSfA + lane * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          *reinterpret_cast<uint4*>(sfs + 2 * kSfA + lane * 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        } else {
+          const uint32_t c0 = e8m0_code(cb0) * 0x01010101u, c1 = e8m0_code(cb1) * 0x01010101u;
+          *reinterpret_cast<uint4*>(sfs + kSfA + lane * 16) = make_uint4(c0, c0, c0, c0);
+          *reinterpret_cast<uint4*>(sfs + 2 * kSfA + lane * 16) = make_uint4(c1, c1, c1, c1);
+        }
         ptx::fence_proxy_async_smem();  // generic-proxy writes -> visible to tcgen05.cp
         __syncwarp();
         if (lane == 0) {
           const uint32_t sa_ = sbase + s * kStage, sb_ = sa_ + kTileA;
-          ptx::mbar_arrive_expect_tx(full0 + s * 8, kStage);
+          // packed e2m1: the transaction counts the bytes read (two codes per byte)
+          ptx::mbar_arrive_expect_tx(full0 + s * 8, BFP4 ? kTileA + kTileB / 2 : kStage);
           ptx::tma_load_2d(sa_, &tmA, kb * BK, row0, full0 + s * 8);
           ptx::tma_load_2d(sb_, &tmB, kb * BK, rb0, full0 + s * 8);
           ptx::tma_load_2d(sb_ + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
@@ -270,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk)
             mma_mx(tmem_base, da + (uint64_t)(kk * UK / 16), db + (uint64_t)(kk * UK / 16),
-                   mx_idesc(BM, BN, (uint32_t)kk), sfcol, sfcol + 4, (kb | kk) != 0);
+                   mx_idesc(BM, BN, (uint32_t)kk, BFP4 ? kFmtE2M1 : kFmtE4M3), sfcol, sfcol + 4,
+                   (kb | kk) != 0);
           ptx::mma_commit(empty0 + s * 8);
         }
         if (!ok) break;
@@ -298,25 +353,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain this thread's 128 accumulator columns, then release the accumulator
       float acc[128];
       if (SWIGLU) {
-        // gate cols [half*64, +64) -> acc[0..64), up cols [128 + half*64, +64) -> acc[64..128)
+        // gate cols [half*64, +64) -> acc[0..64), up cols [128 + half*64, +64) -> acc[64..128);
+        // all four loads in flight before one wait
+        uint32_t raw[4][32];
+        ptx::tmem_ld32(lane_addr + half * 64, raw[0]);
+        ptx::tmem_ld32(lane_addr + half * 64 + 32, raw[1]);
+        ptx::tmem_ld32(lane_addr + 128 + half * 64, raw[2]);
+        ptx::tmem_ld32(lane_addr + 128 + half * 64 + 32, raw[3]);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 64; c += 32) {
-          uint32_t g[32], u[32];
-          ptx::tmem_ld32(lane_addr + half * 64 + c, g);
-          ptx::tmem_ld32(lane_addr + 128 + half * 64 + c, u);
-          ptx::tmem_wait_ld();
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[c + i] = __uint_as_float(g[i]), acc[64 + c + i] = __uint_as_float(u[i]);
-        }
+          for (int i = 0; i < 32; ++i) acc[32 * j + i] = __uint_as_float(raw[j][i]);
       } else {
+        uint32_t raw[4][32];
 #pragma unroll
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t v[32];
-          ptx::tmem_ld32(lane_addr + half * 128 + c, v);
-          ptx::tmem_wait_ld();
+        for (int j = 0; j < 4; ++j) ptx::tmem_ld32(lane_addr + half * 128 + 32 * j, raw[j]);
+        ptx::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[c + i] = __uint_as_float(v[i]);
-        }
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[32 * j + i] = __uint_as_float(raw[j][i]);
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -388,18 +445,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Block-scaled FP8 grouped GEMM with power-of-two scales (see
 // launch_grouped_gemm_fp8 for the operands; scales are fp32 powers of two).
 cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const void* B,
-                                   const float* b_scales, const int32_t* offsets, int M_total,
-                                   int E, int N, int K, int act, void* Cout, float* c_scales,
-                                   int32_t* status, cudaStream_t s, const char** why) {
+                                   const float* b_scales, const uint8_t* b_sf8,
+                                   const int32_t* offsets, int M_total, int E, int N, int K, int act,
+                                   void* Cout, float* c_scales, int32_t* status, cudaStream_t s,
+                                   const char** why) {
   const bool swiglu = act != kActNone;
+  const bool fp4 = b_sf8 != nullptr;
   const int b_rows = swiglu ? 2 * N : N;
   if (!swiglu && N % 256 != 0) {
     *why = "the block-scaled plain GEMM needs N % 256 == 0";
     return cudaErrorInvalidValue;
   }
+  if (fp4 && (reinterpret_cast<uintptr_t>(B) & 31)) {
+    *why = "packed FP4 weights must be 32-byte aligned";
+    return cudaErrorInvalidValue;
+  }
   CUtensorMap tmA, tmB;
-  if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M_total, 128) ||
-      !make_tmap(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (int64_t)E * b_rows, 128)) {
+  const bool okB = fp4 ? make_tmap_fp4(&tmB, B, K, (int64_t)E * b_rows, 128)
+                       : make_tmap(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (int64_t)E * b_rows, 128);
+  if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M_total, 128) || !okB) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
@@ -419,19 +483,27 @@ cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const v
   a.c_scales = c_scales;
   a.a_scales = a_scales;
   a.b_scales = b_scales;
+  a.b_sf8 = b_sf8;
+  a.b_sf_ld = K / 32;
   a.status = status;
   const int64_t tiles_ub = ((int64_t)M_total / ggmx::BM + (M_total < E ? M_total : E)) * a.NT;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_ub));
-#define MOE_MX(ACTV)                                                                      \
-  do {                                                                                    \
-    cudaError_t e = set_smem(ggmx::gemm_mx_kernel<ACTV>, ggmx::kSmem);                    \
-    if (e != cudaSuccess) return e;                                                       \
-    ggmx::gemm_mx_kernel<ACTV><<<grid, ggmx::kThreads, ggmx::kSmem, s>>>(tmA, tmB, a);    \
+#define MOE_MX(ACTV, F4)                                                                      \
+  do {                                                                                        \
+    cudaError_t e = set_smem(ggmx::gemm_mx_kernel<ACTV, F4>, ggmx::kSmem);                    \
+    if (e != cudaSuccess) return e;                                                           \
+    ggmx::gemm_mx_kernel<ACTV, F4><<<grid, ggmx::kThreads, ggmx::kSmem, s>>>(tmA, tmB, a);    \
   } while (0)
-  if (act == kActSilu) MOE_MX(kActSilu);
-  else if (act == kActGelu) MOE_MX(kActGelu);
-  else if (act == kActRelu) MOE_MX(kActRelu);
-  else MOE_MX(kActNone);
+#define MOE_MX_ACT(F4)                         \
+  do {                                         \
+    if (act == kActSilu) MOE_MX(kActSilu, F4); \
+    else if (act == kActGelu) MOE_MX(kActGelu, F4); \
+    else if (act == kActRelu) MOE_MX(kActRelu, F4); \
+    else MOE_MX(kActNone, F4);                 \
+  } while (0)
+  if (fp4) MOE_MX_ACT(true);
+  else MOE_MX_ACT(false);
+#undef MOE_MX_ACT
 #undef MOE_MX
   note_launch();
   return cudaGetLastError();

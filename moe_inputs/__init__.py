@@ -125,6 +125,7 @@ class LayerConfig:
     zipf_s: float = 1.1
     fp8: bool = False
     ue8m0: bool = False         # FP8 scales as powers of two (block-scaled tensor-core path)
+    fp4: bool = False           # FP4 (e2m1) expert weights with e8m0 scales per (row, 32)
     x_sigma: float = 1.0
     w_sigma: float = 0.02
     seed: int = 0
@@ -161,6 +162,13 @@ CONFIGS = {
                                           bias="zipf", subset=512, fp8=True, ue8m0=True,
                                           desc="fine-grained prefill, FP8 experts with power-of-two "
                                                "(UE8M0) scales on the block-scaled MMA"),
+    "fine_grained_fp4": LayerConfig("fine_grained_fp4", 8192, 7168, 2048, 256, 8, bias="zipf",
+                                    subset=512, fp4=True,
+                                    desc="fine-grained prefill, FP4 (e2m1) expert weights with "
+                                         "UE8M0 scales per 32, e4m3 activations"),
+    "mixtral_decode_fp4": LayerConfig("mixtral_decode_fp4", 16, 4096, 14336, 8, 2, fp4=True,
+                                      desc="Mixtral-shaped decode, FP4 expert weights: T=16 "
+                                           "H=4096 I=14336 E=8 k=2"),
     "mixtral_decode_fp8": LayerConfig("mixtral_decode_fp8", 16, 4096, 14336, 8, 2, fp8=True,
                                       desc="Mixtral-shaped decode, FP8 experts: T=16 H=4096 "
                                            "I=14336 E=8 k=2"),

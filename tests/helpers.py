@@ -29,6 +29,20 @@ def check_close(out, ref, tol=BF16_TOL, what="output"):
     return max_rel, l1_rel
 
 
+def quant_pow2_e4m3(h):
+    """Per row, per 128 group: s = smallest power of two >= amax/448 (fp32),
+    q = e4m3(h/s) by torch's cast. Returns (codes uint8, scales fp32)."""
+    import torch
+    rows, cols = h.shape
+    g = h.reshape(rows, cols // 128, 128)
+    amax = np.abs(g).max(2).astype(np.float32)
+    m, e = np.frexp(amax / np.float32(448))
+    s = np.where(amax > 0, np.ldexp(np.float32(1), np.where(m == 0.5, e - 1, e)), 1.0).astype(np.float32)
+    q = torch.from_numpy((g / s[:, :, None]).astype(np.float32).reshape(rows, cols)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return q, s
+
+
 def dev_bf16(a: np.ndarray):
     import torch
     a = np.ascontiguousarray(a, dtype=np.uint16)

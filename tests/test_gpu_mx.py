@@ -12,7 +12,8 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from helpers import FP8_TOL, check_close, dev, dev_bf16, dev_u8, host_bf16, layer_host
+from helpers import (FP8_TOL, check_close, dev, dev_bf16, dev_u8, host_bf16, layer_host,
+                     quant_pow2_e4m3)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -67,19 +68,6 @@ def test_mx_grouped_gemm_plain(counts, N, K, unit):
             check_close(got[lo:hi], A[lo:hi] @ Bd[e].T, (2e-2, 5e-3), f"expert {e}")
 
 
-def _quant_pow2(h):
-    """Per row, per 128 group: s = smallest power of two >= amax/448, q = e4m3(h/s)."""
-    rows, cols = h.shape
-    g = h.reshape(rows, cols // 128, 128)
-    amax = np.abs(g).max(2).astype(np.float32)
-    r = amax / np.float32(448)
-    m, e = np.frexp(r)
-    s = np.where(amax > 0, np.ldexp(np.float32(1), np.where(m == 0.5, e - 1, e)), 1.0).astype(np.float32)
-    q = torch.from_numpy((g / s[:, :, None]).astype(np.float32).reshape(rows, cols)).to(
-        torch.float8_e4m3fn).view(torch.uint8).numpy()
-    return q, s
-
-
 @pytest.mark.parametrize("counts,N,K", [([0, 1, 130, 300], 256, 384), ([256, 7], 512, 256)])
 def test_mx_grouped_gemm_swiglu_quantised_out(counts, N, K):
     E, offsets, M, aq, as_, bq, bs = _problem(counts, 2 * N, K, 93)
@@ -103,7 +91,7 @@ def test_mx_grouped_gemm_swiglu_quantised_out(counts, N, K):
         g = A[lo:hi] @ Bd[e, :N].T
         u = A[lo:hi] @ Bd[e, N:].T
         h = (g / (1 + np.exp(-g)) * u).astype(np.float32)
-        hq, hs = _quant_pow2(h)
+        hq, hs = quant_pow2_e4m3(h)
         ref = dec[hq] * np.repeat(hs, 128, 1)
         check_close(got[lo:hi], ref, FP8_TOL, f"expert {e}")
         assert np.mean(C.cpu().numpy()[lo:hi] != hq) < 0.02
