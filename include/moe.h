@@ -296,12 +296,17 @@ moe_status_t moe_forward_fp8_gated(const void* x_dev, const void* wr_dev, const 
  * per 32 consecutive K elements, the smallest power of two >= amax / 6 (1 for
  * an all-zero block), stored as its e8m0 byte (biased exponent). Byte i of a
  * row holds element 2i in its low nibble and 2i + 1 in its high nibble.
+ * The scale bytes of a [rows, K] matrix are stored in 512-byte chunks, one
+ * per 128 rows x 128 K, chunks ordered (row block, K block); byte
+ * 16 r + 4 g + j of a chunk is the scale of row 32 g + r of the block for
+ * K elements [32 j, 32 j + 32) of the block (the layout the block-scaled MMA
+ * takes its scale factors in).
  * x and the hidden activations are quantised as in moe_forward_fp8_ue8m0
  * (e4m3, power-of-two scale per 128-group); both expert GEMMs run on the
  * block-scaled MMA with e4m3 A and e2m1 B (kind::mxf8f6f4).
- *   w13q_dev u8 [E, 2I, H/2], w13s_dev u8 [E, 2I, H/32]   (moe_quantize_weight_fp4)
- *   w2q_dev  u8 [E, H, I/2],  w2s_dev  u8 [E, H, I/32]
- *   packed weights 32-byte aligned, scales 4-byte aligned; H % 256 == 0
+ *   w13q_dev u8 [E, 2I, H/2], w13s_dev u8 chunks, E * 2I * H / 32 bytes (moe_quantize_weight_fp4)
+ *   w2q_dev  u8 [E, H, I/2],  w2s_dev  u8 chunks, E * H * I / 32 bytes
+ *   packed weights 32-byte aligned, scales 16-byte aligned; H % 256 == 0
  *   ws >= moe_workspace_size(d, MOE_DTYPE_FP4_E2M1) bytes; act as for
  *   moe_forward_gated. */
 moe_status_t moe_forward_fp4(const void* x_dev, const void* wr_dev, const float* bias_dev,
@@ -313,7 +318,8 @@ moe_status_t moe_forward_fp4(const void* x_dev, const void* wr_dev, const float*
  *   A_dev        e4m3 [M_total, K], a_scales_dev fp32 [M_total, K/128] powers of two
  *   B_dev        packed e2m1 [E, N_B, K/2] (32-byte aligned), N_B = 2N for a
  *                gated epilogue (gate rows then up rows), N otherwise
- *   b_scales_dev e8m0 bytes [E, N_B, K/32] (4-byte aligned)
+ *   b_scales_dev e8m0 bytes in the chunk layout of moe_forward_fp4, E * N_B * K / 32
+ *                bytes (16-byte aligned)
  *   C_dev        bf16 [M_total, N] (plain; N % 256 == 0), or with a gated
  *                epilogue e4m3 [M_total, N] + c_scales_dev fp32 [M_total, N/128]
  *                (power-of-two scales), or bf16 when c_scales_dev is NULL
@@ -325,9 +331,10 @@ moe_status_t moe_grouped_gemm_fp4(const void* A_dev, const float* a_scales_dev, 
                                   size_t ws_bytes, void* stream);
 
 /* FP4 weight quantisation (one-time preparation): nb matrices bf16 [rows,
- * cols] (cols % 128 == 0) -> q_dev packed e2m1 [nb, rows, cols/2], s_dev e8m0
- * bytes [nb, rows, cols/32], by the rule of moe_forward_fp4 with IEEE fp32
- * division and round-to-nearest-even (ties to the even code). */
+ * cols] (rows, cols multiples of 128) -> q_dev packed e2m1 [nb, rows, cols/2],
+ * s_dev e8m0 bytes (nb * rows * cols / 32, the chunk layout of
+ * moe_forward_fp4), by the rule of moe_forward_fp4 with IEEE fp32 division
+ * and round-to-nearest-even (ties to the even code). */
 moe_status_t moe_quantize_weight_fp4(const void* w_dev, int64_t nb, int64_t rows, int64_t cols,
                                      void* q_dev, uint8_t* s_dev, void* stream);
 

@@ -402,8 +402,7 @@ moe_status_t moe_grouped_gemm_fp4(const void* A, const float* a_scales, const vo
   MOE_TRY(check_ptr(a_scales, "a_scales"));
   MOE_TRY(check_ptr(B, "B"));
   if (reinterpret_cast<uintptr_t>(B) & 31) return fail(MOE_ERR_INVALID_ARG, "B must be 32-byte aligned");
-  if (!b_scales || (reinterpret_cast<uintptr_t>(b_scales) & 3))
-    return fail(MOE_ERR_INVALID_ARG, "b_scales must be non-NULL and 4-byte aligned");
+  MOE_TRY(check_ptr(b_scales, "b_scales"));
   MOE_TRY(check_ptr(offsets, "expert_offsets"));
   MOE_TRY(check_ptr(C, "C"));
   MOE_TRY(check_ptr(c_scales, "c_scales", true));
@@ -617,8 +616,8 @@ moe_status_t moe_forward_fp4(const void* x, const void* wr, const float* bias, c
   MOE_TRY(check_ptr(w2q, "w2q"));
   if ((reinterpret_cast<uintptr_t>(w13q) | reinterpret_cast<uintptr_t>(w2q)) & 31)
     return fail(MOE_ERR_INVALID_ARG, "packed FP4 weights must be 32-byte aligned");
-  if (!w13s || !w2s || ((reinterpret_cast<uintptr_t>(w13s) | reinterpret_cast<uintptr_t>(w2s)) & 3))
-    return fail(MOE_ERR_INVALID_ARG, "w13s / w2s must be non-NULL and 4-byte aligned");
+  MOE_TRY(check_ptr(w13s, "w13s"));
+  MOE_TRY(check_ptr(w2s, "w2s"));
   MOE_TRY(check_ptr(out, "out"));
   if (d.H % 256) return fail(MOE_ERR_INVALID_ARG, "the FP4 layer needs H %% 256 == 0 (got %d)", d.H);
   MOE_TRY(check_ws(d, MOE_DTYPE_FP4_E2M1, ws, ws_bytes));
@@ -702,11 +701,11 @@ moe_status_t moe_quantize_weight_fp8(const void* w, int64_t nb, int64_t rows, in
 
 moe_status_t moe_quantize_weight_fp4(const void* w, int64_t nb, int64_t rows, int64_t cols,
                                      void* q, uint8_t* sc, void* stream) {
-  if (nb < 1 || rows < 1 || cols < 128 || cols % 128)
-    return fail(MOE_ERR_INVALID_ARG, "nb >= 1, rows >= 1 and cols a multiple of 128");
+  if (nb < 1 || rows < 128 || rows % 128 || cols < 128 || cols % 128)
+    return fail(MOE_ERR_INVALID_ARG, "nb >= 1, rows and cols multiples of 128");
   MOE_TRY(check_ptr(w, "w"));
   MOE_TRY(check_ptr(q, "q"));
-  if (!sc) return fail(MOE_ERR_INVALID_ARG, "s is NULL");
+  MOE_TRY(check_ptr(sc, "s"));
   MOE_TRY(check_device());
   cudaError_t e = launch_quant_weight_fp4(w, nb, rows, cols, q, sc, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "FP4 weight quantisation");

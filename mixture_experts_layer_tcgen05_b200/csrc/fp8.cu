@@ -131,7 +131,10 @@ cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t
 // 32 consecutive K elements (the OCP microscaling block): the smallest power
 // of two >= amax / 6 (fp32 quotient), p clamped to [-127, 127], 1 for an
 // all-zero block, stored as its biased exponent. Element 2i goes to the low
-// nibble of byte i.
+// nibble of byte i. The scale bytes are stored in the block-scaled GEMM's
+// chunk layout: per 128 rows and 128 K one 512-byte chunk whose byte
+// 16 r + 4 g + j is the scale of row 32 g + r for the K elements
+// [32 j, 32 j + 32) of that chunk.
 
 // e2m1 code of v (|v| <= 6 here): nearest of 0, 0.5, 1, 1.5, 2, 3, 4, 6, ties
 // to the even code; larger magnitudes saturate to 6; the sign bit is kept.
@@ -152,11 +155,15 @@ __device__ __forceinline__ uint32_t e2m1_code(float v) {
 // One thread per 32-element block: 64 bytes in, 16 bytes of codes and one
 // scale byte out.
 __global__ void __launch_bounds__(256) quant_weight_fp4_kernel(const uint4* __restrict__ w,
-                                                               int64_t nblocks,
+                                                               int64_t nblocks, int64_t cols,
                                                                uint4* __restrict__ q,
                                                                uint8_t* __restrict__ sc) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nblocks) return;
+  const int64_t row = i / (cols / 32);  // over all nb matrices (rows % 128 == 0)
+  const int b32 = (int)(i % (cols / 32));
+  const int64_t chunk = (row >> 7) * (cols / 128) + (b32 >> 2);
+  const int64_t sidx = chunk * 512 + 16 * (row & 31) + 4 * ((row >> 5) & 3) + (b32 & 3);
   float v[32];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -181,14 +188,14 @@ __global__ void __launch_bounds__(256) quant_weight_fp4_kernel(const uint4* __re
 #pragma unroll
   for (int j = 0; j < 32; ++j) out[j >> 3] |= e2m1_code(__fdiv_rn(v[j], s)) << (4 * (j & 7));
   q[i] = make_uint4(out[0], out[1], out[2], out[3]);
-  sc[i] = (uint8_t)((__float_as_uint(s) >> 23) & 0xFFu);  // 2^-127 is the one code-0 (subnormal) scale
+  sc[sidx] = (uint8_t)((__float_as_uint(s) >> 23) & 0xFFu);  // 2^-127 is the one code-0 (subnormal) scale
 }
 
 cudaError_t launch_quant_weight_fp4(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                     uint8_t* sc, cudaStream_t s) {
   const int64_t nblocks = nb * rows * (cols / 32);
   quant_weight_fp4_kernel<<<(unsigned)ceil_div(nblocks, 256), 256, 0, s>>>(
-      static_cast<const uint4*>(w), nblocks, static_cast<uint4*>(q), sc);
+      static_cast<const uint4*>(w), nblocks, cols, static_cast<uint4*>(q), sc);
   note_launch();
   return cudaGetLastError();
 }

@@ -21,7 +21,9 @@
 // into the 16-byte-aligned unpacked shared layout the f8f6f4 MMA reads (16
 // codes per 16 bytes), so a stage still covers 128 K in 128-byte rows; A stays
 // e4m3 (kind::mxf8f6f4 mixes the two formats). B's scales are e8m0 codes per
-// (row, 32 K): the four bytes of a row for one stage are its four K steps.
+// (row, 32 K), stored already in the chunk layout above (one 512-byte chunk
+// per 128 rows and 128 K), so each stage's two B chunks arrive by two bulk
+// copies on the stage's barrier.
 //
 // Warp roles (320 threads): warp 0 TMA producer, all 32 lanes building the
 // scale chunks; warp 1 TMEM allocator + MMA issuer; warps 2..9 epilogue.
@@ -63,8 +65,7 @@ struct Args {
   float* c_scales;        // power-of-two scales of C's 128-groups
   const float* a_scales;  // [M_total, kblocks], powers of two
   const float* b_scales;  // [E, b_nblk, kblocks], powers of two (e4m3 B)
-  const uint8_t* b_sf8;   // [E * b_rows, K / 32] e8m0 codes (e2m1 B)
-  int b_sf_ld;            // K / 32
+  const uint8_t* b_sf8;   // e2m1 B: e8m0 chunks [E * b_rows / 128][K / 128][512 bytes]
   int32_t* status;
 };
 
@@ -219,49 +220,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = row0 + g * 32 + lane;
         sa[g] = r < row_end ? args.a_scales + (int64_t)r * nkb : nullptr;  // rows past the expert: scale 1
       }
+      // e2m1 B: the stage's scale chunks of the two 128-row boxes (rows rb0, rb1)
+      const unsigned char* sfc0 = BFP4 ? args.b_sf8 + (int64_t)(rb0 >> 7) * nkb * kSfA : nullptr;
+      const unsigned char* sfc1 = BFP4 ? args.b_sf8 + (int64_t)(rb1 >> 7) * nkb * kSfA : nullptr;
       // scales of the next kPre stages, loaded ahead so that their latency
       // overlaps the wait for a free stage
-      const uint8_t* sf8[8];  // e2m1 B: scale rows lane + 32g of both boxes
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        sf8[g] = BFP4 ? args.b_sf8 + (int64_t)(rb0 + 32 * g + lane) * args.b_sf_ld : nullptr;
-        sf8[4 + g] = BFP4 ? args.b_sf8 + (int64_t)(rb1 + 32 * g + lane) * args.b_sf_ld : nullptr;
-      }
       float pa[kPre][4], pb[kPre][2];
-      uint32_t pw[kPre][BFP4 ? 8 : 1];
-      auto fetch = [&](int kb, float (&a)[4], float (&b)[2], uint32_t (&wv)[BFP4 ? 8 : 1]) {
+      auto fetch = [&](int kb, float (&a)[4], float (&b)[2]) {
         if (kb < nkb) {
 #pragma unroll
           for (int g = 0; g < 4; ++g) a[g] = sa[g] ? __ldg(sa[g] + kb) : 1.0f;
-          if constexpr (BFP4) {
-#pragma unroll
-            for (int g = 0; g < 8; ++g) wv[g] = __ldg(reinterpret_cast<const uint32_t*>(sf8[g]) + kb);
-          } else {
+          if constexpr (!BFP4) {
             b[0] = __ldg(sb0 + kb);
             b[1] = __ldg(sb1 + kb);
           }
         }
       };
 #pragma unroll
-      for (int i = 0; i < kPre; ++i) fetch(i, pa[i], pb[i], pw[i]);
+      for (int i = 0; i < kPre; ++i) fetch(i, pa[i], pb[i]);
       for (int kb = 0; kb < nkb; ++kb, ++issued) {
         const int s = (int)(issued % STAGES);
         const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
         float ca[4] = {pa[0][0], pa[0][1], pa[0][2], pa[0][3]};
         const float cb0 = pb[0][0], cb1 = pb[0][1];
-        uint32_t cw[BFP4 ? 8 : 1];
-#pragma unroll
-        for (int g = 0; g < (BFP4 ? 8 : 1); ++g) cw[g] = pw[0][g];
 #pragma unroll
         for (int i = 0; i + 1 < kPre; ++i) {
 #pragma unroll
           for (int g = 0; g < 4; ++g) pa[i][g] = pa[i + 1][g];
           pb[i][0] = pb[i + 1][0];
           pb[i][1] = pb[i + 1][1];
-#pragma unroll
-          for (int g = 0; g < (BFP4 ? 8 : 1); ++g) pw[i][g] = pw[i + 1][g];
         }
-        fetch(kb + kPre, pa[kPre - 1], pb[kPre - 1], pw[kPre - 1]);
+        fetch(kb + kPre, pa[kPre - 1], pb[kPre - 1]);
         int got = 1;
         if (lane == 0) got = ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty);
         if (!__shfl_sync(0xffffffffu, got, 0)) {
@@ -274,10 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 0; g < 4; ++g) w[g] = e8m0_code(ca[g]) * 0x01010101u;  // same for the four K steps
         unsigned char* sfs = sf + s * kSfStage;
         *reinterpret_cast<uint4*>(sfs + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        if constexpr (BFP4) {  // per-row codes, one byte per K step
-          *reinterpret_cast<uint4*>(sfs + kSfA + lane * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          *reinterpret_cast<uint4*>(sfs + 2 * kSfA + lane * 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-        } else {
+        if constexpr (!BFP4) {  // e2m1 B: its chunks arrive by bulk copy below
           const uint32_t c0 = e8m0_code(cb0) * 0x01010101u, c1 = e8m0_code(cb1) * 0x01010101u;
           *reinterpret_cast<uint4*>(sfs + kSfA + lane * 16) = make_uint4(c0, c0, c0, c0);
           *reinterpret_cast<uint4*>(sfs + 2 * kSfA + lane * 16) = make_uint4(c1, c1, c1, c1);
@@ -287,10 +273,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           const uint32_t sa_ = sbase + s * kStage, sb_ = sa_ + kTileA;
           // packed e2m1: the transaction counts the bytes read (two codes per byte)
-          ptx::mbar_arrive_expect_tx(full0 + s * 8, BFP4 ? kTileA + kTileB / 2 : kStage);
+          // plus the two scale chunks
+          ptx::mbar_arrive_expect_tx(full0 + s * 8, BFP4 ? kTileA + kTileB / 2 + 2 * kSfA : kStage);
           ptx::tma_load_2d(sa_, &tmA, kb * BK, row0, full0 + s * 8);
           ptx::tma_load_2d(sb_, &tmB, kb * BK, rb0, full0 + s * 8);
           ptx::tma_load_2d(sb_ + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
+          if constexpr (BFP4) {
+            const uint32_t sfd = sfbase + s * kSfStage;
+            ptx::bulk_load(sfd + kSfA, sfc0 + (int64_t)kb * kSfA, kSfA, full0 + s * 8);
+            ptx::bulk_load(sfd + 2 * kSfA, sfc1 + (int64_t)kb * kSfA, kSfA, full0 + s * 8);
+          }
         }
       }
     }
@@ -456,8 +448,8 @@ cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const v
     *why = "the block-scaled plain GEMM needs N % 256 == 0";
     return cudaErrorInvalidValue;
   }
-  if (fp4 && (reinterpret_cast<uintptr_t>(B) & 31)) {
-    *why = "packed FP4 weights must be 32-byte aligned";
+  if (fp4 && ((reinterpret_cast<uintptr_t>(B) & 31) || (reinterpret_cast<uintptr_t>(b_sf8) & 15))) {
+    *why = "packed FP4 weights must be 32-byte aligned and their scale chunks 16-byte aligned";
     return cudaErrorInvalidValue;
   }
   CUtensorMap tmA, tmB;
@@ -484,7 +476,6 @@ cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const v
   a.a_scales = a_scales;
   a.b_scales = b_scales;
   a.b_sf8 = b_sf8;
-  a.b_sf_ld = K / 32;
   a.status = status;
   const int64_t tiles_ub = ((int64_t)M_total / ggmx::BM + (M_total < E ? M_total : E)) * a.NT;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_ub));

@@ -28,6 +28,14 @@ def _dequant_fp4(q, sc):
     return _E2M1[codes] * np.repeat(2.0 ** (sc.astype(np.float64) - 127), 32, axis=-1)
 
 
+def _chunks(sc):
+    """e8m0 bytes [nb, rows, K/32] -> the chunk layout the GEMM reads: per 128
+    rows and 128 K a 512-byte chunk, byte 16 r + 4 g + j = row 32 g + r, K step j."""
+    nb, rows, kb32 = sc.shape
+    return np.ascontiguousarray(
+        sc.reshape(nb, rows // 128, 4, 32, kb32 // 4, 4).transpose(0, 1, 4, 3, 2, 5)).reshape(-1)
+
+
 def _dequant_e4m3(q, s):
     dec = np.array([oracle.e4m3_decode(c) for c in range(256)])
     return dec[q] * np.repeat(s, 128, axis=-1)
@@ -40,7 +48,7 @@ def _quant_fp4_dev(w, nb, rows, cols):
     return q, sc
 
 
-@pytest.mark.parametrize("nb,rows,cols", [(1, 1, 128), (3, 5, 384), (2, 64, 1024)])
+@pytest.mark.parametrize("nb,rows,cols", [(1, 128, 128), (3, 128, 384), (2, 256, 1024)])
 def test_quantize_weight_fp4_bit_exact(nb, rows, cols):
     rng = np.random.default_rng(rows * cols)
     w = (rng.standard_normal((nb, rows, cols)) * 0.02).astype(np.float32)
@@ -51,7 +59,7 @@ def test_quantize_weight_fp4_bit_exact(nb, rows, cols):
     q, sc = _quant_fp4_dev(wb, nb, rows, cols)
     torch.cuda.synchronize()
     rq, rs = oracle.quant_weight_fp4(wb)
-    np.testing.assert_array_equal(sc.cpu().numpy(), rs)
+    np.testing.assert_array_equal(sc.cpu().numpy().reshape(-1), _chunks(rs))
     np.testing.assert_array_equal(q.cpu().numpy(), rq)
 
 
@@ -72,8 +80,8 @@ def test_fp4_grouped_gemm_plain(counts, N, K):
     E, offsets, M, aq, as_, bq, bs = _problem(counts, N, K, 101)
     C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
-    moe.moe_grouped_gemm_fp4(dev_u8(aq), dev(as_), dev_u8(bq), dev_u8(bs), dev(offsets), M, E, N,
-                             K, moe.MOE_EPILOGUE_NONE, C, None, ws)
+    moe.moe_grouped_gemm_fp4(dev_u8(aq), dev(as_), dev_u8(bq), dev_u8(_chunks(bs)), dev(offsets), M,
+                             E, N, K, moe.MOE_EPILOGUE_NONE, C, None, ws)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(ws) == 0
     A, Bd = _dequant_e4m3(aq, as_), _dequant_fp4(bq, bs)
@@ -90,8 +98,8 @@ def test_fp4_grouped_gemm_swiglu_quantised_out(counts, N, K):
     C = torch.empty(M, N, dtype=torch.uint8, device="cuda")
     cs = torch.empty(M, N // 128, dtype=torch.float32, device="cuda")
     ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
-    moe.moe_grouped_gemm_fp4(dev_u8(aq), dev(as_), dev_u8(bq), dev_u8(bs), dev(offsets), M, E, N,
-                             K, moe.MOE_EPILOGUE_SWIGLU, C, cs, ws)
+    moe.moe_grouped_gemm_fp4(dev_u8(aq), dev(as_), dev_u8(bq), dev_u8(_chunks(bs)), dev(offsets), M,
+                             E, N, K, moe.MOE_EPILOGUE_SWIGLU, C, cs, ws)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(ws) == 0
     A, Bd = _dequant_e4m3(aq, as_), _dequant_fp4(bq, bs)
