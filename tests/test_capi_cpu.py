@@ -112,3 +112,34 @@ def test_stage_events_need_six():
 def test_last_error_is_thread_local_and_cleared():
     moe.moe_set_stage_events(None)
     assert moe.moe_last_error() == ""
+
+
+def test_fp4_entry_points_validate_before_launch():
+    d = (16, 256, 256, 4, 2)
+    assert moe.moe_workspace_size(d, moe.MOE_DTYPE_FP4_E2M1) == \
+        moe.moe_workspace_size(d, moe.MOE_DTYPE_FP8_E4M3_UE8M0) > 0
+    swi = moe.MOE_EPILOGUE_SWIGLU
+    with pytest.raises(moe.MoeError) as ei:  # packed weights must be 32-byte aligned (TMA 4-bit map)
+        moe.moe_forward_fp4(FAKE, FAKE, None, FAKE + 16, FAKE, FAKE, FAKE, d, swi, FAKE, FAKE,
+                            1 << 30, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG and "32-byte" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:  # scale chunks are bulk-copied: 16-byte aligned
+        moe.moe_forward_fp4(FAKE, FAKE, None, FAKE, FAKE + 4, FAKE, FAKE, d, swi, FAKE, FAKE,
+                            1 << 30, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG and "w13s" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_forward_fp4(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, d, moe.MOE_EPILOGUE_NONE,
+                            FAKE, FAKE, 1 << 30, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoeError) as ei:  # the plain FP4 GEMM tiles N by 256
+        moe.moe_grouped_gemm_fp4(FAKE, FAKE, FAKE, FAKE, FAKE, 10, 4, 384, 128,
+                                 moe.MOE_EPILOGUE_NONE, FAKE, None, FAKE, 4096, stream=0)
+    assert "256" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:  # FP4 B scales are bytes: the generic entry refuses
+        moe.moe_grouped_gemm(FAKE, FAKE, FAKE, 10, 4, 256, 128, moe.MOE_DTYPE_FP4_E2M1,
+                             moe.MOE_EPILOGUE_NONE, FAKE, FAKE, FAKE, ws=FAKE, ws_bytes=4096,
+                             stream=0)
+    assert "moe_grouped_gemm_fp4" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:  # scale chunks cover 128 rows
+        moe.moe_quantize_weight_fp4(FAKE, 1, 100, 256, FAKE, FAKE, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
