@@ -376,6 +376,15 @@ moe_status_t moe_get_device_status(const void* ws, int32_t* status_out);
 /* Clears the workspace's device status word (stream-ordered). */
 moe_status_t moe_clear_device_status(void* ws, void* stream);
 
+/* Self-test of the bounded device waits the pipelined kernels use (failure
+ * detection without a GPU fault): one CTA waits on an mbarrier that nothing
+ * arrives at, for budget_cycles SM clocks (1000 .. 2e9), then gives up and
+ * records (MOE_ERR_TIMEOUT << 8) | 7 in the status word of ws, unless the
+ * word already holds a failure, in which case it gives up at once and leaves
+ * the word unchanged. Stream-ordered; read the result with
+ * moe_get_device_status. The context stays usable. */
+moe_status_t moe_check_wait_timeout(void* ws, int64_t budget_cycles, void* stream);
+
 /* Stage timing for moe_forward / moe_forward_fp8 on the calling thread: when
  * set, the next forwards record events[0..5] (cudaEvent_t) on their stream at
  * entry, after routing, after the permutation, after GEMM1, after GEMM2 and

@@ -30,7 +30,7 @@ __all__ = [
     "moe_permute_noalloc",
     "moe_grouped_gemm", "moe_combine", "moe_forward", "moe_forward_fp8", "moe_forward_hostio",
     "moe_quantize_act_fp8", "moe_quantize_weight_fp8", "moe_get_device_status",
-    "moe_clear_device_status", "moe_set_stage_events", "EXPORTED",
+    "moe_clear_device_status", "moe_set_stage_events", "moe_check_wait_timeout", "EXPORTED",
 ]
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_DEVICE = 0, 1, 2
@@ -93,6 +93,7 @@ _SIGS = {
     "moe_quantize_weight_fp8_fmt": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp]),
     "moe_get_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_clear_device_status": (_i32, [_vp, _vp]),
+    "moe_check_wait_timeout": (_i32, [_vp, _i64, _vp]),
     "moe_set_stage_events": (_i32, [ctypes.POINTER(_vp), _i32]),
 }
 EXPORTED = tuple(_SIGS)
@@ -291,6 +292,10 @@ def moe_get_device_status(ws) -> int:
 
 def moe_clear_device_status(ws, stream=None):
     _check(lib().moe_clear_device_status(_p(ws), _s(stream)))
+
+
+def moe_check_wait_timeout(ws, budget_cycles, stream=None):
+    _check(lib().moe_check_wait_timeout(_p(ws), int(budget_cycles), _s(stream)))
 
 
 def moe_set_stage_events(events):

@@ -48,6 +48,7 @@ cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const v
                                    const int32_t* offsets, int M_total, int E, int N, int K, int act,
                                    void* Cout, float* c_scales, int32_t* status, cudaStream_t s,
                                    const char** why);
+cudaError_t launch_wait_selftest(int32_t* status, long long budget, cudaStream_t s);
 cudaError_t launch_quant_weight_fp4(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                     uint8_t* sc, cudaStream_t s);
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
@@ -719,6 +720,18 @@ moe_status_t moe_get_device_status(const void* ws, int32_t* status_out) {
   cudaError_t e = cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "read status");
   *status_out = v;
+  return ok();
+}
+
+moe_status_t moe_check_wait_timeout(void* ws, int64_t budget_cycles, void* stream) {
+  MOE_TRY(check_ptr(ws, "ws"));
+  if (budget_cycles < 1000 || budget_cycles > 2000000000LL)
+    return fail(MOE_ERR_INVALID_ARG, "budget_cycles must be in [1000, 2e9] (got %lld)",
+                (long long)budget_cycles);
+  MOE_TRY(check_device());
+  cudaError_t e = launch_wait_selftest(static_cast<int32_t*>(ws), (long long)budget_cycles,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait self-test");
   return ok();
 }
 

@@ -21,6 +21,7 @@ enum WaitSite : int32_t {
   kSiteEpiAccFull = 4,
   kSiteDrain = 5,
   kSiteBadIndex = 6,  // an expert id / row index outside its range (skipped)
+  kSiteSelfTest = 7,  // the wait of moe_check_wait_timeout
 };
 
 // status word: 0 = ok; else (MOE_ERR_TIMEOUT << 8) | site

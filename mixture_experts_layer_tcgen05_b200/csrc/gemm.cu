@@ -41,7 +41,7 @@ struct RowsCfg {
   static constexpr int STAGES = kSmemBudget / kStage;
   static constexpr int kAccCols = 256;  // column stride between the two accumulators
   static constexpr uint32_t kIdesc = ptx::make_idesc(BM, BN, 1, 1);  // bf16 x bf16 -> fp32
-  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + 2 * (kMaxE + 1) * 4;
+  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4;
 };
 
 // ACT: gated activation of the epilogue (kActNone: plain GEMM).
@@ -85,12 +85,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
     ptx::tmem_relinquish();
   }
-  if (warp == 2) build_tile_starts_mixed<BM>(args.offsets, args.E, args.NT, tile_start);
+  if (warp == 2) build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = mixed_total(tile_start, args.E);
+  const int total = tile_start[args.E];
   const int nkb = args.K / BK;
   // Plain GEMM, BN = 256: when the tiles leave a last wave at most half full,
   // each of its tiles runs as two BN = 128 units (the column halves), so that
@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   auto decode = [&](int tile, int& e, int& m, int& n) {
-    int local;
-    e = mixed_decode(tile_start, args.E, tile, local);
+    e = find_expert(tile_start, args.E, tile);
+    const int local = tile - tile_start[e];
     const int cnt = args.offsets[e + 1] - args.offsets[e];
     const int mt = (cnt + BM - 1) / BM;
     const int bsz = args.band * args.NT;

@@ -62,45 +62,6 @@ __device__ void build_tile_starts(const int32_t* offsets, int E, int NT, int32_t
   if (lane == 0) tile_start[E] = carry;
 }
 
-// The order the persistent CTAs take tiles in. Experts with one row tile
-// stream their whole weight matrix for it (memory-bound tiles); experts with
-// more row tiles share each weight strip among their row tiles (tensor-bound
-// tiles). Both kinds are spread evenly over the schedule, so that at any
-// moment some CTAs stream weights while the others keep the tensor cores
-// busy: ts[0..E] are the tile prefix sums of the multi-tile experts,
-// ts[E+1..2E+1] those of the single-tile experts, and schedule position t is
-// a single-tile one when floor((t+1) NS / N) > floor(t NS / N). Warp-wide.
-template <int kRowsPerTile>
-__device__ void build_tile_starts_mixed(const int32_t* offsets, int E, int NT, int32_t* ts) {
-  const int lane = threadIdx.x & 31;
-  int32_t carry_b = 0, carry_s = 0;
-  for (int e0 = 0; e0 < E; e0 += 32) {
-    const int e = e0 + lane;
-    const int32_t cnt = e < E ? max(offsets[e + 1] - offsets[e], 0) : 0;
-    const int32_t mt = (cnt + kRowsPerTile - 1) / kRowsPerTile;
-    const int32_t tb = mt >= 2 ? mt * NT : 0, tsm = mt == 1 ? NT : 0;
-    int32_t ib = tb, is = tsm;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int32_t vb = __shfl_up_sync(0xffffffffu, ib, off);
-      const int32_t vs = __shfl_up_sync(0xffffffffu, is, off);
-      if (lane >= off) ib += vb, is += vs;
-    }
-    if (e < E) {
-      ts[e] = carry_b + ib - tb;
-      ts[E + 1 + e] = carry_s + is - tsm;
-    }
-    carry_b += __shfl_sync(0xffffffffu, ib, 31);
-    carry_s += __shfl_sync(0xffffffffu, is, 31);
-  }
-  if (lane == 0) {
-    ts[E] = carry_b;
-    ts[2 * E + 1] = carry_s;
-  }
-}
-
-__device__ __forceinline__ int mixed_total(const int32_t* ts, int E) { return ts[E] + ts[2 * E + 1]; }
-
 // Largest e with tile_start[e] <= tile (that expert is non-empty).
 __device__ __forceinline__ int find_expert(const int32_t* tile_start, int E, int tile) {
   int lo = 0, hi = E;
@@ -110,24 +71,6 @@ __device__ __forceinline__ int find_expert(const int32_t* tile_start, int E, int
     else hi = mid;
   }
   return lo;
-}
-
-// Schedule position -> (expert, tile index inside the expert), for the order
-// of build_tile_starts_mixed.
-__device__ __forceinline__ int mixed_decode(const int32_t* ts, int E, int tile, int& local) {
-  const int32_t* big = ts;
-  const int32_t* small = ts + E + 1;
-  const int64_t ns = small[E], n = (int64_t)big[E] + ns;
-  const int sb = (int)((int64_t)tile * ns / n), sa = (int)((int64_t)(tile + 1) * ns / n);
-  if (sa > sb) {
-    const int e = find_expert(small, E, sb);
-    local = sb - small[e];
-    return e;
-  }
-  const int i = tile - sb;
-  const int e = find_expert(big, E, i);
-  local = i - big[e];
-  return e;
 }
 
 // ------------------------------------------------------------------ utils

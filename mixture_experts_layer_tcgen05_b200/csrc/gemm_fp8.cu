@@ -34,7 +34,7 @@ constexpr int kStage = kTileA + kTileB;
 constexpr int STAGES = 4;
 constexpr int kMaxE = 1024;
 constexpr uint32_t kIdesc = ptx::make_idesc(BM, BN, 0, 0);  // e4m3 x e4m3 -> fp32
-constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + 2 * (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
+constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
 
 struct Args {
   const int32_t* offsets;
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // bars: full[STAGES], empty[STAGES], pfull[2], pempty[2], drain, redbar[2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 7);
   int32_t* tile_start = reinterpret_cast<int32_t*>(smem + STAGES * kStage + 256);
-  float* red = reinterpret_cast<float*>(tile_start + 2 * (kMaxE + 1));  // [2 tiles][2 halves][BM]
+  float* red = reinterpret_cast<float*>(tile_start + kMaxE + 1);  // [2 tiles][2 halves][BM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = ptx::smem_addr(smem);
@@ -98,17 +98,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
     ptx::tmem_relinquish();
   }
-  if (warp == 2) gg::build_tile_starts_mixed<BM>(args.offsets, args.E, args.NT, tile_start);
+  if (warp == 2) gg::build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = gg::mixed_total(tile_start, args.E);
+  const int total = tile_start[args.E];
   const int nkb = args.kblocks;
 
   auto decode = [&](int tile, int& e, int& m, int& n) {
-    int local;
-    e = gg::mixed_decode(tile_start, args.E, tile, local);
+    e = gg::find_expert(tile_start, args.E, tile);
+    const int local = tile - tile_start[e];
     const int cnt = args.offsets[e + 1] - args.offsets[e];
     const int mt = (cnt + BM - 1) / BM;
     const int bsz = args.band * args.NT;

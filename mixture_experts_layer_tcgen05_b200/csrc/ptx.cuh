@@ -56,17 +56,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Gives up after
-// kWaitBudgetCycles (or as soon as another thread has recorded a failure),
-// recording the site; returns false then.
+// `budget` cycles (kWaitBudgetCycles, about a second, unless a caller asks
+// for less) or as soon as another thread has recorded a failure, recording
+// the site; returns false then.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* status,
-                                          int site) {
+                                          int site, long long budget = kWaitBudgetCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   uint32_t n = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++n & 255u) == 0) {
       if (*reinterpret_cast<volatile int32_t*>(status) != 0) return false;
-      if (clock64() - t0 > kWaitBudgetCycles) {
+      if (clock64() - t0 > budget) {
         record_timeout(status, site);
         return false;
       }

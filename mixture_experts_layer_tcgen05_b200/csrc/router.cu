@@ -477,6 +477,15 @@ __global__ void __launch_bounds__(256, 1) router_tall_kernel(
   // stage Wr: 8 bf16 per 16-byte load, several loads in flight per thread
   const uint4* w4 = reinterpret_cast<const uint4*>(wr);
   const int nvec = H * E / 8;
+  if (E == EV) {  // no padding: the table is Wr widened in place, two 16-byte stores per load
+#pragma unroll 4
+    for (int v = tid; v < nvec; v += blockDim.x) {
+      const uint4 u = __ldg(w4 + v);
+      float4* d = reinterpret_cast<float4*>(sw + 8 * v);
+      d[0] = make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
+      d[1] = make_float4(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w));
+    }
+  } else {
 #pragma unroll 4
   for (int v = tid; v < nvec; v += blockDim.x) {
     const uint4 u = __ldg(w4 + v);
@@ -487,6 +496,7 @@ __global__ void __launch_bounds__(256, 1) router_tall_kernel(
       sw[h * EV + e] = (q & 1) ? bf16hi_to_f32(uw[q >> 1]) : bf16lo_to_f32(uw[q >> 1]);
       if (++e == E) e = 0, ++h;
     }
+  }
   }
   if (E < EV) {
     const int pad = EV - E;
