@@ -227,6 +227,15 @@ moe_status_t moe_grouped_gemm(const void* A_dev, const int32_t* a_rows_dev, int3
                               int32_t max_rows_per_expert, void* ws, size_t ws_bytes,
                               void* stream);
 
+/* Row gather: dst[i, :] = src[rows[i], :] for i in [0, n), rows of
+ * row_bytes bytes (a multiple of 4; 16-byte vectors when a multiple of 16).
+ * The data movement of the expert-parallel regroup (rows received per source
+ * rank put into local-expert order, and back). An index outside
+ * [0, src_rows) skips its row and records (MOE_ERR_INVALID_ARG << 8) | 6 in
+ * the status word of ws (when ws is not NULL). n == 0 is a no-op. */
+moe_status_t moe_gather_rows(const void* src_dev, int64_t src_rows, const int32_t* rows_dev,
+                             int64_t n, int64_t row_bytes, void* dst_dev, void* ws, void* stream);
+
 /* Weighted combine ([R] pseudocode `y = sum_i weights_i * expert_i(x)`):
  *   out[t, :] = sum_{j = 0..k-1} w[t, j] * y_perm[inv_perm[t, j], :]
  * summed in fp32 in slot order, rounded once to bf16.

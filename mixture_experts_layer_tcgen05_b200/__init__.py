@@ -28,7 +28,7 @@ __all__ = [
     "moe_last_error", "moe_abi_version", "moe_launch_count", "moe_workspace_size",
     "moe_workspace_layout", "moe_route_topk", "moe_topk_from_logits", "moe_permute",
     "moe_permute_noalloc",
-    "moe_grouped_gemm", "moe_combine", "moe_forward", "moe_forward_fp8", "moe_forward_hostio",
+    "moe_grouped_gemm", "moe_combine", "moe_gather_rows", "moe_forward", "moe_forward_fp8", "moe_forward_hostio",
     "moe_quantize_act_fp8", "moe_quantize_weight_fp8", "moe_get_device_status",
     "moe_clear_device_status", "moe_set_stage_events", "moe_check_wait_timeout", "EXPORTED",
 ]
@@ -75,6 +75,7 @@ _SIGS = {
     "moe_grouped_gemm": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp,
                                 _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "moe_combine": (_i32, [_vp, _vp, _vp, Dims, _vp, _vp]),
+    "moe_gather_rows": (_i32, [_vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp]),
     "moe_forward": (_i32, [_vp, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _sz, _vp]),
     "moe_forward_fp8": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _sz, _vp]),
     "moe_forward_hostio": (_i32, [_vp, _vp, _vp, _vp, _vp, Dims, _vp, _vp, _sz, _vp]),
@@ -209,6 +210,11 @@ def moe_grouped_gemm(A, B, offsets, M_total, E, N, K, dt, ep, C, a_scales=None, 
                                   K, dt, ep, _p(C),
                                   _p(a_scales), _p(b_scales), _p(c_scales), max_rows_per_expert,
                                   _p(ws), _nbytes(ws, ws_bytes), _s(stream)))
+
+
+def moe_gather_rows(src, src_rows, rows, n, row_bytes, dst, ws=None, stream=None):
+    _check(lib().moe_gather_rows(_p(src), int(src_rows), _p(rows), int(n), int(row_bytes), _p(dst),
+                                 _p(ws), _s(stream)))
 
 
 def moe_combine(y_perm, w, inv_perm, d, out, stream=None):

@@ -420,6 +420,26 @@ moe_status_t moe_grouped_gemm_fp4(const void* A, const float* a_scales, const vo
   return ok();
 }
 
+moe_status_t moe_gather_rows(const void* src, int64_t src_rows, const int32_t* rows, int64_t n,
+                             int64_t row_bytes, void* dst, void* ws, void* stream) {
+  if (n < 0 || src_rows < 0 || n > INT32_MAX || src_rows > INT32_MAX)
+    return fail(MOE_ERR_INVALID_ARG, "n and src_rows must be in [0, 2^31)");
+  if (row_bytes < 4 || row_bytes % 4 || row_bytes > (1 << 20))
+    return fail(MOE_ERR_INVALID_ARG, "row_bytes must be a multiple of 4 in [4, 2^20] (got %lld)",
+                (long long)row_bytes);
+  if (n == 0) return ok();
+  MOE_TRY(check_ptr(src, "src"));
+  MOE_TRY(check_ptr(rows, "rows"));
+  MOE_TRY(check_ptr(dst, "dst"));
+  MOE_TRY(check_ptr(ws, "ws", true));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_gather_rows(src, rows, (int)n, (int)src_rows, (int)row_bytes, dst,
+                                     ws ? static_cast<int32_t*>(ws) : nullptr,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "row gather");
+  return ok();
+}
+
 moe_status_t moe_combine(const void* y_perm, const float* w, const int32_t* inv_perm, moe_dims_t d,
                          void* out, void* stream) {
   moe_dims_t d2 = d;
