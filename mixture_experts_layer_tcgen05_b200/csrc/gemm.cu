@@ -41,7 +41,7 @@ struct RowsCfg {
   static constexpr int STAGES = kSmemBudget / kStage;
   static constexpr int kAccCols = 256;  // column stride between the two accumulators
   static constexpr uint32_t kIdesc = ptx::make_idesc(BM, BN, 1, 1);  // bf16 x bf16 -> fp32
-  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4;
+  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + 2 * (kMaxE + 1) * 4;
 };
 
 // ACT: gated activation of the epilogue (kActNone: plain GEMM).
@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // bars: full[STAGES], empty[STAGES], accf[2], acce[2], drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   int32_t* tile_start = reinterpret_cast<int32_t*>(smem + STAGES * C::kStage + 256);
+  int32_t* soff = tile_start + kMaxE + 1;  // [E + 1] expert offsets, shared copy
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = ptx::smem_addr(smem);
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
     ptx::tmem_relinquish();
   }
-  if (warp == 2) build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start);
+  if (warp == 2) build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start, soff);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto decode = [&](int tile, int& e, int& m, int& n) {
     e = find_expert(tile_start, args.E, tile);
     const int local = tile - tile_start[e];
-    const int cnt = args.offsets[e + 1] - args.offsets[e];
+    const int cnt = soff[e + 1] - soff[e];
     const int mt = (cnt + BM - 1) / BM;
     const int bsz = args.band * args.NT;
     const int b = local / bsz;
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int e, m, n;
         decode(tile, e, m, n);
         int src_row[4];
-        gather4_tile_rows(args.a_rows, args.offsets[e] + m * BM, args.M_total, args.a_src_rows, lane,
+        gather4_tile_rows(args.a_rows, soff[e] + m * BM, args.M_total, args.a_src_rows, lane,
                          src_row);
         int rb0, rb1;
         if (SWIGLU) {
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tile = unit_tile(u, half);
         int e, m, n;
         decode(tile, e, m, n);
-        const int row_a = args.offsets[e] + m * BM;
+        const int row_a = soff[e] + m * BM;
         int rb0, rb1;
         if (SWIGLU) {
           rb0 = e * args.b_rows + n * 128;
@@ -246,8 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tile = unit_tile(u, half);
       int e, m, n;
       decode(tile, e, m, n);
-      const int row = args.offsets[e] + m * BM + q * 32 + lane;
-      const bool valid = row >= 0 && row < args.offsets[e + 1] && row < args.M_total;
+      const int row = soff[e] + m * BM + q * 32 + lane;
+      const bool valid = row >= 0 && row < soff[e + 1] && row < args.M_total;
       if (!ptx::mbar_wait(accf0 + acc * 8, acc_ph, args.status, kSiteEpiAccFull)) break;
       ptx::tc_fence_after();
       const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
@@ -307,7 +308,7 @@ struct SwapCfg {
   static constexpr int kTmemCols = (2 * kAccCols) <= 32 ? 32 : (2 * kAccCols) <= 64 ? 64
                                    : (2 * kAccCols) <= 128 ? 128 : 256;
   static constexpr uint32_t kIdesc = ptx::make_idesc(BM, BNT, 1, 1);
-  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4;
+  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + 2 * (kMaxE + 1) * 4;
 };
 
 // tmA: weights [E*b_rows, K]; tmB: activation rows [M_total, K].
@@ -325,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStage);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   int32_t* tile_start = reinterpret_cast<int32_t*>(smem + STAGES * C::kStage + 256);
+  int32_t* soff = tile_start + kMaxE + 1;  // [E + 1] expert offsets, shared copy
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = ptx::smem_addr(smem);
@@ -349,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), C::kTmemCols);
     ptx::tmem_relinquish();
   }
-  if (warp == 2) build_tile_starts<BNT>(args.offsets, args.E, args.NT, tile_start);
+  if (warp == 2) build_tile_starts<BNT>(args.offsets, args.E, args.NT, tile_start, soff);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int e, tt, n, kb0;
         decode(tile, e, tt, n, kb0);
-        const int row_b = args.offsets[e] + tt * BNT;
+        const int row_b = soff[e] + tt * BNT;
         const int ra = e * args.b_rows + n * 128;
         for (int kb = kb0; kb < kb0 + nkb; ++kb, ++issued) {
           const int s = (int)(issued % STAGES);
@@ -439,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       int e, tt, n, kb0;
       decode(tile, e, tt, n, kb0);
-      const int row0 = args.offsets[e] + tt * BNT;
-      const int nrows = min(min(BNT, args.offsets[e + 1] - row0), args.M_total - row0);
+      const int row0 = soff[e] + tt * BNT;
+      const int nrows = min(min(BNT, soff[e + 1] - row0), args.M_total - row0);
       const int col = n * 128 + q * 32 + lane;  // output column owned by this thread
       if (!ptx::mbar_wait(accf0 + acc * 8, acc_ph, args.status, kSiteEpiAccFull)) break;
       ptx::tc_fence_after();

@@ -41,10 +41,14 @@ struct Args {
 };
 
 // ------------------------------------------------------------- scheduling
-// tile_start[e] = sum_{e' < e} tiles(e'), tile_start[E] = total. Warp-wide.
+// tile_start[e] = sum_{e' < e} tiles(e'), tile_start[E] = total; soff[0..E]
+// = offsets[0..E], a shared-memory copy every role decodes tiles from (no
+// global-memory latency at a tile switch). Warp-wide.
 template <int kRowsPerTile>
-__device__ void build_tile_starts(const int32_t* offsets, int E, int NT, int32_t* tile_start) {
+__device__ void build_tile_starts(const int32_t* offsets, int E, int NT, int32_t* tile_start,
+                                  int32_t* soff) {
   const int lane = threadIdx.x & 31;
+  for (int e = lane; e <= E; e += 32) soff[e] = offsets[e];
   int32_t carry = 0;
   for (int e0 = 0; e0 < E; e0 += 32) {
     int e = e0 + lane;

@@ -34,7 +34,7 @@ constexpr int kStage = kTileA + kTileB;
 constexpr int STAGES = 4;
 constexpr int kMaxE = 1024;
 constexpr uint32_t kIdesc = ptx::make_idesc(BM, BN, 0, 0);  // e4m3 x e4m3 -> fp32
-constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
+constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + 2 * (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
 
 struct Args {
   const int32_t* offsets;
@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // bars: full[STAGES], empty[STAGES], pfull[2], pempty[2], drain, redbar[2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 7);
   int32_t* tile_start = reinterpret_cast<int32_t*>(smem + STAGES * kStage + 256);
-  float* red = reinterpret_cast<float*>(tile_start + kMaxE + 1);  // [2 tiles][2 halves][BM]
+  int32_t* soff = tile_start + kMaxE + 1;  // [E + 1] expert offsets, shared copy
+  float* red = reinterpret_cast<float*>(soff + kMaxE + 1);  // [2 tiles][2 halves][BM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = ptx::smem_addr(smem);
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
     ptx::tmem_relinquish();
   }
-  if (warp == 2) gg::build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start);
+  if (warp == 2) gg::build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start, soff);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto decode = [&](int tile, int& e, int& m, int& n) {
     e = gg::find_expert(tile_start, args.E, tile);
     const int local = tile - tile_start[e];
-    const int cnt = args.offsets[e + 1] - args.offsets[e];
+    const int cnt = soff[e + 1] - soff[e];
     const int mt = (cnt + BM - 1) / BM;
     const int bsz = args.band * args.NT;
     const int b = local / bsz;
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int e, m, n;
         decode(tile, e, m, n);
         int src_row[4];
-        gg::gather4_tile_rows(args.a_rows, args.offsets[e] + m * BM, args.M_total, args.a_src_rows,
+        gg::gather4_tile_rows(args.a_rows, soff[e] + m * BM, args.M_total, args.a_src_rows,
                              lane, src_row);
         int rb0, rb1;
         if (SWIGLU) {
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int e, m, n;
         decode(tile, e, m, n);
-        const int row_a = args.offsets[e] + m * BM;
+        const int row_a = soff[e] + m * BM;
         int rb0, rb1;
         if (SWIGLU) {
           rb0 = e * args.b_rows + n * 128;
@@ -232,8 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tile_par = tile_iter & 1;
       int e, m, n;
       decode(tile, e, m, n);
-      const int row = args.offsets[e] + m * BM + rl;
-      const bool valid = row >= 0 && row < args.offsets[e + 1] && row < args.M_total;
+      const int row = soff[e] + m * BM + rl;
+      const bool valid = row >= 0 && row < soff[e + 1] && row < args.M_total;
       const int row_c = min(max(row, 0), args.M_total - 1);
       int srow = row_c;
       if (GATHER) {

@@ -54,7 +54,7 @@ constexpr int kMaxE = 1024;
 constexpr int kSfCol0 = 256;     // TMEM columns of the scale-factor ring
 constexpr int kSfColsPerStage = 16;
 constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + (size_t)STAGES * kSfStage + 256 +
-                         (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
+                         2 * (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
 
 struct Args {
   const int32_t* offsets;
@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // bars: full[STAGES], empty[STAGES], accf, acce, drain, redbar[2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
   int32_t* tile_start = reinterpret_cast<int32_t*>(sf + STAGES * kSfStage + 256);
-  float* red = reinterpret_cast<float*>(tile_start + kMaxE + 1);  // [2 tiles][2 halves][BM]
+  int32_t* soff = tile_start + kMaxE + 1;  // [E + 1] expert offsets, shared copy
+  float* red = reinterpret_cast<float*>(soff + kMaxE + 1);  // [2 tiles][2 halves][BM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = ptx::smem_addr(smem), sfbase = ptx::smem_addr(sf);
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
     ptx::tmem_relinquish();
   }
-  if (warp == 2) gg::build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start);
+  if (warp == 2) gg::build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start, soff);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto decode = [&](int tile, int& e, int& m, int& n) {
     e = gg::find_expert(tile_start, args.E, tile);
     const int local = tile - tile_start[e];
-    const int cnt = args.offsets[e + 1] - args.offsets[e];
+    const int cnt = soff[e + 1] - soff[e];
     const int mt = (cnt + BM - 1) / BM;
     const int bsz = args.band * args.NT;
     const int b = local / bsz;
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       int e, m, n;
       decode(tile, e, m, n);
-      const int row0 = args.offsets[e] + m * BM, row_end = args.offsets[e + 1];
+      const int row0 = soff[e] + m * BM, row_end = soff[e + 1];
       int rb0, rb1, nb0, nb1;  // B rows of the two 128-row boxes and their scale blocks
       if (SWIGLU) {
         rb0 = e * args.b_rows + n * 128;
@@ -337,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tile_par = tile_iter & 1;
       int e, m, n;
       decode(tile, e, m, n);
-      const int row = args.offsets[e] + m * BM + rl;
-      const bool valid = row >= 0 && row < args.offsets[e + 1] && row < args.M_total;
+      const int row = soff[e] + m * BM + rl;
+      const bool valid = row >= 0 && row < soff[e + 1] && row < args.M_total;
       if (!ptx::mbar_wait(accf, acc_ph, args.status, kSiteEpiAccFull)) break;
       acc_ph ^= 1;
       ptx::tc_fence_after();
