@@ -16,7 +16,8 @@ namespace moe {
 
 // kernels (router.cu, permute.cu, gemm.cu, fp8.cu)
 cudaError_t launch_route(const void* x, const void* wr, const float* bias, int T, int H, int E,
-                         int k, float* logits, int32_t* ids, float* w, cudaStream_t s);
+                         int k, float* logits, int32_t* ids, float* w, float* part,
+                         size_t part_bytes, cudaStream_t s);
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t s);
 int64_t permute_scratch_bytes(int T, int E);
@@ -256,7 +257,7 @@ moe_status_t moe_route_topk(const void* x, const void* wr, const float* bias, mo
   }
   MOE_TRY(check_device());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_route(x, wr, bias, d.T, d.H, d.E, d.k, logits, ids, w, s);
+  cudaError_t e = launch_route(x, wr, bias, d.T, d.H, d.E, d.k, logits, ids, w, nullptr, 0, s);
   if (e != cudaSuccess) return cuda_fail(e, "router");
   return ok();
 }
@@ -472,7 +473,10 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
   const char* why = "";
   cudaError_t e;
   record(s, 0);
-  if ((e = launch_route(x, wr, bias, T, H, E, k, logits, ids, tw, s)) != cudaSuccess)
+  // the E > 32 router may use the y_perm region (idle until GEMM-2) for its
+  // per-h-block sums
+  if ((e = launch_route(x, wr, bias, T, H, E, k, logits, ids, tw, at<float>(ws, L.y_perm),
+                        (size_t)(L.total - L.y_perm), s)) != cudaSuccess)
     return cuda_fail(e, "router");
   record(s, 1);
   // The permuted copy of x feeds GEMM1's TMA tile loads (a gather inside the

@@ -50,12 +50,15 @@ __device__ __forceinline__ void load_bf16_vec(const uint16_t* p, float (&v)[N]) 
 constexpr int kRouterBlocks = 8;  // h blocks of the fixed summation order
 constexpr int kWideKC = 32;
 
-template <bool VEC>
-__global__ void __launch_bounds__(256, 1) router_wide_kernel(const __nv_bfloat16* __restrict__ x,
-                                                             const __nv_bfloat16* __restrict__ wr,
-                                                             const float* __restrict__ bias,
-                                                             int T, int H, int E,
-                                                             float* __restrict__ logits) {
+// SPLIT: grid.z runs the 8 h blocks as separate CTAs, each writing its
+// block sums to part[b][t][e] (the running total and the bias are then
+// applied by topk_kernel<PER, true>, in the same order); for many more CTAs
+// than the 64-token tiles give and without the running-total registers.
+template <bool VEC, bool SPLIT>
+__global__ void __launch_bounds__(256, 1) router_wide_kernel(
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
+    const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
+    float* __restrict__ part) {
   constexpr int BT = 64, EC = 256, KC = kWideKC;
   constexpr int XVEC = BT * KC / 8 / 256;  // 16-byte x vectors per thread per chunk (1)
   constexpr int WVEC = KC * EC / 8 / 256;  // 16-byte Wr vectors per thread per chunk (4)
@@ -115,15 +118,24 @@ __global__ void __launch_bounds__(256, 1) router_wide_kernel(const __nv_bfloat16
   // acc[a][p]: the current h block's sums of experts (2p, 2p+1) of token a;
   // tot[a][p]: the finished blocks' sums, added left to right (the fixed
   // blocked order: 8 contiguous h blocks, each summed from zero)
-  float2 acc[8][4], tot[8][4];
+  float2 acc[8][4], tot[SPLIT ? 1 : 8][4];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int p = 0; p < 4; ++p) acc[a][p] = tot[a][p] = make_float2(0.0f, 0.0f);
-  const int nchunks = H / KC;
+    for (int p = 0; p < 4; ++p) acc[a][p] = make_float2(0.0f, 0.0f);
+  if constexpr (!SPLIT) {
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+      for (int p = 0; p < 4; ++p) tot[a][p] = make_float2(0.0f, 0.0f);
+  }
   const int L = H / kRouterBlocks;  // a multiple of 16, so blocks end on 16-h steps
+  const int hbase = SPLIT ? (int)blockIdx.z * L : 0;  // SPLIT: L is a multiple of KC
+  const int nchunks = (SPLIT ? L : H) / KC;
   int done = 0;                     // finished blocks
   auto fold = [&]() {
+    if constexpr (SPLIT) return;
+    else {
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
@@ -134,13 +146,14 @@ __global__ void __launch_bounds__(256, 1) router_wide_kernel(const __nv_bfloat16
         acc[a][p] = make_float2(0.0f, 0.0f);
       }
     ++done;
+    }
   };
-  load(0);
+  load(hbase);
   store(0);
   __syncthreads();
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
-    if (c + 1 < nchunks) load((c + 1) * KC);
+    if (c + 1 < nchunks) load(hbase + (c + 1) * KC);
     const float* xb = xs + b * KC * BT + tok0;
     const float* wb = ws + b * KC * EC + eg * 4;
 #pragma unroll 1
@@ -161,7 +174,7 @@ __global__ void __launch_bounds__(256, 1) router_wide_kernel(const __nv_bfloat16
           for (int p = 0; p < 4; ++p) acc[a][p] = __ffma2_rn(xa, wv[p], acc[a][p]);
         }
       }
-      if ((c * KC + h0 + 16) % L == 0) fold();
+      if (!SPLIT && (c * KC + h0 + 16) % L == 0) fold();
     }
     if (c + 1 < nchunks) store(b ^ 1);
     __syncthreads();
@@ -173,8 +186,15 @@ __global__ void __launch_bounds__(256, 1) router_wide_kernel(const __nv_bfloat16
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const int ee = e0 + eg * 8 + 2 * p;
-      if (ee < E) logits[(int64_t)t * E + ee] = __fadd_rn(tot[a][p].x, bias ? bias[ee] : 0.0f);
-      if (ee + 1 < E) logits[(int64_t)t * E + ee + 1] = __fadd_rn(tot[a][p].y, bias ? bias[ee + 1] : 0.0f);
+      if constexpr (SPLIT) {
+        float* d = part + ((int64_t)blockIdx.z * T + t) * E + ee;
+        if (ee < E) d[0] = acc[a][p].x;
+        if (ee + 1 < E) d[1] = acc[a][p].y;
+      } else {
+        if (ee < E) logits[(int64_t)t * E + ee] = __fadd_rn(tot[a][p].x, bias ? bias[ee] : 0.0f);
+        if (ee + 1 < E)
+          logits[(int64_t)t * E + ee + 1] = __fadd_rn(tot[a][p].y, bias ? bias[ee + 1] : 0.0f);
+      }
     }
   }
 }
@@ -182,19 +202,38 @@ __global__ void __launch_bounds__(256, 1) router_wide_kernel(const __nv_bfloat16
 // One warp per token. Lane l holds logits e = l + 32*i. k rounds of a warp
 // argmax on (logit desc, index asc); slot j gets the j-th winner. Weights:
 // w_j = exp(l_j - l_max) / sum_selected exp(l_i - l_max).
-template <int PER>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
+// PART: the logits are first formed from the 8 block sums part[b][t][e] of
+// the split wide kernel, added left to right, then the bias (the fixed
+// blocked order), and written to `logits`.
+template <int PER, bool PART>
+__global__ void __launch_bounds__(256) topk_kernel(float* __restrict__ logits,
+                                                   const float* __restrict__ part,
+                                                   const float* __restrict__ bias, int T, int E,
                                                    int k, int32_t* __restrict__ ids,
                                                    float* __restrict__ w) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
-  const float* l = logits + (int64_t)warp * E;
+  float* l = logits + (int64_t)warp * E;
   float v[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     int e = lane + 32 * i;
-    v[i] = e < E ? l[e] : -INFINITY;
+    if constexpr (PART) {
+      if (e < E) {
+        const float* p = part + (int64_t)warp * E + e;
+        float s = p[0];
+#pragma unroll
+        for (int b = 1; b < kRouterBlocks; ++b) s = __fadd_rn(s, p[(int64_t)b * T * E]);
+        s = __fadd_rn(s, bias ? bias[e] : 0.0f);
+        l[e] = s;
+        v[i] = s;
+      } else {
+        v[i] = -INFINITY;
+      }
+    } else {
+      v[i] = e < E ? l[e] : -INFINITY;
+    }
   }
   uint32_t taken = 0;  // bit i: v[i] already selected (or absent)
 #pragma unroll
@@ -562,16 +601,19 @@ static int narrow_pairs(int E) {
   return ep / 2;
 }
 
-cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                        cudaStream_t s);
+cudaError_t launch_topk_part(float* logits, const float* part, const float* bias, int T, int E,
+                             int k, int32_t* ids, float* w, cudaStream_t s);
 
 // Logits and top-k of T tokens: for E <= 32 the fused tall kernel (many
 // tokens, Wr fits shared memory) or the fused narrow kernel; else the wide
-// logits kernel followed by the warp-per-token selection.
+// logits kernel followed by the warp-per-token selection. With scratch for
+// 8 T E floats (and H a multiple of 256) the wide kernel runs its 8 h blocks
+// as separate CTAs and the selection adds the block sums in order.
 constexpr int kTallMinT = 1024;
 constexpr size_t kTallMaxSmem = 200 * 1024;
 cudaError_t launch_route(const void* x, const void* wr, const float* bias, int T, int H, int E,
-                         int k, float* logits, int32_t* ids, float* w, cudaStream_t s) {
+                         int k, float* logits, int32_t* ids, float* w, float* part,
+                         size_t part_bytes, cudaStream_t s) {
   const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
   const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(wr);
   if (E <= 32 && T >= kTallMinT) {
@@ -619,25 +661,40 @@ cudaError_t launch_route(const void* x, const void* wr, const float* bias, int T
     return cudaGetLastError();
   }
   const size_t smem = 2 * (size_t)kWideKC * (64 + 256) * 4;
-  dim3 grid((unsigned)ceil_div(T, 64), (unsigned)ceil_div(E, 256));
+  const bool split = part && part_bytes >= (size_t)kRouterBlocks * T * E * sizeof(float) &&
+                     (H / kRouterBlocks) % kWideKC == 0;
+  dim3 grid((unsigned)ceil_div(T, 64), (unsigned)ceil_div(E, 256), split ? kRouterBlocks : 1);
+#define MOE_WIDE(VECV, SPLITV)                                                                   \
+  do {                                                                                           \
+    cudaFuncSetAttribute(router_wide_kernel<VECV, SPLITV>,                                        \
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                 \
+    router_wide_kernel<VECV, SPLITV><<<grid, 256, smem, s>>>(xp, wp, bias, T, H, E, logits, part); \
+  } while (0)
   if (E % 8 == 0) {
-    cudaFuncSetAttribute(router_wide_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    router_wide_kernel<true><<<grid, 256, smem, s>>>(xp, wp, bias, T, H, E, logits);
+    if (split) MOE_WIDE(true, true);
+    else MOE_WIDE(true, false);
   } else {
-    cudaFuncSetAttribute(router_wide_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    router_wide_kernel<false><<<grid, 256, smem, s>>>(xp, wp, bias, T, H, E, logits);
+    if (split) MOE_WIDE(false, true);
+    else MOE_WIDE(false, false);
   }
+#undef MOE_WIDE
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_topk(logits, T, E, k, ids, w, s);
+  return launch_topk_part(logits, split ? part : nullptr, bias, T, E, k, ids, w, s);
 }
 
-cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
-                        cudaStream_t s) {
+// Selection of the top k of each token's E logits (a warp per token); with
+// `part`, the logits are first formed from the split kernel's block sums.
+cudaError_t launch_topk_part(float* logits, const float* part, const float* bias, int T, int E,
+                             int k, int32_t* ids, float* w, cudaStream_t s) {
   int per = (E + 31) / 32;
   dim3 grid((unsigned)ceil_div((int64_t)T * 32, 256));
-#define MOE_TOPK(P) topk_kernel<P><<<grid, 256, 0, s>>>(logits, T, E, k, ids, w)
+#define MOE_TOPK(P)                                                              \
+  do {                                                                           \
+    if (part) topk_kernel<P, true><<<grid, 256, 0, s>>>(logits, part, bias, T, E, k, ids, w); \
+    else topk_kernel<P, false><<<grid, 256, 0, s>>>(logits, nullptr, nullptr, T, E, k, ids, w); \
+  } while (0)
   if (per <= 1)
     MOE_TOPK(1);
   else if (per <= 2)
@@ -653,6 +710,11 @@ cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, 
 #undef MOE_TOPK
   note_launch();
   return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                        cudaStream_t s) {
+  return launch_topk_part(const_cast<float*>(logits), nullptr, nullptr, T, E, k, ids, w, s);
 }
 
 }  // namespace moe

@@ -79,6 +79,10 @@ def test_mixtral_decode_all_tokens():
     dict(T=300, E=16, k=1, H=256, I=384),        # Switch top-1, I not a multiple of 256
     dict(T=513, E=32, k=4, H=384, I=256),        # rows spanning several tiles + ragged tail
     dict(T=40, E=8, k=2, H=256, I=128),          # decode-sized (small-M path)
+    # E > 32: the wide router with its h blocks as separate CTAs (H % 256 == 0) or not
+    dict(T=200, E=40, k=4, H=256, I=256, bias="normal"),
+    dict(T=77, E=37, k=3, H=512, I=128),         # E not a multiple of 8
+    dict(T=150, E=48, k=2, H=384, I=256),        # H % 256 != 0: blocks in one CTA
 ])
 def test_edge_shapes(kw):
     cfg = mi.CONFIGS["tiny"].with_(**kw)
