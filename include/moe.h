@@ -145,9 +145,10 @@ moe_status_t moe_workspace_layout(moe_dims_t d, moe_dtype_t dt, moe_ws_layout_t*
  *              fp32 logits go to the lower expert index
  *   w_dev      fp32 [T, k] out: exp(l_j - l_max) / sum over selected
  *   ws/ws_bytes workspace (needed when logits_dev is NULL; may be NULL else)
- * The logits are fp32 sums over h in ascending order of exact bf16 x bf16
- * products, so they (and the ids) are bit-reproducible functions of the
- * inputs. I is ignored. */
+ * The logits are fp32 sums of exact bf16 x bf16 products in a fixed order:
+ * 8 contiguous h blocks of H/8, each summed from zero h ascending, the block
+ * sums added left to right, then the bias. So they (and the ids) are
+ * bit-reproducible functions of the inputs. I is ignored. */
 moe_status_t moe_route_topk(const void* x_dev, const void* wr_dev, const float* bias_dev,
                             moe_dims_t d, float* logits_dev, int32_t* ids_dev, float* w_dev,
                             void* ws, size_t ws_bytes, void* stream);

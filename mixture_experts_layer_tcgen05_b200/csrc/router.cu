@@ -6,12 +6,14 @@
 // the k largest are kept and renormalised over the selected experts.
 //
 // The logits decide integers (the selected ids), so they are computed in a
-// fixed order: one fp32 accumulator per (token, expert), h ascending, one
-// fused multiply-add per term. A bf16 x bf16 product is exact in fp32, so the
-// FMA equals the rounded sum of the exact product and every logit is a fixed
-// function of the inputs. The work is register-tiled on CUDA cores (each
-// thread owns TT tokens x TE experts); tensor cores are not used here because
-// their internal accumulation order is not specified.
+// fixed order: the h range is cut into 8 contiguous blocks of H/8; each block
+// is summed from zero, h ascending, one fp32 fused multiply-add per term (a
+// bf16 x bf16 product is exact in fp32, so the FMA equals the rounded sum of
+// the exact product); the 8 block sums are added left to right, then the
+// bias. Every logit is thus a fixed function of the inputs, whichever kernel
+// computes it (tall, narrow, wide, split or not). The work runs on CUDA cores;
+// tensor cores are not used here because their internal accumulation order
+// is not specified.
 #include "gemm_common.cuh"  // num_sms
 #include "ptx.cuh"
 
