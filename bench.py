@@ -422,6 +422,8 @@ def gpu_arm(args, cfg):
                 "traffic": kernel_traffic(cfg.name, "gemm1"),
                 "kernel": ("gemm_mx_kernel<SwiGLU, e2m1 B> (FP4 GEMM1 + SwiGLU + h quantisation)"
                            if cfg.fp4 else
+                           "gemm_mx_kernel<SwiGLU> (block-scaled FP8 GEMM1 + SwiGLU + h quantisation)"
+                           if cfg.ue8m0 else
                            "gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)"
                            if cfg.fp8 else "gemm_swap_kernel<SwiGLU> (GEMM1, small-M)"),
                 "algorithmic_bytes_per_launch": g1_bytes, "peak_source": peak_src}

@@ -330,15 +330,18 @@ moe_status_t moe_forward_fp4(const void* x_dev, const void* wr_dev, const float*
  *                gated epilogue (gate rows then up rows), N otherwise
  *   b_scales_dev e8m0 bytes in the chunk layout of moe_forward_fp4, E * N_B * K / 32
  *                bytes (16-byte aligned)
- *   C_dev        bf16 [M_total, N] (plain; N % 256 == 0), or with a gated
- *                epilogue e4m3 [M_total, N] + c_scales_dev fp32 [M_total, N/128]
+ *   C_dev        bf16 [M_total, N] (plain; N % 256 == 0 in the tokens-in-M form),
+ *                or with a gated epilogue e4m3 [M_total, N] + c_scales_dev fp32 [M_total, N/128]
  *                (power-of-two scales), or bf16 when c_scales_dev is NULL
- *   offsets, E, ws as for moe_grouped_gemm. */
+ *   offsets, E, ws as for moe_grouped_gemm; max_rows_per_expert in [1, 64]
+ *   (an upper bound on any expert's rows, e.g. the token count of a decode
+ *   batch) selects the weights-in-M (swap-AB) form, 0 the tokens-in-M one. */
 moe_status_t moe_grouped_gemm_fp4(const void* A_dev, const float* a_scales_dev, const void* B_dev,
                                   const uint8_t* b_scales_dev, const int32_t* offsets_dev,
                                   int32_t M_total, int32_t E, int32_t N, int32_t K,
-                                  moe_epilogue_t ep, void* C_dev, float* c_scales_dev, void* ws,
-                                  size_t ws_bytes, void* stream);
+                                  moe_epilogue_t ep, void* C_dev, float* c_scales_dev,
+                                  int32_t max_rows_per_expert, void* ws, size_t ws_bytes,
+                                  void* stream);
 
 /* FP4 weight quantisation (one-time preparation): nb matrices bf16 [rows,
  * cols] (rows, cols multiples of 128) -> q_dev packed e2m1 [nb, rows, cols/2],

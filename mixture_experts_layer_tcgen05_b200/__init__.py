@@ -86,7 +86,7 @@ _SIGS = {
                                      _vp]),
     "moe_forward_fp4": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, Dims, _i32, _vp, _vp, _sz, _vp]),
     "moe_grouped_gemm_fp4": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
-                                    _vp, _vp, _sz, _vp]),
+                                    _vp, _i32, _vp, _sz, _vp]),
     "moe_quantize_weight_fp4": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "moe_quantize_act_fp8": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "moe_quantize_weight_fp8": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
@@ -258,10 +258,11 @@ def moe_forward_fp4(x, wr, bias, w13q, w13s, w2q, w2s, d, act, out, ws, ws_bytes
 
 
 def moe_grouped_gemm_fp4(A, a_scales, B, b_scales, offsets, M_total, E, N, K, ep, C,
-                         c_scales=None, ws=None, ws_bytes=None, stream=None):
+                         c_scales=None, ws=None, ws_bytes=None, stream=None, max_rows_per_expert=0):
     _check(lib().moe_grouped_gemm_fp4(_p(A), _p(a_scales), _p(B), _p(b_scales), _p(offsets),
-                                      M_total, E, N, K, int(ep), _p(C), _p(c_scales), _p(ws),
-                                      _nbytes(ws, ws_bytes), _s(stream)))
+                                      M_total, E, N, K, int(ep), _p(C), _p(c_scales),
+                                      int(max_rows_per_expert), _p(ws), _nbytes(ws, ws_bytes),
+                                      _s(stream)))
 
 
 def moe_quantize_weight_fp4(w, nb, rows, cols, q, s, stream=None):

@@ -50,6 +50,11 @@ cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const v
                                    void* Cout, float* c_scales, int32_t* status, cudaStream_t s,
                                    const char** why);
 cudaError_t launch_wait_selftest(int32_t* status, long long budget, cudaStream_t s);
+cudaError_t launch_grouped_gemm_mx_swap(const void* A, const float* a_scales, const void* B,
+                                        const float* b_scales, const uint8_t* b_sf8,
+                                        const int32_t* offsets, int M_total, int E, int N, int K,
+                                        int act, void* Cout, float* c_scales, int max_rows,
+                                        int32_t* status, cudaStream_t s, const char** why);
 cudaError_t launch_quant_weight_fp4(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                     uint8_t* sc, cudaStream_t s);
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
@@ -381,6 +386,10 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
                                 offsets, M_total, E, N, K,
                                 (int)ep, C, c_scales, max_rows_per_expert,
                                 at<int32_t>(ws, 0), static_cast<cudaStream_t>(stream), &why);
+  else if (max_rows_per_expert > 0 && max_rows_per_expert <= 64)  // decode sizes: weights in M
+    e = launch_grouped_gemm_mx_swap(A, a_scales, B, b_scales, nullptr, offsets, M_total, E, N, K,
+                                    (int)ep, C, c_scales, max_rows_per_expert, at<int32_t>(ws, 0),
+                                    static_cast<cudaStream_t>(stream), &why);
   else
     e = launch_grouped_gemm_mx(A, a_scales, B, b_scales, nullptr, offsets, M_total, E, N, K,
                                (int)ep, C, c_scales, at<int32_t>(ws, 0),
@@ -392,14 +401,16 @@ moe_status_t moe_grouped_gemm(const void* A, const int32_t* a_rows, int32_t a_sr
 moe_status_t moe_grouped_gemm_fp4(const void* A, const float* a_scales, const void* B,
                                   const uint8_t* b_scales, const int32_t* offsets, int32_t M_total,
                                   int32_t E, int32_t N, int32_t K, moe_epilogue_t ep, void* C,
-                                  float* c_scales, void* ws, size_t ws_bytes, void* stream) {
+                                  float* c_scales, int32_t max_rows_per_expert, void* ws,
+                                  size_t ws_bytes, void* stream) {
   if (M_total < 1) return fail(MOE_ERR_INVALID_ARG, "M_total must be >= 1");
   if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 1024]");
   if (N < 128 || N % 128 || K < 128 || K % 128)
     return fail(MOE_ERR_INVALID_ARG, "N and K must be positive multiples of 128 (N=%d K=%d)", N, K);
   if (ep < MOE_EPILOGUE_NONE || ep > MOE_EPILOGUE_REGLU) return fail(MOE_ERR_INVALID_ARG, "bad epilogue");
-  if (ep == MOE_EPILOGUE_NONE && N % 256)
-    return fail(MOE_ERR_INVALID_ARG, "the plain FP4 GEMM needs N %% 256 == 0 (N=%d)", N);
+  const bool small = max_rows_per_expert > 0 && max_rows_per_expert <= 64;
+  if (ep == MOE_EPILOGUE_NONE && N % 256 && !small)
+    return fail(MOE_ERR_INVALID_ARG, "the plain tokens-in-M FP4 GEMM needs N %% 256 == 0 (N=%d)", N);
   MOE_TRY(check_ptr(A, "A"));
   MOE_TRY(check_ptr(a_scales, "a_scales"));
   MOE_TRY(check_ptr(B, "B"));
@@ -414,9 +425,14 @@ moe_status_t moe_grouped_gemm_fp4(const void* A, const float* a_scales, const vo
   if (ws_bytes < 256) return fail(MOE_ERR_WORKSPACE, "workspace too small: %zu bytes", ws_bytes);
   MOE_TRY(check_device());
   const char* why = "";
-  cudaError_t e = launch_grouped_gemm_mx(A, a_scales, B, nullptr, b_scales, offsets, M_total, E, N,
-                                         K, (int)ep, C, c_scales, at<int32_t>(ws, 0),
-                                         static_cast<cudaStream_t>(stream), &why);
+  cudaError_t e =
+      small
+          ? launch_grouped_gemm_mx_swap(A, a_scales, B, nullptr, b_scales, offsets, M_total, E, N, K,
+                                        (int)ep, C, c_scales, max_rows_per_expert, at<int32_t>(ws, 0),
+                                        static_cast<cudaStream_t>(stream), &why)
+          : launch_grouped_gemm_mx(A, a_scales, B, nullptr, b_scales, offsets, M_total, E, N, K,
+                                   (int)ep, C, c_scales, at<int32_t>(ws, 0),
+                                   static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "FP4 grouped GEMM: %s %s", cudaGetErrorString(e), why);
   return ok();
 }
@@ -533,6 +549,8 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
       const float* f2 = fp4 ? nullptr : w2s;
       const uint8_t* b13 = fp4 ? reinterpret_cast<const uint8_t*>(w13s) : nullptr;
       const uint8_t* b2 = fp4 ? reinterpret_cast<const uint8_t*>(w2s) : nullptr;
+      // the tokens-in-M kernel at every batch size: at decode sizes the
+      // weights-in-M form measured no faster (weight streaming bounds both)
       if ((e = launch_grouped_gemm_mx(xq_perm, xs_perm, w13, f13, b13, offsets, R, E, I, H, act, hq,
                                       hs, status, s, &why)) != cudaSuccess)
         return fail(MOE_ERR_CUDA, "%s GEMM1: %s %s", fp4 ? "FP4" : "FP8", cudaGetErrorString(e), why);

@@ -108,9 +108,10 @@ __device__ __forceinline__ void sf_copy(uint32_t tmem, uint64_t desc) {
 // Block-scaled instruction descriptor: e4m3 x (e4m3 or e2m1), fp32
 // accumulate, E8M0 scales, scale-factor ids (the K step) for A and B.
 constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
-__host__ __device__ constexpr uint32_t mx_idesc(int M, int N, uint32_t sf_id, uint32_t b_fmt) {
+__host__ __device__ constexpr uint32_t mx_idesc(int M, int N, uint32_t sf_id, uint32_t b_fmt,
+                                               uint32_t a_fmt = 0) {
   return (sf_id << 4)                    // B scale-factor id
-         | (0u << 7) | (b_fmt << 10)      // A format E4M3; B format E4M3 (0) or E2M1 (5)
+         | (a_fmt << 7) | (b_fmt << 10)   // A, B formats: E4M3 (0) or E2M1 (5)
          | ((uint32_t)(N >> 3) << 17)     // N / 8
          | (1u << 23)                     // scale format E8M0
          | ((uint32_t)(M >> 4) << 24)     // M / 16
@@ -430,6 +431,282 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+
+// ==========================================================================
+// small-M (swap-AB) block-scaled kernel: weights in the MMA's M slot
+// ==========================================================================
+// For decode-sized batches an expert has a few rows, so the tokens-in-M
+// kernel would load (and multiply) 128-row token tiles for them. Here the
+// expert's weight rows take the MMA's M = 128 and its tokens the N = BNT
+// (16, 32 or 64) slot, as in the bf16 small-M kernel: A = weights (e4m3 or
+// e2m1, with their scale chunks), B = token rows (e4m3, power-of-two scales
+// per row and 128-K block). A tile is (expert, token tile, 128 output
+// columns); for a gated epilogue a stage holds the gate and the up rows of
+// those columns and each K step issues two MMAs. The accumulator is
+// transposed (TMEM lane = output column, column = token), double-buffered.
+// Output: bf16, or for a gated epilogue with c_scales e4m3 + power-of-two
+// scales per (row, 128 columns), the 128 columns of a tile being exactly one
+// group (the group maximum is exchanged between the four epilogue warps).
+template <int ACT, bool BFP4, int BNT>
+struct MxSwapCfg {
+  static constexpr bool SWIGLU = ACT != kActNone;
+  static constexpr int kNA = SWIGLU ? 2 : 1;          // weight boxes per stage
+  static constexpr int kTileW = 128 * BK;             // 16 KB (e2m1: unpacked layout)
+  static constexpr int kTileT = BNT * BK;             // token rows of a stage
+  static constexpr int kStage = kNA * kTileW + kTileT;  // a multiple of 1024
+  static constexpr int kSf = (kNA + 1) * kSfA;        // weight chunk(s) + token chunk
+  static constexpr int STAGES = (200 * 1024) / (kStage + kSf) > 8 ? 8 : (200 * 1024) / (kStage + kSf);
+  static constexpr int kAccCols = kNA * BNT;          // per accumulator buffer
+  static constexpr int kSfCol = 256;                  // scale-factor ring after the accumulators
+  static constexpr size_t kSmem = 1024 + (size_t)STAGES * (kStage + kSf) + 256 +
+                                  2 * (kMaxE + 1) * 4 + 2 * 4 * BNT * 4;
+  // transaction bytes of a stage: packed e2m1 counts two codes per byte
+  static constexpr uint32_t kTx = kNA * (BFP4 ? kTileW / 2 + kSfA : kTileW) + kTileT;
+};
+
+template <int ACT, bool BFP4, int BNT>
+__global__ void __launch_bounds__(192, 1)
+    gemm_mx_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
+                        Args args) {
+  using C = MxSwapCfg<ACT, BFP4, BNT>;
+  constexpr bool SWIGLU = C::SWIGLU;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sf = smem + STAGES * C::kStage;  // [STAGES][weight chunk(s), token chunk]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sf + STAGES * C::kSf);
+  // bars: full[STAGES], empty[STAGES], accf[2], acce[2], drain, redbar[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 7);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(sf + STAGES * C::kSf + 256);
+  int32_t* soff = tile_start + kMaxE + 1;  // [E + 1] expert offsets, shared copy
+  float* red = reinterpret_cast<float*>(soff + kMaxE + 1);  // [2 tiles][4 warps][BNT]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = ptx::smem_addr(smem), sfbase = ptx::smem_addr(sf);
+  const uint32_t full0 = ptx::smem_addr(bars), empty0 = full0 + STAGES * 8;
+  const uint32_t accf0 = empty0 + STAGES * 8, acce0 = accf0 + 16, drain = acce0 + 16;
+  const uint32_t redbar0 = drain + 8;  // group-maximum exchange, by tile parity
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full0 + s * 8, 1);
+      ptx::mbar_init(empty0 + s * 8, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(accf0 + a * 8, 1);
+      ptx::mbar_init(acce0 + a * 8, 4);
+      ptx::mbar_init(redbar0 + a * 8, 128);
+    }
+    ptx::mbar_init(drain, 1);
+    ptx::fence_barrier_init();
+    ptx::tma_prefetch_desc(&tmW);
+    ptx::tma_prefetch_desc(&tmT);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 2) gg::build_tile_starts<BNT>(args.offsets, args.E, args.NT, tile_start, soff);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = tile_start[args.E];
+  const int nkb = args.kblocks;
+
+  // tile -> expert, token tile, 128-column output tile
+  auto decode = [&](int tile, int& e, int& tt, int& n) {
+    e = gg::find_expert(tile_start, args.E, tile);
+    const int local = tile - tile_start[e];
+    tt = local / args.NT;
+    n = local % args.NT;
+  };
+
+  if (warp == 0) {
+    // all lanes: scale chunks; lane 0: barriers and TMA loads
+    int64_t issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      int e, tt, n;
+      decode(tile, e, tt, n);
+      const int row0 = soff[e] + tt * BNT, row_end = soff[e + 1];
+      const int rw0 = e * args.b_rows + n * 128;              // gate (or only) weight rows
+      const int rw1 = SWIGLU ? rw0 + args.up_off : rw0;      // up weight rows
+      const float* sw0 = args.b_scales + ((int64_t)e * args.b_nblk + (n * 128 >> 7)) * nkb;
+      const float* sw1 = SWIGLU ? args.b_scales + ((int64_t)e * args.b_nblk + ((args.up_off + n * 128) >> 7)) * nkb
+                                : sw0;
+      const unsigned char* swc0 = BFP4 ? args.b_sf8 + (int64_t)(rw0 >> 7) * nkb * kSfA : nullptr;
+      const unsigned char* swc1 = BFP4 ? args.b_sf8 + (int64_t)(rw1 >> 7) * nkb * kSfA : nullptr;
+      // token rows lane and lane + 32 of the tile (scale 1 past the expert)
+      const int r0 = row0 + lane, r1 = row0 + 32 + lane;
+      const float* st0 = r0 < row_end ? args.a_scales + (int64_t)r0 * nkb : nullptr;
+      const float* st1 = (BNT > 32 && r1 < row_end) ? args.a_scales + (int64_t)r1 * nkb : nullptr;
+      for (int kb = 0; kb < nkb; ++kb, ++issued) {
+        const int s = (int)(issued % STAGES);
+        const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
+        const float t0s = st0 ? __ldg(st0 + kb) : 1.0f;
+        const float t1s = st1 ? __ldg(st1 + kb) : 1.0f;
+        float w0s = 1.0f, w1s = 1.0f;
+        if constexpr (!BFP4) {
+          w0s = __ldg(sw0 + kb);
+          w1s = __ldg(sw1 + kb);
+        }
+        int got = 1;
+        if (lane == 0) got = ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
+        }
+        unsigned char* sfs = sf + s * C::kSf;  // [weight chunk(s)][token chunk]
+        const uint32_t tc0 = e8m0_code(t0s) * 0x01010101u, tc1 = e8m0_code(t1s) * 0x01010101u;
+        *reinterpret_cast<uint4*>(sfs + C::kNA * kSfA + lane * 16) =
+            make_uint4(tc0, tc1, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        if constexpr (!BFP4) {  // one block scale per 128 x 128 weight block: the same code everywhere
+          const uint32_t c0 = e8m0_code(w0s) * 0x01010101u, c1 = e8m0_code(w1s) * 0x01010101u;
+          *reinterpret_cast<uint4*>(sfs + lane * 16) = make_uint4(c0, c0, c0, c0);
+          if (SWIGLU) *reinterpret_cast<uint4*>(sfs + kSfA + lane * 16) = make_uint4(c1, c1, c1, c1);
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t sw = sbase + s * C::kStage, st = sw + C::kNA * C::kTileW;
+          ptx::mbar_arrive_expect_tx(full0 + s * 8, C::kTx);
+          ptx::tma_load_2d(sw, &tmW, kb * BK, rw0, full0 + s * 8);
+          if (SWIGLU) ptx::tma_load_2d(sw + C::kTileW, &tmW, kb * BK, rw1, full0 + s * 8);
+          ptx::tma_load_2d(st, &tmT, kb * BK, row0, full0 + s * 8);
+          if constexpr (BFP4) {
+            const uint32_t sfd = sfbase + s * C::kSf;
+            ptx::bulk_load(sfd, swc0 + (int64_t)kb * kSfA, kSfA, full0 + s * 8);
+            if (SWIGLU) ptx::bulk_load(sfd + kSfA, swc1 + (int64_t)kb * kSfA, kSfA, full0 + s * 8);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) gg::drain_loads<STAGES>(full0, issued, args.status);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int64_t consumed = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      constexpr uint32_t kWFmt = BFP4 ? kFmtE2M1 : kFmtE4M3;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        if (!ptx::mbar_wait(acce0 + acc * 8, acc_ph ^ 1, args.status, kSiteMmaAccEmpty)) break;
+        ptx::tc_fence_after();
+        const uint32_t d = tmem_base + acc * C::kAccCols;
+        for (int kb = 0; kb < nkb; ++kb, ++consumed) {
+          const int s = (int)(consumed % STAGES);
+          const uint32_t ph = (uint32_t)((consumed / STAGES) & 1);
+          if (!ptx::mbar_wait(full0 + s * 8, ph, args.status, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          // scale-factor ring: weight chunk(s) at +0 (+4), token chunk at +8
+          const uint32_t sfcol = tmem_base + C::kSfCol + s * 16;
+          const uint32_t sfs = sfbase + s * C::kSf;
+          sf_copy(sfcol, sf_desc(sfs));
+          if (SWIGLU) sf_copy(sfcol + 4, sf_desc(sfs + kSfA));
+          sf_copy(sfcol + 8, sf_desc(sfs + C::kNA * kSfA));
+          const uint32_t sw = sbase + s * C::kStage, st = sw + C::kNA * C::kTileW;
+          const uint64_t dw = ptx::sw128_kmajor_desc(sw), dt = ptx::sw128_kmajor_desc(st);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk) {
+            const uint64_t ko = (uint64_t)(kk * UK / 16);
+            const uint32_t idesc = mx_idesc(128, BNT, (uint32_t)kk, kFmtE4M3, kWFmt);
+            mma_mx(d, dw + ko, dt + ko, idesc, sfcol, sfcol + 8, (kb | kk) != 0);
+            if (SWIGLU)
+              mma_mx(d + BNT, dw + (uint64_t)(C::kTileW >> 4) + ko, dt + ko, idesc, sfcol + 4,
+                     sfcol + 8, (kb | kk) != 0);
+          }
+          ptx::mma_commit(empty0 + s * 8);
+        }
+        if (!ok) break;
+        ptx::mma_commit(accf0 + acc * 8);
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1;
+      }
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, args.status, kSiteDrain);
+    }
+  } else {
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    int tile_iter = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tile_iter) {
+      int e, tt, n;
+      decode(tile, e, tt, n);
+      const int row0 = soff[e] + tt * BNT;
+      const int nrows = min(min(BNT, soff[e + 1] - row0), args.M_total - row0);
+      const int col = n * 128 + q * 32 + lane;  // output column owned by this thread
+      if (!ptx::mbar_wait(accf0 + acc * 8, acc_ph, args.status, kSiteEpiAccFull)) break;
+      ptx::tc_fence_after();
+      const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
+      float v[BNT];
+#pragma unroll
+      for (int c = 0; c < BNT; c += 16) {
+        uint32_t g[16], u[16];
+        ptx::tmem_ld16(t0 + c, g);
+        if (SWIGLU) ptx::tmem_ld16(t0 + BNT + c, u);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[c + i] = SWIGLU ? gated<ACT>(__uint_as_float(g[i]), __uint_as_float(u[i]))
+                            : __uint_as_float(g[i]);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acce0 + acc * 8);
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1;
+      if (SWIGLU && args.c_scales) {
+        // e4m3 output: the 128 columns of this tile are one group of each row
+        float* rb = red + (tile_iter & 1) * 4 * BNT;
+#pragma unroll
+        for (int t = 0; t < BNT; ++t) {
+          float m = fabsf(v[t]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (lane == 0) rb[q * BNT + t] = m;
+        }
+        // all 128 epilogue threads arrive; a bounded wait, so that a failed
+        // pipeline cannot leave some of them waiting here for good
+        ptx::mbar_arrive(redbar0 + (tile_iter & 1) * 8);
+        if (!ptx::mbar_wait(redbar0 + (tile_iter & 1) * 8, (uint32_t)((tile_iter >> 1) & 1),
+                            args.status, kSiteEpiAccFull))
+          break;
+        uint8_t* cq = static_cast<uint8_t*>(args.C);
+#pragma unroll
+        for (int t = 0; t < BNT; ++t) {
+          if (t < nrows) {
+            const float amax = fmaxf(fmaxf(rb[t], rb[BNT + t]), fmaxf(rb[2 * BNT + t], rb[3 * BNT + t]));
+            const float sc = pow2_scale(amax);
+            const float inv = __frcp_rn(sc);  // exact: sc is a power of two
+            const uint32_t code =
+                __nv_cvt_float2_to_fp8x2(make_float2(v[t] * inv, 0.0f), __NV_SATFINITE, __NV_E4M3) & 0xFFu;
+            cq[(int64_t)(row0 + t) * args.ldc + col] = (uint8_t)code;
+            if (q == 0 && lane == 0) args.c_scales[(int64_t)(row0 + t) * (args.ldc / 128) + n] = sc;
+          }
+        }
+      } else {
+        __nv_bfloat16* cb = static_cast<__nv_bfloat16*>(args.C);
+#pragma unroll
+        for (int t = 0; t < BNT; ++t)
+          if (t < nrows) cb[(int64_t)(row0 + t) * args.ldc + col] = __float2bfloat16_rn(v[t]);
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, 512);
+  }
+}
+
 }  // namespace ggmx
 
 // ==========================================================================
@@ -497,6 +774,79 @@ cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const v
   else MOE_MX_ACT(false);
 #undef MOE_MX_ACT
 #undef MOE_MX
+  note_launch();
+  return cudaGetLastError();
+}
+
+
+// Small-M form of the block-scaled GEMM (weights in M): A = token rows (e4m3,
+// a_scales), B = weights (e4m3 with b_scales, or packed e2m1 with b_sf8
+// chunks); BNT from max_rows (the most rows an expert can have).
+cudaError_t launch_grouped_gemm_mx_swap(const void* A, const float* a_scales, const void* B,
+                                        const float* b_scales, const uint8_t* b_sf8,
+                                        const int32_t* offsets, int M_total, int E, int N, int K,
+                                        int act, void* Cout, float* c_scales, int max_rows,
+                                        int32_t* status, cudaStream_t s, const char** why) {
+  const bool swiglu = act != kActNone;
+  const bool fp4 = b_sf8 != nullptr;
+  const int b_rows = swiglu ? 2 * N : N;
+  if (fp4 && ((reinterpret_cast<uintptr_t>(B) & 31) || (reinterpret_cast<uintptr_t>(b_sf8) & 15))) {
+    *why = "packed FP4 weights must be 32-byte aligned and their scale chunks 16-byte aligned";
+    return cudaErrorInvalidValue;
+  }
+  const int bnt = max_rows <= 16 ? 16 : max_rows <= 32 ? 32 : 64;
+  CUtensorMap tmW, tmT;
+  const bool okW = fp4 ? make_tmap_fp4(&tmW, B, K, (int64_t)E * b_rows, 128)
+                       : make_tmap(&tmW, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (int64_t)E * b_rows, 128);
+  if (!okW || !make_tmap(&tmT, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M_total, bnt)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  ggmx::Args a;
+  a.offsets = offsets;
+  a.E = E;
+  a.K = K;
+  a.ldc = N;
+  a.NT = N / 128;  // 128-column output tiles per expert
+  a.b_rows = b_rows;
+  a.up_off = swiglu ? N : 0;
+  a.band = 0;
+  a.M_total = M_total;
+  a.kblocks = K / 128;
+  a.b_nblk = b_rows / 128;
+  a.C = Cout;
+  a.c_scales = c_scales;
+  a.a_scales = a_scales;
+  a.b_scales = b_scales;
+  a.b_sf8 = b_sf8;
+  a.status = status;
+  const int64_t tiles_ub = ((int64_t)M_total / bnt + (M_total < E ? M_total : E)) * a.NT;
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_ub));
+#define MOE_MXS(ACTV, F4, BN)                                                                      \
+  do {                                                                                             \
+    using Cfg = ggmx::MxSwapCfg<ACTV, F4, BN>;                                                     \
+    cudaError_t e = set_smem(ggmx::gemm_mx_swap_kernel<ACTV, F4, BN>, Cfg::kSmem);                 \
+    if (e != cudaSuccess) return e;                                                                \
+    ggmx::gemm_mx_swap_kernel<ACTV, F4, BN><<<grid, 192, Cfg::kSmem, s>>>(tmW, tmT, a);            \
+  } while (0)
+#define MOE_MXS_BN(ACTV, F4)                          \
+  do {                                                \
+    if (bnt == 16) MOE_MXS(ACTV, F4, 16);             \
+    else if (bnt == 32) MOE_MXS(ACTV, F4, 32);        \
+    else MOE_MXS(ACTV, F4, 64);                       \
+  } while (0)
+#define MOE_MXS_ACT(F4)                               \
+  do {                                                \
+    if (act == kActSilu) MOE_MXS_BN(kActSilu, F4);    \
+    else if (act == kActGelu) MOE_MXS_BN(kActGelu, F4); \
+    else if (act == kActRelu) MOE_MXS_BN(kActRelu, F4); \
+    else MOE_MXS_BN(kActNone, F4);                    \
+  } while (0)
+  if (fp4) MOE_MXS_ACT(true);
+  else MOE_MXS_ACT(false);
+#undef MOE_MXS_ACT
+#undef MOE_MXS_BN
+#undef MOE_MXS
   note_launch();
   return cudaGetLastError();
 }

@@ -169,6 +169,10 @@ CONFIGS = {
     "mixtral_decode_fp4": LayerConfig("mixtral_decode_fp4", 16, 4096, 14336, 8, 2, fp4=True,
                                       desc="Mixtral-shaped decode, FP4 expert weights: T=16 "
                                            "H=4096 I=14336 E=8 k=2"),
+    "mixtral_decode_fp8_ue8m0": LayerConfig("mixtral_decode_fp8_ue8m0", 16, 4096, 14336, 8, 2,
+                                            fp8=True, ue8m0=True,
+                                            desc="Mixtral-shaped decode, FP8 experts with "
+                                                 "power-of-two scales: T=16 H=4096 I=14336 E=8 k=2"),
     "mixtral_decode_fp8": LayerConfig("mixtral_decode_fp8", 16, 4096, 14336, 8, 2, fp8=True,
                                       desc="Mixtral-shaped decode, FP8 experts: T=16 H=4096 "
                                            "I=14336 E=8 k=2"),

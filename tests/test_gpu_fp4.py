@@ -74,14 +74,15 @@ def _problem(counts, NB, K, tag):
     return E, offsets, M, aq, as_, bq, bs
 
 
-@pytest.mark.parametrize("counts,N,K", [([0, 1, 130, 300], 256, 384), ([128, 0, 5], 512, 256),
-                                        ([700], 256, 1024)])
-def test_fp4_grouped_gemm_plain(counts, N, K):
+@pytest.mark.parametrize("counts,N,K,hint", [
+    ([0, 1, 130, 300], 256, 384, 0), ([128, 0, 5], 512, 256, 0), ([700], 256, 1024, 0),
+    ([3, 0, 16, 9], 256, 384, 16), ([1, 30, 2], 384, 256, 32), ([50, 64, 0, 33], 128, 512, 64)])
+def test_fp4_grouped_gemm_plain(counts, N, K, hint):
     E, offsets, M, aq, as_, bq, bs = _problem(counts, N, K, 101)
     C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     moe.moe_grouped_gemm_fp4(dev_u8(aq), dev(as_), dev_u8(bq), dev_u8(_chunks(bs)), dev(offsets), M,
-                             E, N, K, moe.MOE_EPILOGUE_NONE, C, None, ws)
+                             E, N, K, moe.MOE_EPILOGUE_NONE, C, None, ws, max_rows_per_expert=hint)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(ws) == 0
     A, Bd = _dequant_e4m3(aq, as_), _dequant_fp4(bq, bs)
@@ -92,14 +93,15 @@ def test_fp4_grouped_gemm_plain(counts, N, K):
             check_close(got[lo:hi], A[lo:hi] @ Bd[e].T, (2e-2, 5e-3), f"expert {e}")
 
 
-@pytest.mark.parametrize("counts,N,K", [([0, 1, 130, 300], 256, 384), ([256, 7], 512, 256)])
-def test_fp4_grouped_gemm_swiglu_quantised_out(counts, N, K):
+@pytest.mark.parametrize("counts,N,K,hint", [([0, 1, 130, 300], 256, 384, 0), ([256, 7], 512, 256, 0),
+                                             ([3, 0, 16, 9], 256, 384, 16), ([40, 1], 384, 256, 64)])
+def test_fp4_grouped_gemm_swiglu_quantised_out(counts, N, K, hint):
     E, offsets, M, aq, as_, bq, bs = _problem(counts, 2 * N, K, 103)
     C = torch.empty(M, N, dtype=torch.uint8, device="cuda")
     cs = torch.empty(M, N // 128, dtype=torch.float32, device="cuda")
     ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     moe.moe_grouped_gemm_fp4(dev_u8(aq), dev(as_), dev_u8(bq), dev_u8(_chunks(bs)), dev(offsets), M,
-                             E, N, K, moe.MOE_EPILOGUE_SWIGLU, C, cs, ws)
+                             E, N, K, moe.MOE_EPILOGUE_SWIGLU, C, cs, ws, max_rows_per_expert=hint)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(ws) == 0
     A, Bd = _dequant_e4m3(aq, as_), _dequant_fp4(bq, bs)

@@ -48,16 +48,20 @@ def _dense(aq, as_, bq, bs):
 
 
 @pytest.mark.parametrize("unit", [True, False])
-@pytest.mark.parametrize("counts,N,K", [([0, 1, 130, 300], 256, 384), ([128, 0, 5], 512, 256),
-                                        ([700], 256, 1024)])
-def test_mx_grouped_gemm_plain(counts, N, K, unit):
+@pytest.mark.parametrize("counts,N,K,hint", [
+    ([0, 1, 130, 300], 256, 384, 0), ([128, 0, 5], 512, 256, 0), ([700], 256, 1024, 0),
+    # decode sizes: weights in M, 16 / 32 / 64 token columns
+    ([3, 0, 16, 9], 256, 384, 16), ([1, 30, 2], 384, 256, 32), ([50, 64, 0, 33], 128, 512, 64)])
+def test_mx_grouped_gemm_plain(counts, N, K, hint, unit):
     """unit: every scale 1 (the MMA alone); else power-of-two scales per row,
     per 128-row weight block and per 128-K block (the scale-factor layout)."""
+    if hint == 0 and N % 256:
+        pytest.skip("the tokens-in-M form tiles N by 256")
     E, offsets, M, aq, as_, bq, bs = _problem(counts, N, K, 91, unit)
     C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     moe.moe_grouped_gemm(dev_u8(aq), dev_u8(bq), dev(offsets), M, E, N, K, DT,
-                         moe.MOE_EPILOGUE_NONE, C, dev(as_), dev(bs), ws=ws)
+                         moe.MOE_EPILOGUE_NONE, C, dev(as_), dev(bs), max_rows_per_expert=hint, ws=ws)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(ws) == 0
     A, Bd = _dense(aq, as_, bq, bs)
@@ -68,14 +72,16 @@ def test_mx_grouped_gemm_plain(counts, N, K, unit):
             check_close(got[lo:hi], A[lo:hi] @ Bd[e].T, (2e-2, 5e-3), f"expert {e}")
 
 
-@pytest.mark.parametrize("counts,N,K", [([0, 1, 130, 300], 256, 384), ([256, 7], 512, 256)])
-def test_mx_grouped_gemm_swiglu_quantised_out(counts, N, K):
+@pytest.mark.parametrize("counts,N,K,hint", [([0, 1, 130, 300], 256, 384, 0), ([256, 7], 512, 256, 0),
+                                             ([3, 0, 16, 9], 256, 384, 16), ([40, 1], 384, 256, 64)])
+def test_mx_grouped_gemm_swiglu_quantised_out(counts, N, K, hint):
     E, offsets, M, aq, as_, bq, bs = _problem(counts, 2 * N, K, 93)
     C = torch.empty(M, N, dtype=torch.uint8, device="cuda")
     cs = torch.empty(M, N // 128, dtype=torch.float32, device="cuda")
     ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     moe.moe_grouped_gemm(dev_u8(aq), dev_u8(bq), dev(offsets), M, E, N, K, DT,
-                         moe.MOE_EPILOGUE_SWIGLU, C, dev(as_), dev(bs), cs, ws=ws)
+                         moe.MOE_EPILOGUE_SWIGLU, C, dev(as_), dev(bs), cs, max_rows_per_expert=hint,
+                         ws=ws)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(ws) == 0
     dec = _dec_table()
