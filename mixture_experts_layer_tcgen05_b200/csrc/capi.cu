@@ -518,14 +518,19 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
     if ((e = permute_gather(x, H * 2, x_perm, nullptr, 0, nullptr)) != cudaSuccess)
       return cuda_fail(e, "permute");
     record(s, 2);
+    // GEMM scratch: the split-K partials of the small-M kernels (decode), or
+    // the K-split last wave of the plain tokens-in-M GEMM-2, in a region the
+    // GEMM does not touch (x_perm, read by GEMM-1 only)
     void* splitk = L.splitk >= 0 ? at<void>(ws, L.splitk) : nullptr;
     const size_t splitk_bytes = L.splitk >= 0 ? (size_t)(L.y_perm - L.splitk) : 0;
+    const size_t rows_bytes = (size_t)R * H * 2;
     if ((e = launch_grouped_gemm_bf16(x_perm, nullptr, R, w13, offsets, R, E, I, H, act, h, T,
                                       status, splitk, splitk_bytes, s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "GEMM1: %s %s", cudaGetErrorString(e), why);
     record(s, 3);
     if ((e = launch_grouped_gemm_bf16(h, nullptr, R, w2, offsets, R, E, H, I, 0, y_perm, T,
-                                      status, splitk, splitk_bytes, s, &why)) != cudaSuccess)
+                                      status, splitk ? splitk : x_perm, splitk ? splitk_bytes : rows_bytes,
+                                      s, &why)) != cudaSuccess)
       return fail(MOE_ERR_CUDA, "GEMM2: %s %s", cudaGetErrorString(e), why);
     record(s, 4);
   } else {

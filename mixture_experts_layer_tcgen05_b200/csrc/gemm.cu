@@ -93,15 +93,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = tile_start[args.E];
   const int nkb = args.K / BK;
-  // Plain GEMM, BN = 256: when the tiles leave a last wave at most half full,
-  // each of its tiles runs as two BN = 128 units (the column halves), so that
-  // wave ends in about half the time. units >= nfull are those halves.
-  constexpr bool kCanSplit = !SWIGLU && BN == 256 && !GATHER;
+  // Plain GEMM: when the tiles leave a last wave at most half full, each of
+  // its tiles runs as two units over the two halves of K, so that wave ends in
+  // about half the time. Units >= nfull are those halves; each leaves its fp32
+  // accumulator in args.tail_part ([unit - nfull][128 rows][BN columns]) and
+  // tail_reduce_kernel adds the two halves (measured: prefill GEMM-2 777 ->
+  // 753 us; the gated GEMM-1 lost more in its epilogue than it gained).
   const int G = (int)gridDim.x;
   const int nfull = (total / G) * G, ntail = total - nfull;
-  const bool split = kCanSplit && args.tail_split && ntail > 0 && 2 * ntail <= G;
+  const bool split = !SWIGLU && !GATHER && args.tail_part && ntail > 0 && 2 * ntail <= G;
   const int units = split ? nfull + 2 * ntail : total;
-  // unit -> tile and column half (0: all BN columns, 1 / 2: first / second 128)
+  // unit -> tile and K half (0: all of K, 1 / 2: first / second half)
   auto unit_tile = [&](int u, int& half) {
     if (split && u >= nfull) {
       half = 1 + ((u - nfull) & 1);
@@ -109,6 +111,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     half = 0;
     return u;
+  };
+  auto k_range = [&](int half, int& kb0, int& kb1) {
+    kb0 = half == 2 ? nkb / 2 : 0;
+    kb1 = half == 1 ? nkb / 2 : nkb;
   };
 
   auto decode = [&](int tile, int& e, int& m, int& n) {
@@ -179,11 +185,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           rb0 = e * args.b_rows + n * 128;
           rb1 = rb0 + args.up_off;
         } else {
-          rb0 = e * args.b_rows + n * BN + (half == 2 ? 128 : 0);
+          rb0 = e * args.b_rows + n * BN;
           rb1 = rb0 + 128;
         }
-        const bool two_b = BN == 256 && half == 0;  // a column half needs one 128-row B box
-        for (int kb = 0; kb < nkb; ++kb, ++issued) {
+        constexpr bool two_b = BN == 256;
+        int kb0, kb1;
+        k_range(half, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++issued) {
           const int s = (int)(issued % STAGES);
           const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
           if (!ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty)) {
@@ -206,13 +214,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_ph = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        int half;
+        int half, kb0, kb1;
         unit_tile(u, half);
-        const uint32_t idesc = half ? ptx::make_idesc(BM, 128, 1, 1) : C::kIdesc;
+        k_range(half, kb0, kb1);
         if (!ptx::mbar_wait(acce0 + acc * 8, acc_ph ^ 1, args.status, kSiteMmaAccEmpty)) break;
         ptx::tc_fence_after();
         const uint32_t d = tmem_base + acc * C::kAccCols;
-        for (int kb = 0; kb < nkb; ++kb, ++consumed) {
+        for (int kb = kb0; kb < kb1; ++kb, ++consumed) {
           const int s = (int)(consumed % STAGES);
           const uint32_t ph = (uint32_t)((consumed / STAGES) & 1);
           if (!ptx::mbar_wait(full0 + s * 8, ph, args.status, kSiteMmaFull)) {
@@ -225,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk)
             ptx::mma_f16(d, da + (uint64_t)(kk * UK * 2 / 16), db + (uint64_t)(kk * UK * 2 / 16),
-                         idesc, (kb | kk) != 0);
+                         C::kIdesc, kb != kb0 || kk != 0);
           ptx::mma_commit(empty0 + s * 8);
         }
         if (!ok) break;
@@ -252,7 +260,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ptx::mbar_wait(accf0 + acc * 8, acc_ph, args.status, kSiteEpiAccFull)) break;
       ptx::tc_fence_after();
       const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
-      if (SWIGLU) {
+      if (half) {  // one K half of a last-wave tile: the raw fp32 accumulator row
+        float4* dst = reinterpret_cast<float4*>(args.tail_part + ((int64_t)(u - nfull) * BM + q * 32 + lane) * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld32(t0 + c, v);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[c / 4 + i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      } else if (SWIGLU) {
         __nv_bfloat16* dst = args.C + (int64_t)row * args.ldc + n * 128;
 #pragma unroll 1
         for (int c = 0; c < 128; c += 32) {
@@ -266,10 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (valid) store_row32(dst + c, h);
         }
       } else {
-        __nv_bfloat16* dst = args.C + (int64_t)row * args.ldc + n * BN + (half == 2 ? 128 : 0);
-        const int ncols = half ? 128 : BN;
+        __nv_bfloat16* dst = args.C + (int64_t)row * args.ldc + n * BN;
 #pragma unroll 1
-        for (int c = 0; c < ncols; c += 32) {
+        for (int c = 0; c < BN; c += 32) {
           uint32_t v[32];
           ptx::tmem_ld32(t0 + c, v);
           ptx::tmem_wait_ld();
@@ -291,6 +310,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, 512);
+  }
+}
+
+
+// Finishes the K-split last wave of the plain gemm_rows_kernel: block (i, y)
+// takes rows [16 y, 16 y + 16) of tail tile nfull + i (the same tile order,
+// recomputed from the offsets with the GEMM's grid size G), adds its two K
+// halves (first + second, fp32) and writes them as bf16.
+template <int BN>
+__global__ void __launch_bounds__(256) tail_reduce_kernel(Args args, int G) {
+  __shared__ int32_t tile_start[kMaxE + 1];
+  __shared__ int32_t soff[kMaxE + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) build_tile_starts<BM>(args.offsets, args.E, args.NT, tile_start, soff);
+  __syncthreads();
+  const int total = tile_start[args.E];
+  const int nfull = (total / G) * G, ntail = total - nfull;
+  if (!(ntail > 0 && 2 * ntail <= G) || (int)blockIdx.x >= ntail) return;
+  const int tile = nfull + (int)blockIdx.x;
+  const int e = find_expert(tile_start, args.E, tile);
+  const int local = tile - tile_start[e];
+  const int mt = (soff[e + 1] - soff[e] + BM - 1) / BM;
+  const int bsz = args.band * args.NT;
+  const int b = local / bsz;
+  const int rows = min(args.band, mt - b * args.band);
+  const int l2 = local - b * bsz;
+  const int n = l2 / rows, m = b * args.band + l2 % rows;
+  const float* p0 = args.tail_part + (int64_t)(2 * blockIdx.x) * BM * BN;
+  const float* p1 = p0 + (int64_t)BM * BN;
+  for (int r = (int)blockIdx.y * 16 + warp; r < (int)blockIdx.y * 16 + 16; r += 8) {
+    const int row = soff[e] + m * BM + r;
+    if (row >= soff[e + 1] || row >= args.M_total) break;
+    const float* a0 = p0 + (int64_t)r * BN;
+    const float* a1 = p1 + (int64_t)r * BN;
+    for (int c = 4 * lane; c < BN; c += 128) {
+      const float4 v0 = *reinterpret_cast<const float4*>(a0 + c);
+      const float4 v1 = *reinterpret_cast<const float4*>(a1 + c);
+      *reinterpret_cast<uint2*>(args.C + (int64_t)row * args.ldc + n * BN + c) =
+          make_uint2(pack_bf16x2(__fadd_rn(v0.x, v1.x), __fadd_rn(v0.y, v1.y)),
+                     pack_bf16x2(__fadd_rn(v0.z, v1.z), __fadd_rn(v0.w, v1.w)));
+    }
   }
 }
 
@@ -539,7 +599,7 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A
   a.a_src = A;
   a.a_src_rows = A_src_rows;
   a.ksplit = 1;
-  a.tail_split = 1;
+  a.tail_part = nullptr;
   a.partial = nullptr;
   const int64_t a_tmap_rows = A_rows ? A_src_rows : M_total;
   a.status = status;
@@ -623,6 +683,11 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A
   a.band = 8;
   const int64_t tiles_ub = ((int64_t)M_total / gg::BM + (M_total < E ? M_total : E)) * a.NT;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_ub));
+  // plain GEMM: scratch for a K-split last wave, at most `grid` half-tile
+  // partials of 128 x BN fp32
+  const size_t tail_bytes = (size_t)grid * gg::BM * BN * sizeof(float);
+  if (!swiglu && !A_rows && scratch && scratch_bytes >= tail_bytes)
+    a.tail_part = static_cast<float*>(scratch);
 #define MOE_ROWS(SW, BNV)                                                                \
   do {                                                                                   \
     auto k = a.a_rows ? gg::gemm_rows_kernel<SW, BNV, true> : gg::gemm_rows_kernel<SW, BNV, false>; \
@@ -642,6 +707,12 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A
     MOE_ROWS(kActNone, 128);
 #undef MOE_ROWS
   note_launch();
+  if (a.tail_part) {  // finishes the last wave's tiles if the kernel split them
+    const dim3 rgrid(grid, gg::BM / 16);
+    if (BN == 256) gg::tail_reduce_kernel<256><<<rgrid, 256, 0, s>>>(a, (int)grid);
+    else gg::tail_reduce_kernel<128><<<rgrid, 256, 0, s>>>(a, (int)grid);
+    note_launch();
+  }
   return cudaGetLastError();
 }
 

@@ -33,7 +33,7 @@ struct Args {
   const int32_t* a_rows;  // gather: source row of each routed row (nullptr: A is dense)
   const void* a_src;      // gather: source matrix [a_src_rows, K]
   int a_src_rows;
-  int tail_split;    // rows kernel, plain BN = 256: the last partial wave runs as BN = 128 halves
+  float* tail_part;  // rows kernel: fp32 partial sums of a K-split last wave, or nullptr
   int ksplit;        // small-M kernel: K split into ksplit ranges, fp32 partials
   float* partial;    // [ksplit, M_total, pld] with pld = (SwiGLU ? 2 : 1) * ldc
   __nv_bfloat16* C;

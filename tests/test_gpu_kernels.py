@@ -203,23 +203,29 @@ def test_grouped_gemm_plain(counts, N, K, hint):
             check_close(got[lo:hi], ref, BF16_TOL, f"expert {e}")
 
 
-@pytest.mark.parametrize("N", [256, 512])
-def test_grouped_gemm_plain_last_wave_halves(N):
+@pytest.mark.parametrize("swiglu", [False, True])
+@pytest.mark.parametrize("N,K", [(256, 128), (512, 384)])
+def test_grouped_gemm_last_wave_split_over_k(N, K, swiglu):
     """Enough 128 x 256 tiles that the last wave of the 148-CTA grid is at most
-    half full: those tiles run as two 128-column halves."""
+    half full: for the plain GEMM those tiles run as two units over the halves
+    of K, whose fp32 partials a second kernel adds -- given scratch for them;
+    the gated GEMM keeps whole tiles with the same scratch."""
     counts = [20000, 300, 0, 180]
-    E, offsets, M, A, B = _grouped_problem(counts, N, 128, 81)
+    E, offsets, M, A, B = _grouped_problem(counts, 2 * N if swiglu else N, K, 81)
     C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
-    moe.moe_grouped_gemm(dev_bf16(A), dev_bf16(B), dev(offsets), M, E, N, 128, moe.MOE_DTYPE_BF16,
-                         moe.MOE_EPILOGUE_NONE, C, ws=ws)
+    ws = torch.zeros(32 << 20, dtype=torch.uint8, device="cuda")
+    ep = moe.MOE_EPILOGUE_SWIGLU if swiglu else moe.MOE_EPILOGUE_NONE
+    moe.moe_grouped_gemm(dev_bf16(A), dev_bf16(B), dev(offsets), M, E, N, K, moe.MOE_DTYPE_BF16,
+                         ep, C, ws=ws)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(ws) == 0
     got = mi.bf16_to_f32(host_bf16(C))
     for e in range(E):
         lo, hi = offsets[e], offsets[e + 1]
         if hi > lo:
-            check_close(got[lo:hi], oracle.expert_down_rows(A[lo:hi], B[e]), BF16_TOL, f"expert {e}")
+            ref = (oracle.expert_swiglu_rows(A[lo:hi], B[e]) if swiglu
+                   else oracle.expert_down_rows(A[lo:hi], B[e]))
+            check_close(got[lo:hi], ref, BF16_TOL, f"expert {e}")
 
 
 def test_combine_exact_given_y():
