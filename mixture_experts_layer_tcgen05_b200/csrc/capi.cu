@@ -26,6 +26,8 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* off
                            cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, int T,
                                int row_bytes, void* x_perm, int32_t* status, cudaStream_t s);
+cudaError_t launch_scatter_rows(const void* x, const int32_t* inv_perm, int T, int k,
+                                int row_bytes, void* x_perm, int32_t* status, cudaStream_t s);
 cudaError_t launch_permute_gather_small(const int32_t* ids, int T, int E, int k, int32_t* offsets,
                                         int32_t* perm_token, int32_t* inv_perm, const void* x,
                                         int row_bytes, void* x_perm, const void* x2,
@@ -59,6 +61,9 @@ cudaError_t launch_quant_weight_fp4(const void* w, int64_t nb, int64_t rows, int
                                     uint8_t* sc, cudaStream_t s);
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
                              const int32_t* row_map, bool ue8m0, cudaStream_t s);
+cudaError_t launch_quant_act_scatter(const void* x, int64_t rows, int64_t cols,
+                                     const int32_t* inv_perm, int k, void* q_perm, float* sc_perm,
+                                     bool ue8m0, int32_t* status, cudaStream_t s);
 cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                 float* sc, bool ue8m0, cudaStream_t s);
 
@@ -308,9 +313,8 @@ moe_status_t moe_permute(const int32_t* ids, moe_dims_t d, int32_t* offsets, int
                      at<char>(ws, L.scratch), at<int32_t>(ws, L.status), s);
   if (e != cudaSuccess) return cuda_fail(e, "permute");
   if (x) {
-    e = launch_gather_rows(x, perm_token, d.T * d.k, d.T, d.H * 2, x_perm,
-                           at<int32_t>(ws, L.status), s);
-    if (e != cudaSuccess) return cuda_fail(e, "gather");
+    e = launch_scatter_rows(x, inv_perm, d.T, d.k, d.H * 2, x_perm, at<int32_t>(ws, L.status), s);
+    if (e != cudaSuccess) return cuda_fail(e, "row scatter");
   }
   return ok();
 }
@@ -498,25 +502,21 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
   // The permuted copy of x feeds GEMM1's TMA tile loads (a gather inside the
   // GEMM costs the tensor cores more than this copy costs). Decode-sized
   // batches permute and gather in one launch; larger ones use the chunked
-  // permutation, then the gather.
-  auto permute_gather = [&](const void* a, int a_bytes, void* a_perm, const void* b, int b_bytes,
-                            void* b_perm) -> cudaError_t {
-    cudaError_t r = launch_permute_gather_small(ids, T, E, k, offsets, perm_token, inv_perm, a,
-                                                a_bytes, a_perm, b, b_bytes, b_perm, status, s);
-    if (r != cudaErrorNotSupported) return r;
-    if ((r = launch_permute(ids, T, E, k, offsets, perm_token, inv_perm, at<char>(ws, L.scratch),
-                            status, s)) != cudaSuccess)
-      return r;
-    if ((r = launch_gather_rows(a, perm_token, R, T, a_bytes, a_perm, status, s)) != cudaSuccess)
-      return r;
-    if (b) r = launch_gather_rows(b, perm_token, R, T, b_bytes, b_perm, status, s);
-    return r;
+  // permutation, then write each token's row to its k positions.
+  const bool small = R <= kSmallPermRows && E <= 1024;
+  auto permute_large = [&]() {
+    return launch_permute(ids, T, E, k, offsets, perm_token, inv_perm, at<char>(ws, L.scratch),
+                          status, s);
   };
   if (dt == MOE_DTYPE_BF16) {
     void* x_perm = at<void>(ws, L.x_perm);
     void* h = at<void>(ws, L.h);
-    if ((e = permute_gather(x, H * 2, x_perm, nullptr, 0, nullptr)) != cudaSuccess)
-      return cuda_fail(e, "permute");
+    if (small)
+      e = launch_permute_gather_small(ids, T, E, k, offsets, perm_token, inv_perm, x, H * 2, x_perm,
+                                      nullptr, 0, nullptr, status, s);
+    else if ((e = permute_large()) == cudaSuccess)
+      e = launch_scatter_rows(x, inv_perm, T, k, H * 2, x_perm, status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "permute");
     record(s, 2);
     // GEMM scratch: the split-K partials of the small-M kernels (decode), or
     // the K-split last wave of the plain tokens-in-M GEMM-2, in a region the
@@ -540,13 +540,24 @@ static moe_status_t forward_impl(const void* x, const void* wr, const float* bia
     float* xs_perm = at<float>(ws, L.xs_perm);
     void* hq = at<void>(ws, L.hq);
     float* hs = at<float>(ws, L.hs);
-    // x is quantised once per token, then its codes and scales are permuted
+    // x is quantised once per token. Decode-sized batches quantise into xq /
+    // xs, then permute and gather codes and scales in one launch; larger ones
+    // permute first and quantise each token straight into its k permuted rows.
     const bool fp4 = dt == MOE_DTYPE_FP4_E2M1;  // w13s / w2s hold e8m0 bytes then
     const bool ue8m0 = dt == MOE_DTYPE_FP8_E4M3_UE8M0 || fp4;
-    if ((e = launch_quant_act(x, T, H, xq, xs, nullptr, ue8m0, s)) != cudaSuccess)
-      return cuda_fail(e, "activation quantisation");
-    if ((e = permute_gather(xq, H, xq_perm, xs, (H / 128) * 4, xs_perm)) != cudaSuccess)
-      return cuda_fail(e, "permute");
+    if (small) {
+      if ((e = launch_quant_act(x, T, H, xq, xs, nullptr, ue8m0, s)) != cudaSuccess)
+        return cuda_fail(e, "activation quantisation");
+      if ((e = launch_permute_gather_small(ids, T, E, k, offsets, perm_token, inv_perm, xq, H,
+                                           xq_perm, xs, (H / 128) * 4, xs_perm, status, s)) !=
+          cudaSuccess)
+        return cuda_fail(e, "permute");
+    } else {
+      if ((e = permute_large()) != cudaSuccess) return cuda_fail(e, "permute");
+      if ((e = launch_quant_act_scatter(x, T, H, inv_perm, k, xq_perm, xs_perm, ue8m0, status, s)) !=
+          cudaSuccess)
+        return cuda_fail(e, "activation quantisation");
+    }
     record(s, 2);
     if (ue8m0) {
       // power-of-two scales: the block-scaled tensor-core path, no promotion

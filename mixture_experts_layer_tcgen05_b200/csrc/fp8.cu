@@ -32,37 +32,69 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return lo | (hi << 16);
 }
 
-// One warp per output row; each step covers two 128-column groups (lanes
-// 0-15 and 16-31, eight values each). Output row p reads input row
-// row_map[p] (the expert permutation) or p when row_map is NULL.
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint4* __restrict__ x, int64_t rows,
-                                                        int64_t cols,
-                                                        const int32_t* __restrict__ row_map,
-                                                        uint2* __restrict__ q,
-                                                        float* __restrict__ s, bool ue8m0) {
+// One warp per row; each step covers two 128-column groups (lanes 0-15 and
+// 16-31, eight values each). Gather form (SCATTER false): output row p reads
+// input row row_map[p] (the expert permutation) or p when row_map is NULL.
+// Scatter form: input row p is read once and its codes and scales are
+// written to output rows row_map[p*k + j], j < k (the inverse permutation),
+// so the permuted operand is produced without an unpermuted copy; rows
+// outside [0, rows*k) set the status flag and the warp writes nothing.
+constexpr int kQuantScatterMaxK = 16;  // lanes that hold the k output rows
+
+template <bool SCATTER>
+__global__ void __launch_bounds__(256, SCATTER ? 4 : 1) quant_act_kernel(
+    const uint4* __restrict__ x, int64_t rows, int64_t cols, const int32_t* __restrict__ row_map,
+    int k, uint2* __restrict__ q, float* __restrict__ s, bool ue8m0, int32_t* status) {
   const int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (p >= rows) return;
-  const int64_t src = row_map ? row_map[p] : p;
+  if (p >= rows) return;  // warp-uniform
   const int64_t vpr = cols / 8, groups = cols / 128;
+  int64_t src = p;
+  int mine = (int)p;  // scatter: lane j < k holds output row j of this input row
+  if constexpr (SCATTER) {
+    mine = lane < k ? row_map[p * k + lane] : 0;
+    if (__any_sync(0xffffffffu, (unsigned)mine >= (unsigned)(rows * k))) {
+      if (lane == 0) record_bad_index(status);
+      return;
+    }
+  } else {
+    src = row_map ? row_map[p] : p;
+  }
   const uint4* xr = x + src * vpr;
-  uint2* qr = q + p * vpr;
-  for (int64_t v0 = 0; v0 < vpr; v0 += 32) {
-    const int64_t v = v0 + lane;
-    const bool on = v < vpr;  // a trailing single group leaves lanes 16-31 idle
-    const uint4 u = on ? xr[v] : make_uint4(0, 0, 0, 0);
-    const float f[8] = {bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y),
-                        bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w)};
-    float amax = 0.0f;
+  // four 256-column steps per pass: their loads are issued before any is used
+  for (int64_t b0 = 0; b0 < vpr; b0 += 4 * 32) {
+    uint4 ub[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    for (int i = 0; i < 4; ++i) {
+      const int64_t v = b0 + i * 32 + lane;
+      ub[i] = v < vpr ? xr[v] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll 1
+    for (int i = 0; i < 4; ++i) {
+      const int64_t v0 = b0 + i * 32;
+      if (v0 >= vpr) break;  // warp-uniform
+      const int64_t v = v0 + lane;
+      const bool on = v < vpr;  // a trailing single group leaves lanes 16-31 idle
+      const uint4 u = ub[0];
+      ub[0] = ub[1], ub[1] = ub[2], ub[2] = ub[3];  // constant indices: stays in registers
+      const float f[8] = {bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y),
+                          bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w)};
+      float amax = 0.0f;
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const float sc = group_scale(amax, ue8m0);
-    if (on) {
-      qr[v] = make_uint2(e4m3x4(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc), __fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc)),
-                         e4m3x4(__fdiv_rn(f[4], sc), __fdiv_rn(f[5], sc), __fdiv_rn(f[6], sc), __fdiv_rn(f[7], sc)));
-      if ((lane & 15) == 0) s[p * groups + v / 16] = sc;
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const float sc = group_scale(amax, ue8m0);
+      const uint2 code =
+          make_uint2(e4m3x4(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc), __fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc)),
+                     e4m3x4(__fdiv_rn(f[4], sc), __fdiv_rn(f[5], sc), __fdiv_rn(f[6], sc), __fdiv_rn(f[7], sc)));
+      for (int j = 0; j < (SCATTER ? k : 1); ++j) {  // warp-uniform trip count
+        const int64_t d = SCATTER ? __shfl_sync(0xffffffffu, mine, j) : mine;
+        if (on) {
+          q[d * vpr + v] = code;
+          if ((lane & 15) == 0) s[d * groups + v / 16] = sc;
+        }
+      }
     }
   }
 }
@@ -111,8 +143,22 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const __nv_bfloat16* 
 
 cudaError_t launch_quant_act(const void* x, int64_t rows, int64_t cols, void* q, float* sc,
                              const int32_t* row_map, bool ue8m0, cudaStream_t s) {
-  quant_act_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, s>>>(
-      static_cast<const uint4*>(x), rows, cols, row_map, static_cast<uint2*>(q), sc, ue8m0);
+  quant_act_kernel<false><<<(unsigned)ceil_div(rows, 8), 256, 0, s>>>(
+      static_cast<const uint4*>(x), rows, cols, row_map, 1, static_cast<uint2*>(q), sc, ue8m0,
+      nullptr);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// x [rows, cols] quantised per row and 128-column group, each row's codes and
+// scales written to the k permuted rows inv_perm[row*k + j].
+cudaError_t launch_quant_act_scatter(const void* x, int64_t rows, int64_t cols,
+                                     const int32_t* inv_perm, int k, void* q_perm, float* sc_perm,
+                                     bool ue8m0, int32_t* status, cudaStream_t s) {
+  if (k < 1 || k > kQuantScatterMaxK) return cudaErrorNotSupported;
+  quant_act_kernel<true><<<(unsigned)ceil_div(rows, 8), 256, 0, s>>>(
+      static_cast<const uint4*>(x), rows, cols, inv_perm, k, static_cast<uint2*>(q_perm), sc_perm,
+      ue8m0, status);
   note_launch();
   return cudaGetLastError();
 }

@@ -16,8 +16,8 @@ namespace moe {
 cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets,
                            int32_t* perm_token, int32_t* inv_perm, void* scratch, int32_t* status,
                            cudaStream_t s);
-cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, int T,
-                               int row_bytes, void* x_perm, int32_t* status, cudaStream_t s);
+cudaError_t launch_scatter_rows(const void* x, const int32_t* inv_perm, int T, int k,
+                                int row_bytes, void* x_perm, int32_t* status, cudaStream_t s);
 
 // The largest scratch the fixed array provides (see MOE_NOALLOC_SCRATCH_BYTES).
 constexpr int64_t kNoAllocScratch = MOE_NOALLOC_SCRATCH_BYTES;
@@ -61,7 +61,7 @@ cudaError_t launch_permute_noalloc(const int32_t* ids, int T, int H, int E, int 
   // Every scratch word the permutation reads is written earlier in the same
   // call (chunk masks, chunk bases, counts), so the array needs no clearing.
   e = launch_permute(ids, T, E, k, offsets, perm_token, inv_perm, scratch, nullptr, s);
-  if (e == cudaSuccess && x) e = launch_gather_rows(x, perm_token, T * k, T, H * 2, x_perm, nullptr, s);
+  if (e == cudaSuccess && x) e = launch_scatter_rows(x, inv_perm, T, k, H * 2, x_perm, nullptr, s);
   return e;
 }
 

@@ -145,6 +145,49 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const V* __restrict__ 
   for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
 }
 
+// ---- token-major row scatter: x_perm[inv_perm[t, j], :] = x[t, :] -----------
+// The same bytes as the gather, visited from the source side: one warp per
+// token reads its row once and writes it to the row's k positions, so x
+// crosses HBM once however many experts the token chose (the gather reads a
+// row k times, from HBM again once the output stream has evicted it from L2).
+// Four vectors per lane are loaded before their stores, for more loads in
+// flight. k <= 16 (the largest k the entry points accept); destinations
+// outside [0, T*k) set the status flag and the warp writes nothing.
+constexpr int kScatterMaxK = 16;
+
+template <typename V>
+__global__ void __launch_bounds__(256) scatter_rows_kernel(const V* __restrict__ x,
+                                                           const int32_t* __restrict__ inv_perm,
+                                                           int T, int k, int vec_per_row,
+                                                           V* __restrict__ x_perm, int32_t* status) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= T) return;  // warp-uniform
+  const int R = T * k;
+  const int mine = lane < k ? inv_perm[(int64_t)t * k + lane] : 0;
+  if (__any_sync(0xffffffffu, (unsigned)mine >= (unsigned)R)) {
+    if (lane == 0) record_bad_index(status);
+    return;
+  }
+  V* dst[kScatterMaxK];
+#pragma unroll
+  for (int j = 0; j < kScatterMaxK; ++j)
+    dst[j] = x_perm + (int64_t)__shfl_sync(0xffffffffu, mine, j) * vec_per_row;
+  const V* src = x + (int64_t)t * vec_per_row;
+  for (int v0 = lane; v0 < vec_per_row; v0 += 4 * 32) {
+    V u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (v0 + i * 32 < vec_per_row) u[i] = src[v0 + i * 32];
+#pragma unroll
+    for (int j = 0; j < kScatterMaxK; ++j) {
+      if (j >= k) break;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (v0 + i * 32 < vec_per_row) dst[j][v0 + i * 32] = u[i];
+    }
+  }
+}
+
 // ---- small batches: permutation and row gather in one launch ---------------
 // For R = T*k <= 1024 routed rows (decode-sized batches) the three launches of
 // the chunked permutation plus the gather cost more than the work. Here block
@@ -154,7 +197,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const V* __restrict__ 
 // among the earlier pairs of the same expert (the pairs are in token order, so
 // that rank is the token-ascending position) and copies its token's row(s)
 // to the permuted position. The result equals the chunked permutation's.
-constexpr int kSmallPermMaxR = 1024;
+constexpr int kSmallPermMaxR = kSmallPermRows;
 constexpr int kSmallPermThreads = 128;
 
 __global__ void __launch_bounds__(kSmallPermThreads) permute_gather_small_kernel(
@@ -340,6 +383,21 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, 
   else
     gather_rows_kernel<uint32_t><<<(unsigned)ceil_div(R, 8), 256, 0, s>>>(
         static_cast<const uint32_t*>(x), perm_token, R, T, row_bytes / 4,
+        static_cast<uint32_t*>(x_perm), status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_rows(const void* x, const int32_t* inv_perm, int T, int k,
+                                int row_bytes, void* x_perm, int32_t* status, cudaStream_t s) {
+  if (k > kScatterMaxK) return cudaErrorNotSupported;
+  if (row_bytes % 16 == 0)
+    scatter_rows_kernel<uint4><<<(unsigned)ceil_div(T, 8), 256, 0, s>>>(
+        static_cast<const uint4*>(x), inv_perm, T, k, row_bytes / 16, static_cast<uint4*>(x_perm),
+        status);
+  else
+    scatter_rows_kernel<uint32_t><<<(unsigned)ceil_div(T, 8), 256, 0, s>>>(
+        static_cast<const uint32_t*>(x), inv_perm, T, k, row_bytes / 4,
         static_cast<uint32_t*>(x_perm), status);
   note_launch();
   return cudaGetLastError();

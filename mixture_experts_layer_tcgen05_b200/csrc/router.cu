@@ -55,9 +55,10 @@ constexpr int kWideKC = 32;
 // SPLIT: grid.z runs the 8 h blocks as separate CTAs, each writing its
 // block sums to part[b][t][e] (the running total and the bias are then
 // applied by topk_kernel<PER, true>, in the same order); for many more CTAs
-// than the 64-token tiles give and without the running-total registers.
+// than the 64-token tiles give and without the running-total registers;
+// two CTAs per SM (128 registers) for more warps to hide the FMA latency.
 template <bool VEC, bool SPLIT>
-__global__ void __launch_bounds__(256, 1) router_wide_kernel(
+__global__ void __launch_bounds__(256, SPLIT ? 2 : 1) router_wide_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
     const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
     float* __restrict__ part) {

@@ -158,6 +158,8 @@ def check_fp8_layer(cfg, L):
 
 
 @pytest.mark.parametrize("kw", [dict(T=200, H=512, I=256, E=16, k=4, subset=0),
+                                # T*k > 1024: permuted first, each token quantised into its k rows
+                                dict(T=300, H=512, I=256, E=16, k=4, subset=0),
                                 dict(T=33, H=256, I=384, E=8, k=2, subset=0),
                                 dict(T=16, H=1024, I=2048, E=8, k=2, bias="zero", subset=0)])
 def test_fp8_layer_small(kw):

@@ -126,10 +126,11 @@ def _ids_cases():
     return cases
 
 
-@pytest.mark.parametrize("case", range(10))
-def test_permute_bit_exact(case):
+@pytest.mark.parametrize("case,H", [(c, 128) for c in range(10)] +
+                         # rows of several 4-vector steps per lane, the last one partial
+                         [(3, 1152), (5, 7168), (6, 3200)])
+def test_permute_bit_exact(case, H):
     T, E, k, ids = _ids_cases()[case]
-    H = 128
     d = (T, H, 128, E, k)
     ws = torch.zeros(moe.moe_workspace_size(d), dtype=torch.uint8, device="cuda")
     off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
