@@ -122,7 +122,9 @@ size_t moe_workspace_size(moe_dims_t d, moe_dtype_t dt);
  *   perm_token int32 [T*k]               token of permuted row p
  *   inv_perm  int32 [T, k]               permuted row of (token t, slot j)
  *   x_perm    bf16 [T*k, H]  (BF16)      permuted token rows
- *   xq        e4m3 [T, H], xs fp32 [T, H/128]            (FP8: x quantised per token)
+ *   xq        e4m3 [T, H], xs fp32 [T, H/128]            (FP8: x quantised per token;
+ *                                                       written only when T*k <= 1024, larger
+ *                                                       batches quantise into xq_perm directly)
  *   xq_perm   e4m3 [T*k, H], xs_perm fp32 [T*k, H/128]   (FP8: their permuted rows)
  *   h         bf16 [T*k, I]  (BF16)      SwiGLU output per permuted row
  *   hq        e4m3 [T*k, I], hs fp32 [T*k, I/128]        (FP8)

@@ -11,6 +11,7 @@
 #include <string>
 
 #include "common.cuh"
+#include "permute.cuh"
 
 namespace moe {
 

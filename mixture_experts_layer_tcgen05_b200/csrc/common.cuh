@@ -29,10 +29,6 @@ __device__ __forceinline__ void record_timeout(int32_t* status, int site) {
   atomicCAS(status, 0, (MOE_ERR_TIMEOUT << 8) | site);
 }
 
-// Routed rows (T*k) up to which the permutation and the row gather run as one
-// launch (permute_gather_small_kernel); larger batches take the chunked path.
-constexpr int kSmallPermRows = 1024;
-
 __device__ __forceinline__ void record_bad_index(int32_t* status) {
   if (status) atomicCAS(status, 0, (MOE_ERR_INVALID_ARG << 8) | kSiteBadIndex);
 }

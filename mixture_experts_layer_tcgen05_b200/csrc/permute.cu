@@ -14,6 +14,7 @@
 //      (token t, slot j) with expert e is
 //        offsets[e] + chunk_base[chunk(t)][e] + popc(mask[chunk(t)][e] & lanes below t).
 #include "common.cuh"
+#include "permute.cuh"
 
 namespace moe {
 
@@ -288,6 +289,8 @@ __global__ void __launch_bounds__(kSmallPermThreads) permute_gather_small_kernel
 // `y = sum_i weights_i * expert_i(x)`:
 //   out[t, c] = sum_{j ascending} w[t, j] * y_perm[inv_perm[t, j], c]  (fp32) -> bf16
 // Each thread owns 8 consecutive columns (one 16-byte vector) of one token.
+// The routed rows are read four at a time, all four loads issued before the
+// first is used; the sums still run in ascending j.
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const float* __restrict__ w,
                                                       const int32_t* __restrict__ inv_perm, int T,
@@ -299,22 +302,37 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   float acc[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    const float wj = __ldg(w + (int64_t)t * k + j);
-    const int p = __ldg(inv_perm + (int64_t)t * k + j);
-    if ((unsigned)p >= (unsigned)(T * k)) {
-      record_bad_index(status);
-      continue;
+  for (int j0 = 0; j0 < k; j0 += 4) {
+    uint4 y[4];
+    float wj[4];
+    bool use[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u;
+      use[u] = false;
+      if (j < k) {
+        wj[u] = __ldg(w + (int64_t)t * k + j);
+        const int p = __ldg(inv_perm + (int64_t)t * k + j);
+        if ((unsigned)p >= (unsigned)(T * k)) {
+          record_bad_index(status);
+        } else {
+          y[u] = __ldg(y_perm + (int64_t)p * vec_per_row + v);
+          use[u] = true;
+        }
+      }
     }
-    uint4 y = __ldg(y_perm + (int64_t)p * vec_per_row + v);
-    acc[0] = __fmaf_rn(wj, bf16lo_to_f32(y.x), acc[0]);
-    acc[1] = __fmaf_rn(wj, bf16hi_to_f32(y.x), acc[1]);
-    acc[2] = __fmaf_rn(wj, bf16lo_to_f32(y.y), acc[2]);
-    acc[3] = __fmaf_rn(wj, bf16hi_to_f32(y.y), acc[3]);
-    acc[4] = __fmaf_rn(wj, bf16lo_to_f32(y.z), acc[4]);
-    acc[5] = __fmaf_rn(wj, bf16hi_to_f32(y.z), acc[5]);
-    acc[6] = __fmaf_rn(wj, bf16lo_to_f32(y.w), acc[6]);
-    acc[7] = __fmaf_rn(wj, bf16hi_to_f32(y.w), acc[7]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!use[u]) continue;
+      acc[0] = __fmaf_rn(wj[u], bf16lo_to_f32(y[u].x), acc[0]);
+      acc[1] = __fmaf_rn(wj[u], bf16hi_to_f32(y[u].x), acc[1]);
+      acc[2] = __fmaf_rn(wj[u], bf16lo_to_f32(y[u].y), acc[2]);
+      acc[3] = __fmaf_rn(wj[u], bf16hi_to_f32(y[u].y), acc[3]);
+      acc[4] = __fmaf_rn(wj[u], bf16lo_to_f32(y[u].z), acc[4]);
+      acc[5] = __fmaf_rn(wj[u], bf16hi_to_f32(y[u].z), acc[5]);
+      acc[6] = __fmaf_rn(wj[u], bf16lo_to_f32(y[u].w), acc[6]);
+      acc[7] = __fmaf_rn(wj[u], bf16hi_to_f32(y[u].w), acc[7]);
+    }
   }
   uint4 o;
   o.x = pack_bf16x2(acc[0], acc[1]);

@@ -229,15 +229,16 @@ def test_grouped_gemm_last_wave_split_over_k(N, K, swiglu):
             check_close(got[lo:hi], ref, BF16_TOL, f"expert {e}")
 
 
-def test_combine_exact_given_y():
+@pytest.mark.parametrize("k", [1, 3, 4, 6, 9, 16])  # routed rows are read four at a time
+def test_combine_exact_given_y(k):
     rng = np.random.default_rng(5)
-    T, H, k = 37, 256, 3
+    T, H = 37, 256
     R = T * k
     y = mi.normal_bf16(0, 51, 1.0, 1, R, H).reshape(R, H)
     w = rng.random((T, k)).astype(np.float32)
     inv = rng.permutation(R).astype(np.int32).reshape(T, k)
     out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
-    moe.moe_combine(dev_bf16(y), dev(w), dev(inv), (T, H, 128, 8, k), out)
+    moe.moe_combine(dev_bf16(y), dev(w), dev(inv), (T, H, 128, 16, k), out)
     torch.cuda.synchronize()
     yf = mi.bf16_to_f32(y)
     got = mi.bf16_to_f32(host_bf16(out))
