@@ -166,7 +166,8 @@ moe_status_t moe_topk_from_logits(const float* logits_dev, moe_dims_t d, int32_t
  *   offsets_dev    int32 [E + 1] out (exclusive prefix sum of expert counts)
  *   perm_token_dev int32 [T*k] out
  *   inv_perm_dev   int32 [T, k] out
- *   x_dev/x_perm_dev  bf16 [T, H] in / [T*k, H] out, both NULL to skip the row gather
+ *   x_dev/x_perm_dev  bf16 [T, H] in / [T*k, H] out: x_perm[p] = x[perm_token[p]]
+ *                  (each token's row written to its k rows); both NULL to skip it
  *   ws/ws_bytes    workspace of moe_workspace_size(d, BF16) bytes */
 moe_status_t moe_permute(const int32_t* ids_dev, moe_dims_t d, int32_t* offsets_dev,
                          int32_t* perm_token_dev, int32_t* inv_perm_dev, const void* x_dev,
