@@ -143,3 +143,35 @@ def test_fp4_entry_points_validate_before_launch():
     with pytest.raises(moe.MoeError) as ei:  # scale chunks cover 128 rows
         moe.moe_quantize_weight_fp4(FAKE, 1, 100, 256, FAKE, FAKE, stream=0)
     assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+
+
+def test_product_path_never_reaches_the_oracle():
+    """The package (binding, expert-parallel layer, CUDA sources, build script)
+    neither imports the CPU oracle nor links or loads its C library: every step
+    of the layer runs in the CUDA kernels, with no CPU fallback."""
+    pkg = os.path.join(ROOT, "mixture_experts_layer_tcgen05_b200")
+    seen = 0
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if not f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                continue
+            src = open(os.path.join(dirpath, f)).read()
+            seen += 1
+            assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), f
+            assert "moe_oracle" not in src and "liboracle" not in src, f
+    assert seen > 5
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
+    """With the shared library absent the binding raises instead of computing
+    anything another way."""
+    import importlib.util
+    src = os.path.join(ROOT, "mixture_experts_layer_tcgen05_b200", "__init__.py")
+    fake_pkg = tmp_path / "mixture_experts_layer_tcgen05_b200"
+    fake_pkg.mkdir()
+    (fake_pkg / "__init__.py").write_text(open(src).read())
+    spec = importlib.util.spec_from_file_location("moe_nolib", fake_pkg / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    with pytest.raises(ImportError, match="missing"):
+        mod.lib()
