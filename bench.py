@@ -121,6 +121,22 @@ def touched_weight_bytes(cfg, offsets, bytes_per_w=2.0):
     return ne * 3 * cfg.H * cfg.I * bytes_per_w, ne
 
 
+def layer_roofline(flops: float, nbytes: float, ms_per_step: float, peaks: dict, ratio: float,
+                   n_exp: int) -> dict:
+    """The whole layer against both roofs: achieved TFLOP/s and GB/s with their
+    fractions of the measured peaks (the tensor peak x `ratio` for FP8 / FP4),
+    and the roofline time max(FLOPs / tensor peak, bytes / HBM bandwidth) with
+    the fraction of it the step reaches (1.0 = at the roofline)."""
+    s = ms_per_step / 1e3
+    tpk = peaks["bf16_tflops_sustained"] * ratio
+    roof_ms = max(flops / (tpk * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    return {"tflops": flops / s / 1e12, "tflops_frac": flops / s / 1e12 / tpk,
+            "gbs": nbytes / s / 1e9, "gbs_frac": nbytes / s / 1e9 / peaks["hbm_gbs"],
+            "roofline_ms": roof_ms, "roofline_frac": roof_ms / ms_per_step,
+            "bound": "tensor" if flops / (tpk * 1e12) >= nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
+            "touched_experts": n_exp}
+
+
 def kernel_traffic(cfg_name: str, kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if the kernel's sources are unchanged."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -441,7 +457,7 @@ def gpu_arm(args, cfg):
                            "gemm_mx_kernel<SwiGLU> (block-scaled FP8 GEMM1 + SwiGLU + h quantisation)"
                            if cfg.ue8m0 else
                            "gemm_rows_fp8_kernel<SwiGLU> (FP8 GEMM1 + SwiGLU + h quantisation)" if cfg.fp8
-                           else "gemm_rows_kernel<SwiGLU,256> (GEMM1 + SwiGLU, rows gathered)"),
+                           else "gemm_rows_kernel<SwiGLU,256> (GEMM1 + SwiGLU on the permuted rows)"),
                 "algorithmic_flops_per_launch": g1_flops,
                 "peak_source": f"{peak_src} bf16 x {ratio:g} (sustained; burst {pk_burst:.1f} -> frac "
                                f"{ach / pk_burst:.3f})"}
@@ -457,12 +473,7 @@ def gpu_arm(args, cfg):
                    "l2": f"inputs larger than L2: {wbytes / 1e9:.2f} GB of expert weights read "
                          "per step, no flush"},
         "roofline": roof,
-        "layer": {"tflops": flops / (ms_per_step / 1e3) / 1e12,
-                  "tflops_frac": flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]
-                  / (2.0 if quant else 1.0),
-                  "gbs": layer_bytes / (ms_per_step / 1e3) / 1e9,
-                  "gbs_frac": layer_bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
-                  "touched_experts": n_exp},
+        "layer": layer_roofline(flops, layer_bytes, ms_per_step, peaks, 2.0 if quant else 1.0, n_exp),
         "stages_us": {n: round(float(v) * 1e3, 2) for n, v in
                       zip(["route", "permute", "gemm1", "gemm2", "combine"], stage_ms)},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,

@@ -53,3 +53,18 @@ def test_token_parallel_replicas_gloo_world2():
         assert rate == pytest.approx(world * cfg.T / 0.015)
         assert digests[0][1] == digests[1][1]  # same router weights
         assert digests[0][0] != digests[1][0]  # different token batches
+
+
+def test_layer_roofline_time_and_fractions():
+    peaks = {"bf16_tflops_sustained": 1000.0, "hbm_gbs": 5000.0}
+    # compute-bound: 2 TFLOP at 1000 TF/s = 2 ms; 1 GB at 5 TB/s = 0.2 ms
+    r = bench.layer_roofline(2e12, 1e9, 4.0, peaks, 1.0, 8)
+    assert r["bound"] == "tensor" and abs(r["roofline_ms"] - 2.0) < 1e-12
+    assert abs(r["roofline_frac"] - 0.5) < 1e-12 and abs(r["tflops_frac"] - 0.5) < 1e-12
+    assert abs(r["gbs"] - 250.0) < 1e-9 and r["touched_experts"] == 8
+    # the FP8 / FP4 ratio doubles the tensor roof
+    assert abs(bench.layer_roofline(2e12, 1e9, 4.0, peaks, 2.0, 8)["roofline_ms"] - 1.0) < 1e-12
+    # memory-bound: 10 GB at 5 TB/s = 2 ms
+    r = bench.layer_roofline(1e9, 1e10, 2.5, peaks, 1.0, 3)
+    assert r["bound"] == "hbm" and abs(r["roofline_ms"] - 2.0) < 1e-12
+    assert abs(r["roofline_frac"] - 0.8) < 1e-12 and abs(r["gbs_frac"] - 0.8) < 1e-12
