@@ -72,3 +72,30 @@ def layer_host(name: str, **over) -> tuple:
 
 def dims(cfg):
     return (cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
+
+
+# Canary bytes on both sides of a buffer: with no sanitizer on the GPU, a
+# kernel that writes past either end of its output or workspace shows up as
+# a changed guard byte.
+GUARD_BYTES = 4096
+GUARD_FILL = 0xA5
+
+
+class Guarded:
+    """`t` is a `shape`/`dtype` view starting GUARD_BYTES into a byte buffer
+    whose guard bytes hold GUARD_FILL; `intact()` checks both guards. `fill`
+    sets every byte of the view (e.g. 0 for a workspace)."""
+
+    def __init__(self, shape, dtype, device="cuda", fill=None):
+        import torch
+        self.n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self.buf = torch.full((2 * GUARD_BYTES + self.n,), GUARD_FILL, dtype=torch.uint8,
+                              device=device)
+        inner = self.buf[GUARD_BYTES:GUARD_BYTES + self.n]
+        if fill is not None:
+            inner.fill_(fill)
+        self.t = inner.view(dtype).view(tuple(shape))
+
+    def intact(self) -> bool:
+        lo, hi = self.buf[:GUARD_BYTES], self.buf[GUARD_BYTES + self.n:]
+        return bool((lo == GUARD_FILL).all().item()) and bool((hi == GUARD_FILL).all().item())

@@ -175,3 +175,24 @@ def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
     spec.loader.exec_module(mod)
     with pytest.raises(ImportError, match="missing"):
         mod.lib()
+
+
+@pytest.mark.parametrize("dtype,shape", [("bfloat16", (3, 5)), ("float32", (7,)), ("uint8", (2, 3, 4)),
+                                         ("int32", (1, 9))])
+def test_guarded_buffer_detects_writes_past_either_end(dtype, shape):
+    """The GPU tests' canary buffers, checked here on CPU tensors."""
+    import torch
+    from helpers import GUARD_BYTES, Guarded
+    dt = getattr(torch, dtype)
+    g = Guarded(shape, dt, device="cpu", fill=0)
+    assert g.t.shape == shape and g.t.dtype == dt and g.t.is_contiguous()
+    assert g.t.data_ptr() - g.buf.data_ptr() == GUARD_BYTES
+    assert g.t.data_ptr() % 256 == g.buf.data_ptr() % 256  # alignment carried over
+    assert bool((g.t.view(torch.uint8) == 0).all()) and g.intact()
+    g.t.view(torch.uint8).fill_(0x3C)  # writes inside the view leave the guards alone
+    assert g.intact()
+    g.buf[GUARD_BYTES - 1] = 0
+    assert not g.intact()
+    g2 = Guarded(shape, dt, device="cpu")
+    g2.buf[GUARD_BYTES + g2.n] = 0
+    assert not g2.intact()
