@@ -198,7 +198,6 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const V* __restrict__
 // among the earlier pairs of the same expert (the pairs are in token order, so
 // that rank is the token-ascending position) and copies its token's row(s)
 // to the permuted position. The result equals the chunked permutation's.
-constexpr int kSmallPermMaxR = kSmallPermRows;
 constexpr int kSmallPermThreads = 128;
 
 __global__ void __launch_bounds__(kSmallPermThreads) permute_gather_small_kernel(
@@ -381,7 +380,7 @@ cudaError_t launch_permute_gather_small(const int32_t* ids, int T, int E, int k,
                                         int row2_bytes, void* x2_perm, int32_t* status,
                                         cudaStream_t s) {
   const int R = T * k;
-  if (R > kSmallPermMaxR || E > 1024 || (x && row_bytes % 16) || (x2 && row2_bytes % 4))
+  if (R > kSmallPermRows || E > 1024 || (x && row_bytes % 16) || (x2 && row2_bytes % 4))
     return cudaErrorNotSupported;
   const size_t smem = (size_t)(R + E + 1) * sizeof(int32_t);
   permute_gather_small_kernel<<<(unsigned)R, kSmallPermThreads, smem, s>>>(
