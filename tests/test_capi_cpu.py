@@ -196,3 +196,26 @@ def test_guarded_buffer_detects_writes_past_either_end(dtype, shape):
     g2 = Guarded(shape, dt, device="cpu")
     g2.buf[GUARD_BYTES + g2.n] = 0
     assert not g2.intact()
+
+
+def test_every_device_wait_is_bounded():
+    """The kernels wait only through ptx::mbar_wait, which gives up after a
+    clock64 budget (or as soon as another thread has recorded a failure) and
+    records the site in the status word; there is no other spin loop, and no
+    trap or device assert anywhere in the CUDA sources."""
+    csrc = os.path.join(ROOT, "mixture_experts_layer_tcgen05_b200", "csrc")
+    files = sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    assert "ptx.cuh" in files and len(files) > 5
+    for f in files:
+        src = open(os.path.join(csrc, f)).read()
+        code = re.sub(r"//[^\n]*|/\*.*?\*/", "", src, flags=re.S)
+        if f != "ptx.cuh":
+            assert "mbarrier.try_wait" not in code and "mbar_try_wait" not in code, f
+        assert not re.search(r"while\s*\(\s*(1|true)\s*\)|for\s*\(\s*;\s*;\s*\)", code), f
+        assert "__trap" not in code and not re.search(r"\btrap\s*;", code), f
+        assert not re.search(r"\bassert\s*\(", code), f
+    ptx = open(os.path.join(csrc, "ptx.cuh")).read()
+    body = ptx[ptx.index("bool mbar_wait("):]
+    body = body[:body.index("\n}\n")]
+    for needed in ("clock64()", "budget", "record_timeout", "return false"):
+        assert needed in body, needed
