@@ -117,3 +117,28 @@ def test_regroup_plan_is_expert_major_then_source():
     assert off.tolist() == [0, 3, 5, 6]
     src_idx, off = regroup_plan(np.zeros((3, 2), dtype=np.int64))
     assert len(src_idx) == 0 and off.tolist() == [0, 0, 0]
+
+
+def test_regroup_plan_properties_on_random_count_tables():
+    """For any table of received row counts: the plan is a permutation of the
+    received rows, each local expert's rows are one contiguous block in
+    source order (sources ascending, each source's own order kept), and
+    inverse_permutation undoes it."""
+    from mixture_experts_layer_tcgen05_b200.ep import inverse_permutation
+    rng = np.random.default_rng(17)
+    for _ in range(200):
+        G, El = int(rng.integers(1, 6)), int(rng.integers(1, 7))
+        rc = rng.integers(0, 5, size=(G, El)) * (rng.random((G, El)) < 0.7)
+        src_idx, off = regroup_plan(rc)
+        n = int(rc.sum())
+        assert sorted(src_idx.tolist()) == list(range(n))
+        assert off[0] == 0 and off[-1] == n and np.all(np.diff(off) == rc.sum(0))
+        # label each received row with (source, expert, position within that block)
+        labels = [(s, j, i) for s in range(G) for j in range(El) for i in range(rc[s, j])]
+        got = [labels[r] for r in src_idx]
+        for j in range(El):
+            block = got[off[j]:off[j + 1]]
+            assert all(lab[1] == j for lab in block)
+            assert block == sorted(block)  # sources ascending, then the source's own order
+        inv = inverse_permutation(src_idx.astype(np.int64))
+        assert np.array_equal(src_idx[inv], np.arange(n)) if n else len(inv) == 0
