@@ -219,3 +219,31 @@ def test_every_device_wait_is_bounded():
     body = body[:body.index("\n}\n")]
     for needed in ("clock64()", "budget", "record_timeout", "return false"):
         assert needed in body, needed
+
+
+@pytest.mark.parametrize("dt", ["MOE_DTYPE_BF16", "MOE_DTYPE_FP8_E4M3", "MOE_DTYPE_FP8_E4M3_UE8M0",
+                                "MOE_DTYPE_FP4_E2M1"])
+def test_workspace_layout_at_the_largest_accepted_dims(dt):
+    """Sizes far past 2^32 bytes: the layout arithmetic is 64-bit, every region
+    is 256-byte aligned, no two regions overlap at their nominal sizes, and the
+    total covers them all. T = 2^27 - 1 with k = 16 is just under the 2^31
+    routed-row limit of the dims check."""
+    dtype = getattr(moe, dt)
+    T, H, I, E, k = (1 << 27) - 1, 7168, 2048, 1024, 16
+    R = T * k
+    L = moe.moe_workspace_layout((T, H, I, E, k), dtype)
+    assert L.total == moe.moe_workspace_size((T, H, I, E, k), dtype) > R * H
+    q = dtype != moe.MOE_DTYPE_BF16
+    size = {"logits": T * E * 4, "topk_ids": R * 4, "topk_w": R * 4, "offsets": (E + 1) * 4,
+            "perm_token": R * 4, "inv_perm": R * 4, "y_perm": R * H * 2}
+    if q:
+        size.update(xq=T * H, xs=T * (H // 128) * 4, xq_perm=R * H, xs_perm=R * (H // 128) * 4,
+                    hq=R * I, hs=R * (I // 128) * 4)
+    else:
+        size.update(x_perm=R * H * 2, h=R * I * 2)
+    regions = sorted((getattr(L, f), getattr(L, f) + n, f) for f, n in size.items())
+    for lo, hi, f in regions:
+        assert lo % 256 == 0, f
+    for (lo0, hi0, f0), (lo1, hi1, f1) in zip(regions, regions[1:]):
+        assert hi0 <= lo1, (f0, f1)  # no two regions overlap
+    assert regions[-1][1] <= L.total
