@@ -170,6 +170,18 @@ def oracle_inputs(cfg, L):
     return {"w13": L["w13"], "w2": L["w2"]}
 
 
+def cpu_model() -> str | None:
+    """The host CPU's model name (first `model name` line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def oracle_tokens_per_s(cfg, L, budget_s: float, kw=None):
     import oracle
 
@@ -219,7 +231,7 @@ def reference_arm(args, cfg):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": cfg.desc, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
-                         "kind": "oracle", "sample": sample},
+                         "cpu": cpu_model(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -487,7 +499,7 @@ def gpu_arm(args, cfg):
 
         v, n, t = oracle_tokens_per_s(cfg, L, float(os.environ.get("MOE_CPU_BUDGET_S", "20")))
         res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle.threads(),
-                               "kind": "oracle",
+                               "cpu": cpu_model(), "kind": "oracle",
                                "sample": f"{n} of {cfg.T} tokens (seeded subset), whole layer "
                                          f"per token, {t:.1f} s"}
     print(json.dumps(res), flush=True)

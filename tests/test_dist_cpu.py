@@ -68,3 +68,8 @@ def test_layer_roofline_time_and_fractions():
     r = bench.layer_roofline(1e9, 1e10, 2.5, peaks, 1.0, 3)
     assert r["bound"] == "hbm" and abs(r["roofline_ms"] - 2.0) < 1e-12
     assert abs(r["roofline_frac"] - 0.8) < 1e-12 and abs(r["gbs_frac"] - 0.8) < 1e-12
+
+
+def test_cpu_model_is_read_from_the_host():
+    m = bench.cpu_model()
+    assert m is None or (isinstance(m, str) and m and "\n" not in m)
