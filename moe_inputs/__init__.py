@@ -14,7 +14,8 @@ layout the library consumes:
 * ``x``    ``[T, H]`` bf16, N(0, 1)
 * ``wr``   ``[H, E]`` bf16, N(0, 0.02)
 * ``bias`` ``[E]`` fp32: zero, N(0, 0.5), or the Zipf(s=1.1) log-pmf of a seeded
-  rank permutation, ``-1.1 * ln(rank)``
+  rank permutation in units of the logits' own spread,
+  ``-1.1 * sigma_l * ln(rank)`` with ``sigma_l = x_sigma * w_sigma * sqrt(H)``
 * ``w13``  ``[E, 2I, H]`` bf16, K-major: rows ``[0, I)`` are ``Wg[e]^T``, rows
   ``[I, 2I)`` are ``Wu[e]^T``; N(0, 0.02)
 * ``w2``   ``[E, H, I]`` bf16, K-major: ``Wd[e]^T``; N(0, 0.02)
@@ -190,10 +191,15 @@ def make_router(cfg: LayerConfig):
     elif cfg.bias == "normal":
         b = normal_f32(cfg.seed, TAG_BIAS, cfg.bias_sigma, 1, 1, cfg.E).reshape(cfg.E)
     elif cfg.bias == "zipf":
+        # The Zipf(s) log-pmf of each expert's rank, -s*ln(rank) up to a constant, measured
+        # in the logits' own standard deviation sigma_l (the nominal spread of x.Wr), so the
+        # skew it imposes does not shrink as H grows. In plain logit units the router's
+        # own spread (1.69 at H = 7168) flattens it and every expert keeps some tokens.
         perm = permutation(cfg.seed, TAG_ZIPF, cfg.E)
         rank = np.empty(cfg.E, dtype=np.int64)
         rank[perm] = np.arange(1, cfg.E + 1)
-        b = np.array([-cfg.zipf_s * math.log(r) for r in rank], dtype=np.float32)
+        sigma_l = cfg.x_sigma * cfg.w_sigma * math.sqrt(cfg.H)
+        b = np.array([-cfg.zipf_s * sigma_l * math.log(r) for r in rank], dtype=np.float32)
     else:
         raise ValueError(cfg.bias)
     return wr, b

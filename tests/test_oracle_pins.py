@@ -632,5 +632,18 @@ def test_generator_moments():
 def test_zipf_bias_is_log_pmf_of_a_rank_permutation():
     cfg = mi.CONFIGS["fine_grained"]
     _, b = mi.make_router(cfg.with_(H=8))
-    ranks = np.exp(-b.astype(np.float64) / 1.1)
+    sigma_l = 1.0 * 0.02 * np.sqrt(8)  # x ~ N(0,1), Wr ~ N(0,0.02): the logits' spread
+    ranks = np.exp(-b.astype(np.float64) / (1.1 * sigma_l))
     np.testing.assert_allclose(np.sort(ranks), np.arange(1, 257), rtol=1e-5)
+
+
+def test_fine_grained_workload_is_skewed_with_empty_experts():
+    # The fine-grained workload promises Zipf-skewed expert loads "including some empty
+    # experts": route the full-size seed-0 batch with the oracle and check both properties.
+    cfg = mi.CONFIGS["fine_grained"]
+    wr, b = mi.make_router(cfg)
+    ids, _ = oracle.topk(oracle.router_logits(mi.make_x(cfg), wr, b), cfg.k)
+    counts = np.bincount(ids.ravel(), minlength=cfg.E)
+    assert counts.sum() == cfg.T * cfg.k
+    assert np.sum(counts == 0) >= 1
+    assert counts.max() > 8 * counts.mean()
