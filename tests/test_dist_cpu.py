@@ -55,19 +55,44 @@ def test_token_parallel_replicas_gloo_world2():
         assert digests[0][0] != digests[1][0]  # different token batches
 
 
-def test_layer_roofline_time_and_fractions():
-    peaks = {"bf16_tflops_sustained": 1000.0, "hbm_gbs": 5000.0}
-    # compute-bound: 2 TFLOP at 1000 TF/s = 2 ms; 1 GB at 5 TB/s = 0.2 ms
-    r = bench.layer_roofline(2e12, 1e9, 4.0, peaks, 1.0, 8)
-    assert r["bound"] == "tensor" and abs(r["roofline_ms"] - 2.0) < 1e-12
-    assert abs(r["roofline_frac"] - 0.5) < 1e-12 and abs(r["tflops_frac"] - 0.5) < 1e-12
-    assert abs(r["gbs"] - 250.0) < 1e-9 and r["touched_experts"] == 8
-    # the FP8 / FP4 ratio doubles the tensor roof
-    assert abs(bench.layer_roofline(2e12, 1e9, 4.0, peaks, 2.0, 8)["roofline_ms"] - 1.0) < 1e-12
-    # memory-bound: 10 GB at 5 TB/s = 2 ms
-    r = bench.layer_roofline(1e9, 1e10, 2.5, peaks, 1.0, 3)
-    assert r["bound"] == "hbm" and abs(r["roofline_ms"] - 2.0) < 1e-12
-    assert abs(r["roofline_frac"] - 0.8) < 1e-12 and abs(r["gbs_frac"] - 0.8) < 1e-12
+def _cfg(**kw):
+    return mi.CONFIGS["tiny"].with_(**kw)
+
+
+def test_rooflines_layer_time_and_fractions():
+    peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 800.0, "hbm_gbs": 5000.0}
+    # T*k*H*I chosen so 6*T*k*H*I = 2e12 FLOP; one expert of 4 touched with rows
+    cfg = _cfg(T=1000, k=1, H=1000, I=1000 * 1000 // 3, E=4)
+    off = np.array([0, 1000, 1000, 1000, 1000], dtype=np.int32)
+    flops = 6.0 * cfg.T * cfg.k * cfg.H * cfg.I
+    stage = np.array([0.0, 0.0, 2.0, 1.0, 0.0])
+    roof, lay, wbytes = bench.rooflines(cfg, off, 4.0, stage, 200.0, peaks, "measured")
+    assert wbytes == 3 * cfg.H * cfg.I * 2 and lay["touched_experts"] == 1
+    # a region under a second is compared with the burst peak
+    assert roof["peak"] == 1000.0 and "burst" in roof["peak_source"]
+    assert abs(roof["achieved"] - 4.0 * cfg.T * cfg.H * cfg.I / 2e-3 / 1e12) < 1e-9
+    assert abs(roof["frac_of_sustained"] - roof["achieved"] / 800.0) < 1e-12
+    assert lay["bound"] == "tensor"
+    assert abs(lay["roofline_ms"] - flops / 1e15 * 1e3) < 1e-9
+    assert abs(lay["roofline_frac"] - lay["roofline_ms"] / 4.0) < 1e-12
+    # a long region takes the sustained peak
+    roof2, lay2, _ = bench.rooflines(cfg, off, 4.0, stage, 5000.0, peaks, "measured")
+    assert roof2["peak"] == 800.0 and "sustained" in roof2["peak_source"]
+    # FP8 doubles the tensor roof
+    r8, l8, _ = bench.rooflines(cfg.with_(fp8=True), off, 4.0, stage, 200.0, peaks, "measured",
+                                e4m3_tflops=1800.0)
+    assert r8["peak"] == 2000.0 and abs(r8["frac_of_cublas_e4m3"] - r8["achieved"] / 1800) < 1e-12
+
+
+def test_rooflines_decode_is_hbm_bound():
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    cfg = _cfg(T=16, k=2, H=4096, I=14336, E=8)
+    off = np.array([0, 4, 8, 12, 16, 20, 24, 28, 32], dtype=np.int32)
+    stage = np.array([0.0, 0.0, 0.2, 0.1, 0.0])
+    roof, lay, wbytes = bench.rooflines(cfg, off, 0.5, stage, 10.0, peaks, "fallback")
+    g1 = 8 * 2 * cfg.H * cfg.I * 2.0
+    assert roof["bound"] == "hbm" and abs(roof["achieved"] - g1 / 0.2e-3 / 1e9) < 1e-6
+    assert lay["bound"] == "hbm"
 
 
 def test_cpu_model_is_read_from_the_host():
