@@ -177,25 +177,39 @@ moe_status_t moe_permute(const int32_t* ids_dev, moe_dims_t d, int32_t* offsets_
  * this entry point: it exists for callers that cannot allocate device memory
  * when they call it -- for example an engine that plans all of its memory
  * once at start-up and must not call cudaMalloc (or a caching allocator)
- * while serving, or code that runs where allocation is not allowed. Results
- * are identical to moe_permute's.
+ * while serving, or code that runs where allocation is not allowed. For
+ * valid ids the results are identical to moe_permute's.
  *
  * The scratch lives in one fixed device array inside this library,
  * MOE_NOALLOC_SCRATCH_BYTES bytes on every device that loads it, held until
- * the process exits. Dims whose scratch exceeds it (2 * ceil(T/32) * E * 4
- * bytes, each part rounded up to 256, plus E * 4) are rejected with
- * MOE_ERR_INVALID_ARG before anything is launched; E = 256 allows T up to
- * 16352, E = 8 about a million. The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. Every call uses the same array and leaves its
- * contents behind (nothing in it needs clearing: each call writes every word
- * it reads), so calls that can overlap on the GPU -- two streams, or two
- * threads -- race on it: order them on one stream. Nothing here allocates or
- * frees memory. Arguments as for moe_permute (no ws). */
+ * the process exits. Its first 256 bytes are a status word; the rest
+ * (MOE_NOALLOC_SCRATCH_BYTES - 256) is the permutation's scratch. Dims whose
+ * scratch exceeds that (2 * ceil(T/32) * E * 4 bytes, each of the two parts
+ * rounded up to 256, plus E * 4 rounded up to 256) are rejected with
+ * MOE_ERR_INVALID_ARG before anything is launched: E = 256 allows T up to
+ * 16352, E = 8 up to 524032. The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture. Every call uses the same array and
+ * leaves its contents behind (the scratch needs no clearing: each call writes
+ * every scratch word it reads), so calls that can overlap on the GPU -- two
+ * streams, or two threads -- race on it: order them on one stream.
+ * An expert id outside [0, E), or an expert repeated within a token, is
+ * recorded as (MOE_ERR_INVALID_ARG << 8) | 6 in the array's status word
+ * (the first failure is kept; read and clear it with
+ * moe_permute_noalloc_status); such a pair is skipped and its outputs are
+ * left unwritten. Nothing here allocates or frees memory. Arguments as for
+ * moe_permute (no ws). */
 #define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
 moe_status_t moe_permute_noalloc(const int32_t* ids_dev, moe_dims_t d, int32_t* offsets_dev,
                                  int32_t* perm_token_dev, int32_t* inv_perm_dev,
                                  const void* x_dev, void* x_perm_dev, void* stream);
+
+/* The status word of moe_permute_noalloc's fixed array on the current device:
+ * 0, or the first recorded failure. Waits for all work on the device, then
+ * reads it into *status_out; with clear != 0 it then sets it back to 0.
+ * Blocking and synchronising: for checks between batches, not in hot loops
+ * or stream captures. Allocates nothing. */
+moe_status_t moe_permute_noalloc_status(int32_t* status_out, int32_t clear);
 
 /* Grouped GEMM on tcgen05 tensor cores ([X] backend table, grouped_mm and
  * deepgemm rows: one grouped GEMM over expert-sorted rows).
@@ -384,6 +398,23 @@ moe_status_t moe_quantize_act_fp8_fmt(const void* x_dev, int64_t rows, int64_t c
 moe_status_t moe_quantize_weight_fp8_fmt(const void* w_dev, int64_t nb, int64_t rows,
                                          int64_t cols, void* q_dev, float* s_dev,
                                          moe_scale_fmt_t fmt, void* stream);
+
+/* One-time weight packing ([X] backend table, grouped_mm row: each expert's
+ * gate and up projections map H -> I, its down projection I -> H). Takes the
+ * experts' weights in their logical layout and writes the K-major layout
+ * every forward and grouped GEMM above reads:
+ *   wg_dev, wu_dev bf16 [E, H, I]    gate and up projection of each expert
+ *   wd_dev         bf16 [E, I, H]    down projection of each expert
+ *   w13_dev        bf16 [E, 2I, H] out: rows [0, I) = Wg[e]^T, rows [I, 2I) = Wu[e]^T
+ *   w2_dev         bf16 [E, H, I]  out: Wd[e]^T
+ * A pure copy (bit-exact). H and I multiples of 128, 1 <= E <= 65535; the
+ * outputs must not overlap the inputs or each other (MOE_ERR_INVALID_ARG).
+ * Stream-ordered, no workspace; untimed preparation, not part of the layer.
+ * The FP8 / FP4 weights are then quantised from w13 / w2 with
+ * moe_quantize_weight_fp8(_fmt) / moe_quantize_weight_fp4. */
+moe_status_t moe_pack_weights(const void* wg_dev, const void* wu_dev, const void* wd_dev,
+                              int32_t E, int32_t H, int32_t I, void* w13_dev, void* w2_dev,
+                              void* stream);
 
 /* Reads the workspace's device status word (MOE_OK or MOE_ERR_TIMEOUT) into
  * *status_out. Synchronises the device (a blocking copy); not for hot loops. */

@@ -27,9 +27,9 @@ __all__ = [
     "MOE_DTYPE_FP4_E2M1", "moe_forward_fp4", "moe_grouped_gemm_fp4", "moe_quantize_weight_fp4",
     "moe_last_error", "moe_abi_version", "moe_launch_count", "moe_workspace_size",
     "moe_workspace_layout", "moe_route_topk", "moe_topk_from_logits", "moe_permute",
-    "moe_permute_noalloc",
+    "moe_permute_noalloc", "moe_permute_noalloc_status",
     "moe_grouped_gemm", "moe_combine", "moe_gather_rows", "moe_forward", "moe_forward_fp8", "moe_forward_hostio",
-    "moe_quantize_act_fp8", "moe_quantize_weight_fp8", "moe_get_device_status",
+    "moe_quantize_act_fp8", "moe_quantize_weight_fp8", "moe_pack_weights", "moe_get_device_status",
     "moe_clear_device_status", "moe_set_stage_events", "moe_check_wait_timeout", "EXPORTED",
 ]
 
@@ -72,6 +72,7 @@ _SIGS = {
     "moe_topk_from_logits": (_i32, [_vp, Dims, _vp, _vp, _vp]),
     "moe_permute": (_i32, [_vp, Dims, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (_i32, [_vp, Dims, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_permute_noalloc_status": (_i32, [ctypes.POINTER(_i32), _i32]),
     "moe_grouped_gemm": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp,
                                 _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "moe_combine": (_i32, [_vp, _vp, _vp, Dims, _vp, _vp]),
@@ -92,6 +93,7 @@ _SIGS = {
     "moe_quantize_weight_fp8": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "moe_quantize_act_fp8_fmt": (_i32, [_vp, _i64, _i64, _vp, _vp, _i32, _vp]),
     "moe_quantize_weight_fp8_fmt": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp]),
+    "moe_pack_weights": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_get_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_clear_device_status": (_i32, [_vp, _vp]),
     "moe_check_wait_timeout": (_i32, [_vp, _i64, _vp]),
@@ -203,6 +205,12 @@ def moe_permute_noalloc(ids, d, offsets, perm_token, inv_perm, x=None, x_perm=No
                                      _p(x), _p(x_perm), _s(stream)))
 
 
+def moe_permute_noalloc_status(clear: bool = False) -> int:
+    v = ctypes.c_int32(0)
+    _check(lib().moe_permute_noalloc_status(ctypes.byref(v), int(bool(clear))))
+    return v.value
+
+
 def moe_grouped_gemm(A, B, offsets, M_total, E, N, K, dt, ep, C, a_scales=None, b_scales=None,
                      c_scales=None, max_rows_per_expert=0, ws=None, ws_bytes=None, stream=None,
                      a_rows=None, a_src_rows=0):
@@ -289,6 +297,10 @@ def moe_quantize_act_fp8_fmt(x, rows, cols, q, s, fmt, stream=None):
 def moe_quantize_weight_fp8_fmt(w, nb, rows, cols, q, s, fmt, stream=None):
     _check(lib().moe_quantize_weight_fp8_fmt(_p(w), nb, rows, cols, _p(q), _p(s), int(fmt),
                                              _s(stream)))
+
+
+def moe_pack_weights(wg, wu, wd, E, H, I, w13, w2, stream=None):
+    _check(lib().moe_pack_weights(_p(wg), _p(wu), _p(wd), E, H, I, _p(w13), _p(w2), _s(stream)))
 
 
 def moe_get_device_status(ws) -> int:

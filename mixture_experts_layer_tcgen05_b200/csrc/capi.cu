@@ -68,10 +68,14 @@ cudaError_t launch_quant_act_scatter(const void* x, int64_t rows, int64_t cols,
 cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                 float* sc, bool ue8m0, cudaStream_t s);
 
+cudaError_t launch_pack_weights(const void* wg, const void* wu, const void* wd, int E, int H,
+                                int I, void* w13, void* w2, cudaStream_t s);
+
 int64_t noalloc_scratch_capacity();
 cudaError_t launch_permute_noalloc(const int32_t* ids, int T, int H, int E, int k, int32_t* offsets,
                                    int32_t* perm_token, int32_t* inv_perm, const void* x,
                                    void* x_perm, cudaStream_t s);
+cudaError_t noalloc_status(int32_t* out, bool clear);
 
 static std::atomic<int64_t> g_launches{0};
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -344,6 +348,14 @@ moe_status_t moe_permute_noalloc(const int32_t* ids, moe_dims_t d, int32_t* offs
   cudaError_t e = launch_permute_noalloc(ids, d.T, d.H, d.E, d.k, offsets, perm_token, inv_perm, x,
                                          x_perm, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "permute (fixed scratch)");
+  return ok();
+}
+
+moe_status_t moe_permute_noalloc_status(int32_t* status_out, int32_t clear) {
+  if (!status_out) return fail(MOE_ERR_INVALID_ARG, "status_out is NULL");
+  MOE_TRY(check_device());
+  cudaError_t e = noalloc_status(status_out, clear != 0);
+  if (e != cudaSuccess) return cuda_fail(e, "read the fixed array's status word");
   return ok();
 }
 
@@ -769,6 +781,35 @@ moe_status_t moe_quantize_weight_fp4(const void* w, int64_t nb, int64_t rows, in
   MOE_TRY(check_device());
   cudaError_t e = launch_quant_weight_fp4(w, nb, rows, cols, q, sc, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "FP4 weight quantisation");
+  return ok();
+}
+
+moe_status_t moe_pack_weights(const void* wg, const void* wu, const void* wd, int32_t E, int32_t H,
+                              int32_t I, void* w13, void* w2, void* stream) {
+  if (E < 1 || E > 65535) return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 65535] (got %d)", E);
+  if (H < 128 || H % 128)
+    return fail(MOE_ERR_INVALID_ARG, "H must be a positive multiple of 128 (got %d)", H);
+  if (I < 128 || I % 128)
+    return fail(MOE_ERR_INVALID_ARG, "I must be a positive multiple of 128 (got %d)", I);
+  MOE_TRY(check_ptr(wg, "wg"));
+  MOE_TRY(check_ptr(wu, "wu"));
+  MOE_TRY(check_ptr(wd, "wd"));
+  MOE_TRY(check_ptr(w13, "w13"));
+  MOE_TRY(check_ptr(w2, "w2"));
+  // the outputs must not overlap any input (the transposes read and write concurrently)
+  const uint64_t hi = (uint64_t)H * I * 2 * E;
+  auto lo_of = [](const void* p) { return reinterpret_cast<uint64_t>(p); };
+  auto overlap = [&](const void* a, uint64_t na, const void* b, uint64_t nb) {
+    return lo_of(a) < lo_of(b) + nb && lo_of(b) < lo_of(a) + na;
+  };
+  const void* ins[3] = {wg, wu, wd};
+  for (const void* in : ins)
+    if (overlap(w13, 2 * hi, in, hi) || overlap(w2, hi, in, hi))
+      return fail(MOE_ERR_INVALID_ARG, "w13 / w2 overlap an input weight");
+  if (overlap(w13, 2 * hi, w2, hi)) return fail(MOE_ERR_INVALID_ARG, "w13 and w2 overlap");
+  MOE_TRY(check_device());
+  cudaError_t e = launch_pack_weights(wg, wu, wd, E, H, I, w13, w2, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "weight packing");
   return ok();
 }
 

@@ -247,3 +247,63 @@ def test_workspace_layout_at_the_largest_accepted_dims(dt):
     for (lo0, hi0, f0), (lo1, hi1, f1) in zip(regions, regions[1:]):
         assert hi0 <= lo1, (f0, f1)  # no two regions overlap
     assert regions[-1][1] <= L.total
+
+
+def _noalloc_scratch(T, E):
+    # the permutation's scratch: chunk masks and chunk bases (ceil(T/32) x E words each, each
+    # part rounded up to 256 bytes) and E counts (rounded up to 256)
+    def up(n):
+        return (n + 255) // 256 * 256
+    c = (T + 31) // 32
+    return 2 * up(c * E * 4) + up(E * 4)
+
+
+@pytest.mark.parametrize("E", [256, 8])
+def test_noalloc_rejects_exactly_past_its_fixed_array(E, monkeypatch):
+    """The size check runs before the device check: the largest accepted T gets as far as
+    the (faked, refused) device check; one token more is rejected as too large. The
+    array's first 256 bytes are its status word."""
+    monkeypatch.setenv("MOE_FAKE_CC", "90")
+    cap = 1048576 - 256
+    T = max(t for t in range(1, 600000) if _noalloc_scratch(t, E) <= cap) if E == 8 else \
+        max(t for t in range(1, 20000) if _noalloc_scratch(t, E) <= cap)
+    assert T == {256: 16352, 8: 524032}[E]  # the bounds include/moe.h states
+    k = 2
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_permute_noalloc(FAKE, (T, 128, 128, E, k), FAKE, FAKE, FAKE, stream=0)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_DEVICE
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_permute_noalloc(FAKE, (T + 1, 128, 128, E, k), FAKE, FAKE, FAKE, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG and "scratch" in str(ei.value)
+
+
+def test_noalloc_status_validates():
+    assert moe.lib().moe_permute_noalloc_status(None, 0) == moe.MOE_ERR_INVALID_ARG
+    assert "NULL" in moe.moe_last_error()
+
+
+def test_pack_weights_validates_before_launch(monkeypatch):
+    monkeypatch.setenv("MOE_FAKE_CC", "90")
+    E, H, I = 4, 256, 384
+    n = E * H * I * 2
+    wg, wu, wd = FAKE, FAKE + n, FAKE + 2 * n
+    w13, w2 = FAKE + 3 * n, FAKE + 5 * n
+    for bad, msg in [((0, H, I), "E must"), ((E, 100, I), "H must"), ((E, H, 64), "I must")]:
+        with pytest.raises(moe.MoeError) as ei:
+            moe.moe_pack_weights(wg, wu, wd, *bad, w13, w2, stream=0)
+        assert ei.value.status == moe.MOE_ERR_INVALID_ARG and msg in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_pack_weights(None, wu, wd, E, H, I, w13, w2, stream=0)
+    assert "wg is NULL" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_pack_weights(wg, wu, wd + 8, E, H, I, w13, w2, stream=0)
+    assert "aligned" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:  # w13 spans 2n bytes: it would run into w2 at 4n
+        moe.moe_pack_weights(wg, wu, wd, E, H, I, FAKE + 3 * n, FAKE + 4 * n, stream=0)
+    assert "overlap" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:  # output written over an input
+        moe.moe_pack_weights(wg, wu, wd, E, H, I, FAKE + n, w2, stream=0)
+    assert "overlap" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:  # valid: gets as far as the device check
+        moe.moe_pack_weights(wg, wu, wd, E, H, I, w13, w2, stream=0)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_DEVICE
