@@ -35,8 +35,9 @@ __global__ void __launch_bounds__(128) permute_mask_kernel(const int32_t* __rest
     if (t < T)
       for (int j = 0; j < k; ++j) {
         const int e = ids[(int64_t)t * k + j];
-        if ((unsigned)e < (unsigned)E) atomicOr(&m[e], 1u << lane);
-        else record_bad_index(status);
+        if ((unsigned)e >= (unsigned)E) record_bad_index(status);
+        else if (atomicOr(&m[e], 1u << lane) & (1u << lane))  // bit already set: a repeat
+          record_bad_index(status);
       }
   }
   __syncwarp();
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(128) permute_scatter_kernel(
     if ((unsigned)e >= (unsigned)E) continue;  // recorded by the mask kernel
     uint32_t m = masks[(int64_t)chunk * E + e];
     int32_t p = off_smem[e] + chunk_base[(int64_t)chunk * E + e] + __popc(m & below);
-    if ((unsigned)p >= (unsigned)(T * k)) {  // repeated expert within a token
+    if ((unsigned)p >= (unsigned)(T * k)) {  // only for invalid ids (recorded by the mask kernel)
       record_bad_index(status);
       continue;
     }
@@ -255,6 +256,12 @@ __global__ void __launch_bounds__(kSmallPermThreads) permute_gather_small_kernel
     for (int e = tid; e <= E; e += kSmallPermThreads) offsets[e] = soff[e];
   const int b = blockIdx.x, t = b / k, e = sid[b];
   if (e < 0) return;
+  if (tid == 0)  // an expert repeated within the token is recorded (once, by its later slot)
+    for (int p = t * k; p < b; ++p)
+      if (sid[p] == e) {
+        record_bad_index(status);
+        break;
+      }
   // rank of pair b among the earlier pairs that chose the same expert
   int cnt = 0;
   for (int p = tid; p < b; p += kSmallPermThreads) cnt += sid[p] == e;

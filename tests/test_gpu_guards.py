@@ -6,9 +6,8 @@ holding a known byte, and after the call both guards must be unchanged. The
 shapes are ragged (experts whose rows end mid-tile, a last tile hanging past
 the last row, empty experts) so that every masked edge is exercised: the
 row scatter, the split router's block sums, the GEMM epilogues and their
-split-K / K-split partials, the quantised copies and the combine.
-
-Collected last: its calls repeat ones the parity tests make."""
+split-K / K-split partials, the quantised copies and the combine. Its calls
+repeat ones the parity tests make."""
 import numpy as np
 import pytest
 
