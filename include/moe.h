@@ -416,6 +416,54 @@ moe_status_t moe_pack_weights(const void* wg_dev, const void* wu_dev, const void
                               int32_t E, int32_t H, int32_t I, void* w13_dev, void* w2_dev,
                               void* stream);
 
+/* Expert-parallel exchange planned and moved on the device ([X] backend
+ * table, deepgemm_megamoe row: experts spread over ranks, each token's rows
+ * dispatched to the ranks owning their experts and combined back). G ranks
+ * own E / G consecutive experts each (rank g: [g*El, (g+1)*El), El = E / G).
+ * Every rank has routed and permuted its own tokens (moe_route_topk,
+ * moe_permute: rows expert-major) and all ranks hold the same all-gathered
+ * counts_all int32 [G, E] (row s: rank s's rows per expert, e.g. the
+ * differences of its offsets). No count ever goes to the host.
+ *
+ * moe_ep_plan (one small kernel) writes rank `rank`'s plan, int32, into
+ * plan_dev (moe_ep_plan_bytes(E, G) bytes, 16-byte aligned):
+ *   loc_off   [El + 1]   at plan_dev: this rank's receive buffer is
+ *                        expert-major (local expert j, then source rank
+ *                        ascending, then the source's row order); local expert
+ *                        j owns rows [loc_off[j], loc_off[j+1]) -- the offsets
+ *                        to run moe_grouped_gemm on it directly
+ *   send_base [E]        at plan_dev + (El + 1 rounded up to 4): row in rank
+ *                        e / El's receive buffer of this rank's first row for
+ *                        expert e
+ *   ret_lb [El*G + 1], ret_dst [El*G]   then: the return path's blocks
+ * moe_ep_plan_bytes returns 0 for E, G outside 1 <= G <= 64, E <= 1024, E % G == 0.
+ *
+ * moe_ep_dispatch: row p of x_perm_dev [R, row_bytes] (this rank's permuted
+ * rows, offsets_dev [E + 1] from moe_permute) is stored to row
+ * send_base[e] + (p - offsets[e]) of the buffer at dst_bufs_dev[e / El]
+ * (a DEVICE array of G addresses: the ranks' receive buffers, mapped into
+ * this process, e.g. symmetric memory; each dst_rows rows long).
+ * moe_ep_return: row q < loc_off[El] of y_loc_dev [cap_rows, row_bytes]
+ * (this rank's expert outputs in receive order) is stored back to its
+ * source rank s, at the row of src_bufs_dev[s] (the ranks' y_perm buffers,
+ * src_rows rows each) it was dispatched from. cap_rows is any upper bound on
+ * the received rows (the kernel reads the exact count from the plan).
+ * Plain 16-byte stores, each warp's ended by a system-scope fence; the caller
+ * orders them before the other ranks' reads with a cross-rank
+ * synchronisation on the stream (e.g. an NCCL collective). A destination row
+ * outside its buffer is skipped and (MOE_ERR_INVALID_ARG << 8) | 6 recorded
+ * in ws's status word (ws may be NULL). row_bytes a multiple of 16. */
+size_t moe_ep_plan_bytes(int32_t E, int32_t G);
+moe_status_t moe_ep_plan(const int32_t* counts_all_dev, int32_t G, int32_t rank, int32_t E,
+                         int32_t* plan_dev, void* stream);
+moe_status_t moe_ep_dispatch(const void* x_perm_dev, const int32_t* offsets_dev,
+                             const int32_t* plan_dev, int32_t E, int32_t G, int32_t R,
+                             int64_t row_bytes, const uint64_t* dst_bufs_dev, int64_t dst_rows,
+                             void* ws, void* stream);
+moe_status_t moe_ep_return(const void* y_loc_dev, const int32_t* plan_dev, int32_t E, int32_t G,
+                           int64_t cap_rows, int64_t row_bytes, const uint64_t* src_bufs_dev,
+                           int64_t src_rows, void* ws, void* stream);
+
 /* Reads the workspace's device status word (MOE_OK or MOE_ERR_TIMEOUT) into
  * *status_out. Synchronises the device (a blocking copy); not for hot loops. */
 moe_status_t moe_get_device_status(const void* ws, int32_t* status_out);

@@ -30,6 +30,7 @@ __all__ = [
     "moe_permute_noalloc", "moe_permute_noalloc_status",
     "moe_grouped_gemm", "moe_combine", "moe_gather_rows", "moe_forward", "moe_forward_fp8", "moe_forward_hostio",
     "moe_quantize_act_fp8", "moe_quantize_weight_fp8", "moe_pack_weights", "moe_get_device_status",
+    "moe_ep_plan_bytes", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
     "moe_clear_device_status", "moe_set_stage_events", "moe_check_wait_timeout", "EXPORTED",
 ]
 
@@ -94,6 +95,10 @@ _SIGS = {
     "moe_quantize_act_fp8_fmt": (_i32, [_vp, _i64, _i64, _vp, _vp, _i32, _vp]),
     "moe_quantize_weight_fp8_fmt": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp]),
     "moe_pack_weights": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_ep_plan_bytes": (_sz, [_i32, _i32]),
+    "moe_ep_plan": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
+    "moe_ep_dispatch": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _vp, _i64, _vp, _vp]),
+    "moe_ep_return": (_i32, [_vp, _vp, _i32, _i32, _i64, _i64, _vp, _i64, _vp, _vp]),
     "moe_get_device_status": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "moe_clear_device_status": (_i32, [_vp, _vp]),
     "moe_check_wait_timeout": (_i32, [_vp, _i64, _vp]),
@@ -301,6 +306,25 @@ def moe_quantize_weight_fp8_fmt(w, nb, rows, cols, q, s, fmt, stream=None):
 
 def moe_pack_weights(wg, wu, wd, E, H, I, w13, w2, stream=None):
     _check(lib().moe_pack_weights(_p(wg), _p(wu), _p(wd), E, H, I, _p(w13), _p(w2), _s(stream)))
+
+
+def moe_ep_plan_bytes(E, G) -> int:
+    return int(lib().moe_ep_plan_bytes(E, G))
+
+
+def moe_ep_plan(counts_all, G, rank, E, plan, stream=None):
+    _check(lib().moe_ep_plan(_p(counts_all), G, rank, E, _p(plan), _s(stream)))
+
+
+def moe_ep_dispatch(x_perm, offsets, plan, E, G, R, row_bytes, dst_bufs, dst_rows, ws=None,
+                    stream=None):
+    _check(lib().moe_ep_dispatch(_p(x_perm), _p(offsets), _p(plan), E, G, R, row_bytes,
+                                 _p(dst_bufs), dst_rows, _p(ws), _s(stream)))
+
+
+def moe_ep_return(y_loc, plan, E, G, cap_rows, row_bytes, src_bufs, src_rows, ws=None, stream=None):
+    _check(lib().moe_ep_return(_p(y_loc), _p(plan), E, G, cap_rows, row_bytes, _p(src_bufs),
+                               src_rows, _p(ws), _s(stream)))
 
 
 def moe_get_device_status(ws) -> int:

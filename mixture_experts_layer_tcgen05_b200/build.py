@@ -12,7 +12,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 SRCS = ["capi.cu", "router.cu", "permute.cu", "gemm.cu", "gemm_fp8.cu", "gemm_mx.cu", "fp8.cu",
-        "noalloc.cu", "selftest.cu", "pack.cu"]
+        "noalloc.cu", "selftest.cu", "pack.cu", "ep.cu"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

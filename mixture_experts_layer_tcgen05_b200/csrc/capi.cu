@@ -68,6 +68,14 @@ cudaError_t launch_quant_act_scatter(const void* x, int64_t rows, int64_t cols,
 cudaError_t launch_quant_weight(const void* w, int64_t nb, int64_t rows, int64_t cols, void* q,
                                 float* sc, bool ue8m0, cudaStream_t s);
 
+int64_t ep_plan_ints(int E, int G);
+cudaError_t launch_ep_plan(const int32_t* cnt, int G, int E, int rank, int32_t* plan, cudaStream_t s);
+cudaError_t launch_ep_dispatch(const void* x_perm, const int32_t* offsets, const int32_t* plan,
+                               int E, int G, int R, int row_bytes, const uint64_t* dst_bufs,
+                               int64_t dst_rows, int32_t* status, cudaStream_t s);
+cudaError_t launch_ep_return(const void* y_loc, const int32_t* plan, int E, int G, int64_t cap,
+                             int row_bytes, const uint64_t* src_bufs, int64_t src_rows,
+                             int32_t* status, cudaStream_t s);
 cudaError_t launch_pack_weights(const void* wg, const void* wu, const void* wd, int E, int H,
                                 int I, void* w13, void* w2, cudaStream_t s);
 
@@ -810,6 +818,75 @@ moe_status_t moe_pack_weights(const void* wg, const void* wu, const void* wd, in
   MOE_TRY(check_device());
   cudaError_t e = launch_pack_weights(wg, wu, wd, E, H, I, w13, w2, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "weight packing");
+  return ok();
+}
+
+namespace {
+moe_status_t check_ep(int32_t E, int32_t G, int32_t rank) {
+  if (G < 1 || G > 64) return fail(MOE_ERR_INVALID_ARG, "G must be in [1, 64] (got %d)", G);
+  if (E < 1 || E > 1024 || E % G)
+    return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 1024] and a multiple of G (E=%d, G=%d)", E, G);
+  if (rank < 0 || rank >= G) return fail(MOE_ERR_INVALID_ARG, "rank must be in [0, G) (got %d)", rank);
+  return MOE_OK;
+}
+}  // namespace
+
+size_t moe_ep_plan_bytes(int32_t E, int32_t G) {
+  if (check_ep(E, G, 0) != MOE_OK) return 0;
+  return (size_t)ep_plan_ints(E, G) * sizeof(int32_t);
+}
+
+moe_status_t moe_ep_plan(const int32_t* counts_all, int32_t G, int32_t rank, int32_t E,
+                         int32_t* plan, void* stream) {
+  MOE_TRY(check_ep(E, G, rank));
+  MOE_TRY(check_ptr(counts_all, "counts_all"));
+  MOE_TRY(check_ptr(plan, "plan"));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_ep_plan(counts_all, G, E, rank, plan, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel plan");
+  return ok();
+}
+
+moe_status_t moe_ep_dispatch(const void* x_perm, const int32_t* offsets, const int32_t* plan,
+                             int32_t E, int32_t G, int32_t R, int64_t row_bytes,
+                             const uint64_t* dst_bufs, int64_t dst_rows, void* ws, void* stream) {
+  MOE_TRY(check_ep(E, G, 0));
+  if (R < 0) return fail(MOE_ERR_INVALID_ARG, "R must be >= 0 (got %d)", R);
+  if (row_bytes < 16 || row_bytes % 16 || row_bytes > (int64_t)1 << 30)
+    return fail(MOE_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16 (got %lld)",
+                (long long)row_bytes);
+  if (dst_rows < 0) return fail(MOE_ERR_INVALID_ARG, "dst_rows must be >= 0");
+  MOE_TRY(check_ptr(x_perm, "x_perm", R == 0));
+  MOE_TRY(check_ptr(offsets, "offsets"));
+  MOE_TRY(check_ptr(plan, "plan"));
+  MOE_TRY(check_ptr(dst_bufs, "dst_bufs"));
+  MOE_TRY(check_ptr(ws, "ws", true));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_ep_dispatch(x_perm, offsets, plan, E, G, R, (int)row_bytes, dst_bufs,
+                                     dst_rows, static_cast<int32_t*>(ws),
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel dispatch");
+  return ok();
+}
+
+moe_status_t moe_ep_return(const void* y_loc, const int32_t* plan, int32_t E, int32_t G,
+                           int64_t cap_rows, int64_t row_bytes, const uint64_t* src_bufs,
+                           int64_t src_rows, void* ws, void* stream) {
+  MOE_TRY(check_ep(E, G, 0));
+  if (cap_rows < 0 || cap_rows > ((int64_t)1 << 31) * 8)
+    return fail(MOE_ERR_INVALID_ARG, "cap_rows out of range");
+  if (row_bytes < 16 || row_bytes % 16 || row_bytes > (int64_t)1 << 30)
+    return fail(MOE_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16 (got %lld)",
+                (long long)row_bytes);
+  if (src_rows < 0) return fail(MOE_ERR_INVALID_ARG, "src_rows must be >= 0");
+  MOE_TRY(check_ptr(y_loc, "y_loc", cap_rows == 0));
+  MOE_TRY(check_ptr(plan, "plan"));
+  MOE_TRY(check_ptr(src_bufs, "src_bufs"));
+  MOE_TRY(check_ptr(ws, "ws", true));
+  MOE_TRY(check_device());
+  cudaError_t e = launch_ep_return(y_loc, plan, E, G, cap_rows, (int)row_bytes, src_bufs, src_rows,
+                                   static_cast<int32_t*>(ws), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "expert-parallel return");
   return ok();
 }
 

@@ -18,7 +18,17 @@ token exchange over NVLink. Each of G ranks owns E / G consecutive experts
 The per-rank compute steps are the library's CUDA kernels (`CudaExpertOps`);
 the exchanges are NCCL all-to-alls through torch.distributed. The class takes
 the compute steps as an object so that the exchange and regroup logic can be
-exercised by processes without a GPU.
+exercised by processes without a GPU. Its split sizes come to the host once
+per forward (NCCL's variable all-to-all takes them there).
+
+`DeviceExpertParallelMoE` keeps the whole exchange on the device: the counts
+are all-gathered into a device [G, E] matrix, `moe_ep_plan` turns it into
+every row's destination, `moe_ep_dispatch` stores the rows straight into the
+owners' receive buffers (expert-major there, so the grouped GEMMs run on them
+with no regroup) and `moe_ep_return` stores the expert outputs back into the
+sources' y_perm. The receive and y_perm buffers are symmetric memory (every
+rank maps every other rank's), the only host work is launching, and two NCCL
+all-reduces of one word order the stores before the reads.
 """
 from __future__ import annotations
 
@@ -26,8 +36,9 @@ import numpy as np
 import torch
 import torch.distributed as dist
 
-from . import (MOE_DTYPE_BF16, MOE_EPILOGUE_NONE, MOE_EPILOGUE_SWIGLU, moe_combine, moe_gather_rows,
-               moe_grouped_gemm, moe_permute, moe_route_topk, moe_workspace_size)
+from . import (MOE_DTYPE_BF16, MOE_EPILOGUE_NONE, MOE_EPILOGUE_SWIGLU, moe_combine, moe_ep_dispatch,
+               moe_ep_plan, moe_ep_plan_bytes, moe_ep_return, moe_gather_rows, moe_grouped_gemm,
+               moe_permute, moe_route_topk, moe_workspace_size)
 
 
 def regroup_plan(recv_counts) -> tuple[np.ndarray, np.ndarray]:
@@ -157,3 +168,71 @@ class ExpertParallelMoE:
         y_perm = y_recv.new_empty(x_perm.shape[0], y_recv.shape[1])
         dist.all_to_all_single(y_perm, y_recv, send_split, recv_split, group=self.group)
         return ops.combine(y_perm, w, inv_perm)
+
+
+class DeviceExpertParallelMoE:
+    """The bf16 layer with its experts spread over the ranks of `group`, the
+    exchange planned and moved on the device (no count reaches the host).
+
+    ops: this rank's `CudaExpertOps`. T_max: the most tokens a rank passes to
+    forward. Buffers are sized for the worst case: a rank receives at most
+    G * T_max * min(k, E / G) rows (a token holds each expert once)."""
+
+    def __init__(self, ops: CudaExpertOps, E: int, T_max: int, group=None):
+        import torch.distributed._symmetric_memory as symm_mem
+
+        self.ops, self.E, self.group = ops, E, group
+        self.G = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if E % self.G:
+            raise ValueError(f"E={E} does not split over {self.G} ranks")
+        self.El = E // self.G
+        self.T_max = T_max
+        k, H, dev = ops.k, ops.H, ops.device
+        self.cap = self.G * T_max * min(k, self.El)   # receive rows, worst case
+        self.R_max = T_max * k                         # a rank's own routed rows
+        gname = group.group_name if group is not None else dist.group.WORLD.group_name
+        self.x_recv = symm_mem.empty(self.cap, H, dtype=torch.bfloat16, device=dev)
+        self.y_perm = symm_mem.empty(self.R_max, H, dtype=torch.bfloat16, device=dev)
+        hx = symm_mem.rendezvous(self.x_recv, gname)
+        hy = symm_mem.rendezvous(self.y_perm, gname)
+        self.recv_ptrs = torch.tensor(list(hx.buffer_ptrs), dtype=torch.int64, device=dev)
+        self.yperm_ptrs = torch.tensor(list(hy.buffer_ptrs), dtype=torch.int64, device=dev)
+        self._handles = (hx, hy)
+        self.counts_all = torch.zeros(self.G, E, dtype=torch.int32, device=dev)
+        self.plan = torch.zeros(moe_ep_plan_bytes(E, self.G) // 4, dtype=torch.int32, device=dev)
+        self.h = torch.empty(self.cap, ops.I, dtype=torch.bfloat16, device=dev)
+        self.y_loc = torch.empty(self.cap, H, dtype=torch.bfloat16, device=dev)
+        self.status = torch.zeros(64, dtype=torch.int32, device=dev)
+        self._sync = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def _order(self):
+        """Every rank's stores so far are visible to every rank's later reads: an
+        all-reduce of one word on the stream (the host does not wait)."""
+        dist.all_reduce(self._sync, group=self.group)
+
+    def forward(self, x):
+        """x [T, H] bf16, this rank's tokens (1 <= T <= T_max); returns out [T, H]."""
+        ops, G, E, El = self.ops, self.G, self.E, self.El
+        T, H = x.shape
+        if not 1 <= T <= self.T_max:
+            raise ValueError(f"T={T} outside [1, {self.T_max}]")
+        ids, w = ops.route(x)
+        offsets, inv_perm, x_perm = ops.permute(ids, x)
+        counts = (offsets[1:] - offsets[:-1]).to(torch.int32).contiguous()
+        dist.all_gather_into_tensor(self.counts_all, counts, group=self.group)
+        moe_ep_plan(self.counts_all, G, self.rank, E, self.plan)
+        row_bytes = H * 2
+        moe_ep_dispatch(x_perm, offsets, self.plan, E, G, T * ops.k, row_bytes, self.recv_ptrs,
+                        self.cap, self.status)
+        self._order()
+        loc_off = self.plan[:El + 1]
+        ws = ops._workspace(1)
+        moe_grouped_gemm(self.x_recv, ops.w13, loc_off, self.cap, El, ops.I, H, MOE_DTYPE_BF16,
+                         MOE_EPILOGUE_SWIGLU, self.h, ws=ws)
+        moe_grouped_gemm(self.h, ops.w2, loc_off, self.cap, El, H, ops.I, MOE_DTYPE_BF16,
+                         MOE_EPILOGUE_NONE, self.y_loc, ws=ws)
+        moe_ep_return(self.y_loc, self.plan, E, G, self.cap, row_bytes, self.yperm_ptrs,
+                      self.R_max, self.status)
+        self._order()
+        return ops.combine(self.y_perm[:T * ops.k], w, inv_perm)

@@ -307,3 +307,22 @@ def test_pack_weights_validates_before_launch(monkeypatch):
     with pytest.raises(moe.MoeError) as ei:  # valid: gets as far as the device check
         moe.moe_pack_weights(wg, wu, wd, E, H, I, w13, w2, stream=0)
     assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_DEVICE
+
+
+def test_expert_parallel_exchange_validates_before_launch(monkeypatch):
+    monkeypatch.setenv("MOE_FAKE_CC", "90")
+    assert moe.moe_ep_plan_bytes(12, 3) == 4 * (8 + 12 + 13 + 12)  # loc_off padded to 4 ints
+    for E, G in [(10, 3), (0, 1), (2048, 2), (64, 0), (64, 65)]:
+        assert moe.moe_ep_plan_bytes(E, G) == 0
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ep_plan(FAKE, 3, 3, 12, FAKE, stream=0)  # rank outside [0, G)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG and "rank" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ep_dispatch(FAKE, FAKE, FAKE, 12, 3, 10, 100, FAKE, 64, stream=0)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG and "row_bytes" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ep_return(FAKE, FAKE, 12, 3, 64, 256, None, 64, stream=0)
+    assert "src_bufs is NULL" in str(ei.value)
+    with pytest.raises(moe.MoeError) as ei:  # valid: as far as the device check
+        moe.moe_ep_dispatch(FAKE, FAKE, FAKE, 12, 3, 10, 256, FAKE, 64, stream=0)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_DEVICE
