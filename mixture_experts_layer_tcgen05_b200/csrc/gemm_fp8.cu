@@ -258,22 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       // plain GEMM: scales are read two k-blocks ahead of their use (measured
       // faster there; with SwiGLU the extra registers cost more than they save)
-      float pa[2], pb0[2];
-      if (!SWIGLU) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int kj = j < nkb ? j : 0;
-          pa[j] = sa_p[kj], pb0[j] = sb0[kj];
-        }
-      }
+      // scales of k-block kb + 1 loaded while kb is promoted (rotated scalars)
+      float a_n = sa_p[0], b0_n = sb0[0], b1_n = sb1[0];
       for (int kb = 0; kb < nkb; ++kb, ++seq) {
-        float s0, s1;
-        if (SWIGLU) {
-          const float sa = sa_p[kb];
-          s0 = sa * sb0[kb], s1 = sa * sb1[kb];
-        } else {
-          s0 = s1 = pa[kb & 1] * pb0[kb & 1];
-          if (kb + 2 < nkb) pa[kb & 1] = sa_p[kb + 2], pb0[kb & 1] = sb0[kb + 2];
+        const float s0 = a_n * b0_n, s1 = SWIGLU ? a_n * b1_n : s0;
+        if (kb + 1 < nkb) {
+          a_n = sa_p[kb + 1], b0_n = sb0[kb + 1];
+          if (SWIGLU) b1_n = sb1[kb + 1];
         }
         const int pb = (int)(seq & 1);
         const uint32_t pph = (uint32_t)((seq >> 1) & 1);
@@ -291,10 +282,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_ld16(pbase + half * 64 + c, g);
             ptx::tmem_ld16(pbase + 128 + half * 64 + c, u);
             ptx::tmem_wait_ld();
+            const float2 s0p = make_float2(s0, s0), s1p = make_float2(s1, s1);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              acc[c + i] = __fmaf_rn(__uint_as_float(g[i]), s0, acc[c + i]);
-              acc[64 + c + i] = __fmaf_rn(__uint_as_float(u[i]), s1, acc[64 + c + i]);
+            for (int i = 0; i < 16; i += 2) {  // paired FMAs: two IEEE fmas per instruction
+              float2 a = __ffma2_rn(make_float2(__uint_as_float(g[i]), __uint_as_float(g[i + 1])), s0p,
+                                    make_float2(acc[c + i], acc[c + i + 1]));
+              acc[c + i] = a.x, acc[c + i + 1] = a.y;
+              float2 b = __ffma2_rn(make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])), s1p,
+                                    make_float2(acc[64 + c + i], acc[65 + c + i]));
+              acc[64 + c + i] = b.x, acc[65 + c + i] = b.y;
             }
           }
         } else {
