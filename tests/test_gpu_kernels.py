@@ -166,6 +166,9 @@ GEMM_CASES = [
     ([31, 2, 32, 0, 9], 384, 256, 32),
     # large experts: many m-tiles per expert, banded raster
     ([1500, 0, 700], 256, 384, 0),
+    # partial m-tiles of many sizes (1 row short of a 16-row step, on one, one past),
+    # alone and after full tiles
+    ([95, 96, 97, 15, 16, 17, 33, 112, 127, 128, 129, 224, 352], 256, 384, 0),
     ([2048, 1, 255], 512, 256, 0),
 ]
 
