@@ -314,6 +314,212 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
+// ==========================================================================
+// tokens-in-M kernel with two-half tiles
+// ==========================================================================
+// Plain GEMMs with a long K (>= 4096). A tile is 256 routed rows (two halves
+// of 128) by 256 weight columns. Each K step loads the two A halves and ONE
+// 256-row weight tile and issues the MMAs of both halves against it, so a
+// stage (64 KB) carries two thirds of the bytes per FLOP of a 128-row tile
+// and takes twice the MMA time to consume: the three-stage ring hides about
+// 2000 cycles of load latency instead of 1500. A half with no rows of the
+// expert is neither loaded nor multiplied. The two accumulators (128 lanes x
+// 256 columns each) fill TMEM, so there is no second buffer: eight epilogue
+// warps (four per half) drain the two halves in parallel, and the next
+// tile's MMAs into a half start as soon as that half is drained. Measured
+// (same box): Mixtral-shaped GEMM-2 (K = 14336) 718-725 vs 767-768 us with
+// 128-row tiles; the gated GEMM-1 (K = 4096 or 7168) was 2-4 % slower, its
+// shorter tiles exposing the undoubled epilogue, so it keeps 128-row tiles.
+struct Rows2Cfg {
+  static constexpr int BN = 256;
+  static constexpr int kTileB = BN * BK * 2;            // 32 KB
+  static constexpr int kStage = 2 * kTileA + kTileB;    // 64 KB
+  static constexpr int STAGES = kSmemBudget / kStage;   // 3
+  static constexpr int kThreads2 = 320;
+  static constexpr uint32_t kIdesc = ptx::make_idesc(BM, BN, 1, 1);
+  static constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + 2 * (kMaxE + 1) * 4;
+};
+
+__global__ void __launch_bounds__(Rows2Cfg::kThreads2, 1)
+    gemm_rows2_kernel(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, Args args) {
+  using C = Rows2Cfg;
+  constexpr int STAGES = C::STAGES;
+  constexpr int BM2 = 2 * BM;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStage);
+  // bars: full[STAGES], empty[STAGES], accf, acce[2], drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(smem + STAGES * C::kStage + 256);
+  int32_t* soff = tile_start + kMaxE + 1;  // [E + 1] expert offsets, shared copy
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const uint32_t full0 = ptx::smem_addr(bars), empty0 = full0 + STAGES * 8;
+  const uint32_t accf = empty0 + STAGES * 8, acce0 = accf + 8, drain = acce0 + 16;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full0 + s * 8, 1);
+      ptx::mbar_init(empty0 + s * 8, 1);
+    }
+    ptx::mbar_init(accf, 1);
+    ptx::mbar_init(acce0, 4);
+    ptx::mbar_init(acce0 + 8, 4);
+    ptx::mbar_init(drain, 1);
+    ptx::fence_barrier_init();
+    ptx::tma_prefetch_desc(&tmA);
+    ptx::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 2) build_tile_starts<BM2>(args.offsets, args.E, args.NT, tile_start, soff);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = tile_start[args.E];
+  const int nkb = args.K / BK;
+
+  auto decode = [&](int tile, int& e, int& m, int& n) {
+    e = find_expert(tile_start, args.E, tile);
+    const int local = tile - tile_start[e];
+    const int cnt = soff[e + 1] - soff[e];
+    const int mt = (cnt + BM2 - 1) / BM2;
+    const int bsz = args.band * args.NT;
+    const int b = local / bsz;
+    const int rows = min(args.band, mt - b * args.band);
+    const int l2 = local - b * bsz;
+    n = l2 / rows;
+    m = b * args.band + l2 % rows;
+  };
+  // the tile's second half holds rows of its expert
+  auto has_half1 = [&](int e, int m) {
+    return min(soff[e + 1], args.M_total) - (soff[e] + m * BM2) > BM;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, m, n;
+        decode(tile, e, m, n);
+        const int row_a = soff[e] + m * BM2;
+        const bool h1 = has_half1(e, m);
+        const int rb0 = e * args.b_rows + n * C::BN, rb1 = rb0 + 128;
+        for (int kb = 0; kb < nkb; ++kb, ++issued) {
+          const int s = (int)(issued % STAGES);
+          const uint32_t ph = (uint32_t)((issued / STAGES) & 1);
+          if (!ptx::mbar_wait(empty0 + s * 8, ph ^ 1, args.status, kSiteProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + s * C::kStage, sb = sa + 2 * kTileA;
+          ptx::mbar_arrive_expect_tx(full0 + s * 8, (h1 ? 2 * kTileA : kTileA) + C::kTileB);
+          ptx::tma_load_2d(sa, &tmA, kb * BK, row_a, full0 + s * 8);
+          if (h1) ptx::tma_load_2d(sa + kTileA, &tmA, kb * BK, row_a + BM, full0 + s * 8);
+          ptx::tma_load_2d(sb, &tmB, kb * BK, rb0, full0 + s * 8);
+          ptx::tma_load_2d(sb + 128 * 128, &tmB, kb * BK, rb1, full0 + s * 8);
+        }
+      }
+      drain_loads<STAGES>(full0, issued, args.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int64_t consumed = 0;
+      bool ok = true;
+      int t = 0;  // tiles of this CTA so far
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++t) {
+        int e, m, n;
+        decode(tile, e, m, n);
+        const bool h1 = has_half1(e, m);
+        // a half's accumulator is free once the epilogue has drained it for the previous tile
+        const uint32_t par = (uint32_t)((t & 1) ^ 1);
+        if (!ptx::mbar_wait(acce0, par, args.status, kSiteMmaAccEmpty)) break;
+        ptx::tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb, ++consumed) {
+          const int s = (int)(consumed % STAGES);
+          const uint32_t ph = (uint32_t)((consumed / STAGES) & 1);
+          if (!ptx::mbar_wait(full0 + s * 8, ph, args.status, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa = sbase + s * C::kStage, sb = sa + 2 * kTileA;
+          const uint64_t da0 = ptx::sw128_kmajor_desc(sa), db = ptx::sw128_kmajor_desc(sb);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk)
+            ptx::mma_f16(tmem_base, da0 + (uint64_t)(kk * UK * 2 / 16),
+                         db + (uint64_t)(kk * UK * 2 / 16), C::kIdesc, kb != 0 || kk != 0);
+          if (h1) {
+            if (kb == 0) {
+              if (!ptx::mbar_wait(acce0 + 8, par, args.status, kSiteMmaAccEmpty)) {
+                ok = false;
+                break;
+              }
+              ptx::tc_fence_after();
+            }
+            const uint64_t da1 = ptx::sw128_kmajor_desc(sa + kTileA);
+#pragma unroll
+            for (int kk = 0; kk < BK / UK; ++kk)
+              ptx::mma_f16(tmem_base + C::BN, da1 + (uint64_t)(kk * UK * 2 / 16),
+                           db + (uint64_t)(kk * UK * 2 / 16), C::kIdesc, kb != 0 || kk != 0);
+          }
+          ptx::mma_commit(empty0 + s * 8);
+        }
+        if (!ok) break;
+        ptx::mma_commit(accf);
+      }
+      // every MMA this thread issued has completed once `drain` fires
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, args.status, kSiteDrain);
+    }
+  } else {
+    // epilogue warps 2..9: half h = (warp - 2) / 4, TMEM lane quarter warp % 4
+    const int h = (warp - 2) >> 2;
+    const int q = warp & 3;
+    int t = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++t) {
+      int e, m, n;
+      decode(tile, e, m, n);
+      const int row0 = soff[e] + m * BM2 + h * BM;
+      const int row = row0 + q * 32 + lane;
+      const bool valid = row >= 0 && row < soff[e + 1] && row < args.M_total;
+      const bool any = h == 0 || has_half1(e, m);
+      if (!ptx::mbar_wait(accf, (uint32_t)(t & 1), args.status, kSiteEpiAccFull)) break;
+      ptx::tc_fence_after();
+      const uint32_t t0 = tmem_base + ((uint32_t)(q * 32) << 16) + h * C::BN;
+      if (any) {
+        __nv_bfloat16* dst = args.C + (int64_t)row * args.ldc + n * C::BN;
+#pragma unroll 1
+        for (int c = 0; c < C::BN; c += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld32(t0 + c, v);
+          ptx::tmem_wait_ld();
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v[i]);
+          if (valid) store_row32(dst + c, y);
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acce0 + h * 8);
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, 512);
+  }
+}
+
 // Finishes the K-split last wave of the plain gemm_rows_kernel: block (i, y)
 // takes rows [16 y, 16 y + 16) of tail tile nfull + i (the same tile order,
 // recomputed from the offsets with the GEMM's grid size G), adds its two K
@@ -681,6 +887,19 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A
   }
   a.NT = swiglu ? N / 128 : N / BN;
   a.band = 8;
+  // Plain GEMMs with a long K take two-half (256-row) tiles; the gated GEMM and
+  // short-K plain GEMMs keep 128-row tiles, whose second accumulator buffer
+  // hides their epilogue (and whose last wave can split over K).
+  if (!A_rows && !swiglu && BN == 256 && K >= 4096) {
+    a.band = 4;
+    const int64_t tiles2 = ((int64_t)M_total / (2 * gg::BM) + (M_total < E ? M_total : E)) * a.NT;
+    const unsigned grid2 = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sms, tiles2));
+    cudaError_t e = set_smem(gg::gemm_rows2_kernel, gg::Rows2Cfg::kSmem);
+    if (e != cudaSuccess) return e;
+    gg::gemm_rows2_kernel<<<grid2, gg::Rows2Cfg::kThreads2, gg::Rows2Cfg::kSmem, s>>>(tmA, tmB, a);
+    note_launch();
+    return cudaGetLastError();
+  }
   const int64_t tiles_ub = ((int64_t)M_total / gg::BM + (M_total < E ? M_total : E)) * a.NT;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sms, tiles_ub));
   // plain GEMM: scratch for a K-split last wave, at most `grid` half-tile

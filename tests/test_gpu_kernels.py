@@ -169,6 +169,9 @@ GEMM_CASES = [
     # partial m-tiles of many sizes (1 row short of a 16-row step, on one, one past),
     # alone and after full tiles
     ([95, 96, 97, 15, 16, 17, 33, 112, 127, 128, 129, 224, 352], 256, 384, 0),
+    # K >= 4096: the plain GEMM takes two-half (256-row) tiles as the gated one always
+    # does; halves with no rows, a half with one row, several 256-row tiles
+    ([0, 1, 130, 300, 513, 256], 256, 4096, 0),
     ([2048, 1, 255], 512, 256, 0),
 ]
 
