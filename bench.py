@@ -409,8 +409,9 @@ def rooflines(cfg, offsets, ms_per_step: float, stage_ms, region_ms: float, peak
 
 
 def time_steps(torch, moe, w: Workload, steps: int, warmup: int, barrier, clocks=None):
-    """`steps` forwards on the current stream between a barrier and a synchronise, with
-    per-stage events; returns (ms for all steps, mean stage ms [5], launches)."""
+    """`steps` forwards on the current stream between a barrier and a synchronise (the
+    timed region: nothing but the forwards), then `steps` more with per-stage events for
+    the breakdown; returns (ms of the timed steps, mean stage ms [5], launches, clocks)."""
     stream = torch.cuda.current_stream()
     for _ in range(max(3, warmup)):
         w.step()
@@ -418,7 +419,6 @@ def time_steps(torch, moe, w: Workload, steps: int, warmup: int, barrier, clocks
     status = moe.moe_get_device_status(w.ws)
     if status != 0:
         raise SystemExit(f"device status {status} after warm-up ({w.cfg.name})")
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if clocks is not None:
         clocks.start()
@@ -426,15 +426,20 @@ def time_steps(torch, moe, w: Workload, steps: int, warmup: int, barrier, clocks
     torch.cuda.synchronize()
     n0 = moe.moe_launch_count()
     t0.record(stream)
-    for i in range(steps):
-        moe.moe_set_stage_events(stage_ev[i])
+    for _ in range(steps):
         w.step()
     t1.record(stream)
-    moe.moe_set_stage_events(None)
     torch.cuda.synchronize()
     barrier()
     launches = moe.moe_launch_count() - n0
     clk = clocks.stop() if clocks is not None else None
+    # the stage breakdown, from a second run of the same steps
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for i in range(steps):
+        moe.moe_set_stage_events(stage_ev[i])
+        w.step()
+    moe.moe_set_stage_events(None)
+    torch.cuda.synchronize()
     stages = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(5)] for ev in stage_ev])
     return t0.elapsed_time(t1), stages.mean(0), launches, clk
 
