@@ -35,6 +35,7 @@ def _problem(counts, N2, K, tag):
     ([0, 1, 130, 300], 256, 384, 0, 4096),          # tokens-in-M kernel
     ([0, 1, 17, 64], 256, 256, 64, 4096),           # small-M kernel
     ([3, 0, 16], 128, 4096, 16, 64 << 20),          # small-M kernel with split-K
+    ([0, 1, 130, 300, 257], 256, 4096, 0, 4096),    # K >= 4096: two-half (256-row) tiles
 ])
 def test_grouped_gemm_gated(ep, act, counts, N, K, hint, ws_bytes):
     E, offsets, M, A, B = _problem(counts, 2 * N, K, 71)
