@@ -31,10 +31,20 @@ constexpr int kThreads = 320;
 constexpr int kTileA = BM * BK;  // 16 KB
 constexpr int kTileB = BN * BK;  // 32 KB
 constexpr int kStage = kTileA + kTileB;
-constexpr int STAGES = 4;
 constexpr int kMaxE = 1024;
 constexpr uint32_t kIdesc = ptx::make_idesc(BM, BN, 0, 0);  // e4m3 x e4m3 -> fp32
-constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + 256 + 2 * (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
+// The plain GEMM stages its bf16 output tile (128 x 256, 64 KB) in shared
+// memory and writes it with asynchronous bulk copies, so the promotion warps
+// go on to the next tile at once; that buffer takes the fourth ring stage.
+__host__ __device__ constexpr int stages_of(bool plain) { return plain ? 3 : 4; }
+// Staging rows are BN * 2 + 16 bytes apart: consecutive rows start 16 bytes further along the
+// banks, so the 32 rows a warp writes at once spread over them (four wavefronts a store).
+constexpr int kStgRow = BN * 2 + 16;
+__host__ __device__ constexpr int staging_of(bool plain) { return plain ? BM * kStgRow : 0; }
+__host__ __device__ constexpr size_t smem_of(bool plain) {
+  return 1024 + (size_t)stages_of(plain) * kStage + staging_of(plain) + 256 + 2 * (kMaxE + 1) * 4 +
+         2 * 2 * BM * 4;
+}
 
 struct Args {
   const int32_t* offsets;
@@ -63,13 +73,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_rows_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, Args args) {
   constexpr bool SWIGLU = ACT != kActNone;
+  constexpr int STAGES = stages_of(!SWIGLU);
+  constexpr int kStaging = staging_of(!SWIGLU);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * kStage);
+  unsigned char* staging = smem + STAGES * kStage;  // plain: [BM rows][BN cols] bf16
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + kStaging);
   // bars: full[STAGES], empty[STAGES], pfull[2], pempty[2], drain, redbar[2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 7);
-  int32_t* tile_start = reinterpret_cast<int32_t*>(smem + STAGES * kStage + 256);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(staging + kStaging + 256);
   int32_t* soff = tile_start + kMaxE + 1;  // [E + 1] expert offsets, shared copy
   float* red = reinterpret_cast<float*>(soff + kMaxE + 1);  // [2 tiles][2 halves][BM]
 
@@ -365,16 +378,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             d4[v] = make_uint4(pack_bf16x2(h[8 * v], h[8 * v + 1]), pack_bf16x2(h[8 * v + 2], h[8 * v + 3]),
                                pack_bf16x2(h[8 * v + 4], h[8 * v + 5]), pack_bf16x2(h[8 * v + 6], h[8 * v + 7]));
         }
-      } else if (valid) {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.C) + (int64_t)row * args.ldc + n * BN + half * 128;
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+      } else {
+        // this thread's 128 columns of its row: into the staging tile, then one
+        // asynchronous bulk copy of those 256 bytes to C (rows of the expert only)
+        unsigned char* srow = staging + (size_t)rl * kStgRow + half * 256;
+        if (tile_iter > 0) ptx::bulk_wait_read0();  // the previous tile's copy has read it
 #pragma unroll
-        for (int v = 0; v < 16; ++v)
-          d4[v] = make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
-                             pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+        for (int v = 0; v < 16; ++v) {
+          *reinterpret_cast<uint4*>(srow + v * 16) =
+              make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                         pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+        }
+        ptx::fence_proxy_async_smem();  // the generic-proxy writes -> visible to the bulk copy
+        if (valid) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.C) + (int64_t)row * args.ldc + n * BN + half * 128;
+          ptx::bulk_store(dst, ptx::smem_addr(srow), 256);
+        }
+        ptx::bulk_commit();
       }
     }
   }
+  if (!SWIGLU && warp >= 2) ptx::bulk_wait_all();  // every output copy has landed
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -431,9 +455,10 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_ub));
 #define MOE_FP8(SW, G)                                                                    \
   do {                                                                                    \
-    cudaError_t e = set_smem(gg8::gemm_rows_fp8_kernel<SW, G>, gg8::kSmem);               \
+    constexpr size_t smem = gg8::smem_of(SW == kActNone);                                 \
+    cudaError_t e = set_smem(gg8::gemm_rows_fp8_kernel<SW, G>, smem);                     \
     if (e != cudaSuccess) return e;                                                       \
-    gg8::gemm_rows_fp8_kernel<SW, G><<<grid, gg8::kThreads, gg8::kSmem, s>>>(tmA, tmB, a); \
+    gg8::gemm_rows_fp8_kernel<SW, G><<<grid, gg8::kThreads, smem, s>>>(tmA, tmB, a);      \
   } while (0)
 #define MOE_FP8_ACT(ACTV)           \
   do {                              \
