@@ -409,9 +409,11 @@ def rooflines(cfg, offsets, ms_per_step: float, stage_ms, region_ms: float, peak
 
 
 def time_steps(torch, moe, w: Workload, steps: int, warmup: int, barrier, clocks=None):
-    """`steps` forwards on the current stream between a barrier and a synchronise (the
-    timed region: nothing but the forwards), then `steps` more with per-stage events for
-    the breakdown; returns (ms of the timed steps, mean stage ms [5], launches, clocks)."""
+    """After the warm-up, `steps` forwards with per-stage events for the breakdown, then
+    the timed region: `steps` forwards and nothing else, between a barrier and a
+    synchronise. The breakdown runs first so that both passes see the GPU in the same
+    steady state (clock under the power cap). Returns (ms of the timed steps, mean stage
+    ms [5], launches, clocks)."""
     stream = torch.cuda.current_stream()
     for _ in range(max(3, warmup)):
         w.step()
@@ -419,6 +421,13 @@ def time_steps(torch, moe, w: Workload, steps: int, warmup: int, barrier, clocks
     status = moe.moe_get_device_status(w.ws)
     if status != 0:
         raise SystemExit(f"device status {status} after warm-up ({w.cfg.name})")
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for i in range(steps):
+        moe.moe_set_stage_events(stage_ev[i])
+        w.step()
+    moe.moe_set_stage_events(None)
+    torch.cuda.synchronize()
+    stages = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(5)] for ev in stage_ev])
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if clocks is not None:
         clocks.start()
@@ -433,14 +442,6 @@ def time_steps(torch, moe, w: Workload, steps: int, warmup: int, barrier, clocks
     barrier()
     launches = moe.moe_launch_count() - n0
     clk = clocks.stop() if clocks is not None else None
-    # the stage breakdown, from a second run of the same steps
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
-    for i in range(steps):
-        moe.moe_set_stage_events(stage_ev[i])
-        w.step()
-    moe.moe_set_stage_events(None)
-    torch.cuda.synchronize()
-    stages = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(5)] for ev in stage_ev])
     return t0.elapsed_time(t1), stages.mean(0), launches, clk
 
 
