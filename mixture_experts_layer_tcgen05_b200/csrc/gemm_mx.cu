@@ -53,8 +53,16 @@ constexpr int kSfStage = 3 * kSfA;  // A chunk + two B chunks
 constexpr int kMaxE = 1024;
 constexpr int kSfCol0 = 256;     // TMEM columns of the scale-factor ring
 constexpr int kSfColsPerStage = 16;
-constexpr size_t kSmem = 1024 + (size_t)STAGES * kStage + (size_t)STAGES * kSfStage + 256 +
-                         2 * (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
+// The plain GEMM stages its bf16 output tile in shared memory (rows 16 bytes
+// apart beyond their 512, so a warp's 16-byte stores spread over the banks)
+// and writes it with asynchronous bulk copies: the epilogue warps are free
+// to drain the next accumulator at once. That buffer takes the fourth stage.
+constexpr int kStgRow = BN * 2 + 16;
+__host__ __device__ constexpr int mx_stages(bool plain) { return plain ? 3 : STAGES; }
+__host__ __device__ constexpr size_t mx_smem(bool plain) {
+  return 1024 + (size_t)mx_stages(plain) * (kStage + kSfStage) + (plain ? (size_t)BM * kStgRow : 0) +
+         256 + 2 * (kMaxE + 1) * 4 + 2 * 2 * BM * 4;
+}
 
 struct Args {
   const int32_t* offsets;
@@ -137,14 +145,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    Args args) {
   constexpr bool SWIGLU = ACT != kActNone;
+  constexpr int STAGES = mx_stages(!SWIGLU);
+  constexpr int kStaging = SWIGLU ? 0 : BM * kStgRow;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sf = smem + STAGES * kStage;  // [STAGES][A chunk, B chunk 0, B chunk 1]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sf + STAGES * kSfStage);
+  unsigned char* staging = sf + STAGES * kSfStage;  // plain: [BM rows][kStgRow bytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + kStaging);
   // bars: full[STAGES], empty[STAGES], accf, acce, drain, redbar[2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
-  int32_t* tile_start = reinterpret_cast<int32_t*>(sf + STAGES * kSfStage + 256);
+  int32_t* tile_start = reinterpret_cast<int32_t*>(staging + kStaging + 256);
   int32_t* soff = tile_start + kMaxE + 1;  // [E + 1] expert offsets, shared copy
   float* red = reinterpret_cast<float*>(soff + kMaxE + 1);  // [2 tiles][2 halves][BM]
 
@@ -413,16 +424,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             d4[v] = make_uint4(pack_bf16x2(h[8 * v], h[8 * v + 1]), pack_bf16x2(h[8 * v + 2], h[8 * v + 3]),
                                pack_bf16x2(h[8 * v + 4], h[8 * v + 5]), pack_bf16x2(h[8 * v + 6], h[8 * v + 7]));
         }
-      } else if (valid) {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.C) + (int64_t)row * args.ldc + n * BN + half * 128;
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+      } else {
+        // this thread's 128 columns: into the staging tile, then one asynchronous bulk
+        // copy of those 256 bytes to C (rows of the expert only)
+        unsigned char* srow = staging + (size_t)rl * kStgRow + half * 256;
+        if (tile_iter > 0) ptx::bulk_wait_read0();  // the previous tile's copy has read it
 #pragma unroll
         for (int v = 0; v < 16; ++v)
-          d4[v] = make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
-                             pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+          *reinterpret_cast<uint4*>(srow + v * 16) =
+              make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                         pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+        ptx::fence_proxy_async_smem();  // the generic-proxy writes -> visible to the bulk copy
+        if (valid) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.C) + (int64_t)row * args.ldc + n * BN + half * 128;
+          ptx::bulk_store(dst, ptx::smem_addr(srow), 256);
+        }
+        ptx::bulk_commit();
       }
     }
   }
+  if (!SWIGLU && warp >= 2) ptx::bulk_wait_all();  // every output copy has landed
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -759,9 +780,10 @@ cudaError_t launch_grouped_gemm_mx(const void* A, const float* a_scales, const v
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles_ub));
 #define MOE_MX(ACTV, F4)                                                                      \
   do {                                                                                        \
-    cudaError_t e = set_smem(ggmx::gemm_mx_kernel<ACTV, F4>, ggmx::kSmem);                    \
+    constexpr size_t smem = ggmx::mx_smem(ACTV == kActNone);                                  \
+    cudaError_t e = set_smem(ggmx::gemm_mx_kernel<ACTV, F4>, smem);                           \
     if (e != cudaSuccess) return e;                                                           \
-    ggmx::gemm_mx_kernel<ACTV, F4><<<grid, ggmx::kThreads, ggmx::kSmem, s>>>(tmA, tmB, a);    \
+    ggmx::gemm_mx_kernel<ACTV, F4><<<grid, ggmx::kThreads, smem, s>>>(tmA, tmB, a);           \
   } while (0)
 #define MOE_MX_ACT(F4)                         \
   do {                                         \
