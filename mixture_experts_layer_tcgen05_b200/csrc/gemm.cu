@@ -886,7 +886,7 @@ cudaError_t launch_grouped_gemm_bf16(const void* A, const int32_t* A_rows, int A
     return cudaErrorInvalidValue;
   }
   a.NT = swiglu ? N / 128 : N / BN;
-  a.band = 8;
+  a.band = 16;
   // Plain GEMMs with a long K take two-half (256-row) tiles; the gated GEMM and
   // short-K plain GEMMs keep 128-row tiles, whose second accumulator buffer
   // hides their epilogue (and whose last wave can split over K).
