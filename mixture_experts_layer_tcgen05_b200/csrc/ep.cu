@@ -21,7 +21,7 @@
 //
 // Rows move by plain stores through the destination pointers (the buffers of
 // the other ranks mapped into this process, e.g. symmetric memory), 16 bytes
-// per lane; no TMA, no multicast. Each warp ends with a system-scope fence so
+// per lane; no TMA copies touch peer memory. Each warp ends with a system-scope fence so
 // its stores are visible to the other ranks once the stream's next
 // cross-rank synchronisation (a collective) has run.
 #include "common.cuh"
