@@ -18,6 +18,8 @@
 // (row, 128-column group) to e4m3 with scale amax/448 (the next GEMM's input).
 #include <cuda_fp8.h>
 
+#include <cstring>
+
 #include "gemm_common.cuh"
 
 namespace moe {
@@ -34,13 +36,15 @@ constexpr int kStage = kTileA + kTileB;
 constexpr int kMaxE = 1024;
 constexpr uint32_t kIdesc = ptx::make_idesc(BM, BN, 0, 0);  // e4m3 x e4m3 -> fp32
 // The plain GEMM stages its bf16 output tile (128 x 256, 64 KB) in shared
-// memory and writes it with asynchronous bulk copies, so the promotion warps
-// go on to the next tile at once; that buffer takes the fourth ring stage.
+// memory and writes it with tiled TMA stores, so the promotion warps go on
+// to the next tile at once; that buffer takes the fourth ring stage. Each
+// promotion warp owns 8 KB: its 32 rows x 128 columns as two boxes of 64
+// columns in the 128-byte-swizzled layout (row r's 16-byte chunk c at
+// r * 128 + ((c ^ (r % 8)) * 16)), which spreads the 32 rows a warp writes
+// at once over all banks and is what the store's tensor map expects.
 __host__ __device__ constexpr int stages_of(bool plain) { return plain ? 3 : 4; }
-// Staging rows are BN * 2 + 16 bytes apart: consecutive rows start 16 bytes further along the
-// banks, so the 32 rows a warp writes at once spread over them (four wavefronts a store).
-constexpr int kStgRow = BN * 2 + 16;
-__host__ __device__ constexpr int staging_of(bool plain) { return plain ? BM * kStgRow : 0; }
+constexpr int kStgWarp = 32 * 128 * 2;  // bytes of one promotion warp's two boxes
+__host__ __device__ constexpr int staging_of(bool plain) { return plain ? 8 * kStgWarp : 0; }
 __host__ __device__ constexpr size_t smem_of(bool plain) {
   return 1024 + (size_t)stages_of(plain) * kStage + staging_of(plain) + 256 + 2 * (kMaxE + 1) * 4 +
          2 * 2 * BM * 4;
@@ -71,7 +75,8 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 template <int ACT, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_rows_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ CUtensorMap tmB, Args args) {
+                         const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmC, Args args) {
   constexpr bool SWIGLU = ACT != kActNone;
   constexpr int STAGES = stages_of(!SWIGLU);
   constexpr int kStaging = staging_of(!SWIGLU);
@@ -107,6 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_barrier_init();
     ptx::tma_prefetch_desc(&tmA);
     ptx::tma_prefetch_desc(&tmB);
+    if (!SWIGLU) ptx::tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), 512);
@@ -379,22 +385,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                                pack_bf16x2(h[8 * v + 4], h[8 * v + 5]), pack_bf16x2(h[8 * v + 6], h[8 * v + 7]));
         }
       } else {
-        // this thread's 128 columns of its row: into the staging tile, then one
-        // asynchronous bulk copy of those 256 bytes to C (rows of the expert only)
-        unsigned char* srow = staging + (size_t)rl * kStgRow + half * 256;
-        if (tile_iter > 0) ptx::bulk_wait_read0();  // the previous tile's copy has read it
+        // this warp's 32 rows x 128 columns: two swizzled 64-column boxes in its
+        // staging region, then two tiled TMA stores issued by lane 0 when all 32
+        // rows belong to the expert; a row group that runs past the expert's
+        // rows stores its valid rows directly instead (a box store would
+        // overwrite the first rows of the next expert's output)
+        unsigned char* region = staging + (size_t)(warp - 2) * kStgWarp;
+        if (tile_iter > 0) {  // the previous tile's stores have read the region
+          if (lane == 0) ptx::bulk_wait_read0();
+          __syncwarp();
+        }
+        const int g0 = soff[e] + m * BM + q * 32;
+        const int nvalid = min(32, min(soff[e + 1], args.M_total) - g0);
+        if (nvalid == 32) {
 #pragma unroll
-        for (int v = 0; v < 16; ++v) {
-          *reinterpret_cast<uint4*>(srow + v * 16) =
-              make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
-                         pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+          for (int b = 0; b < 2; ++b)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float* a8 = acc + b * 64 + c * 8;
+              *reinterpret_cast<uint4*>(region + b * 4096 + lane * 128 + ((c ^ (lane & 7)) * 16)) =
+                  make_uint4(pack_bf16x2(a8[0], a8[1]), pack_bf16x2(a8[2], a8[3]),
+                             pack_bf16x2(a8[4], a8[5]), pack_bf16x2(a8[6], a8[7]));
+            }
+          ptx::fence_proxy_async_smem();  // the generic-proxy writes -> visible to the TMA store
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t src = ptx::smem_addr(region);
+            ptx::tma_store_2d(&tmC, src, n * BN + half * 128, g0);
+            ptx::tma_store_2d(&tmC, src + 4096, n * BN + half * 128 + 64, g0);
+            ptx::bulk_commit();
+          }
+        } else if (valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.C) + (int64_t)row * args.ldc +
+                                               n * BN + half * 128);
+#pragma unroll
+          for (int v = 0; v < 16; ++v)
+            d4[v] = make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                               pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
         }
-        ptx::fence_proxy_async_smem();  // the generic-proxy writes -> visible to the bulk copy
-        if (valid) {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.C) + (int64_t)row * args.ldc + n * BN + half * 128;
-          ptx::bulk_store(dst, ptx::smem_addr(srow), 256);
-        }
-        ptx::bulk_commit();
       }
     }
   }
@@ -423,11 +451,14 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_
     *why = "FP8 GEMM without SwiGLU needs N % 256 == 0";
     return cudaErrorInvalidValue;
   }
-  CUtensorMap tmA, tmB;
-  // a gathered A is read by tile::gather4 from a map whose box is one row high
+  CUtensorMap tmA, tmB, tmC;
+  std::memset(&tmC, 0, sizeof(tmC));
+  // a gathered A is read by tile::gather4 from a map whose box is one row high;
+  // the plain GEMM's bf16 output is written in 64-column x 32-row swizzled boxes
   if (!make_tmap(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, A_rows ? A_src_rows : M_total,
                  A_rows ? 1 : 128) ||
-      !make_tmap(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (int64_t)E * b_rows, 128)) {
+      !make_tmap(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (int64_t)E * b_rows, 128) ||
+      (!swiglu && !make_tmap(&tmC, Cout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M_total, 32))) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
@@ -458,7 +489,7 @@ cudaError_t launch_grouped_gemm_fp8(const void* A, const int32_t* A_rows, int A_
     constexpr size_t smem = gg8::smem_of(SW == kActNone);                                 \
     cudaError_t e = set_smem(gg8::gemm_rows_fp8_kernel<SW, G>, smem);                     \
     if (e != cudaSuccess) return e;                                                       \
-    gg8::gemm_rows_fp8_kernel<SW, G><<<grid, gg8::kThreads, smem, s>>>(tmA, tmB, a);      \
+    gg8::gemm_rows_fp8_kernel<SW, G><<<grid, gg8::kThreads, smem, s>>>(tmA, tmB, tmC, a); \
   } while (0)
 #define MOE_FP8_ACT(ACTV)           \
   do {                              \

@@ -92,6 +92,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int3
       : "memory");
 }
 
+// 2-D tiled store of the box at shared address `src` (laid out as the tensor
+// map's swizzle mode prescribes) to {c0 (inner), c1 (outer)}, tracked in this
+// thread's bulk async-groups. Both coordinates must be >= 0; rows past the
+// tensor's extent are not written.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+
 // Contiguous global -> shared copy of `bytes` (a multiple of 16, both
 // addresses 16-byte aligned); the transaction bytes complete on `bar`.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
