@@ -104,7 +104,12 @@ def _quant_f32(h):
     return q, s
 
 
-@pytest.mark.parametrize("counts,N,K", [([0, 1, 130, 300], 256, 384), ([256, 7], 512, 256)])
+# The plain GEMM stores 32-row groups of its output tile as whole boxes when all
+# 32 rows belong to the expert and row by row otherwise: experts ending exactly
+# on a 32-row group next to other experts' rows, groups of 1 and 31 rows, a
+# tile whose last groups hold no rows of its expert.
+@pytest.mark.parametrize("counts,N,K", [([0, 1, 130, 300], 256, 384), ([256, 7], 512, 256),
+                                        ([32, 33, 95, 64, 1, 31, 160], 256, 256)])
 def test_fp8_grouped_gemm_plain(counts, N, K):
     E, offsets, M, aq, as_, bq, bs = _fp8_problem(counts, N, K, 81)
     C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
