@@ -22,6 +22,7 @@ enum WaitSite : int32_t {
   kSiteDrain = 5,
   kSiteBadIndex = 6,  // an expert id / row index outside its range (skipped)
   kSiteSelfTest = 7,  // the wait of moe_check_wait_timeout
+  kSiteRowCopy = 8,   // a row's bulk load in the row scatter
 };
 
 // status word: 0 = ok; else (MOE_ERR_TIMEOUT << 8) | site

@@ -13,8 +13,11 @@
 //   3. offsets = exclusive scan of the totals over experts; the row of
 //      (token t, slot j) with expert e is
 //        offsets[e] + chunk_base[chunk(t)][e] + popc(mask[chunk(t)][e] & lanes below t).
+#include <algorithm>
+
 #include "common.cuh"
 #include "permute.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -188,6 +191,55 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const V* __restrict__
         if (v0 + i * 32 < vec_per_row) dst[j][v0 + i * 32] = u[i];
     }
   }
+}
+
+// The same scatter with the bulk-copy engine (rows a multiple of 16 bytes):
+// each warp loads its token's row into shared memory with one asynchronous
+// bulk copy, waits for it on an mbarrier (bounded), and lanes j < k each issue
+// one bulk store of the whole row to position inv_perm[t, j]; before the
+// buffer takes the next row, the lanes wait until their stores have read it.
+// The warp issues a handful of copy instructions per row instead of 32 vector
+// stores per lane per 2 KB, and the copies run while it waits.
+constexpr int kBulkWarps = 4;
+
+__global__ void __launch_bounds__(kBulkWarps * 32) scatter_rows_bulk_kernel(
+    const unsigned char* __restrict__ x, const int32_t* __restrict__ inv_perm, int T, int k,
+    int row_bytes, unsigned char* __restrict__ x_perm, int32_t* status) {
+  extern __shared__ __align__(128) unsigned char bulk_rows[];  // [kBulkWarps][row_bytes]
+  __shared__ __align__(8) uint64_t bar[kBulkWarps];
+  __shared__ int32_t local_status;  // the waits' status word when the caller passes none
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) local_status = 0;
+  if (lane == 0) ptx::mbar_init(ptx::smem_addr(&bar[warp]), 1);
+  ptx::fence_barrier_init();
+  __syncthreads();
+  int32_t* st = status ? status : &local_status;
+  const uint32_t buf = ptx::smem_addr(bulk_rows + (size_t)warp * row_bytes);
+  const uint32_t b = ptx::smem_addr(&bar[warp]);
+  const int R = T * k;
+  uint32_t phase = 0;
+  for (int t = blockIdx.x * kBulkWarps + warp; t < T; t += gridDim.x * kBulkWarps) {
+    const int mine = lane < k ? inv_perm[(int64_t)t * k + lane] : 0;
+    if (__any_sync(0xffffffffu, (unsigned)mine >= (unsigned)R)) {
+      if (lane == 0) record_bad_index(status);
+      continue;
+    }
+    ptx::bulk_wait_read0();  // this lane's stores of the previous row have read the buffer
+    __syncwarp();
+    int ok = 1;
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx(b, (uint32_t)row_bytes);
+      ptx::bulk_load(buf, x + (int64_t)t * row_bytes, (uint32_t)row_bytes, b);
+      ok = ptx::mbar_wait(b, phase, st, kSiteRowCopy);
+    }
+    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    phase ^= 1;
+    if (lane < k) {
+      ptx::bulk_store(x_perm + (int64_t)mine * row_bytes, buf, (uint32_t)row_bytes);
+      ptx::bulk_commit();
+    }
+  }
+  ptx::bulk_wait_all();  // every store has completed before the block's shared memory goes
 }
 
 // ---- small batches: permutation and row gather in one launch ---------------
@@ -415,7 +467,19 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int R, 
 cudaError_t launch_scatter_rows(const void* x, const int32_t* inv_perm, int T, int k,
                                 int row_bytes, void* x_perm, int32_t* status, cudaStream_t s) {
   if (k > kScatterMaxK) return cudaErrorNotSupported;
-  if (row_bytes % 16 == 0)
+  const size_t bulk_smem = (size_t)kBulkWarps * row_bytes;
+  if (row_bytes % 16 == 0 && bulk_smem <= 64 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(scatter_rows_bulk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bulk_smem);
+    if (e != cudaSuccess) return e;
+    int sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t blocks = std::min<int64_t>(ceil_div(T, kBulkWarps), (int64_t)std::max(sms, 1) * 3);
+    scatter_rows_bulk_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), kBulkWarps * 32, bulk_smem, s>>>(
+        static_cast<const unsigned char*>(x), inv_perm, T, k, row_bytes,
+        static_cast<unsigned char*>(x_perm), status);
+  } else if (row_bytes % 16 == 0)
     scatter_rows_kernel<uint4><<<(unsigned)ceil_div(T, 8), 256, 0, s>>>(
         static_cast<const uint4*>(x), inv_perm, T, k, row_bytes / 16, static_cast<uint4*>(x_perm),
         status);
