@@ -464,8 +464,15 @@ moe_status_t moe_ep_return(const void* y_loc_dev, const int32_t* plan_dev, int32
                            int64_t cap_rows, int64_t row_bytes, const uint64_t* src_bufs_dev,
                            int64_t src_rows, void* ws, void* stream);
 
-/* Reads the workspace's device status word (MOE_OK or MOE_ERR_TIMEOUT) into
- * *status_out. Synchronises the device (a blocking copy); not for hot loops. */
+/* Reads the workspace's device status word into *status_out: 0 (MOE_OK), or
+ * (code << 8) | site for the first failure a kernel recorded. code is
+ * MOE_ERR_TIMEOUT for a bounded wait that ran out, the site naming it: 1 a
+ * GEMM producer waiting for a free stage, 2 an MMA thread waiting for its
+ * operands, 3 an MMA thread waiting for a free accumulator, 4 an epilogue
+ * waiting for a full accumulator, 5 the final drain, 7 the self-test below,
+ * 8 a row load of the row scatter; code MOE_ERR_INVALID_ARG with site 6 means
+ * an expert id or row index out of range was met and skipped. Synchronises
+ * the device (a blocking copy); not for hot loops. */
 moe_status_t moe_get_device_status(const void* ws, int32_t* status_out);
 
 /* Clears the workspace's device status word (stream-ordered). */
