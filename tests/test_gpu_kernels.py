@@ -128,7 +128,9 @@ def _ids_cases():
 
 @pytest.mark.parametrize("case,H", [(c, 128) for c in range(10)] +
                          # rows of several 4-vector steps per lane, the last one partial
-                         [(3, 1152), (5, 7168), (6, 3200)])
+                         [(3, 1152), (5, 7168), (6, 3200),
+                          # rows above 16 KB: the vector-store scatter instead of bulk copies
+                          (3, 8320)])
 def test_permute_bit_exact(case, H):
     T, E, k, ids = _ids_cases()[case]
     d = (T, H, 128, E, k)
