@@ -9,7 +9,10 @@
 // up to one rounding, so saturation never changes a value).
 #include <cuda_fp8.h>
 
+#include <algorithm>
+
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -99,6 +102,75 @@ __global__ void __launch_bounds__(256, SCATTER ? 4 : 1) quant_act_kernel(
   }
 }
 
+// The scatter form with the bulk-copy engine, for rows whose scales fill whole
+// 16-byte units (cols % 512 == 0): each warp quantises its token's row as
+// above into a shared buffer (the codes, then the row's scales), and lanes
+// j < k each issue two bulk stores, the codes to row inv_perm[p*k + j] of q
+// and the scales to the same row of s; before the buffer takes the next
+// token the lanes wait until their stores have read it.
+constexpr int kQBulkWarps = 4;
+
+__global__ void __launch_bounds__(kQBulkWarps * 32) quant_act_scatter_bulk_kernel(
+    const uint4* __restrict__ x, int64_t rows, int64_t cols, const int32_t* __restrict__ inv_perm,
+    int k, unsigned char* __restrict__ q, float* __restrict__ s, bool ue8m0, int32_t* status) {
+  extern __shared__ __align__(16) unsigned char qrows[];  // [kQBulkWarps][cols + groups * 4]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t vpr = cols / 8, groups = cols / 128;
+  unsigned char* buf = qrows + (size_t)warp * (cols + groups * 4);
+  const uint32_t sbuf = ptx::smem_addr(buf);
+  const int64_t R = rows * k;
+  for (int64_t p = (int64_t)blockIdx.x * kQBulkWarps + warp; p < rows;
+       p += (int64_t)gridDim.x * kQBulkWarps) {
+    const int mine = lane < k ? inv_perm[p * k + lane] : 0;
+    if (__any_sync(0xffffffffu, (unsigned)mine >= (unsigned)R)) {
+      if (lane == 0) record_bad_index(status);
+      continue;
+    }
+    ptx::bulk_wait_read0();  // this lane's stores of the previous row have read the buffer
+    __syncwarp();
+    const uint4* xr = x + p * vpr;
+    for (int64_t b0 = 0; b0 < vpr; b0 += 4 * 32) {
+      uint4 ub[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t v = b0 + i * 32 + lane;
+        ub[i] = v < vpr ? xr[v] : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i) {
+        const int64_t v0 = b0 + i * 32;
+        if (v0 >= vpr) break;  // warp-uniform
+        const int64_t v = v0 + lane;
+        const bool on = v < vpr;
+        const uint4 u = ub[0];
+        ub[0] = ub[1], ub[1] = ub[2], ub[2] = ub[3];
+        const float f[8] = {bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y),
+                            bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w)};
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float sc = group_scale(amax, ue8m0);
+        if (on) {
+          *reinterpret_cast<uint2*>(buf + v * 8) =
+              make_uint2(e4m3x4(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc), __fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc)),
+                         e4m3x4(__fdiv_rn(f[4], sc), __fdiv_rn(f[5], sc), __fdiv_rn(f[6], sc), __fdiv_rn(f[7], sc)));
+          if ((lane & 15) == 0) *reinterpret_cast<float*>(buf + cols + (v / 16) * 4) = sc;
+        }
+      }
+    }
+    ptx::fence_proxy_async_smem();  // the generic-proxy writes -> visible to the bulk copies
+    __syncwarp();
+    if (lane < k) {
+      ptx::bulk_store(q + (int64_t)mine * cols, sbuf, (uint32_t)cols);
+      ptx::bulk_store(s + (int64_t)mine * groups, sbuf + (uint32_t)cols, (uint32_t)(groups * 4));
+      ptx::bulk_commit();
+    }
+  }
+  ptx::bulk_wait_all();  // every store has completed before the block's shared memory goes
+}
+
 // One block (256 threads) per 128 x 128 weight block.
 __global__ void __launch_bounds__(256) quant_weight_kernel(const __nv_bfloat16* __restrict__ w,
                                                            int64_t rows, int64_t cols,
@@ -156,9 +228,23 @@ cudaError_t launch_quant_act_scatter(const void* x, int64_t rows, int64_t cols,
                                      const int32_t* inv_perm, int k, void* q_perm, float* sc_perm,
                                      bool ue8m0, int32_t* status, cudaStream_t s) {
   if (k < 1 || k > kQuantScatterMaxK) return cudaErrorNotSupported;
-  quant_act_kernel<true><<<(unsigned)ceil_div(rows, 8), 256, 0, s>>>(
-      static_cast<const uint4*>(x), rows, cols, inv_perm, k, static_cast<uint2*>(q_perm), sc_perm,
-      ue8m0, status);
+  const size_t bulk_smem = (size_t)kQBulkWarps * (cols + cols / 128 * 4);
+  if (cols % 512 == 0 && bulk_smem <= 64 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(quant_act_scatter_bulk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bulk_smem);
+    if (e != cudaSuccess) return e;
+    int sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t blocks = std::min<int64_t>(ceil_div(rows, kQBulkWarps), (int64_t)std::max(sms, 1) * 6);
+    quant_act_scatter_bulk_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), kQBulkWarps * 32, bulk_smem,
+                                    s>>>(static_cast<const uint4*>(x), rows, cols, inv_perm, k,
+                                         static_cast<unsigned char*>(q_perm), sc_perm, ue8m0, status);
+  } else {
+    quant_act_kernel<true><<<(unsigned)ceil_div(rows, 8), 256, 0, s>>>(
+        static_cast<const uint4*>(x), rows, cols, inv_perm, k, static_cast<uint2*>(q_perm), sc_perm,
+        ue8m0, status);
+  }
   note_launch();
   return cudaGetLastError();
 }

@@ -212,3 +212,42 @@ def test_fp8_grouped_gemm_row_gather():
             g = A[lo:hi] @ Bd[e, :N].T
             u = A[lo:hi] @ Bd[e, N:].T
             check_close(got[lo:hi], g / (1 + np.exp(-g)) * u, (2e-2, 5e-3), f"expert {e}")
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+@pytest.mark.parametrize("H", [512, 768])  # 4 scale groups a row, and 6 (not 16-byte scale rows)
+def test_fp8_forward_scattered_codes_bit_exact(H, ue8m0):
+    """With more than 1024 routed rows the FP8 forwards quantise each token once and write its
+    codes and scales to the token's k permuted rows; every permuted row must hold exactly the
+    oracle's quantisation of its token (codes and scales byte for byte)."""
+    cfg = mi.CONFIGS["tiny"].with_(T=300, H=H, I=256, E=16, k=4, bias="normal")
+    L = mi.make_layer(cfg)
+    T, E, k = cfg.T, cfg.E, cfg.k
+    R = T * k
+    d = (T, H, cfg.I, E, k)
+    fmt = moe.MOE_SCALE_UE8M0 if ue8m0 else moe.MOE_SCALE_F32
+    w13q = torch.empty(E, 2 * cfg.I, H, dtype=torch.uint8, device="cuda")
+    w13s = torch.empty(E, 2 * cfg.I // 128, H // 128, dtype=torch.float32, device="cuda")
+    w2q = torch.empty(E, H, cfg.I, dtype=torch.uint8, device="cuda")
+    w2s = torch.empty(E, H // 128, cfg.I // 128, dtype=torch.float32, device="cuda")
+    moe.moe_quantize_weight_fp8_fmt(dev_bf16(L["w13"]), E, 2 * cfg.I, H, w13q, w13s, fmt)
+    moe.moe_quantize_weight_fp8_fmt(dev_bf16(L["w2"]), E, H, cfg.I, w2q, w2s, fmt)
+    ws = torch.zeros(moe.moe_workspace_size(d, moe.MOE_DTYPE_FP8_E4M3), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    args = (dev_bf16(L["x"]), dev_bf16(L["wr"]), dev(L["bias"]), w13q, w13s, w2q, w2s, d)
+    if ue8m0:
+        moe.moe_forward_fp8_ue8m0(*args, moe.MOE_EPILOGUE_SWIGLU, out, ws)
+    else:
+        moe.moe_forward_fp8(*args, out, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    lay = moe.moe_workspace_layout(d, moe.MOE_DTYPE_FP8_E4M3)
+    wsh = ws.cpu().numpy()
+    ids = wsh[lay.topk_ids:lay.topk_ids + 4 * R].view(np.int32).reshape(T, k)
+    xq = wsh[lay.xq_perm:lay.xq_perm + R * H].reshape(R, H)
+    xs = wsh[lay.xs_perm:lay.xs_perm + R * (H // 128) * 4].view(np.uint32).reshape(R, H // 128)
+    _, perm_token, _, _ = oracle.permute(ids, E)
+    rq, rs = oracle.quant_act_fp8(L["x"], ue8m0=ue8m0)
+    np.testing.assert_array_equal(xq, rq[perm_token])
+    np.testing.assert_array_equal(xs, rs.view(np.uint32)[perm_token])
